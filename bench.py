@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark one decode step of the paged KV cache on B200: the new token's K/V
+append (reshape_and_cache) followed by paged decode attention over every
+running sequence, on a seeded synthetic batch resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). ``value`` is the step's algorithmic bytes
+(K/V tiles of every distinct referenced block, q, out, block tables and
+seq_lens, plus the append's rows and slots) per second of device time, summed
+over ranks (each rank runs its own replica: the path has no exchange step).
+``roofline`` reports the decode kernel alone against the measured HBM copy
+bandwidth. ``e2e`` repeats the step with every per-step input copied in from
+pinned host memory and the output copied back inside the timed region.
+``--impl reference`` times the CPU oracle (fp64, one core) on the same
+workload, a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+from paged_kv_cache_462_b200 import accounting as acct  # noqa: E402
+
+METRIC = "paged decode KV GB/s & seq-steps/s vs B200 HBM roofline; oracle CPU time"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=1, help="workload 0..4 (default 1, Llama-3-8B bf16)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--partitions", type=int, default=0, help="decode runs (0 = automatic)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def describe(b: W.DecodeBatch) -> str:
+    sp = b.spec
+    return (f"{sp.name}: {sp.num_seqs} seqs, lengths {sp.lengths}, {sp.num_heads}q/{sp.num_kv_heads}kv heads, "
+            f"head_dim {sp.head_dim}, block {sp.block_size}, pool {b.num_blocks} blocks, kv {sp.kv_dtype}, q {sp.q_dtype}"
+            + (f", prefix groups of {sp.share_group} sharing <= {sp.share_blocks} blocks" if sp.share_group else ""))
+
+
+def step_bytes(b: W.DecodeBatch):
+    sp = b.spec
+    dec = acct.decode_bytes(b.seq_lens, b.block_tables, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                            sp.block_size, sp.kv_dtype, sp.q_dtype)
+    app = acct.append_bytes(int((b.new_slots >= 0).sum()), sp.num_kv_heads, sp.head_dim, sp.in_dtype, sp.kv_dtype)
+    return dec, app
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(config: int):
+    """DRAM bytes per decode launch from the committed ncu summary, if it matches this kernel build."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_sha") != kernel_sha() or int(rec.get("config", -1)) != config:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("decode_kernel.cuh", "device.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_462_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.on = False
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if self.on:
+                self.samples.append([x.strip() for x in line.split(",")])
+
+    def start(self):
+        self.on = True
+
+    def stop(self):
+        self.on = False
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in self.samples:
+            try:
+                sm.append(float(s[1]))
+                mx.append(float(s[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, s[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def smi_index(torch, dev: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if dev < len(parts):
+            return parts[dev]
+    return str(dev)
+
+
+# ----------------------------------------------------------------------------- device state
+
+class DeviceState:
+    def __init__(self, torch, pkv, b: W.DecodeBatch, device, partitions: int):
+        self.torch, self.pkv, self.b, self.dev = torch, pkv, b, device
+        sp = b.spec
+        self.q = self._dev(b.q, sp.q_dtype)
+        self.bt = torch.from_numpy(b.block_tables).to(device)
+        self.sl = torch.from_numpy(b.seq_lens).to(device)
+        self.new_k = self._dev(b.new_k, sp.in_dtype)
+        self.new_v = self._dev(b.new_v, sp.in_dtype)
+        self.new_slots = torch.from_numpy(b.new_slots).to(device)
+        cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[sp.kv_dtype]
+        shape = (b.num_blocks, sp.num_kv_heads, sp.block_size, sp.head_dim)
+        self.kc = torch.zeros(shape, dtype=cdt, device=device)
+        self.vc = torch.zeros(shape, dtype=cdt, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.out = torch.empty_like(self.q)
+        self.partitions = partitions
+        self.ws = pkv.new_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, partitions, device)
+        for i in range(0, b.hist_slots.size, 1 << 16):      # history already in the cache before the step
+            pkv.reshape_and_cache(self._dev(b.hist_k[i:i + (1 << 16)], sp.in_dtype),
+                                  self._dev(b.hist_v[i:i + (1 << 16)], sp.in_dtype), self.kc, self.vc,
+                                  torch.from_numpy(b.hist_slots[i:i + (1 << 16)]).to(device),
+                                  float(b.k_scale), float(b.v_scale), self.err)
+        torch.cuda.synchronize(device)
+
+    def _dev(self, a, name):
+        t = self.torch
+        if name == "bf16":
+            return t.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(t.bfloat16).to(self.dev)
+        return t.from_numpy(np.ascontiguousarray(a)).to(self.dev)
+
+    def append(self):
+        b = self.b
+        self.pkv.reshape_and_cache(self.new_k, self.new_v, self.kc, self.vc, self.new_slots,
+                                   float(b.k_scale), float(b.v_scale), self.err)
+
+    def decode(self):
+        b = self.b
+        self.pkv.paged_attention_decode(self.out, self.q, self.kc, self.vc, self.bt, self.sl, float(b.scale),
+                                        float(b.k_scale), float(b.v_scale), self.partitions, self.ws)
+
+    def errors(self):
+        self.torch.cuda.synchronize(self.dev)
+        return int(self.err.item()) | self.pkv.read_device_error(self.ws)
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_pair_sampler(b: W.DecodeBatch):
+    """Single (sequence, KV head 0) attention problems cut from the batch, for timing the oracle.
+
+    Returns a list of (callable, bytes). The data preparation (history fill through
+    the oracle's own append, slicing of KV head 0) is done here, outside the timing.
+    """
+    import oracle
+    sp = b.spec
+    G = sp.num_heads // sp.num_kv_heads
+    rng = np.random.default_rng(0)
+    seqs = rng.permutation(b.num_seqs)[: min(b.num_seqs, 16)].tolist()
+    _, kc, vc = oracle.run_step(b, seqs=seqs)
+    kc0 = np.ascontiguousarray(kc[:, 0:1])
+    vc0 = np.ascontiguousarray(vc[:, 0:1])
+    q0 = np.ascontiguousarray(b.q[:, 0:G])
+    nk0 = np.ascontiguousarray(b.new_k[:, 0:1])
+    nv0 = np.ascontiguousarray(b.new_v[:, 0:1])
+    items = []
+    for s in seqs:
+        L = int(b.seq_lens[s])
+        nbytes = (acct.decode_bytes(b.seq_lens[s:s + 1], b.block_tables[s:s + 1], G, 1, sp.head_dim,
+                                    sp.block_size, sp.kv_dtype, sp.q_dtype)["total"]
+                  + acct.append_bytes(1, 1, sp.head_dim, sp.in_dtype, sp.kv_dtype))
+
+        def run(s=s):
+            oracle.reshape_and_cache(nk0, nv0, sp.in_dtype, kc0, vc0, sp.kv_dtype, b.new_slots, 1, sp.head_dim,
+                                     sp.block_size, b.num_blocks, b.k_scale, b.v_scale, rows=[s])
+            oracle.paged_decode(q0, sp.q_dtype, kc0, vc0, sp.kv_dtype, b.block_tables, b.seq_lens, G, 1,
+                                sp.head_dim, sp.block_size, b.num_blocks, b.scale, b.k_scale, b.v_scale, seqs=[s])
+        items.append((run, nbytes, L))
+    return items
+
+
+def time_oracle(items, seconds: float):
+    done_bytes, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        run, nbytes, _ = items[n % len(items)]
+        run()
+        done_bytes += nbytes
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done_bytes / el / 1e9, n, el
+
+
+# ----------------------------------------------------------------------------- arms
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    b = W.config_batch(args.config)
+    items = oracle_pair_sampler(b)
+    # size each step to a bounded sample: one (sequence, kv head) pair, so the run stays within minutes
+    for i in range(args.warmup):
+        items[i % len(items)][0]()
+    times, nbytes = [], 0
+    for i in range(args.steps):
+        run, nb, _ = items[i % len(items)]
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+        nbytes += nb
+    total = sum(times)
+    value = nbytes / total / 1e9
+    sample = (f"one (sequence, KV head 0) attention problem per step, cycling over {len(items)} sequences "
+              f"of the workload, append of its new token included; fp64 C oracle, single thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(b), "config_index": args.config},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ours_arm(args):
+    import torch
+    import paged_kv_cache_462_b200 as pkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    pkv.load_library()
+
+    spec = W.config_spec(args.config)
+    b = W.build_batch(spec, seed=spec.seed + 1000 * rank)
+    state = DeviceState(torch, pkv, b, dev, args.partitions)
+    dec, app = step_bytes(b)
+    bytes_step = dec["total"] + app
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        state.append()
+        state.decode()
+    torch.cuda.synchronize(dev)
+    if state.errors():
+        raise SystemExit(f"device error word {state.errors()} after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(smi_index(torch, local)) if rank == 0 else None
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+    for i in range(K):
+        flush.zero_()                     # cold L2 for every step (outside the step's events)
+        ev[i][0].record(stream)
+        state.append()
+        ev[i][1].record(stream)
+        state.decode()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.stop()
+    if dist:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    app_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    ms = sum(step_ms) / K
+    errs = state.errors()
+
+    # end to end: per-step inputs from pinned host memory, output back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        host = {n: getattr(state, n).detach().cpu().pin_memory() for n in ("q", "new_k", "new_v", "new_slots", "sl", "bt")}
+        out_h = torch.empty(state.out.shape, dtype=state.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        Ke = K
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+        for i in range(Ke + args.warmup):
+            flush.zero_()
+            rec = i >= args.warmup
+            if rec:
+                ee[i - args.warmup][0].record(stream)
+            for n, t in host.items():
+                getattr(state, n).copy_(t, non_blocking=True)
+            state.append()
+            state.decode()
+            out_h.copy_(state.out, non_blocking=True)
+            if rec:
+                ee[i - args.warmup][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = sum(a.elapsed_time(c) for a, c in ee) / Ke
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    # aggregate over ranks: max time, summed bytes
+    vals = torch.tensor([ms, sum(dec_ms) / K, e2e["ms"] if e2e else 0.0, float(bytes_step), float(errs)],
+                        dtype=torch.float64, device=dev)
+    if dist:
+        mx = vals.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        tot = vals.clone()
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        ms_max, dec_max, e2e_max = mx[0].item(), mx[1].item(), mx[2].item()
+        bytes_all = tot[3].item()
+        errs_all = int(mx[4].item())
+    else:
+        ms_max, dec_max, e2e_max, bytes_all, errs_all = ms, sum(dec_ms) / K, (e2e["ms"] if e2e else 0.0), bytes_step, errs
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        dec_gbs = dec["total"] / (sum(dec_ms) / K * 1e-3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": bytes_all / (ms_max * 1e-3) / 1e9,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": describe(b), "config_index": args.config,
+                "kv_storage": spec.kv_dtype, "partitions": args.partitions or pkv.default_partitions(
+                    spec.head_dim, spec.block_size, spec.num_heads, spec.num_kv_heads,
+                    {"f32": 0, "bf16": 1, "e4m3": 2}[spec.kv_dtype]),
+                "step": "reshape_and_cache of one new token per sequence + paged_attention_decode",
+                "l2": "flushed before every step (256 MiB write outside the step's CUDA events)",
+                "replicas": world,
+            },
+            "seq_steps_per_s": world * spec.num_seqs / (ms_max * 1e-3),
+            "decode_us": dec_max * 1e3,
+            "append_us": sum(app_ms) / K * 1e3,
+            "kv_logical_gbs": dec["kv_logical"] / (sum(dec_ms) / K * 1e-3) / 1e9,
+            "step_bytes": bytes_step,
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "paged_decode_kernel",
+                "achieved": dec_gbs,
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": dec_gbs / peak,
+                "traffic": kernel_traffic(args.config),
+                "algorithmic_bytes": dec["total"],
+            },
+            "gpu_launches": 2 * K,
+            "clocks": clocks.summary() if clocks else None,
+            "device_errors": errs_all,
+        }
+        if e2e:
+            line["e2e"] = {"value": bytes_all / (e2e_max * 1e-3) / 1e9, "unit": "GB/s",
+                           "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_max}
+        if world == 1 and not args.no_cpu_baseline:
+            items = oracle_pair_sampler(b)
+            v, n, el = time_oracle(items, args.cpu_seconds)
+            line["cpu_baseline"] = {
+                "value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                "sample": f"{n} single (sequence, KV head 0) problems of this workload cycled for {el:.1f} s "
+                          f"(append + attention each), fp64 C oracle, one thread"}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return ours_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

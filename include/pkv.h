@@ -1,0 +1,165 @@
+/*
+ * pkv.h — C ABI of the B200 paged KV-cache decode library (libpagedkv.so).
+ *
+ * Two operations make up one decode step of a vLLM-style serving loop:
+ *
+ *   reshape_and_cache       append each new token's K and V rows to the paged
+ *                           cache at the slot the scheduler gave it
+ *                           ("vLLM inference cost optimisation",
+ *                           developer.aliyun.com, section 1: the decode loop
+ *                           generates new K/V and writes them into the KV cache).
+ *   paged_attention_decode  for every running sequence, the single new query of
+ *                           each head attends over all cached tokens,
+ *                           out = softmax(q K^T * scale) V (same article, section 2),
+ *                           reading K/V block by block through the sequence's
+ *                           block table, which maps logical blocks to scattered
+ *                           physical blocks of a shared pool (same article,
+ *                           section 4 "PagedAttention"; wzjinhao.cn vLLM
+ *                           write-up, section 2.1).
+ *
+ * Layouts (row-major; the pages fix none of them):
+ *   k_cache, v_cache   [num_blocks][num_kv_heads][block_size][head_dim]
+ *                      elements of kv_dtype. One (block, kv head) tile is
+ *                      block_size*head_dim elements, contiguous.
+ *   q, out             [num_seqs][num_heads][head_dim], q_dtype (out has q's dtype).
+ *   block_tables       int32 [num_seqs][max_blocks_per_seq]; entry j of row s
+ *                      is the physical block of logical block j of sequence s.
+ *                      Only entries j < ceil(seq_lens[s] / block_size) are read.
+ *   seq_lens           int32 [num_seqs]: cached tokens to attend over,
+ *                      including the token being decoded. 0 gives a zero row.
+ *   k, v (append)      [num_tokens][num_kv_heads][head_dim] of in_dtype.
+ *   slot_mapping       int64 [num_tokens]: slot = block * block_size + offset;
+ *                      a negative slot writes nothing.
+ * Grouped-query attention: query head g reads KV head g / (num_heads / num_kv_heads)
+ * (a group of query heads shares one KV head: Aliyun article, GQA/MQA section).
+ *
+ * dtypes: q_dtype/kv_dtype pairs (F32, F32), (BF16, BF16), (BF16, FP8_E4M3).
+ * FP8 caches hold OCP E4M3 codes of x / scale with per-tensor fp32 scales
+ * (Aliyun article, section 15 "the KV cache itself can be quantized";
+ * promptx.wiki tutorial, per-tensor KV scales). Arithmetic is fp32 throughout.
+ * head_dim in {64, 128}; block_size in {8, 16, 32};
+ * num_heads / num_kv_heads in {1, 2, 4, 5, 8}.
+ *
+ * Ownership and synchronisation: every pointer except `stream` is DEVICE
+ * memory owned by the caller. The library never allocates, never frees and
+ * never synchronises; all work is enqueued on `stream` (a cudaStream_t, NULL =
+ * the legacy default stream) and the calls return as soon as it is queued.
+ *
+ * Errors: problems visible on the host (null pointers, unsupported sizes or
+ * dtypes, a workspace that is too small) return a non-zero pkv_status before
+ * anything is launched. A failed launch returns PKV_ERR_LAUNCH. Bad DATA
+ * (a block id outside [0, num_blocks), a seq_len outside
+ * [0, max_blocks_per_seq * block_size], a slot past the end of the pool) is
+ * never read or written: the kernels skip the access and OR one of the
+ * PKV_DEVERR_* bits into a device error word, which the caller reads with
+ * pkv_read_device_error().
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_NULL = 1,        /* a required pointer is NULL */
+    PKV_ERR_SHAPE = 2,       /* unsupported or inconsistent size */
+    PKV_ERR_DTYPE = 3,       /* unsupported dtype or dtype pair */
+    PKV_ERR_WORKSPACE = 4,   /* workspace missing or smaller than paged_attention_workspace_size() */
+    PKV_ERR_LAUNCH = 5,      /* the CUDA runtime refused or failed the launch */
+    PKV_ERR_DEVICE = 6       /* device query failed (no device, bad context) */
+} pkv_status;
+
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks): block skipped */
+#define PKV_DEVERR_SEQ_LEN 2   /* seq_len < 0 or > max_blocks_per_seq * block_size: clamped */
+#define PKV_DEVERR_SLOT 4      /* append slot >= num_blocks * block_size: row skipped */
+#define PKV_DEVERR_TIMEOUT 8   /* a bounded pipeline wait gave up (output incomplete) */
+
+/*
+ * Bytes of device workspace paged_attention_decode needs: an error word, one
+ * arrival counter per (sequence, kv head) and fp32 split-KV partials
+ * (o[G][head_dim], m[G], l[G]) for up to num_partitions + num_seqs*num_kv_heads
+ * segments. num_partitions = 0 sizes it for the automatic partition count on
+ * the current device. Returns 0 for unsupported sizes.
+ */
+PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                      int num_partitions);
+
+/*
+ * Zero a workspace (asynchronously on `stream`). Required once after the
+ * workspace is allocated, and again after a call that reported
+ * PKV_DEVERR_TIMEOUT; every normal call leaves the counters at zero.
+ */
+PKV_API int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Paged decode attention. One launch: the total work, sum over (sequence,
+ * kv head) of ceil(seq_len / block_size) blocks, is cut into num_partitions
+ * equal runs of blocks (0 = one or more per SM, from the occupancy); a run
+ * may cover several (sequence, kv head) pairs and a pair may be split across
+ * runs. Each run streams its K/V tiles through shared memory and keeps an
+ * online softmax; a pair split across runs is finished by whichever run
+ * arrives last, which merges the fp32 partials from the workspace (the
+ * log-sum-exp combination), so no run ever waits for another.
+ *
+ *   out          [num_seqs][num_heads][head_dim], q_dtype
+ *   q            [num_seqs][num_heads][head_dim], q_dtype
+ *   scale        softmax scale (1/sqrt(head_dim) for standard attention)
+ *   k_scale, v_scale  per-tensor dequantisation scales for FP8 caches
+ *                (ignored for F32/BF16 caches)
+ *   workspace    device buffer of >= paged_attention_workspace_size(...,
+ *                num_partitions) bytes, zeroed once by pkv_workspace_init;
+ *                calls that share a workspace must not overlap on the GPU.
+ */
+PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                           int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                           float k_scale, float v_scale, int num_partitions,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode-step append: for every token t with slot_mapping[t] >= 0, write
+ * k[t][h][:] to k_cache[slot / block_size][h][slot % block_size][:] (and v the
+ * same way) for every kv head h. Same dtype: a bit copy. FP8_E4M3 cache from
+ * F32 or BF16 rows: code = E4M3(x / k_scale) with an IEEE fp32 division and
+ * round-to-nearest-even, saturating to +-448 (v with v_scale).
+ * Duplicate non-negative slots in one call give an unspecified winner.
+ * device_error: optional int32 device word that receives PKV_DEVERR_SLOT.
+ */
+PKV_API int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                      const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, int in_dtype, int kv_dtype,
+                      float k_scale, float v_scale, int32_t* device_error, void* stream);
+
+/*
+ * Copy the workspace's device error word to *host_error (synchronising on
+ * `stream`); clear != 0 also resets it to zero.
+ */
+PKV_API int pkv_read_device_error(void* workspace, size_t workspace_bytes, int32_t* host_error, int clear,
+                          void* stream);
+
+/* Number of partitions num_partitions = 0 resolves to for this configuration on the current device. */
+PKV_API int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_kv_heads, int kv_dtype);
+
+/* Static description of a status code. */
+PKV_API const char* pkv_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

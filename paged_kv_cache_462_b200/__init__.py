@@ -1,0 +1,196 @@
+"""Paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of ``libpagedkv.so`` (C ABI declared in ``include/pkv.h``).
+Functions here only check and marshal torch tensors (device pointers, sizes,
+dtypes, the current CUDA stream); every step of the computation runs in the
+library's CUDA kernels. There is no CPU fallback: without the built library
+(``python -m paged_kv_cache_462_b200.build``) every call raises.
+
+Entry points (same names as the C ABI):
+
+* ``reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, ...)`` — append
+  the decode step's new K/V rows into their cache slots.
+* ``paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens,
+  scale, ...)`` — single-query grouped attention for every sequence, reading
+  K/V block by block through the block table.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpagedkv.so")
+
+F32, BF16, FP8_E4M3 = 0, 1, 2
+DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+_TORCH_DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3}
+
+_lib = None
+
+
+class PkvError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: status {status} ({status_string(status)})")
+
+
+def load_library():
+    """Load libpagedkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_462_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.paged_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.paged_attention_workspace_size.restype = sz
+    lib.pkv_workspace_init.argtypes = [P, sz, P]
+    lib.pkv_workspace_init.restype = i32
+    lib.paged_attention_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                           f32, f32, i32, P, sz, P]
+    lib.paged_attention_decode.restype = i32
+    lib.reshape_and_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, f32, P, P]
+    lib.reshape_and_cache.restype = i32
+    lib.pkv_read_device_error.argtypes = [P, sz, ctypes.POINTER(ctypes.c_int32), i32, P]
+    lib.pkv_read_device_error.restype = i32
+    lib.pkv_default_partitions.argtypes = [i32, i32, i32, i32, i32]
+    lib.pkv_default_partitions.restype = i32
+    lib.pkv_status_string.argtypes = [i32]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().pkv_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != 0:
+        raise PkvError(fn, status)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _TORCH_DTYPE[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _cuda(name, t: torch.Tensor):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions=0) -> int:
+    n = load_library().paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions)
+    if n == 0:
+        raise PkvError("paged_attention_workspace_size", 2)
+    return int(n)
+
+
+def new_workspace(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions=0, device=None) -> torch.Tensor:
+    """A zeroed (i.e. initialised) workspace tensor for paged_attention_decode."""
+    n = workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _check("pkv_workspace_init",
+           load_library().pkv_workspace_init(_cuda("workspace", workspace), workspace.numel(), _stream_handle(stream)))
+
+
+def default_partitions(head_dim, block_size, num_heads, num_kv_heads, kv_dtype) -> int:
+    code = kv_dtype if isinstance(kv_dtype, int) else _TORCH_DTYPE[kv_dtype]
+    n = load_library().pkv_default_partitions(head_dim, block_size, num_heads, num_kv_heads, code)
+    if n <= 0:
+        raise PkvError("pkv_default_partitions", -n)
+    return n
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale,
+                           k_scale=1.0, v_scale=1.0, num_partitions=0, workspace=None, stream=None) -> None:
+    """out[s, g] = softmax(scale * q[s, g] . K) V over the seq_lens[s] cached tokens of sequence s.
+
+    q, out: [num_seqs, num_heads, head_dim] (float32 or bfloat16);
+    k_cache, v_cache: [num_blocks, num_kv_heads, block_size, head_dim]
+    (float32, bfloat16, or uint8/float8_e4m3fn E4M3 codes with k_scale/v_scale);
+    block_tables: int32 [num_seqs, max_blocks_per_seq]; seq_lens: int32 [num_seqs].
+    """
+    S, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q/out and the caches")
+    if out.dtype != q.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("out must match q's dtype and v_cache k_cache's")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
+    if workspace is None:
+        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, q.device)
+    st = load_library().paged_attention_decode(
+        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
+        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
+        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _stream_handle(stream))
+    _check("paged_attention_decode", st)
+
+
+def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=1.0, v_scale=1.0,
+                      device_error=None, stream=None) -> None:
+    """Write k[t], v[t] ([num_tokens, num_kv_heads, head_dim]) into slot slot_mapping[t] of the caches."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, BS, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between rows and caches")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise TypeError("slot_mapping must be int64 [num_tokens]")
+    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error)
+    st = load_library().reshape_and_cache(
+        _cuda("k", k), _cuda("v", v), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+        _cuda("slot_mapping", slot_mapping), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
+        float(k_scale), float(v_scale), err, _stream_handle(stream))
+    _check("reshape_and_cache", st)
+
+
+def read_device_error(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:
+    """The workspace's device error word (PKV_DEVERR_* bits); synchronises the stream."""
+    v = ctypes.c_int32(0)
+    _check("pkv_read_device_error", load_library().pkv_read_device_error(
+        _cuda("workspace", workspace), workspace.numel(), ctypes.byref(v), int(clear), _stream_handle(stream)))
+    return int(v.value)
+
+
+_ws_cache: dict = {}
+
+
+def _cached_workspace(S, Hq, Hkv, D, parts, device):
+    n = workspace_size(S, Hq, Hkv, D, parts)
+    key = (str(device), parts)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < n:
+        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+__all__ = [
+    "paged_attention_decode", "reshape_and_cache", "workspace_size", "new_workspace", "workspace_init",
+    "read_device_error", "default_partitions", "status_string", "load_library", "PkvError",
+    "F32", "BF16", "FP8_E4M3",
+]

@@ -1,0 +1,287 @@
+// C ABI of libpagedkv: argument validation, workspace layout and launch.
+// Every entry point validates what the host can see and returns a pkv_status
+// before launching anything; nothing here allocates, frees or synchronises
+// (pkv_read_device_error excepted, which synchronises by design).
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include <cuda_runtime.h>
+
+#include "pkv_internal.h"
+
+namespace pkv {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634074f;
+
+std::mutex g_mu;
+std::map<std::pair<const void*, int>, size_t> g_smem_set;   // (kernel, device) -> dynamic smem limit set
+std::map<int, int> g_sm_count;                                // device -> SMs
+
+int current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return -1;
+    return dev;
+}
+
+int sm_count(int dev)
+{
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_sm_count.find(dev);
+    if (it != g_sm_count.end())
+        return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    g_sm_count[dev] = n;
+    return n;
+}
+
+bool group_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 5 || g == 8; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int slot_floats_for(int group, int head_dim) { return (int)round_up((size_t)group * (head_dim + 2), 4); }
+
+struct WorkspaceLayout {
+    size_t counters_off, partials_off, bytes;
+};
+
+WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_dim, long long runs)
+{
+    WorkspaceLayout w;
+    const long long pairs = (long long)num_seqs * num_kv_heads;
+    w.counters_off = kWorkspaceHeader;
+    w.partials_off = w.counters_off + round_up((size_t)pairs * 4, 256);
+    w.bytes = w.partials_off + (size_t)(runs + pairs) * slot_floats_for(group, head_dim) * 4;
+    return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool ensure_smem_attribute(const void* kernel, size_t bytes)
+{
+    const int dev = current_device();
+    if (dev < 0)
+        return false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto key = std::make_pair(kernel, dev);
+    auto it = g_smem_set.find(key);
+    if (it != g_smem_set.end() && it->second >= bytes)
+        return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    g_smem_set[key] = bytes;
+    return true;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(int status)
+{
+    switch (status) {
+    case PKV_OK:
+        return "ok";
+    case PKV_ERR_NULL:
+        return "a required pointer is NULL";
+    case PKV_ERR_SHAPE:
+        return "unsupported or inconsistent size, or a misaligned cache/row pointer";
+    case PKV_ERR_DTYPE:
+        return "unsupported dtype or dtype pair";
+    case PKV_ERR_WORKSPACE:
+        return "workspace missing or too small";
+    case PKV_ERR_LAUNCH:
+        return "kernel launch failed";
+    case PKV_ERR_DEVICE:
+        return "CUDA device query failed";
+    default:
+        return "unknown status";
+    }
+}
+
+size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                      int num_partitions)
+{
+    if (num_seqs < 0 || num_kv_heads <= 0 || num_heads <= 0 || num_heads % num_kv_heads != 0)
+        return 0;
+    const int group = num_heads / num_kv_heads;
+    if (!group_supported(group) || (head_dim != 64 && head_dim != 128) || num_partitions < 0)
+        return 0;
+    long long runs = num_partitions;
+    if (runs == 0) {
+        const int dev = current_device();
+        const int sms = dev >= 0 ? sm_count(dev) : 0;
+        if (sms <= 0)
+            return 0;
+        runs = (long long)sms * kMaxRunsPerSM;
+    }
+    return layout_for(num_seqs, num_kv_heads, group, head_dim, runs).bytes;
+}
+
+int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!workspace)
+        return PKV_ERR_NULL;
+    if (workspace_bytes < kWorkspaceHeader)
+        return PKV_ERR_WORKSPACE;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_LAUNCH;
+}
+
+int pkv_read_device_error(void* workspace, size_t workspace_bytes, int32_t* host_error, int clear, void* stream)
+{
+    if (!workspace || !host_error)
+        return PKV_ERR_NULL;
+    if (workspace_bytes < kWorkspaceHeader)
+        return PKV_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return PKV_ERR_LAUNCH;
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return PKV_ERR_LAUNCH;
+    *host_error = v;
+    if (clear && v != 0) {
+        if (cudaMemsetAsync(workspace, 0, sizeof v, st) != cudaSuccess)
+            return PKV_ERR_LAUNCH;
+    }
+    return PKV_OK;
+}
+
+int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_kv_heads, int kv_dtype)
+{
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+        return -PKV_ERR_SHAPE;
+    const int dev = current_device();
+    const int sms = dev >= 0 ? sm_count(dev) : 0;
+    if (sms <= 0)
+        return -PKV_ERR_DEVICE;
+    const int q_dtype = kv_dtype == PKV_F32 ? PKV_F32 : PKV_BF16;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.num_seqs = 1;
+    int occ = 0;
+    const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, p, 0,
+                                   nullptr, &occ);
+    if (st != PKV_OK)
+        return -st;
+    if (occ < 1)
+        occ = 1;
+    if (occ > kMaxRunsPerSM)
+        occ = kMaxRunsPerSM;
+    return sms * occ;
+}
+
+int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                           int num_blocks, int q_dtype, int kv_dtype, float k_scale, float v_scale,
+                           int num_partitions, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads != 0 || num_partitions < 0)
+        return PKV_ERR_SHAPE;
+    const int group = num_heads / num_kv_heads;
+    if (!group_supported(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_ERR_SHAPE;
+    if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
+          (q_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3)))
+        return PKV_ERR_DTYPE;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
+        return PKV_ERR_NULL;
+    if (!workspace)
+        return PKV_ERR_WORKSPACE;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return PKV_ERR_SHAPE;
+    if ((long long)num_seqs * max_blocks_per_seq * num_kv_heads >= (1ll << 31) ||
+        (long long)max_blocks_per_seq * block_size >= (1ll << 31))
+        return PKV_ERR_SHAPE;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
+        return PKV_ERR_SHAPE;
+
+    int runs = num_partitions;
+    if (runs == 0) {
+        const int dev = current_device();
+        const int sms = dev >= 0 ? sm_count(dev) : 0;
+        if (sms <= 0)
+            return PKV_ERR_DEVICE;
+        DecodeParams probe;
+        std::memset(&probe, 0, sizeof probe);
+        probe.num_seqs = num_seqs;
+        int occ = 0;
+        const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, probe, 0, nullptr, &occ);
+        if (st != PKV_OK)
+            return st;
+        if (occ < 1)
+            return PKV_ERR_SHAPE;
+        runs = sms * (occ > kMaxRunsPerSM ? kMaxRunsPerSM : occ);
+    }
+    const WorkspaceLayout lay = layout_for(num_seqs, num_kv_heads, group, head_dim, runs);
+    if (workspace_bytes < lay.bytes)
+        return PKV_ERR_WORKSPACE;
+
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.out = out;
+    p.q = q;
+    p.k_cache = static_cast<const uint8_t*>(k_cache);
+    p.v_cache = static_cast<const uint8_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.q_scale = scale * kLog2e * (fp8 ? k_scale * kv_unbias(kv_dtype) : 1.0f);
+    p.v_scale = fp8 ? v_scale * kv_unbias(kv_dtype) : 1.0f;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.err = reinterpret_cast<int32_t*>(ws);
+    p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
+    p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
+    p.slot_floats = slot_floats_for(group, head_dim);
+    return decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, p, runs,
+                           static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                      int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
+                      int kv_dtype, float k_scale, float v_scale, int32_t* device_error, void* stream)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_ERR_SHAPE;
+    if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) &&
+          (kv_dtype == in_dtype || kv_dtype == PKV_FP8_E4M3)))
+        return PKV_ERR_DTYPE;
+    if (num_tokens == 0)
+        return PKV_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping)
+        return PKV_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return PKV_ERR_SHAPE;
+    if (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.0f && v_scale > 0.0f))
+        return PKV_ERR_SHAPE;
+    return cache_dispatch(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                          num_blocks, in_dtype, kv_dtype, k_scale, v_scale, device_error,
+                          static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

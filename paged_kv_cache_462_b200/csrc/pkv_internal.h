@@ -1,0 +1,50 @@
+// Internal declarations shared by the translation units of libpagedkv.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+constexpr int kMaxSmemPerBlock = 227 * 1024;
+constexpr int kMaxSeqs = 16384;         // per call: the per-sequence tile prefix lives in shared memory
+constexpr int kMaxRunsPerSM = 4;        // automatic partition count is at most 4 runs per SM
+constexpr size_t kWorkspaceHeader = 256;
+
+struct DecodeParams {
+    void* out;
+    const void* q;
+    const uint8_t* k_cache;
+    const uint8_t* v_cache;
+    const int32_t* block_tables;
+    const int32_t* seq_lens;
+    int num_seqs;
+    int num_heads;
+    int num_kv_heads;
+    int max_blocks_per_seq;
+    int num_blocks;
+    float q_scale;     // scale * log2(e) * k_scale * (2^120 for E4M3 caches)
+    float v_scale;     // v_scale * (2^120 for E4M3 caches)
+    int32_t* err;      // workspace error word
+    int32_t* counters; // [num_seqs * num_kv_heads] arrivals, zero between calls
+    float* partials;   // [(runs + pairs)][slot_floats]
+    int slot_floats;
+    int stages_per_warp; // set by the launcher
+};
+
+int decode_dispatch(int q_dtype, int kv_dtype, int head_dim, int block_size, int group,
+                    const DecodeParams& p, int nruns, cudaStream_t stream, int* occupancy_out);
+float kv_unbias(int kv_dtype);
+
+int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                   int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                   int in_dtype, int kv_dtype, float k_scale, float v_scale, int32_t* err, cudaStream_t stream);
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device (cached).
+bool ensure_smem_attribute(const void* kernel, size_t bytes);
+
+}  // namespace pkv

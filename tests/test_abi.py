@@ -1,0 +1,93 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol and
+rejects bad host-visible arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_462_b200 as pkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_462_b200 import build
+    build.build()
+    return pkv.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) >= {"paged_attention_decode", "reshape_and_cache", "paged_attention_workspace_size"}
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert pkv.status_string(code)
+    assert pkv.status_string(0) == "ok"
+
+
+def test_workspace_size_with_explicit_partitions(lib):
+    # 64 seqs, 32/8 heads, d=128, 296 runs: header + counters + (296 + 512) slots of 4*(128+2) floats
+    n = lib.paged_attention_workspace_size(64, 32, 8, 128, 296)
+    slot = 4 * (128 + 2)
+    assert n == 256 + 2048 + (296 + 512) * slot * 4
+    assert lib.paged_attention_workspace_size(64, 30, 8, 128, 296) == 0     # 30 % 8 != 0
+    assert lib.paged_attention_workspace_size(64, 24, 8, 128, 296) == 0     # group 3 unsupported
+    assert lib.paged_attention_workspace_size(64, 32, 8, 96, 296) == 0      # head_dim 96 unsupported
+
+
+def _decode(lib, **kw):
+    a = dict(out=None, q=None, k=None, v=None, bt=None, sl=None, S=4, Hq=8, Hkv=2, D=64, BS=16, scale=0.125,
+             MB=4, NB=32, qdt=0, kvdt=0, ks=1.0, vs=1.0, parts=0, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return lib.paged_attention_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["sl"], a["S"], a["Hq"], a["Hkv"],
+                                      a["D"], a["BS"], a["scale"], a["MB"], a["NB"], a["qdt"], a["kvdt"], a["ks"],
+                                      a["vs"], a["parts"], a["ws"], a["wsb"], a["stream"])
+
+
+FAKE = 0x10000  # never dereferenced: every case below fails host validation first
+
+
+def test_decode_host_validation(lib):
+    ptrs = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, ws=FAKE, wsb=1 << 20)
+    assert _decode(lib, **ptrs, Hq=6, Hkv=4) == 2          # heads not a multiple
+    assert _decode(lib, **ptrs, D=96) == 2                  # head_dim
+    assert _decode(lib, **ptrs, BS=12) == 2                 # block size
+    assert _decode(lib, **ptrs, qdt=1, kvdt=0) == 3         # dtype pair
+    assert _decode(lib, **ptrs, qdt=2, kvdt=2) == 3
+    assert _decode(lib, **dict(ptrs, q=None)) == 1          # null
+    assert _decode(lib, **dict(ptrs, ws=None)) == 4         # no workspace
+    assert _decode(lib, **ptrs, MB=0) == 2
+    assert _decode(lib, **dict(ptrs, k=FAKE + 8)) == 2      # misaligned cache for the bulk copies
+    assert _decode(lib, S=0) == 0                           # empty batch: nothing to do
+
+
+def test_append_host_validation(lib):
+    f = lib.reshape_and_cache
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 96, 16, 8, 0, 0, 1.0, 1.0, None, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 0, 1.0, 1.0, None, None) == 3   # bf16 -> f32
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 2, 2, 1.0, 1.0, None, None) == 3   # e4m3 input
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 4, 2, 64, 16, 8, 0, 0, 1.0, 1.0, None, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 2, 0.0, 1.0, None, None) == 2   # zero fp8 scale
+    assert f(None, None, None, None, None, 0, 2, 64, 16, 8, 0, 0, 1.0, 1.0, None, None) == 0   # nothing to append
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 8, 64)
+    kc = torch.zeros(4, 2, 16, 64)
+    with pytest.raises(ValueError):
+        pkv.paged_attention_decode(q.clone(), q, kc, kc.clone(), torch.zeros(1, 4, dtype=torch.int32),
+                                   torch.ones(1, dtype=torch.int32), 0.125, workspace=torch.zeros(1 << 20, dtype=torch.uint8))

@@ -1,0 +1,228 @@
+"""CUDA path against the CPU oracle, element by element, through the C ABI.
+
+Tolerances (max |gpu - oracle| over every output element, oracle in fp64 on the
+same rounded inputs): 1e-5 for fp32 caches, 1e-2 for bf16, 3e-2 for FP8-E4M3.
+The append (reshape_and_cache) must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_462_b200 as pkv
+import workloads as W
+from gpu_harness import TOL, GpuStep, cache_bytes, max_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _spec(name, S, Hq, Hkv, D, BS, kv, lengths, pool=None, seed=1, share=0):
+    q = "f32" if kv == "f32" else "bf16"
+    nb = max(1, -(-max(lengths) // BS))
+    pool = pool or ("fixed", max(8, 2 * sum(-(-L // BS) for L in lengths) + 3))
+    return W.Spec(name, S, Hq, Hkv, D, BS, q, q, kv, ("list", tuple(lengths)), pool,
+                  share_group=share, share_blocks=4 if share else 0, max_blocks_per_seq=nb + 1, seed=seed)
+
+
+def _check_step(batch, partitions=(0,)):
+    ref, okc, ovc = oracle.run_step(batch)
+    g = GpuStep(batch)
+    g.append()
+    torch.cuda.synchronize()
+    assert np.array_equal(cache_bytes(g.kc), okc), "K cache differs from the oracle's append"
+    assert np.array_equal(cache_bytes(g.vc), ovc), "V cache differs from the oracle's append"
+    for parts in partitions:
+        out = g.decode(parts)
+        e = max_err(out, ref)
+        assert e <= TOL[batch.spec.kv_dtype], (parts, e)
+        assert g.device_errors() == 0
+    return g, ref
+
+
+# ------------------------------------------------------------------ append
+
+def test_append_fp8_special_values():
+    """Saturation, ties, subnormals and signed zero through the hardware E4M3 conversion."""
+    vals = np.array([0.0, -0.0, 448.0, 449.0, 1e9, -1e9, np.inf, -np.inf, 2.0 ** -10, -(2.0 ** -10),
+                     3 * 2.0 ** -11, 1.0625, 1.1875, 17.0, 19.0, 240.0, 248.0, 2.0 ** -9, 1e-30, 0.3],
+                    dtype=np.float32)
+    D = 64
+    rows = np.resize(vals, (3, 1, D)).astype(np.float32)
+    rows[1] *= -1.5
+    rows[2] = np.random.default_rng(3).standard_normal((1, D)).astype(np.float32) * 1000
+    slots = np.array([3, 17, 40], np.int64)
+    okc = oracle.empty_cache(4, 1, 16, D, "e4m3"); ovc = oracle.empty_cache(4, 1, 16, D, "e4m3")
+    oracle.reshape_and_cache(rows, rows, "f32", okc, ovc, "e4m3", slots, 1, D, 16, 4, 1.0, 0.5)
+    kc = torch.zeros(4, 1, 16, D, dtype=torch.uint8, device="cuda"); vc = torch.zeros_like(kc)
+    t = torch.from_numpy(rows).cuda()
+    pkv.reshape_and_cache(t, t.clone(), kc, vc, torch.from_numpy(slots).cuda(), 1.0, 0.5)
+    assert np.array_equal(kc.cpu().numpy(), okc)
+    assert np.array_equal(vc.cpu().numpy(), ovc)
+
+
+@pytest.mark.parametrize("kv,inp", [("f32", "f32"), ("bf16", "bf16"), ("e4m3", "bf16"), ("e4m3", "f32")])
+def test_append_bit_exact_and_padding(kv, inp):
+    rng = np.random.default_rng(5)
+    T, Hkv, D, BS, NB = 300, 4, 128, 16, 40
+    rows_k = rng.standard_normal((T, Hkv, D)).astype(np.float32) * 3
+    rows_v = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+    if inp == "bf16":
+        rows_k, rows_v = W.f32_to_bf16_bits(rows_k), W.f32_to_bf16_bits(rows_v)
+    slots = rng.permutation(NB * BS)[:T].astype(np.int64)
+    slots[::7] = -1                                          # padding rows write nothing
+    ks, vs = (np.float32(3 * 4.5 / 448), np.float32(4.5 / 448)) if kv == "e4m3" else (np.float32(1), np.float32(1))
+    okc = oracle.empty_cache(NB, Hkv, BS, D, kv); ovc = oracle.empty_cache(NB, Hkv, BS, D, kv)
+    oracle.reshape_and_cache(rows_k, rows_v, inp, okc, ovc, kv, slots, Hkv, D, BS, NB, ks, vs)
+    kc = torch.zeros(okc.shape, dtype={"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[kv],
+                     device="cuda")
+    vc = torch.zeros_like(kc)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.reshape_and_cache(to_dev(rows_k, inp), to_dev(rows_v, inp), kc, vc, torch.from_numpy(slots).cuda(),
+                          float(ks), float(vs), err)
+    assert np.array_equal(cache_bytes(kc), okc) and np.array_equal(cache_bytes(vc), ovc)
+    assert int(err.item()) == 0
+
+
+def test_append_slot_past_pool_is_flagged_not_written():
+    k = torch.ones(3, 2, 64, device="cuda")
+    kc = torch.zeros(2, 2, 16, 64, device="cuda"); vc = torch.zeros_like(kc)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.reshape_and_cache(k, k, kc, vc, torch.tensor([1, 32, 5000], device="cuda"), device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pkv.DEVERR_SLOT
+    assert kc.sum().item() == 2 * 64 and kc[0, :, 1].eq(1).all()
+
+
+# ------------------------------------------------------------------ decode
+
+def test_config0_full():
+    b = W.config_batch(0)
+    _check_step(b, partitions=(0, 1, 2, 3, 7, 16, 1000))
+
+
+@pytest.mark.parametrize("kv", ["f32", "bf16", "e4m3"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("BS", [8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 5, 8])
+def test_shapes_grid(kv, D, BS, G):
+    Hkv = 2
+    lengths = [0, 1, BS, BS + 1, 3 * BS - 1, 97, 200]
+    b = W.build_batch(_spec(f"grid_{kv}_{D}_{BS}_{G}", len(lengths), G * Hkv, Hkv, D, BS, kv, lengths,
+                            seed=D * 1000 + BS * 10 + G))
+    g, _ = _check_step(b, partitions=(0, 5))
+    out = g.out.float().cpu().numpy()
+    assert np.all(out[0] == 0)                               # empty sequence: zero row
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_configs_cut_down_every_output(cfg):
+    """Same distributions as the full workloads, a few sequences: every output element checked."""
+    over = {1: dict(num_seqs=6), 2: dict(num_seqs=2, lengths=("fixed", 2000)),
+            3: dict(num_seqs=16), 4: dict(num_seqs=5)}[cfg]
+    b = W.config_batch(cfg, **over)
+    _check_step(b, partitions=(0, 1, 3, 17, 148))
+
+
+def test_split_invariance_sweep():
+    b = W.config_batch(1, num_seqs=8)
+    ref, _, _ = oracle.run_step(b)
+    g = GpuStep(b)
+    g.append()
+    for parts in (1, 2, 3, 4, 5, 8, 13, 16, 37, 64, 148, 296, 592, 2000):
+        e = max_err(g.decode(parts), ref)
+        assert e <= TOL["bf16"], (parts, e)
+    assert g.device_errors() == 0
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_full_size_sampled(cfg):
+    """Full workload in the benchmark's launch configuration; sampled sequences checked one by one."""
+    b = W.config_batch(cfg)
+    g = GpuStep(b)
+    out = g.step(0)
+    torch.cuda.synchronize()
+    assert g.device_errors() == 0
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(cfg)
+    seqs = sorted(set(rng.choice(b.num_seqs, size=min(6, b.num_seqs), replace=False).tolist())
+                  | {int(np.argmax(b.seq_lens)), int(np.argmin(b.seq_lens))})
+    ref, okc, ovc = oracle.run_step(b, seqs=seqs)
+    e = max_err(out, ref, seqs)
+    assert e <= TOL[b.spec.kv_dtype], e
+    # every block those sequences read (history fill + the step's append) is bit-exact
+    bs = b.spec.block_size
+    nb = b.nblocks()
+    blocks = np.unique(np.concatenate([b.block_tables[s, :nb[s]] for s in seqs]))
+    idx = torch.from_numpy(blocks.astype(np.int64)).cuda()
+    assert np.array_equal(cache_bytes(g.kc[idx]), okc[blocks])
+    assert np.array_equal(cache_bytes(g.vc[idx]), ovc[blocks])
+
+
+def test_prefix_sharing_equals_private_copies():
+    """Shared prefix blocks are read-only reuse: duplicating them physically changes nothing."""
+    b = W.config_batch(3, num_seqs=16)
+    g1 = GpuStep(b)
+    o1 = g1.step(7).clone()
+    # private copy of every shared block, appended to the pool
+    bs = b.spec.block_size
+    nb = b.nblocks()
+    used = {}
+    tables = b.block_tables.copy()
+    extra_src = []
+    for s in range(b.num_seqs):
+        for j in range(nb[s]):
+            p = int(tables[s, j])
+            if p in used:
+                tables[s, j] = b.num_blocks + len(extra_src)
+                extra_src.append(p)
+            used.setdefault(p, s)
+    assert extra_src, "workload has no shared blocks"
+    g2 = GpuStep(b)
+    g2.append()
+    kc2 = torch.cat([g2.kc, g2.kc[torch.tensor(extra_src, device="cuda")]])
+    vc2 = torch.cat([g2.vc, g2.vc[torch.tensor(extra_src, device="cuda")]])
+    out2 = torch.empty_like(g2.q)
+    ws = pkv.new_workspace(b.num_seqs, b.spec.num_heads, b.spec.num_kv_heads, b.spec.head_dim, 7)
+    pkv.paged_attention_decode(out2, g2.q, kc2, vc2, torch.from_numpy(tables).cuda(), g2.sl, float(b.scale),
+                               num_partitions=7, workspace=ws)
+    assert torch.equal(o1, out2)
+
+
+def test_permutation_invariance_bit_exact():
+    b = W.config_batch(1, num_seqs=8)
+    g = GpuStep(b)
+    o1 = g.step(11).clone()
+    perm = torch.from_numpy(np.random.default_rng(9).permutation(b.num_blocks)).cuda()
+    kc2 = torch.empty_like(g.kc); vc2 = torch.empty_like(g.vc)
+    kc2[perm] = g.kc; vc2[perm] = g.vc
+    bt = torch.from_numpy(b.block_tables).cuda()
+    bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].int(), bt)
+    out2 = torch.empty_like(g.q)
+    pkv.paged_attention_decode(out2, g.q, kc2, vc2, bt2, g.sl, float(b.scale), num_partitions=11,
+                               workspace=pkv.new_workspace(8, 32, 8, 128, 11))
+    assert torch.equal(o1, out2)
+
+
+def test_bad_block_id_is_flagged_and_skipped():
+    b = W.config_batch(1, num_seqs=4)
+    g = GpuStep(b)
+    g.append()
+    bt = b.block_tables.copy()
+    bt[2, 3] = b.num_blocks + 5                              # outside the pool
+    g.bt = torch.from_numpy(bt).cuda()
+    out = g.decode(0)
+    torch.cuda.synchronize()
+    assert g.device_errors() & pkv.DEVERR_BLOCK_ID
+    ref, _, _ = oracle.run_step(b, seqs=[0, 1, 3])
+    assert max_err(out, ref, [0, 1, 3]) <= TOL["bf16"]       # other sequences untouched
+
+
+def test_bad_seq_len_is_flagged_and_clamped():
+    b = W.config_batch(0)
+    g = GpuStep(b)
+    g.append()
+    sl = b.seq_lens.copy()
+    sl[1] = 10_000                                           # beyond max_blocks_per_seq * block_size
+    g.sl = torch.from_numpy(sl).cuda()
+    g.decode(0)
+    assert g.device_errors() & pkv.DEVERR_SEQ_LEN
