@@ -16,8 +16,8 @@
 //    runs and CTA c owns run c (one CTA per SM by default). A run may cover
 //    several pairs and a pair may span several runs; the part of a pair inside
 //    one run is a "segment".
-//  * The 8 warps of a CTA take the run's tiles round-robin (tile k -> warp
-//    k % 8). Each warp owns P shared-memory stages (K tile + V tile) and is its
+//  * The W warps of a CTA (8, or 4 when 8 stages would not fit) take the run's
+//    tiles round-robin (tile k -> warp k % W). Each warp owns P shared-memory stages (K tile + V tile) and is its
 //    own producer: lane 0 issues one bulk copy (TMA, non-tensor) per tile half
 //    into a stage and re-arms the stage's mbarrier as soon as the warp has
 //    finished reading it, so P tiles per warp (up to ~200 KB per SM) are in
@@ -32,7 +32,7 @@
 //    over its LPT lanes by a transposing butterfly that leaves each lane with
 //    one head's score; the online softmax keeps its running max until a new
 //    block max passes it by 8 (log2 units), so most blocks skip the rescale.
-//  * At the end of a segment the 8 warps merge in shared memory. A segment
+//  * At the end of a segment the W warps merge in shared memory. A segment
 //    that covers its whole pair writes the output; otherwise it stores fp32
 //    (o, m, l) partials in the workspace and the last run to arrive on the
 //    pair's counter (atomic, then reset to zero) merges them with the
@@ -49,8 +49,6 @@
 namespace pkv {
 
 constexpr float kRescaleSlack = 8.0f;  // log2 units
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 constexpr int kMaxStagesPerWarp = 8;
 
 template <class KV, class QT, int D, int BS, int G>
@@ -66,7 +64,10 @@ struct Cfg {
     static constexpr int kTile = BS * kRowBytes;                // one (block, kv head) tile
     static constexpr int kStageBytes = 2 * kTile;               // K + V
     static constexpr int kIters = BS / TPP;                     // warp passes per tile
-    static constexpr int kScratchFloats = kWarps * (G * D + 2 * G);
+    // 8 warps, each with at least one stage, unless the stages do not fit: then 4
+    static constexpr int W = (8 * (kStageBytes + 12) + 8 * (G * D + 2 * G) * 4 + 4096 <= kMaxSmemPerBlock) ? 8 : 4;
+    static constexpr int kThreads = W * 32;
+    static constexpr int kScratchFloats = W * (G * D + 2 * G);
     static_assert(kEPL * LPT == D, "lane split");
     static_assert(kChunk == 4 || kChunk == 8 || kChunk == 16, "chunk size");
     static_assert(kTile % 16 == 0, "bulk copies move multiples of 16 bytes");
@@ -161,10 +162,11 @@ __device__ __forceinline__ long long tile_offset(const DecodeParams& p, const in
 }
 
 template <class KV, class QT, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 1) paged_decode_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(Cfg<KV, QT, D, BS, G>::kThreads, 1) paged_decode_kernel(const DecodeParams p)
 {
     using C = Cfg<KV, QT, D, BS, G>;
-    constexpr int W = kWarps;
+    constexpr int W = C::W;
+    constexpr int kThreads = C::kThreads;
     constexpr int LPT = C::LPT;
     const int P = p.stages_per_warp;
     const int S = W * P;
@@ -558,7 +560,7 @@ struct DecodeLauncher {
     static int stages_per_warp(int num_seqs)
     {
         const long long room = (long long)kMaxSmemPerBlock - (long long)fixed_smem(num_seqs);
-        const long long per = (long long)kWarps * (C::kStageBytes + 12);   // stage + barrier + skip flag
+        const long long per = (long long)C::W * (C::kStageBytes + 12);   // stage + barrier + skip flag
         long long P = room / per;
         if (P > kMaxStagesPerWarp)
             P = kMaxStagesPerWarp;
@@ -567,7 +569,7 @@ struct DecodeLauncher {
 
     static size_t smem_bytes(int num_seqs, int P)
     {
-        return fixed_smem(num_seqs) + (size_t)kWarps * P * (C::kStageBytes + 12);
+        return fixed_smem(num_seqs) + (size_t)C::W * P * (C::kStageBytes + 12);
     }
 
     static int occupancy(int num_seqs)
@@ -580,7 +582,7 @@ struct DecodeLauncher {
         const size_t smem = smem_bytes(num_seqs, P);
         if (!ensure_smem_attribute((const void*)kern, smem))
             return 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, C::kThreads, smem) != cudaSuccess)
             return 0;
         return n;
     }
@@ -595,7 +597,7 @@ struct DecodeLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = P;
-        kern<<<nruns, kThreads, smem, stream>>>(p);
+        kern<<<nruns, C::kThreads, smem, stream>>>(p);
         return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
     }
 };
