@@ -42,6 +42,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include "device.cuh"
 #include "pkv_internal.h"
@@ -61,6 +62,7 @@ struct Cfg {
     static constexpr int kEPC = kChunk / kElt;                  // elements per chunk
     static constexpr int kCPL = kRowBytes / (LPT * kChunk);     // chunks per lane per row
     static constexpr int kEPL = kEPC * kCPL;                    // elements per lane = D / LPT
+    static constexpr int kPairs = kEPL / 2;                     // fp32 pairs per lane per row
     static constexpr int kTile = BS * kRowBytes;                // one (block, kv head) tile
     static constexpr int kStageBytes = 2 * kTile;               // K + V
     static constexpr int kIters = BS / TPP;                     // warp passes per tile
@@ -303,33 +305,37 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, BS, G>::kThreads, 1) paged_deco
         int L = p.seq_lens[s];
         L = L < 0 ? 0 : (L > capacity ? capacity : L);
 
-        float qr[G][C::kEPL];
+        // q rows of the group as fp32 pairs, pre-scaled (scale * log2(e) [* k_scale * 2^120])
+        float2 q2[G][C::kPairs];
         {
             const QT* qp = reinterpret_cast<const QT*>(p.q) + ((size_t)s * p.num_heads + (size_t)h * G) * D;
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int e = 0; e < C::kEPL; ++e) {
-                    const int d = ((e / C::kEPC) * LPT + j) * C::kEPC + (e % C::kEPC);
-                    qr[g][e] = to_float(qp[g * D + d]) * p.q_scale;
+                for (int c = 0; c < C::kCPL; ++c) {
+                    float t[C::kEPC];
+                    load_q<C::kEPC>(qp + g * D + (c * LPT + j) * C::kEPC, t);
+#pragma unroll
+                    for (int i = 0; i < C::kEPC / 2; ++i)
+                        q2[g][c * (C::kEPC / 2) + i] = make_float2(t[2 * i] * p.q_scale, t[2 * i + 1] * p.q_scale);
                 }
         }
-        float o[G][C::kEPL];
+        float2 o2[G][C::kPairs];
         float m[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             m[g] = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < C::kEPL; ++e)
-                o[g][e] = 0.f;
+            for (int e = 0; e < C::kPairs; ++e)
+                o2[g][e] = make_float2(0.f, 0.f);
         }
         float l_own = 0.f, m_own = -INFINITY;
 
-        // own tiles inside [x, seg_end): k = warp + W*own
-        for (; own < own_count && run_begin + warp + W * own < seg_end; ++own) {
-            const int k = warp + W * own;
-            const int st = warp + W * (own % P);
-            const uint32_t parity = (own / P) & 1;
+        // own tiles inside [x, seg_end): tile k = warp + W*own; two tiles per step
+        // give each warp two independent q.K / p.V streams and one shared max reduction
+        auto wait_tile = [&](int o) {
+            const int st = warp + W * (o % P);
+            const uint32_t parity = (o / P) & 1;
             bool ok = true;
             if (!aborted)
                 ok = !*abort_flag && mbar_wait_bounded(&full[st], parity);
@@ -340,108 +346,153 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, BS, G>::kThreads, 1) paged_deco
                 }
                 aborted = true;
             }
-            const int jb = (run_begin + k) - pair_begin;   // logical block
-            const int valid = min(BS, L - jb * BS);
-            if (!aborted && skip[st] == 0 && valid > 0) {
-                const uint8_t* kt = stages + (size_t)st * C::kStageBytes;
-                const uint8_t* vt = kt + C::kTile;
-                float sc[C::kIters];
+        };
+        auto tiles = [&](auto nt_tag) {
+            constexpr int NT = decltype(nt_tag)::value;
+            const uint8_t* kt[NT];
+            int valid[NT];
+            bool live[NT];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const int st = warp + W * ((own + t) % P);
+                const int jb = run_begin + warp + W * (own + t) - pair_begin;   // logical block
+                valid[t] = min(BS, L - jb * BS);
+                live[t] = !aborted && skip[st] == 0 && valid[t] > 0;        // warp-uniform
+                kt[t] = stages + (size_t)st * C::kStageBytes;
+            }
+            // ---- scores for this lane's head and tokens tq + TPP*it of each tile
+            float sc[NT][C::kIters];
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
 #pragma unroll
                 for (int it = 0; it < C::kIters; ++it) {
-                    const uint8_t* row = kt + (tq + C::TPP * it) * C::kRowBytes;
+                    const uint8_t* row = kt[t] + (tq + C::TPP * it) * C::kRowBytes;
+                    float2 acc2[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+                        acc2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < C::kCPL; ++c) {
+                        float2 kf[C::kEPC / 2];
+                        load_widen2<KV, C::kChunk>(row + (c * LPT + j) * C::kChunk, kf);
+#pragma unroll
+                        for (int i = 0; i < C::kEPC / 2; ++i)
+#pragma unroll
+                            for (int g = 0; g < G; ++g)
+                                acc2[g] = __ffma2_rn(q2[g][c * (C::kEPC / 2) + i], kf[i], acc2[g]);
+                    }
                     float acc[G];
 #pragma unroll
                     for (int g = 0; g < G; ++g)
-                        acc[g] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < C::kCPL; ++c) {
-                        float kf[C::kEPC];
-                        load_widen<KV, C::kChunk>(row + (c * LPT + j) * C::kChunk, kf);
-#pragma unroll
-                        for (int i = 0; i < C::kEPC; ++i)
-#pragma unroll
-                            for (int g = 0; g < G; ++g)
-                                acc[g] = fmaf(qr[g][c * C::kEPC + i], kf[i], acc[g]);
-                    }
-                    sc[it] = tr_reduce_from<G, LPT / 2>(acc, j);
-                    if (tq + C::TPP * it >= valid)
-                        sc[it] = -INFINITY;
+                        acc[g] = acc2[g].x + acc2[g].y;
+                    const float v = tr_reduce_from<G, LPT / 2>(acc, j);
+                    sc[t][it] = (live[t] && tq + C::TPP * it < valid[t]) ? v : -INFINITY;
                 }
-                float bm = sc[0];
+            // ---- running max per head (lazy: move it only when the block max passes it by the slack)
+            float bm = sc[0][0];
 #pragma unroll
-                for (int it = 1; it < C::kIters; ++it)
-                    bm = fmaxf(bm, sc[it]);
+            for (int t = 0; t < NT; ++t)
 #pragma unroll
-                for (int off = LPT; off < 32; off <<= 1)
-                    bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, off));
-                bool moved = false;
-                float alpha[G];
+                for (int it = 0; it < C::kIters; ++it)
+                    bm = fmaxf(bm, sc[t][it]);
+#pragma unroll
+            for (int off = LPT; off < 32; off <<= 1)
+                bm = fmaxf(bm, __shfl_xor_sync(kFullMask, bm, off));
+            bool moved = false;
+            float alpha[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float b = __shfl_sync(kFullMask, bm, head_src_lane<G, LPT>(g));
+                const bool up = b > m[g] + kRescaleSlack;
+                const float mn = up ? b : m[g];
+                alpha[g] = up ? fast_exp2(m[g] - mn) : 1.f;
+                moved |= up;
+                m[g] = mn;
+            }
+            if (moved) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float b = __shfl_sync(kFullMask, bm, head_src_lane<G, LPT>(g));
-                    const bool up = b > m[g] + kRescaleSlack;
-                    const float mn = up ? b : m[g];
-                    alpha[g] = up ? fast_exp2(m[g] - mn) : 1.f;
-                    moved |= up;
-                    m[g] = mn;
-                }
-                if (moved) {
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-#pragma unroll
-                        for (int e = 0; e < C::kEPL; ++e)
-                            o[g][e] *= alpha[g];
-                        if (g == myhead) {
-                            l_own *= alpha[g];
-                            m_own = m[g];
-                        }
+                    for (int e = 0; e < C::kPairs; ++e)
+                        o2[g][e] = make_float2(o2[g][e].x * alpha[g], o2[g][e].y * alpha[g]);
+                    if (g == myhead) {
+                        l_own *= alpha[g];
+                        m_own = m[g];
                     }
                 }
-                float pr[C::kIters];
+            }
+            float pr[NT][C::kIters];
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
 #pragma unroll
                 for (int it = 0; it < C::kIters; ++it) {
-                    pr[it] = fast_exp2(sc[it] - m_own);
-                    l_own += pr[it];
+                    pr[t][it] = (sc[t][it] == -INFINITY) ? 0.f : fast_exp2(sc[t][it] - m_own);
+                    l_own += pr[t][it];
                 }
+            // ---- o += p V for every head of the group
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (!live[t])
+                    continue;
+                const uint8_t* vt = kt[t] + C::kTile;
 #pragma unroll
                 for (int it = 0; it < C::kIters; ++it) {
-                    float pg[G];
+                    float2 pg[G];
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        pg[g] = __shfl_sync(kFullMask, pr[it], group_base | head_src_lane<G, LPT>(g));
-                    if (tq + C::TPP * it < valid) {
+                    for (int g = 0; g < G; ++g) {
+                        const float pv = __shfl_sync(kFullMask, pr[t][it], group_base | head_src_lane<G, LPT>(g));
+                        pg[g] = make_float2(pv, pv);
+                    }
+                    if (tq + C::TPP * it < valid[t]) {
                         const uint8_t* row = vt + (tq + C::TPP * it) * C::kRowBytes;
 #pragma unroll
                         for (int c = 0; c < C::kCPL; ++c) {
-                            float vf[C::kEPC];
-                            load_widen<KV, C::kChunk>(row + (c * LPT + j) * C::kChunk, vf);
+                            float2 vf[C::kEPC / 2];
+                            load_widen2<KV, C::kChunk>(row + (c * LPT + j) * C::kChunk, vf);
 #pragma unroll
-                            for (int i = 0; i < C::kEPC; ++i)
+                            for (int i = 0; i < C::kEPC / 2; ++i)
 #pragma unroll
                                 for (int g = 0; g < G; ++g)
-                                    o[g][c * C::kEPC + i] = fmaf(pg[g], vf[i], o[g][c * C::kEPC + i]);
+                                    o2[g][c * (C::kEPC / 2) + i] =
+                                        __ffma2_rn(pg[g], vf[i], o2[g][c * (C::kEPC / 2) + i]);
                         }
                     }
                 }
             }
-            // stage st is free again: refill it with this warp's tile own + P
-            __syncwarp();
-            if (!aborted && next_issue < own_count) {
-                fence_proxy_async_smem();
-                issue_next();
+        };
+        while (own < own_count && run_begin + warp + W * own < seg_end) {
+            const bool two = own + 1 < next_issue && run_begin + warp + W * (own + 1) < seg_end;
+            wait_tile(own);
+            if (two) {
+                wait_tile(own + 1);
+                tiles(std::integral_constant<int, 2>{});
+            } else {
+                tiles(std::integral_constant<int, 1>{});
             }
+            // the consumed stages are free again: refill them with this warp's tiles own + P (+1)
+            __syncwarp();
+            const int done = two ? 2 : 1;
+            for (int r = 0; r < done; ++r) {
+                if (!aborted && next_issue < own_count) {
+                    fence_proxy_async_smem();
+                    issue_next();
+                }
+            }
+            own += done;
         }
 
         // ---- fold the token groups of the warp, then merge the warps
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < C::kEPL; ++e) {
-                float v = o[g][e];
+            for (int e = 0; e < C::kPairs; ++e) {
+                float2 v = o2[g][e];
 #pragma unroll
-                for (int off = LPT; off < 32; off <<= 1)
-                    v += __shfl_xor_sync(kFullMask, v, off);
-                o[g][e] = v;
+                for (int off = LPT; off < 32; off <<= 1) {
+                    v.x += __shfl_xor_sync(kFullMask, v.x, off);
+                    v.y += __shfl_xor_sync(kFullMask, v.y, off);
+                }
+                o2[g][e] = v;
             }
 #pragma unroll
         for (int off = LPT; off < 32; off <<= 1)
@@ -450,9 +501,9 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, BS, G>::kThreads, 1) paged_deco
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int e = 0; e < C::kEPL; ++e) {
-                    const int d = ((e / C::kEPC) * LPT + j) * C::kEPC + (e % C::kEPC);
-                    scr_o[(warp * G + g) * D + d] = o[g][e];
+                for (int e = 0; e < C::kPairs; ++e) {
+                    const int d = ((2 * e / C::kEPC) * LPT + j) * C::kEPC + (2 * e % C::kEPC);
+                    *reinterpret_cast<float2*>(&scr_o[(warp * G + g) * D + d]) = o2[g][e];
                 }
             if (myhead >= 0)
                 scr_l[warp * G + myhead] = l_own;

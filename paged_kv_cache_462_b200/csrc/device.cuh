@@ -172,6 +172,83 @@ __device__ __forceinline__ void load_widen(const uint8_t* p, float* f)
     }
 }
 
+// Load CHUNK bytes of cache elements from shared memory as fp32 pairs
+// (element 2i in .x, 2i+1 in .y), for the packed fp32x2 FMA.
+__device__ __forceinline__ void widen_word2(KvBF16, uint32_t w, float2* f)
+{
+    f[0] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ void widen_word2(KvE4M3, uint32_t w, float2* f)
+{
+    float t[4];
+    widen_word(KvE4M3{}, w, t);
+    f[0] = make_float2(t[0], t[1]);
+    f[1] = make_float2(t[2], t[3]);
+}
+
+template <class KV, int CHUNK>
+__device__ __forceinline__ void load_widen2(const uint8_t* p, float2* f)
+{
+    if constexpr (KV::kBytes == 4) {
+        static_assert(CHUNK == 16 || CHUNK == 8, "fp32 chunk");
+        if constexpr (CHUNK == 16) {
+            const float4 u = *reinterpret_cast<const float4*>(p);
+            f[0] = make_float2(u.x, u.y);
+            f[1] = make_float2(u.z, u.w);
+        } else {
+            f[0] = *reinterpret_cast<const float2*>(p);
+        }
+    } else {
+        constexpr int kPairsPerWord = 2 / KV::kBytes;   // bf16: 1, e4m3: 2
+        if constexpr (CHUNK == 16) {
+            const uint4 u = *reinterpret_cast<const uint4*>(p);
+            widen_word2(KV{}, u.x, f + 0 * kPairsPerWord);
+            widen_word2(KV{}, u.y, f + 1 * kPairsPerWord);
+            widen_word2(KV{}, u.z, f + 2 * kPairsPerWord);
+            widen_word2(KV{}, u.w, f + 3 * kPairsPerWord);
+        } else if constexpr (CHUNK == 8) {
+            const uint2 u = *reinterpret_cast<const uint2*>(p);
+            widen_word2(KV{}, u.x, f + 0 * kPairsPerWord);
+            widen_word2(KV{}, u.y, f + 1 * kPairsPerWord);
+        } else {
+            static_assert(CHUNK == 4, "chunk is 4, 8 or 16 bytes");
+            widen_word2(KV{}, *reinterpret_cast<const uint32_t*>(p), f);
+        }
+    }
+}
+
+// Load N consecutive q elements (8 or 16 bytes per vector) from global memory as fp32.
+template <int N>
+__device__ __forceinline__ void load_q(const float* p, float* f)
+{
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(p + i));
+        f[i] = u.x; f[i + 1] = u.y; f[i + 2] = u.z; f[i + 3] = u.w;
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void load_q(const __nv_bfloat16* p, float* f)
+{
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 8) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(p + i));
+            widen_word(KvBF16{}, u.x, f + i);
+            widen_word(KvBF16{}, u.y, f + i + 2);
+            widen_word(KvBF16{}, u.z, f + i + 4);
+            widen_word(KvBF16{}, u.w, f + i + 6);
+        }
+    } else {
+        static_assert(N == 4, "q vector of 4 or a multiple of 8 elements");
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+        widen_word(KvBF16{}, u.x, f);
+        widen_word(KvBF16{}, u.y, f + 2);
+    }
+}
+
 __device__ __forceinline__ float to_float(float x) { return x; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ void from_float(float v, float* p) { *p = v; }

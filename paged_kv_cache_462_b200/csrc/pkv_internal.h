@@ -6,7 +6,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/pkv.h"
+#include "pkv.h"
 
 namespace pkv {
 
