@@ -8,6 +8,7 @@
 #include <mutex>
 #include <utility>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "pkv_internal.h"
@@ -15,8 +16,6 @@
 namespace pkv {
 
 namespace {
-
-constexpr float kLog2e = 1.4426950408889634074f;
 
 std::mutex g_mu;
 std::map<std::pair<const void*, int>, size_t> g_smem_set;   // (kernel, device) -> dynamic smem limit set
@@ -59,13 +58,52 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
     const long long pairs = (long long)num_seqs * num_kv_heads;
     w.counters_off = kWorkspaceHeader;
     w.partials_off = w.counters_off + round_up((size_t)pairs * 4, 256);
-    w.bytes = w.partials_off + (size_t)(runs + pairs) * slot_floats_for(group, head_dim) * 4;
+    // a run writes at most one partial per (stream it touches, head of the stream's group)
+    w.bytes = w.partials_off + (size_t)(runs * kMaxHeadGroup + pairs) * slot_floats_for(group, head_dim) * 4;
     return w;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
 }  // namespace
+
+bool make_cache_tensormap(CUtensorMap* map, const void* base, int kv_dtype, int head_dim, long long rows,
+                          int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const int elt = kv_dtype == PKV_BF16 ? 2 : 1;
+    const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)head_dim * elt};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / elt), (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, kv_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 bool ensure_smem_attribute(const void* kernel, size_t bytes)
 {
@@ -173,6 +211,7 @@ int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
     p.num_seqs = 1;
+    p.num_kv_heads = num_kv_heads;
     int occ = 0;
     const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, num_heads / num_kv_heads, p, 0,
                                    nullptr, &occ);
@@ -210,7 +249,8 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     if (max_blocks_per_seq <= 0 || num_blocks <= 0)
         return PKV_ERR_SHAPE;
     if ((long long)num_seqs * max_blocks_per_seq * num_kv_heads >= (1ll << 31) ||
-        (long long)max_blocks_per_seq * block_size >= (1ll << 31))
+        (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
+        (long long)num_blocks * num_kv_heads * block_size >= (1ll << 31))
         return PKV_ERR_SHAPE;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
         return PKV_ERR_SHAPE;
@@ -224,6 +264,7 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
         DecodeParams probe;
         std::memset(&probe, 0, sizeof probe);
         probe.num_seqs = num_seqs;
+        probe.num_kv_heads = num_kv_heads;
         int occ = 0;
         const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, probe, 0, nullptr, &occ);
         if (st != PKV_OK)
@@ -250,8 +291,9 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     p.num_kv_heads = num_kv_heads;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.num_blocks = num_blocks;
-    p.q_scale = scale * kLog2e * (fp8 ? k_scale * kv_unbias(kv_dtype) : 1.0f);
-    p.v_scale = fp8 ? v_scale * kv_unbias(kv_dtype) : 1.0f;
+    p.scale = scale;
+    p.k_scale = fp8 ? k_scale : 1.0f;
+    p.v_scale_in = fp8 ? v_scale : 1.0f;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.err = reinterpret_cast<int32_t*>(ws);
     p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);

@@ -1,5 +1,6 @@
-// Dispatch of paged_attention_decode to the kernel instantiation for the
-// (q dtype, cache dtype) pair; the kernel itself is in decode_kernel.cuh.
+// Dispatch of paged_attention_decode: the warp-MMA kernel (decode_mma.cuh) for
+// bf16 / E4M3 caches of the shapes it covers, the CUDA-core kernel
+// (decode_kernel.cuh) for fp32 caches and every other supported shape.
 #include "decode_kernel.cuh"
 
 namespace pkv {
@@ -7,10 +8,53 @@ namespace pkv {
 int decode_dispatch_f32(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
 int decode_dispatch_bf16(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
 int decode_dispatch_e4m3(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
+int decode_mma_dispatch_bf16(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
+                             int* occ);
+int decode_mma_dispatch_e4m3(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
+                             int* occ);
+
+int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
+                        cudaStream_t st, int* occ)
+{
+    if (kv_dtype == PKV_BF16)
+        return decode_mma_dispatch_bf16(D, BS, G, HG, p, nruns, st, occ);
+    if (kv_dtype == PKV_FP8_E4M3)
+        return decode_mma_dispatch_e4m3(D, BS, G, HG, p, nruns, st, occ);
+    return PKV_ERR_DTYPE;
+}
+
+bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)
+{
+    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3)
+        return false;
+    if (block_size != 16 && block_size != 32)
+        return false;
+    if (group > 8)
+        return false;
+    if (kv_dtype == PKV_BF16 ? (head_dim != 64 && head_dim != 128) : head_dim != 128)
+        return false;
+    return mma_head_group(kv_dtype, head_dim, block_size, num_kv_heads) > 0;
+}
+
+// Largest head group in {8, 4, 2, 1} that divides num_kv_heads and keeps a stage (K + V) within 64 KB.
+int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads)
+{
+    const int elt = kv_dtype == PKV_BF16 ? 2 : 1;
+    for (int hg = kMaxHeadGroup; hg >= 1; hg /= 2) {
+        if (num_kv_heads % hg != 0)
+            continue;
+        if (2ll * hg * block_size * head_dim * elt <= 64 * 1024)
+            return hg;
+    }
+    return 0;
+}
 
 int decode_dispatch(int q_dtype, int kv_dtype, int D, int BS, int G, const DecodeParams& p, int nruns,
                     cudaStream_t st, int* occupancy_out)
 {
+    if (q_dtype == PKV_BF16 && mma_supported(kv_dtype, D, BS, G, p.num_kv_heads))
+        return decode_mma_dispatch(kv_dtype, D, BS, G, mma_head_group(kv_dtype, D, BS, p.num_kv_heads), p, nruns,
+                                   st, occupancy_out);
     if (q_dtype == PKV_F32 && kv_dtype == PKV_F32)
         return decode_dispatch_f32(D, BS, G, p, nruns, st, occupancy_out);
     if (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16)
@@ -19,7 +63,5 @@ int decode_dispatch(int q_dtype, int kv_dtype, int D, int BS, int G, const Decod
         return decode_dispatch_e4m3(D, BS, G, p, nruns, st, occupancy_out);
     return PKV_ERR_DTYPE;
 }
-
-float kv_unbias(int kv_dtype) { return kv_dtype == PKV_FP8_E4M3 ? kE4M3Unbias : 1.0f; }
 
 }  // namespace pkv

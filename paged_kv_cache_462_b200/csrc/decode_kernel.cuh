@@ -131,22 +131,6 @@ __host__ __device__ constexpr int head_src_lane(int g)
     return 0;
 }
 
-// prefix[s] = num_kv_heads * sum_{s' < s} nblocks(s'); pair (s, h) owns the
-// global tiles [prefix[s] + h*nb_s, prefix[s] + (h+1)*nb_s). Returns the s with
-// prefix[s] <= x < prefix[s+1] (empty sequences are never returned).
-__device__ __forceinline__ int find_seq(const int* prefix, int num_seqs, int x)
-{
-    int lo = 0, hi = num_seqs;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (prefix[mid] <= x)
-            lo = mid;
-        else
-            hi = mid;
-    }
-    return lo;
-}
-
 // Byte offset in the cache of global tile x, -2 for a bad block id.
 template <int TILE>
 __device__ __forceinline__ long long tile_offset(const DecodeParams& p, const int* prefix, int x)
@@ -648,6 +632,9 @@ struct DecodeLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = P;
+        // E4M3 codes are widened to fp32 with a 2^-120 bias (see device.cuh): fold 2^120 into the scales
+        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 ? p.k_scale * KV::kUnbias : 1.0f);
+        p.v_scale = KV::kBytes == 1 ? p.v_scale_in * KV::kUnbias : 1.0f;
         kern<<<nruns, C::kThreads, smem, stream>>>(p);
         return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
     }

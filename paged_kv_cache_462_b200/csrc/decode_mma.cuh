@@ -1,0 +1,694 @@
+// Paged decode attention for bf16 and E4M3 caches on sm_100a: whole-block TMA
+// tiles, one warp per KV head, warp-level tensor-core MMA with fp32 accumulation.
+//
+// Same result as the CUDA-core kernel (decode_kernel.cuh): for every sequence s
+// and query head g, out[s][g] = softmax_t(scale * q . K_t) V_t over the
+// seq_lens[s] cached tokens, K_t/V_t read through the block table
+// ("vLLM inference cost optimisation", developer.aliyun.com, sections 2 and 4;
+// wzjinhao.cn vLLM write-up, section 2.1), GQA head g -> KV head g / G.
+//
+// Why a second kernel: on the CUDA cores the q.K and p.V products of one
+// 16-token tile cost ~900 (bf16) to ~1450 (E4M3, G = 5) warp instructions, so
+// the decode step stayed issue-bound (measured with every tile resident in L2)
+// well below the HBM rate. Here one tile costs ~100 instructions.
+//
+// Layout of the work:
+//  * Unit = (sequence, head group of HG <= 8 KV heads, logical block). The K
+//    rows of a unit are HG*block_size consecutive rows of the pool
+//    ([block][kv head][token][d]), i.e. one contiguous run (32 KB for bf16, 8
+//    heads, block 16, d 128), fetched with 2-D TMA tensor copies whose 128-byte
+//    swizzle makes the ldmatrix reads below bank-conflict free. Same for V.
+//  * Units in (sequence, head group, block) order are cut into gridDim.x equal
+//    runs (one CTA per SM). Warp HG is the producer (block-table lookups, one
+//    TMA copy per 128-byte-wide box, a ring of stages with full/empty
+//    mbarriers); warps 0..HG-1 are consumers, warp w owning KV head
+//    hg*HG + w of every unit, so a run's segment of one (sequence, head)
+//    stream is finished by one warp without any CTA-wide barrier.
+//  * Per 16-token tile: S^T = K Q^T with m16n8k16 MMA (16 tokens x 8 query
+//    heads of the group, k = head_dim), scale, mask, online softmax with a lazy
+//    running max (moved only when a tile max passes it by 8, in log2 units),
+//    P^T re-laid out with 4 shuffles into the B operand of O^T += V^T P^T
+//    (head_dim x 8 heads, k = 16 tokens). bf16 caches use bf16 MMA; E4M3 codes
+//    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2) and use f16 MMA, the
+//    per-tensor scales applied to the fp32 scores and outputs.
+//  * Split streams: the same last-arriver log-sum-exp merge as the CUDA-core
+//    kernel, per (sequence, KV head), done by one warp.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda.h>
+
+#include "device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+constexpr float kMmaRescaleSlack = 8.0f;  // log2 units
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    if constexpr (F16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+}
+
+// two E4M3 codes (low byte first) -> f16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes)
+{
+    uint32_t r;
+    const uint16_t v = static_cast<uint16_t>(two_codes);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    if constexpr (F16) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ configuration
+
+template <class KV, int D, int BS, int G, int HG>
+struct MmaCfg {
+    static constexpr bool kF16 = KV::kBytes == 1;            // E4M3 widened to f16; bf16 stays bf16
+    static constexpr int kRowBytes = D * KV::kBytes;          // one token row of one head
+    static constexpr int kBoxCols = 128 / KV::kBytes;         // elements per 128-byte box row
+    static constexpr int kBoxes = kRowBytes / 128;            // boxes across head_dim
+    static constexpr int kRows = HG * BS;                     // box rows: head-major, token-minor
+    static constexpr int kBoxBytes = kRows * 128;
+    static constexpr int kHalf = kBoxes * kBoxBytes;          // K (or V) part of a stage
+    static constexpr int kStage = 2 * kHalf;
+    static constexpr int kTT = BS / 16;                       // 16-token tiles per block
+    static constexpr int kKS = D / 16;                        // q.K k-steps (16 d each)
+    static constexpr int kDT = D / 16;                        // p.V m-tiles (16 d each)
+    static constexpr int W = HG;                              // consumer warps
+    static constexpr int kThreads = (W + 1) * 32;
+    static_assert(kRowBytes % 128 == 0, "rows are whole 128-byte swizzle spans");
+    static_assert(BS % 16 == 0 && G <= 8 && HG <= 8, "tile shape");
+    static_assert(kRows <= 256, "TMA box height");
+};
+
+// Byte offset of the 16-byte chunk `c` (0..7) of box row `r` in a 128B-swizzled box.
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// ------------------------------------------------------------------ kernel
+
+template <class KV, class QT, int D, int BS, int G, int HG>
+__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 1)
+    paged_decode_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                            const DecodeParams p)
+{
+    using C = MmaCfg<KV, D, BS, G, HG>;
+    constexpr int W = C::W;
+    constexpr bool F16 = C::kF16;
+    const int S = p.stages_per_warp;   // ring depth (stages of the CTA)
+    const int Hkv = p.num_kv_heads;
+    const int NHG = Hkv / HG;          // head groups per sequence
+    const int capacity = p.max_blocks_per_seq * BS;
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* stages = smem;                                                    // [S][kStage], 1024-aligned
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)S * C::kStage);
+    uint64_t* empty = full + S;
+    int* skip = reinterpret_cast<int*>(empty + S);
+    volatile int* abort_flag = skip + S;
+    int* prefix = const_cast<int*>(abort_flag + 1);                           // [num_seqs + 1]
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if ((smem_addr(smem) & 1023u) != 0u) {   // the 128-byte swizzle needs 1024-byte aligned stages
+        if (tid == 0)
+            atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+        return;
+    }
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], W);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    bool bad_len = false;
+    for (int s = tid; s < p.num_seqs; s += C::kThreads) {
+        int L = p.seq_lens[s];
+        if (L < 0 || L > capacity) {
+            bad_len = true;
+            L = L < 0 ? 0 : capacity;
+        }
+        prefix[s + 1] = ((L + BS - 1) / BS) * NHG;
+    }
+    if (bad_len && blockIdx.x == 0)
+        atomicOr(p.err, PKV_DEVERR_SEQ_LEN);
+    if (tid == 0)
+        prefix[0] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < p.num_seqs; base += 32) {
+            const int i = base + lane + 1;
+            int v = (i <= p.num_seqs) ? prefix[i] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(kFullMask, v, o);
+                if (lane >= o)
+                    v += u;
+            }
+            v += carry;
+            if (i <= p.num_seqs)
+                prefix[i] = v;
+            carry = __shfl_sync(kFullMask, v, 31);
+        }
+    }
+    __syncthreads();
+
+    const int total = prefix[p.num_seqs];
+    const int nruns = gridDim.x;
+    const int per_run = (total + nruns - 1) / nruns;
+    const int run_begin = min(total, (int)blockIdx.x * per_run);
+    const int run_end = min(total, run_begin + per_run);
+    const int nunits = run_end - run_begin;
+
+    // zero rows of empty sequences (one run per sequence)
+    for (int s = blockIdx.x; s < p.num_seqs; s += nruns) {
+        if (prefix[s + 1] == prefix[s]) {
+            QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * p.num_heads * D;
+            for (int i = tid; i < p.num_heads * D; i += C::kThreads)
+                from_float(0.f, o + i);
+        }
+    }
+
+    // =========================== producer warp ===============================
+    if (warp == W) {
+        if (nunits <= 0)
+            return;
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        // lane l resolves unit (batch + l): pool row of its head group, or -1 for a bad block id
+        auto locate = [&](int k) -> int {
+            if (k >= nunits)
+                return -1;
+            const int x = run_begin + k;
+            const int s = find_seq(prefix, p.num_seqs, x);
+            const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+            const int r = x - prefix[s];
+            const int hg = r / nb, j = r - hg * nb;
+            const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + j);
+            if (phys < 0 || phys >= p.num_blocks) {
+                atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
+                return -1;
+            }
+            return (phys * Hkv + hg * HG) * BS;
+        };
+        int cur = locate(lane), ahead = locate(32 + lane);
+        bool aborted = false;
+        int issued = 0;
+        for (int k0 = 0; k0 < nunits; k0 += 32) {
+            if (k0 > 0) {
+                cur = ahead;
+                ahead = locate(k0 + 32 + lane);
+            }
+            const int cnt = min(32, nunits - k0);
+            for (int i = 0; i < cnt; ++i) {
+                const int row = __shfl_sync(kFullMask, cur, i);
+                if (lane == 0 && !aborted) {
+                    const int k = k0 + i;
+                    const int st = k % S;
+                    if (*abort_flag) {
+                        aborted = true;
+                    } else if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
+                        aborted = true;
+                        *abort_flag = 1;
+                        atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                    } else if (row < 0) {
+                        skip[st] = 1;
+                        mbar_arrive(&full[st]);
+                        issued = k + 1;
+                    } else {
+                        skip[st] = 0;
+                        uint8_t* dst = stages + (size_t)st * C::kStage;
+                        mbar_arrive_expect_tx(&full[st], C::kStage);
+#pragma unroll
+                        for (int bx = 0; bx < C::kBoxes; ++bx) {
+                            tma_load_2d(dst + bx * C::kBoxBytes, &kmap, bx * C::kBoxCols, row, &full[st]);
+                            tma_load_2d(dst + C::kHalf + bx * C::kBoxBytes, &vmap, bx * C::kBoxCols, row, &full[st]);
+                        }
+                        issued = k + 1;
+                    }
+                }
+            }
+        }
+        if (lane == 0 && aborted) {
+            for (int k = max(0, issued - S); k < issued; ++k)
+                (void)mbar_wait_bounded(&full[k % S], (k / S) & 1);
+        }
+        return;
+    }
+
+    // =========================== consumer warps ==============================
+    const int g = lane >> 2;   // MMA row group
+    const int t = lane & 3;    // MMA column pair
+    const float qk_scale = p.q_scale;
+
+    // A run's split segments (a stream that continues in another run) are at most its
+    // first and its last; their counters and merges wait until the run is streamed.
+    int nsplit = 0;
+    int split_seq[2] = {0, 0}, split_stream[2] = {0, 0}, split_first[2] = {0, 0}, split_last[2] = {0, 0};
+
+    int x = run_begin;
+    int k = 0;                 // unit index within the run
+    while (x < run_end) {
+        const int s = find_seq(prefix, p.num_seqs, x);
+        const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+        const int hg = (x - prefix[s]) / nb;
+        const int stream_begin = prefix[s] + hg * nb;
+        const int stream_end = stream_begin + nb;
+        const int seg_end = min(run_end, stream_end);
+        const int head = hg * HG + warp;           // this warp's KV head
+        int L = p.seq_lens[s];
+        L = L < 0 ? 0 : (L > capacity ? capacity : L);
+
+        // Q^T as the B operand: b0 = (k: d pair, n: query head g); rows g >= G are zero.
+        uint32_t qb[C::kKS][2];
+        {
+            const QT* qp = reinterpret_cast<const QT*>(p.q) + ((size_t)s * p.num_heads + (size_t)head * G + g) * D;
+#pragma unroll
+            for (int ks = 0; ks < C::kKS; ++ks) {
+                if (g < G) {
+                    if constexpr (F16) {
+                        // k order permuted to match the E4M3 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
+                        float f[4];
+                        load_q<4>(qp + ks * 16 + 4 * t, f);
+                        qb[ks][0] = pack2<true>(f[0], f[1]);
+                        qb[ks][1] = pack2<true>(f[2], f[3]);
+                    } else {
+                        qb[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t));
+                        qb[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t + 8));
+                    }
+                } else {
+                    qb[ks][0] = qb[ks][1] = 0u;
+                }
+            }
+        }
+        float o[C::kDT][4];
+#pragma unroll
+        for (int dt = 0; dt < C::kDT; ++dt)
+            o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+        float m[2] = {-INFINITY, -INFINITY};   // running reference for heads 2t, 2t+1
+        float l[2] = {0.f, 0.f};
+
+        for (; x < seg_end; ++x, ++k) {
+            const int st = k % S;
+            bool ok = !*abort_flag && mbar_wait_bounded(&full[st], (k / S) & 1);
+            if (__any_sync(kFullMask, !ok)) {
+                if (lane == 0 && !*abort_flag) {
+                    *abort_flag = 1;
+                    atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                ok = false;
+            }
+            const int jb = x - stream_begin;         // logical block
+            const int valid = min(BS, L - jb * BS);
+            if (ok && skip[st] == 0 && valid > 0) {
+                const uint32_t kbase = smem_addr(stages + (size_t)st * C::kStage);
+                const uint32_t vbase = kbase + C::kHalf;
+                const int r0 = warp * BS;            // this head's first box row
+#pragma unroll
+                for (int tt = 0; tt < C::kTT; ++tt) {
+                    // ---- S^T = K Q^T : 16 tokens x 8 heads
+                    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                    float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
+                    const int mi = lane >> 3, rr = lane & 7;
+                    if constexpr (F16) {
+#pragma unroll
+                        for (int ks = 0; ks < C::kKS; ks += 2) {
+                            // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each
+                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                            uint32_t r[4];
+                            ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
+                                const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi),
+                                                       e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16)};
+                                mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < C::kKS; ++ks) {
+                            // matrices: (tok 0-7, d 0-7), (tok 8-15, d 0-7), (tok 0-7, d 8-15), (tok 8-15, d 8-15)
+                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                            const int box = ks / 4, chunk = (ks % 4) * 2 + (mi >> 1);
+                            uint32_t a[4];
+                            ldsm_x4(kbase + box * C::kBoxBytes + swz(row, chunk), a);
+                            mma_16816<false>((ks & 1) ? sd : sc, a, qb[ks][0], qb[ks][1]);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        sc[i] += sd[i];
+                    // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
+                    const int tok0 = tt * 16 + g;
+                    sc[0] = (tok0 < valid) ? sc[0] * qk_scale : -INFINITY;
+                    sc[1] = (tok0 < valid) ? sc[1] * qk_scale : -INFINITY;
+                    sc[2] = (tok0 + 8 < valid) ? sc[2] * qk_scale : -INFINITY;
+                    sc[3] = (tok0 + 8 < valid) ? sc[3] * qk_scale : -INFINITY;
+                    float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
+                        bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
+                    }
+                    const bool up0 = bm0 > m[0] + kMmaRescaleSlack, up1 = bm1 > m[1] + kMmaRescaleSlack;
+                    if (__any_sync(kFullMask, up0 || up1)) {
+                        const float n0 = up0 ? bm0 : m[0], n1 = up1 ? bm1 : m[1];
+                        const float a0 = up0 ? fast_exp2(m[0] - n0) : 1.f, a1 = up1 ? fast_exp2(m[1] - n1) : 1.f;
+                        m[0] = n0;
+                        m[1] = n1;
+                        l[0] *= a0;
+                        l[1] *= a1;
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; ++dt) {
+                            o[dt][0] *= a0;
+                            o[dt][1] *= a1;
+                            o[dt][2] *= a0;
+                            o[dt][3] *= a1;
+                        }
+                    }
+                    float pr[4];
+                    pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - m[0]);
+                    pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - m[1]);
+                    pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - m[0]);
+                    pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - m[1]);
+                    l[0] += pr[0] + pr[2];
+                    l[1] += pr[1] + pr[3];
+                    // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
+                    const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
+                    const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
+                    const int srcA = (2 * t) * 4 + (g >> 1), srcB = (2 * t + 1) * 4 + (g >> 1);
+                    const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
+                    const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
+                    const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
+                    const uint32_t pb0 = (g < G) ? __byte_perm(va, vb, 0x5410) : 0u;
+                    const uint32_t pb1 = (g < G) ? __byte_perm(va, vb, 0x7632) : 0u;
+                    // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
+                    const bool partial = valid < tt * 16 + 16;
+                    if constexpr (F16) {
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; dt += 2) {
+                            // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
+                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                            uint32_t r[4];
+                            ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
+                                if (partial) {
+                                    const int tk = tt * 16 + 2 * t;
+                                    lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                    hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                }
+                                // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1)
+                                const uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020)),
+                                                       e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031)),
+                                                       e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020)),
+                                                       e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031))};
+                                mma_16816<true>(o[dt + h2], a, pb0, pb1);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; ++dt) {
+                            // matrices: (d 0-7, tok 0-7), (d 8-15, tok 0-7), (d 0-7, tok 8-15), (d 8-15, tok 8-15)
+                            const int row = r0 + tt * 16 + (mi >> 1) * 8 + rr;
+                            const int box = dt / 4, chunk = (dt % 4) * 2 + (mi & 1);
+                            uint32_t a[4];
+                            ldsm_x4_t(vbase + box * C::kBoxBytes + swz(row, chunk), a);
+                            if (partial) {
+                                const int tk = tt * 16 + 2 * t;
+                                const uint32_t m01 = (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                const uint32_t m89 = (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                a[0] &= m01;
+                                a[1] &= m01;
+                                a[2] &= m89;
+                                a[3] &= m89;
+                            }
+                            mma_16816<false>(o[dt], a, pb0, pb1);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
+        }
+
+        // ---- end of this warp's segment: l over the 8 row groups, then write or merge
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l[0] += __shfl_xor_sync(kFullMask, l[0], off);
+            l[1] += __shfl_xor_sync(kFullMask, l[1], off);
+        }
+        const int first_run = stream_begin / per_run;
+        const int last_run = (stream_end - 1) / per_run;
+        const int stream = s * NHG + hg;
+        // element (head column c, row d) of this lane's accumulators
+        auto d_of = [&](int dt, int half) -> int {
+            return F16 ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
+        };
+        if (first_run == last_run) {
+            QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
+            const float inv0 = l[0] > 0.f ? p.v_scale / l[0] : 0.f;
+            const float inv1 = l[1] > 0.f ? p.v_scale / l[1] : 0.f;
+#pragma unroll
+            for (int dt = 0; dt < C::kDT; ++dt)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int d = d_of(dt, half);
+                    if (2 * t < G)
+                        from_float(o[dt][2 * half] * inv0, out + (2 * t) * D + d);
+                    if (2 * t + 1 < G)
+                        from_float(o[dt][2 * half + 1] * inv1, out + (2 * t + 1) * D + d);
+                }
+        } else {
+            float* part = p.partials + ((size_t)(blockIdx.x + stream) * HG + warp) * p.slot_floats;
+#pragma unroll
+            for (int dt = 0; dt < C::kDT; ++dt)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int d = d_of(dt, half);
+                    if (2 * t < G)
+                        part[(2 * t) * D + d] = o[dt][2 * half];
+                    if (2 * t + 1 < G)
+                        part[(2 * t + 1) * D + d] = o[dt][2 * half + 1];
+                }
+            if (g == 0) {
+                if (2 * t < G) {
+                    part[G * D + 2 * t] = m[0];
+                    part[G * D + G + 2 * t] = l[0];
+                }
+                if (2 * t + 1 < G) {
+                    part[G * D + 2 * t + 1] = m[1];
+                    part[G * D + G + 2 * t + 1] = l[1];
+                }
+            }
+            if (nsplit < 2) {
+                split_seq[nsplit] = s;
+                split_stream[nsplit] = stream;
+                split_first[nsplit] = first_run;
+                split_last[nsplit] = last_run;
+                ++nsplit;
+            }
+        }
+    }
+
+    // ---- split streams: publish, count arrivals; the last run to arrive merges (log-sum-exp)
+    for (int i = 0; i < nsplit; ++i) {
+        const int s = split_seq[i], stream = split_stream[i];
+        const int first_run = split_first[i], last_run = split_last[i];
+        const int head = (stream - s * NHG) * HG + warp;
+        const int pair = s * Hkv + head;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            const int arrived = atomicAdd(&p.counters[pair], 1);
+            last = (arrived == last_run - first_run) ? 1 : 0;
+            if (last)
+                p.counters[pair] = 0;
+        }
+        last = __shfl_sync(kFullMask, last, 0);
+        if (!last)
+            continue;
+        __threadfence();
+        QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
+        constexpr int NV = (G * D + 127) / 128;        // float4 groups per lane
+        float4 acc[NV];
+        float mx[NV], ls[NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            mx[v] = -INFINITY;
+            ls[v] = 0.f;
+        }
+        // pass 1: the largest reference max of each element's head over the segments
+        for (int c = first_run; c <= last_run; ++c) {
+            const float* q = p.partials + ((size_t)(c + stream) * HG + warp) * p.slot_floats;
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const int idx = 4 * lane + 128 * v;
+                if (idx < G * D)
+                    mx[v] = fmaxf(mx[v], __ldcg(q + G * D + idx / D));
+            }
+        }
+        // pass 2: weighted sums of o and l
+        for (int c = first_run; c <= last_run; ++c) {
+            const float* q = p.partials + ((size_t)(c + stream) * HG + warp) * p.slot_floats;
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const int idx = 4 * lane + 128 * v;
+                if (idx < G * D && mx[v] != -INFINITY) {
+                    const int gq = idx / D;
+                    const float mc = __ldcg(q + G * D + gq);
+                    const float a = (mc == -INFINITY) ? 0.f : fast_exp2(mc - mx[v]);
+                    const float4 ov = __ldcg(reinterpret_cast<const float4*>(q + idx));
+                    acc[v].x = fmaf(a, ov.x, acc[v].x);
+                    acc[v].y = fmaf(a, ov.y, acc[v].y);
+                    acc[v].z = fmaf(a, ov.z, acc[v].z);
+                    acc[v].w = fmaf(a, ov.w, acc[v].w);
+                    ls[v] = fmaf(a, __ldcg(q + G * D + G + gq), ls[v]);
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const int idx = 4 * lane + 128 * v;
+            if (idx < G * D) {
+                const float inv = ls[v] > 0.f ? p.v_scale / ls[v] : 0.f;
+                from_float(acc[v].x * inv, out + idx);
+                from_float(acc[v].y * inv, out + idx + 1);
+                from_float(acc[v].z * inv, out + idx + 2);
+                from_float(acc[v].w * inv, out + idx + 3);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+// Encode a 2-D tensor map over a cache: rows = num_blocks * num_kv_heads * block_size,
+// row = head_dim elements, box = 128 bytes x box_rows, 128-byte swizzle.
+bool make_cache_tensormap(CUtensorMap* map, const void* base, int kv_dtype, int head_dim, long long rows,
+                          int box_rows);
+
+template <class KV, class QT, int D, int BS, int G, int HG>
+struct MmaLauncher {
+    using C = MmaCfg<KV, D, BS, G, HG>;
+
+    static size_t smem_bytes(int num_seqs, int S)
+    {
+        return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + (size_t)(num_seqs + 1) * 4 + 64;
+    }
+
+    static int stages(int num_seqs)
+    {
+        const long long room = (long long)kMaxSmemPerBlock - 1024 - 16 - (long long)(num_seqs + 1) * 4 - 64;
+        long long S = room / (C::kStage + 20);
+        if (S > 8)
+            S = 8;
+        return (int)S;
+    }
+
+    static int occupancy(int num_seqs)
+    {
+        const int S = stages(num_seqs);
+        if (S < 2)
+            return 0;
+        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG>;
+        const size_t smem = smem_bytes(num_seqs, S);
+        if (!ensure_smem_attribute((const void*)kern, smem))
+            return 0;
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, C::kThreads, smem) != cudaSuccess)
+            return 0;
+        return n;
+    }
+
+    static int launch(DecodeParams p, int nruns, cudaStream_t stream)
+    {
+        const int S = stages(p.num_seqs);
+        if (S < 2)
+            return PKV_ERR_SHAPE;
+        const long long rows = (long long)p.num_blocks * p.num_kv_heads * BS;
+        const int kvdt = KV::kBytes == 1 ? PKV_FP8_E4M3 : PKV_BF16;
+        CUtensorMap kmap, vmap;
+        if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, D, rows, C::kRows) ||
+            !make_cache_tensormap(&vmap, p.v_cache, kvdt, D, rows, C::kRows))
+            return PKV_ERR_LAUNCH;
+        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG>;
+        const size_t smem = smem_bytes(p.num_seqs, S);
+        if (!ensure_smem_attribute((const void*)kern, smem))
+            return PKV_ERR_LAUNCH;
+        p.stages_per_warp = S;
+        // E4M3 -> f16 widening is exact: only the per-tensor scales remain
+        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 ? p.k_scale : 1.0f);
+        p.v_scale = KV::kBytes == 1 ? p.v_scale_in : 1.0f;
+        kern<<<nruns, C::kThreads, smem, stream>>>(kmap, vmap, p);
+        return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+    }
+};
+
+}  // namespace pkv

@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -101,6 +102,21 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 __device__ __forceinline__ void named_barrier_sync(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// prefix[] is a per-sequence exclusive prefix sum of work units; returns the s with
+// prefix[s] <= x < prefix[s+1] (sequences without units are never returned).
+__device__ __forceinline__ int find_seq(const int* prefix, int num_seqs, int x)
+{
+    int lo = 0, hi = num_seqs;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= x)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
 }
 
 __device__ __forceinline__ float fast_exp2(float x)

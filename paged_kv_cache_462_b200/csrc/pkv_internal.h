@@ -14,6 +14,8 @@ constexpr int kMaxSmemPerBlock = 227 * 1024;
 constexpr int kMaxSeqs = 16384;         // per call: the per-sequence tile prefix lives in shared memory
 constexpr int kMaxRunsPerSM = 4;        // automatic partition count is at most 4 runs per SM
 constexpr size_t kWorkspaceHeader = 256;
+constexpr int kMaxHeadGroup = 8;        // KV heads per MMA work unit (partial slots reserved per run)
+constexpr float kLog2e = 1.4426950408889634074f;
 
 struct DecodeParams {
     void* out;
@@ -27,8 +29,11 @@ struct DecodeParams {
     int num_kv_heads;
     int max_blocks_per_seq;
     int num_blocks;
-    float q_scale;     // scale * log2(e) * k_scale * (2^120 for E4M3 caches)
-    float v_scale;     // v_scale * (2^120 for E4M3 caches)
+    float scale;       // softmax scale as given
+    float k_scale;     // per-tensor dequantisation scales (1 for bf16 / f32 caches)
+    float v_scale_in;
+    float q_scale;     // set by the launcher: factor applied to q.K to get log2-domain scores
+    float v_scale;     // set by the launcher: factor applied to the output
     int32_t* err;      // workspace error word
     int32_t* counters; // [num_seqs * num_kv_heads] arrivals, zero between calls
     float* partials;   // [(runs + pairs)][slot_floats]
@@ -36,9 +41,14 @@ struct DecodeParams {
     int stages_per_warp; // set by the launcher
 };
 
+// Kernel selection: warp-MMA kernel for bf16 / E4M3 caches of supported shapes,
+// CUDA-core kernel otherwise. Returns PKV_ERR_SHAPE for unsupported shapes.
 int decode_dispatch(int q_dtype, int kv_dtype, int head_dim, int block_size, int group,
                     const DecodeParams& p, int nruns, cudaStream_t stream, int* occupancy_out);
-float kv_unbias(int kv_dtype);
+bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads);
+int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads);
+int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
+                        cudaStream_t st, int* occ);
 
 int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                    int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
