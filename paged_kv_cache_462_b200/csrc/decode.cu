@@ -36,14 +36,15 @@ bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int nu
     return mma_head_group(kv_dtype, head_dim, block_size, num_kv_heads) > 0;
 }
 
-// Largest head group in {8, 4, 2, 1} that divides num_kv_heads and keeps a stage (K + V) within 64 KB.
+// Largest head group in {4, 2, 1} that divides num_kv_heads and keeps a stage (K + V) within
+// 32 KB: two CTAs (two independent copy pipelines) per SM, 5 warps each.
 int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads)
 {
     const int elt = kv_dtype == PKV_BF16 ? 2 : 1;
-    for (int hg = kMaxHeadGroup; hg >= 1; hg /= 2) {
+    for (int hg = 4; hg >= 1; hg /= 2) {
         if (num_kv_heads % hg != 0)
             continue;
-        if (2ll * hg * block_size * head_dim * elt <= 64 * 1024)
+        if (2ll * hg * block_size * head_dim * elt <= 32 * 1024)
             return hg;
     }
     return 0;

@@ -143,7 +143,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 12
 // ------------------------------------------------------------------ kernel
 
 template <class KV, class QT, int D, int BS, int G, int HG>
-__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 1)
+__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
     paged_decode_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                             const DecodeParams p)
 {
@@ -643,12 +643,19 @@ struct MmaLauncher {
         return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + (size_t)(num_seqs + 1) * 4 + 64;
     }
 
+    // Ring depth: about 96 KB of stages per CTA so that two CTAs share an SM.
     static int stages(int num_seqs)
     {
-        const long long room = (long long)kMaxSmemPerBlock - 1024 - 16 - (long long)(num_seqs + 1) * 4 - 64;
+        const long long budget = kMaxSmemPerBlock / 2 - 1024;
+        const long long room = budget - 16 - (long long)(num_seqs + 1) * 4 - 64;
         long long S = room / (C::kStage + 20);
         if (S > 8)
             S = 8;
+        if (S < 2) {   // many sequences: fall back to one CTA per SM
+            S = ((long long)kMaxSmemPerBlock - 1024 - 16 - (long long)(num_seqs + 1) * 4 - 64) / (C::kStage + 20);
+            if (S > 8)
+                S = 8;
+        }
         return (int)S;
     }
 

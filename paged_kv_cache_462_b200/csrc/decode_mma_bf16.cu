@@ -19,7 +19,6 @@ int by_hg(int HG, const DecodeParams& p, int nruns, cudaStream_t st, int* occ)
         PKV_HG(1)
         PKV_HG(2)
         PKV_HG(4)
-        PKV_HG(8)
 #undef PKV_HG
     default:
         return PKV_ERR_SHAPE;
