@@ -132,6 +132,32 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * paged_attention_decode without a caller workspace, for callers that cannot
+ * allocate device memory: code running while a CUDA graph is captured,
+ * plug-ins whose host framework owns every allocation, hosts that reserve all
+ * memory at start-up. (The pages have no counterpart; this is an interface
+ * convenience, same arithmetic as paged_attention_decode.)
+ *
+ * Arguments are those of paged_attention_decode minus the workspace. The
+ * scratch is a fixed 32 MiB array inside the library, present on every GPU
+ * that loads it until the process exits; a call whose
+ * paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+ * num_partitions) exceeds 32 MiB returns PKV_ERR_WORKSPACE without launching.
+ * Nothing is allocated. The first call on each device looks up the array's
+ * device address (with that device current), so make that first call before
+ * any stream capture. Every call clears the array's counters and error word on
+ * `stream` and then shares the array: calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller. The
+ * device error word is not readable through this entry point.
+ */
+PKV_API int paged_attention_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                          int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                          float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                                          int kv_dtype, float k_scale, float v_scale, int num_partitions,
+                                          void* stream);
+
+/*
  * Decode-step append: for every token t with slot_mapping[t] >= 0, write
  * k[t][h][:] to k_cache[slot / block_size][h][slot % block_size][:] (and v the
  * same way) for every kv head h. Same dtype: a bit copy. FP8_E4M3 cache from
