@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
             }
             const int jb = x - stream_begin;         // logical block
             const int valid = min(BS, L - jb * BS);
+            bool released = false;
             if (ok && skip[st] == 0 && valid > 0) {
                 const uint32_t kbase = smem_addr(stages + (size_t)st * C::kStage);
                 const uint32_t vbase = kbase + C::kHalf;
@@ -400,6 +401,39 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         sc[i] += sd[i];
+                    // V fragments of this tile into registers; after the block's last tile the
+                    // stage goes back to the producer before the softmax and p.V arithmetic
+                    uint32_t vf[C::kDT * 4 / (F16 ? 2 : 1)];
+                    if constexpr (F16) {
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; dt += 2) {
+                            // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
+                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                            uint32_t r[4];
+                            ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                vf[2 * dt + i] = r[i];
+                        }
+                    } else {
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; ++dt) {
+                            // matrices: (d 0-7, tok 0-7), (d 8-15, tok 0-7), (d 0-7, tok 8-15), (d 8-15, tok 8-15)
+                            const int row = r0 + tt * 16 + (mi >> 1) * 8 + rr;
+                            const int box = dt / 4, chunk = (dt % 4) * 2 + (mi & 1);
+                            uint32_t r[4];
+                            ldsm_x4_t(vbase + box * C::kBoxBytes + swz(row, chunk), r);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                vf[4 * dt + i] = r[i];
+                        }
+                    }
+                    if (tt == C::kTT - 1) {
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&empty[st]);
+                        released = true;
+                    }
                     // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
                     const int tok0 = tt * 16 + g;
                     sc[0] = (tok0 < valid) ? sc[0] * qk_scale : -INFINITY;
@@ -449,13 +483,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
                     if constexpr (F16) {
 #pragma unroll
                         for (int dt = 0; dt < C::kDT; dt += 2) {
-                            // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
-                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                            uint32_t r[4];
-                            ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
-                                uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
+                                uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
                                 if (partial) {
                                     const int tk = tt * 16 + 2 * t;
                                     lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
@@ -472,11 +502,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
                     } else {
 #pragma unroll
                         for (int dt = 0; dt < C::kDT; ++dt) {
-                            // matrices: (d 0-7, tok 0-7), (d 8-15, tok 0-7), (d 0-7, tok 8-15), (d 8-15, tok 8-15)
-                            const int row = r0 + tt * 16 + (mi >> 1) * 8 + rr;
-                            const int box = dt / 4, chunk = (dt % 4) * 2 + (mi & 1);
-                            uint32_t a[4];
-                            ldsm_x4_t(vbase + box * C::kBoxBytes + swz(row, chunk), a);
+                            uint32_t a[4] = {vf[4 * dt], vf[4 * dt + 1], vf[4 * dt + 2], vf[4 * dt + 3]};
                             if (partial) {
                                 const int tk = tt * 16 + 2 * t;
                                 const uint32_t m01 = (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
@@ -491,9 +517,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[st]);
+            if (!released) {
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[st]);
+            }
         }
 
         // ---- end of this warp's segment: l over the 8 row groups, then write or merge
@@ -575,41 +603,79 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
             continue;
         __threadfence();
         QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
-        constexpr int NV = (G * D + 127) / 128;        // float4 groups per lane
-        float4 acc[NV];
-        float mx[NV], ls[NV];
+        const int nseg = last_run - first_run + 1;
+        auto slot = [&](int c) -> const float* {
+            return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
+        };
+        // weights: lane c owns segment c (32 at a time); per head the largest reference max
+        float M[G], Lsum[G];
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            mx[v] = -INFINITY;
-            ls[v] = 0.f;
+        for (int gq = 0; gq < G; ++gq) {
+            M[gq] = -INFINITY;
+            Lsum[gq] = 0.f;
         }
-        // pass 1: the largest reference max of each element's head over the segments
-        for (int c = first_run; c <= last_run; ++c) {
-            const float* q = p.partials + ((size_t)(c + stream) * HG + warp) * p.slot_floats;
+        for (int c0 = 0; c0 < nseg; c0 += 32) {
+            const bool mine = c0 + lane < nseg;
 #pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                const int idx = 4 * lane + 128 * v;
-                if (idx < G * D)
-                    mx[v] = fmaxf(mx[v], __ldcg(q + G * D + idx / D));
+            for (int gq = 0; gq < G; ++gq) {
+                float v = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
+                M[gq] = fmaxf(M[gq], v);
             }
         }
-        // pass 2: weighted sums of o and l
-        for (int c = first_run; c <= last_run; ++c) {
-            const float* q = p.partials + ((size_t)(c + stream) * HG + warp) * p.slot_floats;
+        constexpr int NV = (G * D + 127) / 128;        // float4 groups per lane
+        float4 acc[NV];
 #pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                const int idx = 4 * lane + 128 * v;
-                if (idx < G * D && mx[v] != -INFINITY) {
-                    const int gq = idx / D;
-                    const float mc = __ldcg(q + G * D + gq);
-                    const float a = (mc == -INFINITY) ? 0.f : fast_exp2(mc - mx[v]);
-                    const float4 ov = __ldcg(reinterpret_cast<const float4*>(q + idx));
-                    acc[v].x = fmaf(a, ov.x, acc[v].x);
-                    acc[v].y = fmaf(a, ov.y, acc[v].y);
-                    acc[v].z = fmaf(a, ov.z, acc[v].z);
-                    acc[v].w = fmaf(a, ov.w, acc[v].w);
-                    ls[v] = fmaf(a, __ldcg(q + G * D + G + gq), ls[v]);
+        for (int v = 0; v < NV; ++v)
+            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = 0; c0 < nseg; c0 += 32) {
+            const bool mine = c0 + lane < nseg;
+            float w[G];                                 // this lane's segment weights
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+                const float mc = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
+                const float lc = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
+                w[gq] = (mc == -INFINITY || M[gq] == -INFINITY) ? 0.f : fast_exp2(mc - M[gq]);
+                float lw = w[gq] * lc;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    lw += __shfl_xor_sync(kFullMask, lw, off);
+                Lsum[gq] += lw;
+            }
+            const int cnt = min(32, nseg - c0);
+            for (int j = 0; j < cnt; j += 4) {          // four segments' loads in flight
+                float4 ov[4][NV];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) {
+                        const int idx = 4 * lane + 128 * v;
+                        ov[u][v] = (j + u < cnt && idx < G * D)
+                                       ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float wu[G];
+#pragma unroll
+                    for (int gq = 0; gq < G; ++gq)
+                        wu[gq] = __shfl_sync(kFullMask, w[gq], (j + u) & 31);
+                    if (j + u < cnt) {
+#pragma unroll
+                        for (int v = 0; v < NV; ++v) {
+                            const int gv = (4 * lane + 128 * v) / D;
+                            float a = 0.f;
+#pragma unroll
+                            for (int gq = 0; gq < G; ++gq)
+                                a = (gq == gv) ? wu[gq] : a;
+                            acc[v].x = fmaf(a, ov[u][v].x, acc[v].x);
+                            acc[v].y = fmaf(a, ov[u][v].y, acc[v].y);
+                            acc[v].z = fmaf(a, ov[u][v].z, acc[v].z);
+                            acc[v].w = fmaf(a, ov[u][v].w, acc[v].w);
+                        }
+                    }
                 }
             }
         }
@@ -617,7 +683,12 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
         for (int v = 0; v < NV; ++v) {
             const int idx = 4 * lane + 128 * v;
             if (idx < G * D) {
-                const float inv = ls[v] > 0.f ? p.v_scale / ls[v] : 0.f;
+                const int gv = idx / D;
+                float L = 0.f;
+#pragma unroll
+                for (int gq = 0; gq < G; ++gq)
+                    L = (gq == gv) ? Lsum[gq] : L;
+                const float inv = L > 0.f ? p.v_scale / L : 0.f;
                 from_float(acc[v].x * inv, out + idx);
                 from_float(acc[v].y * inv, out + idx + 1);
                 from_float(acc[v].z * inv, out + idx + 2);
