@@ -166,6 +166,30 @@ def smi_index(torch, dev: int) -> str:
     return str(dev)
 
 
+# ----------------------------------------------------------------------------- ranks
+
+MAX_KEYS = ("ms", "decode_ms", "e2e_ms", "errors")      # timed over ranks: the slowest rank counts
+SUM_KEYS = ("step_bytes",)                               # work: every replica's bytes count
+
+
+def aggregate_ranks(torch, dist, device, **vals):
+    """Whole-job figures: the max over ranks of the times and error words, the sum of the bytes.
+
+    With dist None (one process) the values are returned unchanged. Works on any process-group
+    backend (NCCL with a CUDA device, gloo with the CPU)."""
+    if dist is None:
+        return dict(vals)
+    keys = list(vals)
+    t = torch.tensor([float(vals[k]) for k in keys], dtype=torch.float64, device=device)
+    mx, tot = t.clone(), t.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    out = {}
+    for i, k in enumerate(keys):
+        out[k] = tot[i].item() if k in SUM_KEYS else mx[i].item()
+    return out
+
+
 # ----------------------------------------------------------------------------- device state
 
 class DeviceState:
@@ -388,18 +412,10 @@ def ours_arm(args):
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
     # aggregate over ranks: max time, summed bytes
-    vals = torch.tensor([ms, sum(dec_ms) / K, e2e["ms"] if e2e else 0.0, float(bytes_step), float(errs)],
-                        dtype=torch.float64, device=dev)
-    if dist:
-        mx = vals.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        tot = vals.clone()
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-        ms_max, dec_max, e2e_max = mx[0].item(), mx[1].item(), mx[2].item()
-        bytes_all = tot[3].item()
-        errs_all = int(mx[4].item())
-    else:
-        ms_max, dec_max, e2e_max, bytes_all, errs_all = ms, sum(dec_ms) / K, (e2e["ms"] if e2e else 0.0), bytes_step, errs
+    agg = aggregate_ranks(torch, dist, dev, ms=ms, decode_ms=sum(dec_ms) / K,
+                          e2e_ms=e2e["ms"] if e2e else 0.0, step_bytes=float(bytes_step), errors=float(errs))
+    ms_max, dec_max, e2e_max = agg["ms"], agg["decode_ms"], agg["e2e_ms"]
+    bytes_all, errs_all = agg["step_bytes"], int(agg["errors"])
 
     if rank == 0:
         peak, peak_kind = measured_peak()
