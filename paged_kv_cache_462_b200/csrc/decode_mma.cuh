@@ -584,78 +584,111 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
     }
 
     // ---- split streams: publish, count arrivals; the last run to arrive merges (log-sum-exp)
-    for (int i = 0; i < nsplit; ++i) {
-        const int s = split_seq[i], stream = split_stream[i];
-        const int first_run = split_first[i], last_run = split_last[i];
-        const int head = (stream - s * NHG) * HG + warp;
-        const int pair = s * Hkv + head;
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            const int arrived = atomicAdd(&p.counters[pair], 1);
-            last = (arrived == last_run - first_run) ? 1 : 0;
-            if (last)
-                p.counters[pair] = 0;
+    if (nsplit == 0)
+        return;
+    __threadfence();                               // this warp's partials are visible before it counts
+    __syncwarp();
+    int last_bits = 0;
+    if (lane == 0) {
+        int arrived[2] = {0, 0};
+        for (int i = 0; i < nsplit; ++i) {
+            const int head = (split_stream[i] - split_seq[i] * NHG) * HG + warp;
+            arrived[i] = atomicAdd(&p.counters[split_seq[i] * Hkv + head], 1);
         }
-        last = __shfl_sync(kFullMask, last, 0);
-        if (!last)
+        for (int i = 0; i < nsplit; ++i) {
+            if (arrived[i] == split_last[i] - split_first[i]) {
+                const int head = (split_stream[i] - split_seq[i] * NHG) * HG + warp;
+                p.counters[split_seq[i] * Hkv + head] = 0;
+                last_bits |= 1 << i;
+            }
+        }
+    }
+    last_bits = __shfl_sync(kFullMask, last_bits, 0);
+    if (last_bits == 0)
+        return;
+    __threadfence();
+    for (int i = 0; i < nsplit; ++i) {
+        if (!((last_bits >> i) & 1))
             continue;
-        __threadfence();
+        const int s = split_seq[i], stream = split_stream[i];
+        const int first_run = split_first[i];
+        const int nseg = split_last[i] - first_run + 1;
+        const int head = (stream - s * NHG) * HG + warp;
         QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
-        const int nseg = last_run - first_run + 1;
         auto slot = [&](int c) -> const float* {
             return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
         };
-        // weights: lane c owns segment c (32 at a time); per head the largest reference max
-        float M[G], Lsum[G];
-#pragma unroll
-        for (int gq = 0; gq < G; ++gq) {
-            M[gq] = -INFINITY;
-            Lsum[gq] = 0.f;
-        }
-        for (int c0 = 0; c0 < nseg; c0 += 32) {
-            const bool mine = c0 + lane < nseg;
-#pragma unroll
-            for (int gq = 0; gq < G; ++gq) {
-                float v = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1)
-                    v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
-                M[gq] = fmaxf(M[gq], v);
-            }
-        }
-        constexpr int NV = (G * D + 127) / 128;        // float4 groups per lane
+        constexpr int NV = (G * D + 127) / 128;    // float4 groups per lane
         float4 acc[NV];
 #pragma unroll
         for (int v = 0; v < NV; ++v)
             acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum[G];
+        float Mcur[G];                             // running reference over the 32-segment chunks
+#pragma unroll
+        for (int gq = 0; gq < G; ++gq) {
+            Lsum[gq] = 0.f;
+            Mcur[gq] = -INFINITY;
+        }
         for (int c0 = 0; c0 < nseg; c0 += 32) {
-            const bool mine = c0 + lane < nseg;
-            float w[G];                                 // this lane's segment weights
+            const int cnt = min(32, nseg - c0);
+            const bool mine = lane < cnt;
+            // one round trip: lane c's segment (m, l), and every lane's slice of the first four segments' o
+            float mc[G], lc[G];
 #pragma unroll
             for (int gq = 0; gq < G; ++gq) {
-                const float mc = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
-                const float lc = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
-                w[gq] = (mc == -INFINITY || M[gq] == -INFINITY) ? 0.f : fast_exp2(mc - M[gq]);
-                float lw = w[gq] * lc;
+                mc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
+                lc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
+            }
+            float4 ov[4][NV];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    const int idx = 4 * lane + 128 * v;
+                    ov[u][v] = (u < cnt && idx < G * D) ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + u) + idx))
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            // chunk reference max, rescale what earlier chunks accumulated
+            float w[G];
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+                float mx = mc[gq];
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+                const float Mn = fmaxf(Mcur[gq], mx);
+                const float rescale = (Mcur[gq] == -INFINITY) ? 0.f : fast_exp2(Mcur[gq] - Mn);
+                Lsum[gq] *= rescale;
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    if ((4 * lane + 128 * v) / D == gq) {
+                        acc[v].x *= rescale;
+                        acc[v].y *= rescale;
+                        acc[v].z *= rescale;
+                        acc[v].w *= rescale;
+                    }
+                }
+                Mcur[gq] = Mn;
+                w[gq] = (mc[gq] == -INFINITY || Mn == -INFINITY) ? 0.f : fast_exp2(mc[gq] - Mn);
+                float lw = w[gq] * lc[gq];
 #pragma unroll
                 for (int off = 16; off >= 1; off >>= 1)
                     lw += __shfl_xor_sync(kFullMask, lw, off);
                 Lsum[gq] += lw;
             }
-            const int cnt = min(32, nseg - c0);
-            for (int j = 0; j < cnt; j += 4) {          // four segments' loads in flight
-                float4 ov[4][NV];
+            for (int j = 0; j < cnt; j += 4) {
+                if (j > 0) {                         // later groups of four segments
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
+                    for (int u = 0; u < 4; ++u)
 #pragma unroll
-                    for (int v = 0; v < NV; ++v) {
-                        const int idx = 4 * lane + 128 * v;
-                        ov[u][v] = (j + u < cnt && idx < G * D)
-                                       ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
+                        for (int v = 0; v < NV; ++v) {
+                            const int idx = 4 * lane + 128 * v;
+                            ov[u][v] = (j + u < cnt && idx < G * D)
+                                           ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     float wu[G];
