@@ -132,6 +132,31 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * One whole decode step: the append of each sequence's new token (reshape_and_cache of
+ * new_k/new_v row s at slot_mapping[s], one new token per sequence) followed by
+ * paged_attention_decode over the cache that includes it. For bf16 and E4M3 caches of
+ * the shapes the tensor-core decode kernel covers (block_size 16 or 32, group <= 8,
+ * head_dim 64/128 for bf16, 128 for E4M3) both happen in ONE launch: the warp that
+ * streams a sequence's last block first writes the new rows into it. Other shapes run
+ * the two calls in stream order. Results are those of the two calls.
+ *
+ *   new_k, new_v   [num_seqs][num_kv_heads][head_dim] of in_dtype (F32 or BF16)
+ *   slot_mapping   int64 [num_seqs]; a non-negative slot must lie in the block that
+ *                  holds position seq_lens[s] - 1 of sequence s (its last block), so
+ *                  seq_lens[s] >= 1; a negative slot appends nothing.
+ * Other arguments as paged_attention_decode; slot errors go to the workspace error word.
+ * The one-launch form raises PKV_DEVERR_SLOT for a slot outside the last block (still
+ * written, but sequence s's output is then unspecified) and for a non-negative slot of
+ * a sequence with seq_lens[s] == 0 (nothing written).
+ */
+PKV_API int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, const int32_t* block_tables,
+                              const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                              int block_size, float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                              int kv_dtype, float k_scale, float v_scale, int num_partitions, void* workspace,
+                              size_t workspace_bytes, const void* new_k, const void* new_v,
+                              const int64_t* slot_mapping, int in_dtype, void* stream);
+
+/*
  * paged_attention_decode without a caller workspace, for callers that cannot
  * allocate device memory: code running while a CUDA graph is captured,
  * plug-ins whose host framework owns every allocation, hosts that reserve all

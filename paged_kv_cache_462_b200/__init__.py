@@ -54,6 +54,9 @@ def load_library():
     lib.paged_attention_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                            f32, f32, i32, P, sz, P]
     lib.paged_attention_decode.restype = i32
+    lib.paged_decode_step.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                      f32, f32, i32, P, sz, P, P, P, i32, P]
+    lib.paged_decode_step.restype = i32
     lib.reshape_and_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, f32, P, P]
     lib.reshape_and_cache.restype = i32
     lib.pkv_read_device_error.argtypes = [P, sz, ctypes.POINTER(ctypes.c_int32), i32, P]
@@ -151,6 +154,34 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
     _check("paged_attention_decode", st)
 
 
+def paged_decode_step(out, q, k_cache, v_cache, block_tables, seq_lens, new_k, new_v, slot_mapping, scale,
+                      k_scale=1.0, v_scale=1.0, num_partitions=0, workspace=None, stream=None) -> None:
+    """One decode step: append new_k/new_v row s at slot_mapping[s] (one new token per sequence,
+    in its last block), then paged_attention_decode over the cache. One launch where the
+    tensor-core decode kernel applies."""
+    S, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q/out and the caches")
+    if tuple(new_k.shape) != (S, Hkv, D) or tuple(new_v.shape) != (S, Hkv, D) or new_v.dtype != new_k.dtype:
+        raise ValueError("new_k/new_v must be [num_seqs, num_kv_heads, head_dim] of one dtype")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (S,):
+        raise TypeError("slot_mapping must be int64 [num_seqs]")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
+    if workspace is None:
+        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, q.device)
+    st = load_library().paged_decode_step(
+        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
+        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
+        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _cuda("new_k", new_k),
+        _cuda("new_v", new_v), _cuda("slot_mapping", slot_mapping), _dtype_code(new_k), _stream_handle(stream))
+    _check("paged_decode_step", st)
+
+
 def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=1.0, v_scale=1.0,
                       device_error=None, stream=None) -> None:
     """Write k[t], v[t] ([num_tokens, num_kv_heads, head_dim]) into slot slot_mapping[t] of the caches."""
@@ -190,7 +221,7 @@ def _cached_workspace(S, Hq, Hkv, D, parts, device):
 
 
 __all__ = [
-    "paged_attention_decode", "reshape_and_cache", "workspace_size", "new_workspace", "workspace_init",
+    "paged_attention_decode", "paged_decode_step", "reshape_and_cache", "workspace_size", "new_workspace", "workspace_init",
     "read_device_error", "default_partitions", "status_string", "load_library", "PkvError",
     "F32", "BF16", "FP8_E4M3",
 ]

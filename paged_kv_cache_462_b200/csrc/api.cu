@@ -224,11 +224,22 @@ int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_
     return sms * occ;
 }
 
-int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
-                           int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
-                           int num_blocks, int q_dtype, int kv_dtype, float k_scale, float v_scale,
-                           int num_partitions, void* workspace, size_t workspace_bytes, void* stream)
+}  // extern "C"
+
+namespace {
+
+struct AppendArgs {
+    const void* k;
+    const void* v;
+    const int64_t* slots;
+    int in_dtype;
+};
+
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
+                float v_scale, int num_partitions, void* workspace, size_t workspace_bytes, void* stream,
+                const AppendArgs* app)
 {
     if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads != 0 || num_partitions < 0)
@@ -299,8 +310,67 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
+    if (app) {
+        p.new_k = app->k;
+        p.new_v = app->v;
+        p.new_slots = app->slots;
+        p.in_dtype = app->in_dtype;
+    }
     return decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, p, runs,
                            static_cast<cudaStream_t>(stream), nullptr);
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                           int num_blocks, int q_dtype, int kv_dtype, float k_scale, float v_scale,
+                           int num_partitions, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                       block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
+                       num_partitions, workspace, workspace_bytes, stream, nullptr);
+}
+
+int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, const int32_t* block_tables,
+                      const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                      int block_size, float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                      float k_scale, float v_scale, int num_partitions, void* workspace, size_t workspace_bytes,
+                      const void* new_k, const void* new_v, const int64_t* slot_mapping, int in_dtype, void* stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+        return PKV_ERR_SHAPE;
+    if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) && (kv_dtype == in_dtype || kv_dtype == PKV_FP8_E4M3)))
+        return PKV_ERR_DTYPE;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (!new_k || !new_v || !slot_mapping)
+        return PKV_ERR_NULL;
+    if (!workspace)
+        return PKV_ERR_WORKSPACE;
+    if (!aligned16(new_k) || !aligned16(new_v))
+        return PKV_ERR_SHAPE;
+    if (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.0f && v_scale > 0.0f))
+        return PKV_ERR_SHAPE;
+    const int group = num_heads / num_kv_heads;
+    if (q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)) {
+        const AppendArgs app{new_k, new_v, slot_mapping, in_dtype};
+        return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                           head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                           v_scale, num_partitions, workspace, workspace_bytes, stream, &app);
+    }
+    // shapes the fused kernel does not cover: the two calls in stream order
+    const int st = reshape_and_cache(new_k, new_v, k_cache, v_cache, slot_mapping, num_seqs, num_kv_heads, head_dim,
+                                     block_size, num_blocks, in_dtype, kv_dtype, k_scale, v_scale,
+                                     static_cast<int32_t*>(workspace), stream);
+    if (st != PKV_OK)
+        return st;
+    return paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                                  head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
+                                  k_scale, v_scale, num_partitions, workspace, workspace_bytes, stream);
 }
 
 int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,

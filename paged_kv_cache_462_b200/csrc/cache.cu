@@ -21,54 +21,6 @@ namespace pkv {
 
 namespace {
 
-__device__ __forceinline__ void load8(const float* p, float* f)
-{
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    const float4 b = *reinterpret_cast<const float4*>(p + 4);
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f)
-{
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    widen_word(KvBF16{}, u.x, f + 0);
-    widen_word(KvBF16{}, u.y, f + 2);
-    widen_word(KvBF16{}, u.z, f + 4);
-    widen_word(KvBF16{}, u.w, f + 6);
-}
-
-template <class T>
-__device__ __forceinline__ void copy8(const T* src, T* dst)
-{
-    if constexpr (sizeof(T) == 4) {
-        reinterpret_cast<float4*>(dst)[0] = reinterpret_cast<const float4*>(src)[0];
-        reinterpret_cast<float4*>(dst)[1] = reinterpret_cast<const float4*>(src)[1];
-    } else {
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-    }
-}
-
-template <class TIN>
-__device__ __forceinline__ void quant8(const TIN* src, uint8_t* dst, float scale)
-{
-    float f[8];
-    load8(src, f);
-    uint32_t w[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t packed = 0;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float2 y = make_float2(__fdiv_rn(f[4 * h + 2 * i], scale), __fdiv_rn(f[4 * h + 2 * i + 1], scale));
-            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
-            packed |= static_cast<uint32_t>(c) << (16 * i);
-        }
-        w[h] = packed;
-    }
-    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-}
-
 // TIN: float or bf16 input rows; TC: cache element (same as TIN, or uint8_t E4M3 codes).
 template <class TIN, class TC>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(

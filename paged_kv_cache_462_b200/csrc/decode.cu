@@ -36,6 +36,11 @@ bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int nu
     return mma_head_group(kv_dtype, head_dim, block_size, num_kv_heads) > 0;
 }
 
+bool step_fusable(int q_dtype, int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)
+{
+    return q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads);
+}
+
 // Largest head group in {4, 2, 1} that divides num_kv_heads and keeps a stage (K + V) within
 // 32 KB: two CTAs (two independent copy pipelines) per SM, 5 warps each.
 int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads)

@@ -115,6 +115,65 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Decode-step append fused into the producer warp: write the new token of sequence s (row s of
+// new_k / new_v) for KV heads h0 .. h0+nh-1 into its slot, with the conversion reshape_and_cache
+// uses, then order those writes before this warp's later TMA reads of the same block.
+template <class TC>
+__device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0, int nh, int D, int BS, int lane,
+                                            long long slot)
+{
+    const int pieces = D / 8;
+    const long long blk = slot / BS, off = slot - blk * BS;
+    TC* kc = reinterpret_cast<TC*>(const_cast<uint8_t*>(p.k_cache));
+    TC* vc = reinterpret_cast<TC*>(const_cast<uint8_t*>(p.v_cache));
+    for (int it = lane; it < 2 * nh * pieces; it += 32) {
+        const bool is_v = it >= nh * pieces;
+        const int r = is_v ? it - nh * pieces : it;
+        const int h = h0 + r / pieces, c = r % pieces;
+        const long long src_off = ((long long)s * p.num_kv_heads + h) * D + c * 8;
+        TC* dst = (is_v ? vc : kc) + ((blk * p.num_kv_heads + h) * BS + off) * D + c * 8;
+        if (p.in_dtype == PKV_F32) {
+            const float* src = static_cast<const float*>(is_v ? p.new_v : p.new_k) + src_off;
+            if constexpr (sizeof(TC) == 1)
+                quant8(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+        } else {
+            const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.new_v : p.new_k) + src_off;
+            if constexpr (sizeof(TC) == 1)
+                quant8(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+            else
+                copy8(src, reinterpret_cast<__nv_bfloat16*>(dst));
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// `last_phys`: physical block the sequence's last position maps to (-1 when its id was bad);
+// a slot outside it is still written but flagged, since the decode may not see it
+template <int KVBYTES>
+__device__ __forceinline__ void append_new_token_impl(const DecodeParams& p, int s, int h0, int nh, int D, int BS,
+                                                      int lane, int last_phys)
+{
+    const long long slot = __ldg(p.new_slots + s);
+    if (slot >= 0) {
+        if (lane == 0 && last_phys >= 0 && slot / BS != last_phys)
+            atomicOr(p.err, PKV_DEVERR_SLOT);
+        if (slot >= (long long)p.num_blocks * BS) {
+            if (lane == 0)
+                atomicOr(p.err, PKV_DEVERR_SLOT);
+        } else if constexpr (KVBYTES == 1) {
+            append_rows<uint8_t>(p, s, h0, nh, D, BS, lane, slot);
+        } else {
+            append_rows<__nv_bfloat16>(p, s, h0, nh, D, BS, lane, slot);
+        }
+    }
+    fence_proxy_async_global();
+    __syncwarp();
+}
+
 // ------------------------------------------------------------------ configuration
 
 template <class KV, int D, int BS, int G, int HG>
@@ -222,6 +281,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
     // zero rows of empty sequences (one run per sequence)
     for (int s = blockIdx.x; s < p.num_seqs; s += nruns) {
         if (prefix[s + 1] == prefix[s]) {
+            // a new token needs a position in the sequence: seq_lens[s] >= 1
+            if (tid == 0 && p.new_k != nullptr && __ldg(p.new_slots + s) >= 0)
+                atomicOr(p.err, PKV_DEVERR_SLOT);
             QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * p.num_heads * D;
             for (int i = tid; i < p.num_heads * D; i += C::kThreads)
                 from_float(0.f, o + i);
@@ -236,8 +298,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
         }
-        // lane l resolves unit (batch + l): pool row of its head group, or -1 for a bad block id
-        auto locate = [&](int k) -> int {
+        // lane l resolves unit (batch + l): pool row of its head group, or -1 for a bad block id;
+        // `app` is the stream (sequence * NHG + head group) whose new token lands in this unit
+        // (its last block) when the launch also appends, else -1
+        auto locate = [&](int k, int& app) -> int {
+            app = -1;
             if (k >= nunits)
                 return -1;
             const int x = run_begin + k;
@@ -245,6 +310,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
             const int nb = (prefix[s + 1] - prefix[s]) / NHG;
             const int r = x - prefix[s];
             const int hg = r / nb, j = r - hg * nb;
+            if (p.new_k != nullptr && j == nb - 1)
+                app = s * NHG + hg;
             const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + j);
             if (phys < 0 || phys >= p.num_blocks) {
                 atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
@@ -252,17 +319,23 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
             }
             return (phys * Hkv + hg * HG) * BS;
         };
-        int cur = locate(lane), ahead = locate(32 + lane);
+        int cur_app, ahead_app;
+        int cur = locate(lane, cur_app), ahead = locate(32 + lane, ahead_app);
         bool aborted = false;
         int issued = 0;
         for (int k0 = 0; k0 < nunits; k0 += 32) {
             if (k0 > 0) {
                 cur = ahead;
-                ahead = locate(k0 + 32 + lane);
+                cur_app = ahead_app;
+                ahead = locate(k0 + 32 + lane, ahead_app);
             }
             const int cnt = min(32, nunits - k0);
             for (int i = 0; i < cnt; ++i) {
                 const int row = __shfl_sync(kFullMask, cur, i);
+                const int app = __shfl_sync(kFullMask, cur_app, i);
+                if (app >= 0)   // the decode-step append of this stream, before its last block is read
+                    append_new_token_impl<KV::kBytes>(p, app / NHG, (app % NHG) * HG, HG, D, BS, lane,
+                                                      row < 0 ? -1 : row / (Hkv * BS));
                 if (lane == 0 && !aborted) {
                     const int k = k0 + i;
                     const int st = k % S;

@@ -39,6 +39,12 @@ struct DecodeParams {
     float* partials;   // [(runs + pairs)][slot_floats]
     int slot_floats;
     int stages_per_warp; // set by the launcher
+    // fused decode-step append (null new_k: none): row s of new_k/new_v ([num_seqs][num_kv_heads]
+    // [head_dim], in_dtype) goes to slot new_slots[s], which lies in sequence s's last block
+    const void* new_k;
+    const void* new_v;
+    const int64_t* new_slots;
+    int in_dtype;
 };
 
 // Kernel selection: warp-MMA kernel for bf16 / E4M3 caches of supported shapes,
@@ -49,6 +55,9 @@ bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int nu
 int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads);
 int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
                         cudaStream_t st, int* occ);
+
+// The fused step's append + decode in one launch (warp-MMA kernel only).
+bool step_fusable(int q_dtype, int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads);
 
 int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                    int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,

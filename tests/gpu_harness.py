@@ -78,6 +78,18 @@ class GpuStep:
         self.append()
         return self.decode(num_partitions)
 
+    def fused_step(self, num_partitions=0, workspace=None):
+        """The step through paged_decode_step (append fused into the decode launch where it applies)."""
+        b = self.b
+        sp = b.spec
+        if workspace is None:
+            workspace = pkv.new_workspace(b.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, num_partitions)
+        self.ws = workspace
+        pkv.paged_decode_step(self.out, self.q, self.kc, self.vc, self.bt, self.sl, self.new_k, self.new_v,
+                              self.new_slots, float(b.scale), float(b.k_scale), float(b.v_scale), num_partitions,
+                              workspace)
+        return self.out
+
     def device_errors(self):
         torch.cuda.synchronize()
         e = int(self.err.item())

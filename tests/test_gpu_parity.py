@@ -226,3 +226,73 @@ def test_bad_seq_len_is_flagged_and_clamped():
     g.sl = torch.from_numpy(sl).cuda()
     g.decode(0)
     assert g.device_errors() & pkv.DEVERR_SEQ_LEN
+
+
+# ------------------------------------------------------------------ fused step
+
+@pytest.mark.parametrize("cfg,over", [(0, {}), (1, dict(num_seqs=8)), (3, dict(num_seqs=16)), (4, dict(num_seqs=6)),
+                                      (2, dict(num_seqs=2, lengths=("fixed", 1000)))])
+@pytest.mark.parametrize("parts", [0, 3, 64])
+def test_fused_step_matches_oracle_and_two_calls(cfg, over, parts):
+    """paged_decode_step = reshape_and_cache + paged_attention_decode: same caches (bit-exact),
+    outputs within tolerance of the oracle and identical to the two separate calls."""
+    b = W.config_batch(cfg, **over)
+    ref, okc, ovc = oracle.run_step(b)
+    g1 = GpuStep(b)
+    out1 = g1.fused_step(parts).clone()
+    assert g1.device_errors() == 0
+    assert np.array_equal(cache_bytes(g1.kc), okc) and np.array_equal(cache_bytes(g1.vc), ovc)
+    assert max_err(out1, ref) <= TOL[b.spec.kv_dtype]
+    g2 = GpuStep(b)
+    out2 = g2.step(parts)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+@pytest.mark.parametrize("BS", [8, 16, 32])
+def test_fused_step_shapes(kv, BS):
+    lengths = [1, BS, BS + 1, 3 * BS - 1, 97, 200, 0]
+    b = W.build_batch(_spec(f"fused_{kv}_{BS}", len(lengths), 8, 2, 128, BS, kv, lengths, seed=77 + BS))
+    ref, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    out = g.fused_step(5)
+    assert g.device_errors() == 0
+    assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
+    assert max_err(out, ref) <= TOL[kv]
+
+
+def test_fused_step_negative_slot_appends_nothing():
+    """A negative slot skips that sequence's append; its decode then reads the (zero) row."""
+    b = W.config_batch(1, num_seqs=6)
+    b.new_slots[[1, 4]] = -1
+    ref, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    out = g.fused_step(0)
+    assert g.device_errors() == 0
+    assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
+    assert max_err(out, ref) <= TOL["bf16"]
+
+
+def test_fused_step_flags_slot_outside_last_block():
+    b = W.config_batch(1, num_seqs=4)
+    g = GpuStep(b)
+    slots = b.new_slots.copy()
+    slots[2] = int(b.block_tables[2, 0]) * b.spec.block_size    # first block, not the last
+    g.new_slots = torch.from_numpy(slots).cuda()
+    out = g.fused_step(0)
+    assert g.device_errors() & pkv.DEVERR_SLOT
+    ref, _, _ = oracle.run_step(b, seqs=[0, 1, 3])
+    assert max_err(out, ref, [0, 1, 3]) <= TOL["bf16"]           # other sequences untouched
+
+
+def test_fused_step_flags_slot_of_empty_sequence():
+    lengths = [40, 0, 17]
+    b = W.build_batch(_spec("fused_empty_slot", len(lengths), 8, 2, 128, 16, "bf16", lengths, seed=5))
+    g = GpuStep(b)
+    slots = b.new_slots.copy()
+    slots[1] = 0
+    g.new_slots = torch.from_numpy(slots).cuda()
+    out = g.fused_step(0)
+    assert g.device_errors() & pkv.DEVERR_SLOT
+    assert not torch.any(out[1].float() != 0)
