@@ -462,7 +462,8 @@ def ours_arm(args):
                 "traffic": kernel_traffic(args.config),
                 "algorithmic_bytes": kern_bytes,
             },
-            "gpu_launches": (1 if fused else 2) * K,
+            # fused: the decode kernel (append inside) + the merge kernel; else append + decode
+            "gpu_launches": 2 * K,
             "clocks": clocks.summary() if clocks else None,
             "device_errors": errs_all,
         }

@@ -31,8 +31,13 @@
 //    (head_dim x 8 heads, k = 16 tokens). bf16 caches use bf16 MMA; E4M3 codes
 //    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2) and use f16 MMA, the
 //    per-tensor scales applied to the fp32 scores and outputs.
-//  * Split streams: the same last-arriver log-sum-exp merge as the CUDA-core
-//    kernel, per (sequence, KV head), done by one warp.
+//  * Split streams (a stream cut by a run boundary): each run's warp stores its
+//    piece's fp32 partial (o, m, l) and moves on. A second, small kernel
+//    launched as a programmatic dependent launch merges them (log-sum-exp, a
+//    warp per stream and KV head) once the decode grid has finished: no fence,
+//    atomic or merge ever sits in the streaming kernel, whose memory system is
+//    saturated (a global round trip there costs microseconds), and the result
+//    does not depend on timing.
 #pragma once
 
 #include <cstdint>
@@ -199,6 +204,45 @@ struct MmaCfg {
 // Byte offset of the 16-byte chunk `c` (0..7) of box row `r` in a 128B-swizzled box.
 __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// prefix[s] = units (head group x logical block) of sequences before s, units of a sequence =
+// ceil(L / block_size) * groups with L clamped to [0, capacity]. All threads of the CTA; ends
+// with a barrier. False if some seq_len needed clamping.
+__device__ __forceinline__ bool build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity)
+{
+    const int tid = threadIdx.x, lane = tid & 31;
+    bool bad_len = false;
+    for (int s = tid; s < p.num_seqs; s += blockDim.x) {
+        int L = p.seq_lens[s];
+        if (L < 0 || L > capacity) {
+            bad_len = true;
+            L = L < 0 ? 0 : capacity;
+        }
+        prefix[s + 1] = ((L + BS - 1) / BS) * NHG;
+    }
+    if (tid == 0)
+        prefix[0] = 0;
+    const bool any_bad = __syncthreads_or(bad_len);
+    if (tid < 32) {
+        int carry = 0;
+        for (int base = 0; base < p.num_seqs; base += 32) {
+            const int i = base + lane + 1;
+            int v = (i <= p.num_seqs) ? prefix[i] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(kFullMask, v, o);
+                if (lane >= o)
+                    v += u;
+            }
+            v += carry;
+            if (i <= p.num_seqs)
+                prefix[i] = v;
+            carry = __shfl_sync(kFullMask, v, 31);
+        }
+    }
+    __syncthreads();
+    return !any_bad;
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <class KV, class QT, int D, int BS, int G, int HG>
@@ -224,6 +268,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    // the merge kernel that follows may be scheduled now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((smem_addr(smem) & 1023u) != 0u) {   // the 128-byte swizzle needs 1024-byte aligned stages
         if (tid == 0)
             atomicOr(p.err, PKV_DEVERR_TIMEOUT);
@@ -238,38 +284,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    bool bad_len = false;
-    for (int s = tid; s < p.num_seqs; s += C::kThreads) {
-        int L = p.seq_lens[s];
-        if (L < 0 || L > capacity) {
-            bad_len = true;
-            L = L < 0 ? 0 : capacity;
-        }
-        prefix[s + 1] = ((L + BS - 1) / BS) * NHG;
-    }
-    if (bad_len && blockIdx.x == 0)
+    if (!build_unit_prefix(p, prefix, BS, NHG, capacity) && blockIdx.x == 0 && tid == 0)
         atomicOr(p.err, PKV_DEVERR_SEQ_LEN);
-    if (tid == 0)
-        prefix[0] = 0;
-    __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 0; base < p.num_seqs; base += 32) {
-            const int i = base + lane + 1;
-            int v = (i <= p.num_seqs) ? prefix[i] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(kFullMask, v, o);
-                if (lane >= o)
-                    v += u;
-            }
-            v += carry;
-            if (i <= p.num_seqs)
-                prefix[i] = v;
-            carry = __shfl_sync(kFullMask, v, 31);
-        }
-    }
-    __syncthreads();
 
     const int total = prefix[p.num_seqs];
     const int nruns = gridDim.x;
@@ -375,10 +391,6 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
     const int t = lane & 3;    // MMA column pair
     const float qk_scale = p.q_scale;
 
-    // A run's split segments (a stream that continues in another run) are at most its
-    // first and its last; their counters and merges wait until the run is streamed.
-    int nsplit = 0;
-    int split_seq[2] = {0, 0}, split_stream[2] = {0, 0}, split_first[2] = {0, 0}, split_last[2] = {0, 0};
 
     int x = run_begin;
     int k = 0;                 // unit index within the run
@@ -646,161 +658,164 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
                     part[G * D + G + 2 * t + 1] = l[1];
                 }
             }
-            if (nsplit < 2) {
-                split_seq[nsplit] = s;
-                split_stream[nsplit] = stream;
-                split_first[nsplit] = first_run;
-                split_last[nsplit] = last_run;
-                ++nsplit;
-            }
         }
     }
+}
 
-    // ---- split streams: publish, count arrivals; the last run to arrive merges (log-sum-exp)
-    if (nsplit == 0)
-        return;
-    __threadfence();                               // this warp's partials are visible before it counts
-    __syncwarp();
-    int last_bits = 0;
-    if (lane == 0) {
-        int arrived[2] = {0, 0};
-        for (int i = 0; i < nsplit; ++i) {
-            const int head = (split_stream[i] - split_seq[i] * NHG) * HG + warp;
-            arrived[i] = atomicAdd(&p.counters[split_seq[i] * Hkv + head], 1);
-        }
-        for (int i = 0; i < nsplit; ++i) {
-            if (arrived[i] == split_last[i] - split_first[i]) {
-                const int head = (split_stream[i] - split_seq[i] * NHG) * HG + warp;
-                p.counters[split_seq[i] * Hkv + head] = 0;
-                last_bits |= 1 << i;
-            }
-        }
-    }
-    last_bits = __shfl_sync(kFullMask, last_bits, 0);
-    if (last_bits == 0)
-        return;
-    __threadfence();
-    for (int i = 0; i < nsplit; ++i) {
-        if (!((last_bits >> i) & 1))
-            continue;
-        const int s = split_seq[i], stream = split_stream[i];
-        const int first_run = split_first[i];
-        const int nseg = split_last[i] - first_run + 1;
-        const int head = (stream - s * NHG) * HG + warp;
-        QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
-        auto slot = [&](int c) -> const float* {
-            return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
-        };
-        constexpr int NV = (G * D + 127) / 128;    // float4 groups per lane
-        float4 acc[NV];
+// Log-sum-exp merge of the nseg partials of KV head (stream's head group) * HG + warp of sequence
+// s, written by runs first_run .. first_run + nseg - 1, into out. One warp.
+template <class QT, int D, int G, int HG>
+__device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int stream, int first_run, int nseg, int NHG,
+                                           int warp, int lane)
+{
+    const int head = (stream - s * NHG) * HG + warp;
+    QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
+    auto slot = [&](int c) -> const float* {
+        return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
+    };
+    constexpr int NV = (G * D + 127) / 128;    // float4 groups per lane
+    float4 acc[NV];
 #pragma unroll
-        for (int v = 0; v < NV; ++v)
-            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        float Lsum[G];
-        float Mcur[G];                             // running reference over the 32-segment chunks
+    for (int v = 0; v < NV; ++v)
+        acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lsum[G];
+    float Mcur[G];                             // running reference over the 32-segment chunks
+#pragma unroll
+    for (int gq = 0; gq < G; ++gq) {
+        Lsum[gq] = 0.f;
+        Mcur[gq] = -INFINITY;
+    }
+    for (int c0 = 0; c0 < nseg; c0 += 32) {
+        const int cnt = min(32, nseg - c0);
+        const bool mine = lane < cnt;
+        // one round trip: lane c's segment (m, l), and every lane's slice of the first four segments' o
+        float mc[G], lc[G];
 #pragma unroll
         for (int gq = 0; gq < G; ++gq) {
-            Lsum[gq] = 0.f;
-            Mcur[gq] = -INFINITY;
+            mc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
+            lc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
         }
-        for (int c0 = 0; c0 < nseg; c0 += 32) {
-            const int cnt = min(32, nseg - c0);
-            const bool mine = lane < cnt;
-            // one round trip: lane c's segment (m, l), and every lane's slice of the first four segments' o
-            float mc[G], lc[G];
+        float4 ov[4][NV];
 #pragma unroll
-            for (int gq = 0; gq < G; ++gq) {
-                mc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
-                lc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                const int idx = 4 * lane + 128 * v;
+                ov[u][v] = (u < cnt && idx < G * D) ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + u) + idx))
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            float4 ov[4][NV];
+        // chunk reference max, rescale what earlier chunks accumulated
+        float w[G];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+        for (int gq = 0; gq < G; ++gq) {
+            float mx = mc[gq];
 #pragma unroll
-                for (int v = 0; v < NV; ++v) {
-                    const int idx = 4 * lane + 128 * v;
-                    ov[u][v] = (u < cnt && idx < G * D) ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + u) + idx))
-                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            // chunk reference max, rescale what earlier chunks accumulated
-            float w[G];
+            for (int off = 16; off >= 1; off >>= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+            const float Mn = fmaxf(Mcur[gq], mx);
+            const float rescale = (Mcur[gq] == -INFINITY) ? 0.f : fast_exp2(Mcur[gq] - Mn);
+            Lsum[gq] *= rescale;
 #pragma unroll
-            for (int gq = 0; gq < G; ++gq) {
-                float mx = mc[gq];
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1)
-                    mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
-                const float Mn = fmaxf(Mcur[gq], mx);
-                const float rescale = (Mcur[gq] == -INFINITY) ? 0.f : fast_exp2(Mcur[gq] - Mn);
-                Lsum[gq] *= rescale;
-#pragma unroll
-                for (int v = 0; v < NV; ++v) {
-                    if ((4 * lane + 128 * v) / D == gq) {
-                        acc[v].x *= rescale;
-                        acc[v].y *= rescale;
-                        acc[v].z *= rescale;
-                        acc[v].w *= rescale;
-                    }
-                }
-                Mcur[gq] = Mn;
-                w[gq] = (mc[gq] == -INFINITY || Mn == -INFINITY) ? 0.f : fast_exp2(mc[gq] - Mn);
-                float lw = w[gq] * lc[gq];
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1)
-                    lw += __shfl_xor_sync(kFullMask, lw, off);
-                Lsum[gq] += lw;
-            }
-            for (int j = 0; j < cnt; j += 4) {
-                if (j > 0) {                         // later groups of four segments
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-#pragma unroll
-                        for (int v = 0; v < NV; ++v) {
-                            const int idx = 4 * lane + 128 * v;
-                            ov[u][v] = (j + u < cnt && idx < G * D)
-                                           ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float wu[G];
-#pragma unroll
-                    for (int gq = 0; gq < G; ++gq)
-                        wu[gq] = __shfl_sync(kFullMask, w[gq], (j + u) & 31);
-                    if (j + u < cnt) {
-#pragma unroll
-                        for (int v = 0; v < NV; ++v) {
-                            const int gv = (4 * lane + 128 * v) / D;
-                            float a = 0.f;
-#pragma unroll
-                            for (int gq = 0; gq < G; ++gq)
-                                a = (gq == gv) ? wu[gq] : a;
-                            acc[v].x = fmaf(a, ov[u][v].x, acc[v].x);
-                            acc[v].y = fmaf(a, ov[u][v].y, acc[v].y);
-                            acc[v].z = fmaf(a, ov[u][v].z, acc[v].z);
-                            acc[v].w = fmaf(a, ov[u][v].w, acc[v].w);
-                        }
-                    }
+            for (int v = 0; v < NV; ++v) {
+                if ((4 * lane + 128 * v) / D == gq) {
+                    acc[v].x *= rescale;
+                    acc[v].y *= rescale;
+                    acc[v].z *= rescale;
+                    acc[v].w *= rescale;
                 }
             }
+            Mcur[gq] = Mn;
+            w[gq] = (mc[gq] == -INFINITY || Mn == -INFINITY) ? 0.f : fast_exp2(mc[gq] - Mn);
+            float lw = w[gq] * lc[gq];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+                lw += __shfl_xor_sync(kFullMask, lw, off);
+            Lsum[gq] += lw;
         }
+        for (int j = 0; j < cnt; j += 4) {
+            if (j > 0) {                         // later groups of four segments
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const int idx = 4 * lane + 128 * v;
-            if (idx < G * D) {
-                const int gv = idx / D;
-                float L = 0.f;
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) {
+                        const int idx = 4 * lane + 128 * v;
+                        ov[u][v] = (j + u < cnt && idx < G * D)
+                                       ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float wu[G];
 #pragma unroll
                 for (int gq = 0; gq < G; ++gq)
-                    L = (gq == gv) ? Lsum[gq] : L;
-                const float inv = L > 0.f ? p.v_scale / L : 0.f;
-                from_float(acc[v].x * inv, out + idx);
-                from_float(acc[v].y * inv, out + idx + 1);
-                from_float(acc[v].z * inv, out + idx + 2);
-                from_float(acc[v].w * inv, out + idx + 3);
+                    wu[gq] = __shfl_sync(kFullMask, w[gq], (j + u) & 31);
+                if (j + u < cnt) {
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) {
+                        const int gv = (4 * lane + 128 * v) / D;
+                        float a = 0.f;
+#pragma unroll
+                        for (int gq = 0; gq < G; ++gq)
+                            a = (gq == gv) ? wu[gq] : a;
+                        acc[v].x = fmaf(a, ov[u][v].x, acc[v].x);
+                        acc[v].y = fmaf(a, ov[u][v].y, acc[v].y);
+                        acc[v].z = fmaf(a, ov[u][v].z, acc[v].z);
+                        acc[v].w = fmaf(a, ov[u][v].w, acc[v].w);
+                    }
+                }
             }
         }
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+        const int idx = 4 * lane + 128 * v;
+        if (idx < G * D) {
+            const int gv = idx / D;
+            float L = 0.f;
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq)
+                L = (gq == gv) ? Lsum[gq] : L;
+            const float inv = L > 0.f ? p.v_scale / L : 0.f;
+            from_float(acc[v].x * inv, out + idx);
+            from_float(acc[v].y * inv, out + idx + 1);
+            from_float(acc[v].z * inv, out + idx + 2);
+            from_float(acc[v].w * inv, out + idx + 3);
+        }
+    }
+}
+
+
+// Merge of the streams the decode kernel split across runs: one warp per (stream, KV head of its
+// group), launched behind the decode kernel as a programmatic dependent launch. The prefix is
+// built while the decode kernel still runs (it reads only seq_lens); griddepcontrol.wait then
+// holds until the decode grid has finished and its partials are visible.
+constexpr int kMergeThreads = 128;
+
+template <class QT, int D, int BS, int G, int HG>
+__global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeParams p, int decode_runs)
+{
+    extern __shared__ int prefix[];   // [num_seqs + 1]
+    const int NHG = p.num_kv_heads / HG;
+    (void)build_unit_prefix(p, prefix, BS, NHG, p.max_blocks_per_seq * BS);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int total = prefix[p.num_seqs];
+    if (total == 0)
+        return;
+    const int per_run = (total + decode_runs - 1) / decode_runs;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (kMergeThreads / 32);
+    const int items = p.num_seqs * NHG * HG;
+    for (int it = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5); it < items; it += warps) {
+        const int stream = it / HG, w = it - stream * HG;
+        const int s = stream / NHG, hg = stream - s * NHG;
+        const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+        if (nb == 0)
+            continue;
+        const int sb = prefix[s] + hg * nb;
+        const int first_run = sb / per_run, last_run = (sb + nb - 1) / per_run;
+        if (first_run != last_run)
+            merge_split<QT, D, G, HG>(p, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
     }
 }
 
@@ -871,7 +886,29 @@ struct MmaLauncher {
         p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 ? p.k_scale : 1.0f);
         p.v_scale = KV::kBytes == 1 ? p.v_scale_in : 1.0f;
         kern<<<nruns, C::kThreads, smem, stream>>>(kmap, vmap, p);
-        return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+        if (cudaGetLastError() != cudaSuccess)
+            return PKV_ERR_LAUNCH;
+        // the merge of split streams, allowed to start while the decode grid drains
+        auto merge = paged_decode_merge_kernel<QT, D, BS, G, HG>;
+        const size_t msmem = (size_t)(p.num_seqs + 1) * 4;
+        if (!ensure_smem_attribute((const void*)merge, msmem))
+            return PKV_ERR_LAUNCH;
+        const int items = p.num_seqs * p.num_kv_heads;
+        const int per_cta = kMergeThreads / 32;
+        int mgrid = (items + per_cta - 1) / per_cta;
+        if (mgrid > nruns)
+            mgrid = nruns;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(mgrid);
+        cfg.blockDim = dim3(kMergeThreads);
+        cfg.dynamicSmemBytes = msmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, merge, p, nruns) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
     }
 };
 
