@@ -434,7 +434,8 @@ def ours_arm(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32",
+            # arithmetic: tensor-core products in bf16 (E4M3 codes widened exactly to f16), fp32 sums
+            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "f16"}[spec.kv_dtype],
             "data": "synthetic",
             "config": {
                 "workload": describe(b), "config_index": args.config,
@@ -453,7 +454,9 @@ def ours_arm(args):
             "step_bytes": bytes_step,
             "roofline": {
                 "bound": "hbm",
-                "kernel": "paged_decode_mma_kernel (decode with the append fused)" if fused else "paged_decode_kernel",
+                # events bracket the whole step: the decode kernel (append fused) and its merge kernel
+                "kernel": ("paged_decode_mma_kernel (append fused) + paged_decode_merge_kernel" if fused
+                           else "reshape_and_cache_kernel + paged_decode_kernel"),
                 "achieved": kern_gbs,
                 "peak": peak,
                 "peak_kind": peak_kind,
