@@ -49,10 +49,24 @@ def parse_args():
     ap.add_argument("--config", type=int, default=1, help="workload 0..4 (default 1, Llama-3-8B bf16)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partitions", type=int, default=0, help="decode runs (0 = automatic)")
+    ap.add_argument("--kv-dtype", choices=["bf16", "e4m3"], default=None,
+                    help="run the workload with this cache dtype instead of its own (configs 1-4)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
+
+
+def workload_spec(args) -> W.Spec:
+    """The config's workload, with the cache dtype replaced when --kv-dtype asks for it (q and the
+    appended rows stay bf16; an E4M3 cache gets per-tensor absmax/448 scales)."""
+    spec = W.config_spec(args.config)
+    if args.kv_dtype is not None:
+        if spec.q_dtype != "bf16":
+            raise SystemExit("--kv-dtype applies to the bf16-query workloads (configs 1-4)")
+        spec.kv_dtype = args.kv_dtype
+        spec.name = f"{spec.name}_{args.kv_dtype}kv" if args.kv_dtype not in spec.name else spec.name
+    return spec
 
 
 def describe(b: W.DecodeBatch) -> str:
@@ -298,7 +312,7 @@ def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    b = W.config_batch(args.config)
+    b = W.build_batch(workload_spec(args))
     items = oracle_pair_sampler(b)
     # size each step to a bounded sample: one (sequence, kv head) pair, so the run stays within minutes
     for i in range(args.warmup):
@@ -344,7 +358,7 @@ def ours_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pkv.load_library()
 
-    spec = W.config_spec(args.config)
+    spec = workload_spec(args)
     b = W.build_batch(spec, seed=spec.seed + 1000 * rank)
     state = DeviceState(torch, pkv, b, dev, args.partitions)
     dec, app = step_bytes(b)

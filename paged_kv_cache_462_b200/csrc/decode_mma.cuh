@@ -196,6 +196,9 @@ struct MmaCfg {
     static constexpr int kDT = D / 16;                        // p.V m-tiles (16 d each)
     static constexpr int W = HG;                              // consumer warps
     static constexpr int kThreads = (W + 1) * 32;
+    // CTAs per SM: E4M3 tiles (16 KB stages) take three, for 12 consumer warps per SM to hide the
+    // widening chain's latency; the same ~192 KB of stages per SM stay in flight either way
+    static constexpr int kCtasPerSM = (KV::kBytes == 1 && kStage <= 16384) ? 3 : 2;
     static_assert(kRowBytes % 128 == 0, "rows are whole 128-byte swizzle spans");
     static_assert(BS % 16 == 0 && G <= 8 && HG <= 8, "tile shape");
     static_assert(kRows <= 256, "TMA box height");
@@ -246,7 +249,7 @@ __device__ __forceinline__ bool build_unit_prefix(const DecodeParams& p, int* pr
 // ------------------------------------------------------------------ kernel
 
 template <class KV, class QT, int D, int BS, int G, int HG>
-__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, 2)
+__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV, D, BS, G, HG>::kCtasPerSM)
     paged_decode_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                             const DecodeParams p)
 {
@@ -835,10 +838,10 @@ struct MmaLauncher {
         return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + (size_t)(num_seqs + 1) * 4 + 64;
     }
 
-    // Ring depth: about 96 KB of stages per CTA so that two CTAs share an SM.
+    // Ring depth: the SM's shared memory split between kCtasPerSM CTAs (~96 KB or ~64 KB of stages).
     static int stages(int num_seqs)
     {
-        const long long budget = kMaxSmemPerBlock / 2 - 1024;
+        const long long budget = kMaxSmemPerBlock / C::kCtasPerSM - 1024;
         const long long room = budget - 16 - (long long)(num_seqs + 1) * 4 - 64;
         long long S = room / (C::kStage + 20);
         if (S > 8)

@@ -12,7 +12,7 @@ namespace pkv {
 
 constexpr int kMaxSmemPerBlock = 227 * 1024;
 constexpr int kMaxSeqs = 16384;         // per call: the per-sequence tile prefix lives in shared memory
-constexpr int kMaxRunsPerSM = 2;        // automatic partition count is at most 2 runs per SM
+constexpr int kMaxRunsPerSM = 3;        // automatic partition count is at most 3 runs per SM
 constexpr size_t kWorkspaceHeader = 256;
 constexpr int kMaxHeadGroup = 4;        // KV heads per MMA work unit (partial slots reserved per run)
 constexpr float kLog2e = 1.4426950408889634074f;
