@@ -528,14 +528,17 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                     sc[1] = (tok0 < valid) ? sc[1] * qk_scale : -INFINITY;
                     sc[2] = (tok0 + 8 < valid) ? sc[2] * qk_scale : -INFINITY;
                     sc[3] = (tok0 + 8 < valid) ? sc[3] * qk_scale : -INFINITY;
+                    // The reference moves only when some score passes it by the slack; each lane
+                    // tests its own scores first, so the butterfly max runs only when one does
+                    // (same result as reducing first: the tile max passes iff some lane's does).
                     float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
+                    if (__any_sync(kFullMask, bm0 > m[0] + kMmaRescaleSlack || bm1 > m[1] + kMmaRescaleSlack)) {
 #pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
-                        bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
-                    }
-                    const bool up0 = bm0 > m[0] + kMmaRescaleSlack, up1 = bm1 > m[1] + kMmaRescaleSlack;
-                    if (__any_sync(kFullMask, up0 || up1)) {
+                        for (int off = 4; off < 32; off <<= 1) {
+                            bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
+                            bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
+                        }
+                        const bool up0 = bm0 > m[0] + kMmaRescaleSlack, up1 = bm1 > m[1] + kMmaRescaleSlack;
                         const float n0 = up0 ? bm0 : m[0], n1 = up1 ? bm1 : m[1];
                         const float a0 = up0 ? fast_exp2(m[0] - n0) : 1.f, a1 = up1 ? fast_exp2(m[1] - n1) : 1.f;
                         m[0] = n0;
