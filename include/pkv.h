@@ -157,6 +157,26 @@ PKV_API int paged_decode_step(void* out, const void* q, void* k_cache, void* v_c
                               const int64_t* slot_mapping, int in_dtype, void* stream);
 
 /*
+ * Test hook for the failure path (no counterpart in the pages). The same call
+ * as paged_attention_decode, except that the producer warp that owns unit
+ * `withheld_unit` (units = (sequence, KV-head group, block) in order) never
+ * hands that unit's stage to its consumer warps and issues nothing after it.
+ * The consumers' bounded wait (about one second) runs out, the launch sets
+ * PKV_DEVERR_TIMEOUT in the workspace error word and returns; nothing faults or
+ * hangs and the CUDA context stays usable. The output of that CTA's streams is
+ * incomplete, and the workspace must be re-initialised (pkv_workspace_init)
+ * before its next use. Only the tensor-core kernel has the hook: bf16 q with
+ * bf16 or E4M3 caches of block size 16 or 32; other shapes return
+ * PKV_ERR_SHAPE, as does withheld_unit < 0.
+ */
+PKV_API int pkv_test_decode_timeout(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                    int num_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                                    int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                                    float k_scale, float v_scale, int num_partitions, void* workspace,
+                                    size_t workspace_bytes, int withheld_unit, void* stream);
+
+/*
  * paged_attention_decode without a caller workspace, for callers that cannot
  * allocate device memory: code running while a CUDA graph is captured,
  * plug-ins whose host framework owns every allocation, hosts that reserve all

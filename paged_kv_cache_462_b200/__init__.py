@@ -57,6 +57,9 @@ def load_library():
     lib.paged_decode_step.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                       f32, f32, i32, P, sz, P, P, P, i32, P]
     lib.paged_decode_step.restype = i32
+    lib.pkv_test_decode_timeout.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                            f32, f32, i32, P, sz, i32, P]
+    lib.pkv_test_decode_timeout.restype = i32
     lib.reshape_and_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, f32, P, P]
     lib.reshape_and_cache.restype = i32
     lib.pkv_read_device_error.argtypes = [P, sz, ctypes.POINTER(ctypes.c_int32), i32, P]
@@ -134,6 +137,15 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
     (float32, bfloat16, or uint8/float8_e4m3fn E4M3 codes with k_scale/v_scale);
     block_tables: int32 [num_seqs, max_blocks_per_seq]; seq_lens: int32 [num_seqs].
     """
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale,
+                        num_partitions, workspace)
+    st = load_library().paged_attention_decode(*args, _stream_handle(stream))
+    _check("paged_attention_decode", st)
+
+
+def _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale, num_partitions,
+                 workspace):
+    """Checked C arguments of a decode call, up to (not including) the stream."""
     S, Hq, D = q.shape
     NB, Hkv, BS, D2 = k_cache.shape
     if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
@@ -146,12 +158,21 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
         raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
     if workspace is None:
         workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, q.device)
-    st = load_library().paged_attention_decode(
-        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
-        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
-        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _stream_handle(stream))
-    _check("paged_attention_decode", st)
+    return (_cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+            _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
+            block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
+            int(num_partitions), _cuda("workspace", workspace), workspace.numel())
+
+
+def withheld_unit_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, withheld_unit, workspace,
+                        k_scale=1.0, v_scale=1.0, num_partitions=0, stream=None) -> None:
+    """Failure-path test hook: paged_attention_decode with unit `withheld_unit`'s stage never handed
+    to its consumers, so their bounded wait runs out and the workspace error word gets
+    DEVERR_TIMEOUT (read it with read_device_error, then workspace_init before reuse)."""
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale,
+                        num_partitions, workspace)
+    st = load_library().pkv_test_decode_timeout(*args, int(withheld_unit), _stream_handle(stream))
+    _check("pkv_test_decode_timeout", st)
 
 
 def paged_decode_step(out, q, k_cache, v_cache, block_tables, seq_lens, new_k, new_v, slot_mapping, scale,

@@ -239,7 +239,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                 float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
                 float v_scale, int num_partitions, void* workspace, size_t workspace_bytes, void* stream,
-                const AppendArgs* app)
+                const AppendArgs* app, int withheld_unit = -1)
 {
     if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads != 0 || num_partitions < 0)
@@ -310,6 +310,11 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
+    if (withheld_unit >= 0) {
+        if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
+            return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
+        p.withheld_unit = withheld_unit + 1;
+    }
     if (app) {
         p.new_k = app->k;
         p.new_v = app->v;
@@ -333,6 +338,20 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
                        block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
                        num_partitions, workspace, workspace_bytes, stream, nullptr);
+}
+
+int pkv_test_decode_timeout(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                            int num_blocks, int q_dtype, int kv_dtype, float k_scale, float v_scale,
+                            int num_partitions, void* workspace, size_t workspace_bytes, int withheld_unit,
+                            void* stream)
+{
+    if (withheld_unit < 0)
+        return PKV_ERR_SHAPE;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                       block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
+                       num_partitions, workspace, workspace_bytes, stream, nullptr, withheld_unit);
 }
 
 int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, const int32_t* block_tables,

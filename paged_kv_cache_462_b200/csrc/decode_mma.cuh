@@ -364,6 +364,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                         aborted = true;
                         *abort_flag = 1;
                         atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                    } else if (p.withheld_unit != 0 && run_begin + k == p.withheld_unit - 1) {
+                        aborted = true;   // test hook: this stage never fills; issue nothing more
                     } else if (row < 0) {
                         skip[st] = 1;
                         mbar_arrive(&full[st]);

@@ -45,6 +45,9 @@ struct DecodeParams {
     const void* new_v;
     const int64_t* new_slots;
     int in_dtype;
+    // failure-path test hook (tensor-core kernel): 1 + the unit whose stage the producer never
+    // hands to its consumers, so their bounded wait runs out; 0 = none
+    int withheld_unit;
 };
 
 // Kernel selection: warp-MMA kernel for bf16 / E4M3 caches of supported shapes,

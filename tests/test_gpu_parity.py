@@ -296,3 +296,49 @@ def test_fused_step_flags_slot_of_empty_sequence():
     out = g.fused_step(0)
     assert g.device_errors() & pkv.DEVERR_SLOT
     assert not torch.any(out[1].float() != 0)
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    """Failure path: a stage that never fills makes the consumers' bounded wait run out (~1 s);
+    the launch returns with DEVERR_TIMEOUT in the workspace and the context keeps working."""
+    b = W.config_batch(1, num_seqs=8)
+    g = GpuStep(b)
+    g.append()
+    ws = pkv.new_workspace(b.num_seqs, b.spec.num_heads, b.spec.num_kv_heads, b.spec.head_dim, 0)
+    pkv.withheld_unit_decode(g.out, g.q, g.kc, g.vc, g.bt, g.sl, float(b.scale), 5, ws)
+    torch.cuda.synchronize()
+    assert pkv.read_device_error(ws) & pkv.DEVERR_TIMEOUT
+    with pytest.raises(pkv.PkvError):
+        pkv.withheld_unit_decode(g.out, g.q, g.kc, g.vc, g.bt, g.sl, float(b.scale), -1, ws)
+    pkv.workspace_init(ws)
+    out = g.decode(0, ws)
+    torch.cuda.synchronize()
+    assert pkv.read_device_error(ws) == 0
+    ref, _, _ = oracle.run_step(b)
+    assert max_err(out, ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("cfg", [1, 4])
+@pytest.mark.parametrize("parts", [0, 7])
+def test_guard_regions_untouched(cfg, parts):
+    """Canaries before and after `out` and after the workspace survive a fused step."""
+    b = W.config_batch(cfg, num_seqs=6)
+    sp = b.spec
+    g = GpuStep(b)
+    guard = 4096
+    n = g.out.numel()
+    big = torch.empty(guard + n + guard, dtype=g.out.dtype, device=g.out.device)
+    big.view(torch.int16).fill_(0x7FC1)                      # a NaN pattern no result takes
+    g.out = big[guard:guard + n].view_as(g.q)
+    wbytes = pkv.workspace_size(b.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, parts)
+    wbig = torch.zeros(wbytes + 65536, dtype=torch.uint8, device=g.out.device)
+    wbig[wbytes:].fill_(0xA5)
+    ws = wbig[:wbytes]
+    pkv.workspace_init(ws)
+    g.fused_step(parts, ws)
+    torch.cuda.synchronize()
+    assert pkv.read_device_error(ws) == 0
+    assert bool((big[:guard].view(torch.int16) == 0x7FC1).all()) and bool((big[guard + n:].view(torch.int16) == 0x7FC1).all())
+    assert bool((wbig[wbytes:] == 0xA5).all())
+    ref, _, _ = oracle.run_step(b)
+    assert max_err(g.out, ref) <= TOL[sp.kv_dtype]
