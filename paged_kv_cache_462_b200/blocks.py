@@ -1,0 +1,109 @@
+"""ctypes binding of the host block manager (include/pkv_blocks.h): argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import PkvError, load_library
+
+NO_BLOCKS, UNKNOWN_SEQ, DUPLICATE_SEQ, TABLE_FULL = 20, 21, 22, 23
+
+_bound = False
+
+
+def _lib():
+    global _bound
+    lib = load_library()
+    if not _bound:
+        P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.pkv_bm_create.argtypes = [i32, i32, i32]
+        lib.pkv_bm_create.restype = P
+        lib.pkv_bm_destroy.argtypes = [P]
+        lib.pkv_bm_destroy.restype = None
+        lib.pkv_bm_add.argtypes = [P, i64, i32]
+        lib.pkv_bm_fork.argtypes = [P, i64, i64]
+        lib.pkv_bm_append.argtypes = [P, i64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.POINTER(ctypes.c_int32)]
+        lib.pkv_bm_free.argtypes = [P, i64]
+        lib.pkv_bm_num_free.argtypes = [P]
+        lib.pkv_bm_seq_len.argtypes = [P, i64]
+        lib.pkv_bm_ref_count.argtypes = [P, i32]
+        lib.pkv_bm_step.argtypes = [P, P, i32, P, P, P, P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+        lib.pkv_bm_tables.argtypes = [P, P, i32, P, P]
+        for n in ("pkv_bm_add", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_num_free", "pkv_bm_seq_len",
+                  "pkv_bm_ref_count", "pkv_bm_step", "pkv_bm_tables"):
+            getattr(lib, n).restype = i32
+        _bound = True
+    return lib
+
+
+class BlockManager:
+    """Pool of `num_blocks` blocks of `block_size` tokens; tables `max_blocks_per_seq` wide.
+
+    Status-returning calls return the C status (0 = ok, NO_BLOCKS, UNKNOWN_SEQ, ...)."""
+
+    def __init__(self, num_blocks: int, block_size: int, max_blocks_per_seq: int):
+        self._lib = _lib()
+        self.block_size = block_size
+        self.max_blocks = max_blocks_per_seq
+        self._h = self._lib.pkv_bm_create(num_blocks, block_size, max_blocks_per_seq)
+        if not self._h:
+            raise PkvError("pkv_bm_create", 2)
+
+    def close(self):
+        if self._h:
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add(self, seq_id: int, prompt_len: int) -> int:
+        return self._lib.pkv_bm_add(self._h, seq_id, prompt_len)
+
+    def fork(self, parent: int, child: int) -> int:
+        return self._lib.pkv_bm_fork(self._h, parent, child)
+
+    def append(self, seq_id: int):
+        """(status, slot, cow_src, cow_dst)"""
+        slot, src, dst = ctypes.c_int64(-1), ctypes.c_int32(-1), ctypes.c_int32(-1)
+        st = self._lib.pkv_bm_append(self._h, seq_id, ctypes.byref(slot), ctypes.byref(src), ctypes.byref(dst))
+        return st, slot.value, src.value, dst.value
+
+    def free(self, seq_id: int) -> int:
+        return self._lib.pkv_bm_free(self._h, seq_id)
+
+    def num_free(self) -> int:
+        return self._lib.pkv_bm_num_free(self._h)
+
+    def seq_len(self, seq_id: int) -> int:
+        return self._lib.pkv_bm_seq_len(self._h, seq_id)
+
+    def ref_count(self, block: int) -> int:
+        return self._lib.pkv_bm_ref_count(self._h, block)
+
+    def step(self, seq_ids):
+        """Append one token to each sequence; returns
+        (status, slot_mapping int64[n], block_tables int32[n, max_blocks], seq_lens int32[n],
+        cow_pairs int32[k, 2], n_done)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.full(n, -1, dtype=np.int64)
+        tables = np.full((n, self.max_blocks), -1, dtype=np.int32)
+        lens = np.zeros(n, dtype=np.int32)
+        cows = np.full((max(n, 1), 2), -1, dtype=np.int32)
+        n_cow, n_done = ctypes.c_int(0), ctypes.c_int(0)
+        st = self._lib.pkv_bm_step(self._h, ids.ctypes.data, n, slots.ctypes.data, tables.ctypes.data,
+                                   lens.ctypes.data, cows.ctypes.data, ctypes.byref(n_cow), ctypes.byref(n_done))
+        return st, slots, tables, lens, cows[:n_cow.value].copy(), n_done.value
+
+    def tables(self, seq_ids):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = np.full((ids.size, self.max_blocks), -1, dtype=np.int32)
+        lens = np.zeros(ids.size, dtype=np.int32)
+        st = self._lib.pkv_bm_tables(self._h, ids.ctypes.data, ids.size, tables.ctypes.data, lens.ctypes.data)
+        return st, tables, lens

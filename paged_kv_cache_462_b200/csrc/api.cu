@@ -11,6 +11,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "pkv_blocks.h"
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -144,6 +145,14 @@ const char* pkv_status_string(int status)
         return "kernel launch failed";
     case PKV_ERR_DEVICE:
         return "CUDA device query failed";
+    case PKV_BM_NO_BLOCKS:
+        return "block pool has no free block";
+    case PKV_BM_UNKNOWN_SEQ:
+        return "unknown sequence id";
+    case PKV_BM_DUPLICATE_SEQ:
+        return "sequence id already present";
+    case PKV_BM_TABLE_FULL:
+        return "sequence would exceed max_blocks_per_seq";
     default:
         return "unknown status";
     }

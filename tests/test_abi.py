@@ -9,13 +9,16 @@ import pytest
 import paged_kv_cache_462_b200 as pkv
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "pkv.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+    names = set()
+    for h in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -27,7 +30,8 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_functions()
-    assert set(names) >= {"paged_attention_decode", "reshape_and_cache", "paged_attention_workspace_size"}
+    assert set(names) >= {"paged_attention_decode", "reshape_and_cache", "paged_attention_workspace_size",
+                          "paged_decode_step", "pkv_bm_create", "pkv_bm_step"}
     for n in names:
         assert hasattr(lib, n), n
 
