@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
-DT = {"f32": 0, "bf16": 1, "e4m3": 2}
-NP_DT = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8}
+DT = {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3}
+NP_DT = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8, "e5m2": np.uint8}
 
 _lib = None
 
@@ -45,6 +45,10 @@ def _bind(lib):
     lib.orc_e4m3_encode.restype = ctypes.c_uint8
     lib.orc_e4m3_encode_array.argtypes = [P, P, i64]
     lib.orc_e4m3_encode_array.restype = None
+    lib.orc_e5m2_value.argtypes = [ctypes.c_uint8]
+    lib.orc_e5m2_value.restype = f64
+    lib.orc_e5m2_encode_array.argtypes = [P, P, i64]
+    lib.orc_e5m2_encode_array.restype = None
     lib.orc_paged_decode.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
                                      f64, f64, f64, P, i32]
     lib.orc_paged_decode.restype = i32
@@ -80,6 +84,18 @@ def e4m3_encode(x, lib=None) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
     out = np.empty(x.size, dtype=np.uint8)
     lib.orc_e4m3_encode_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def e5m2_value(code: int, lib=None) -> float:
+    return (lib or load()).orc_e5m2_value(int(code))
+
+
+def e5m2_encode(x, lib=None) -> np.ndarray:
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1)
+    out = np.empty(x.size, dtype=np.uint8)
+    lib.orc_e5m2_encode_array(_ptr(x), _ptr(out), x.size)
     return out
 
 

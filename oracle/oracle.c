@@ -34,6 +34,12 @@
  *               division in IEEE binary32 and the encode rounding to nearest,
  *               ties to even, saturating to +-448; dequantised value =
  *               decode(code) * scale.
+ *               E5M2 (the other OCP 8-bit format; the wzjinhao.cn write-up,
+ *               section 2.4, reports its accuracy drift as a KV format):
+ *               bias 15, 2-bit mantissa, S.11111.00 = infinity, S.11111.xx
+ *               (xx != 0) = NaN, largest finite 57344; the same encode rule
+ *               (round to nearest even, magnitudes at or above 57344 saturate
+ *               to it, NaN stays NaN).
  *
  * Layouts (a reading: the pages give none):
  *   cache     [num_blocks][num_kv_heads][block_size][head_dim]
@@ -128,6 +134,74 @@ void orc_e4m3_encode_array(const float* x, uint8_t* codes, int64_t n)
         codes[i] = orc_e4m3_encode(x[i]);
 }
 
+/* OCP E5M2: sign, 5-bit exponent with bias 15, 2-bit mantissa; exponent 0
+ * holds the subnormals m/4 * 2^-14; exponent 31 is infinity (m = 0) or NaN. */
+double orc_e5m2_value(uint8_t code)
+{
+    int s = code >> 7;
+    int e = (code >> 2) & 0x1F;
+    int m = code & 0x3;
+    double v;
+    if (e == 0x1F)
+        v = m == 0 ? INFINITY : NAN;
+    else if (e == 0)
+        v = ldexp((double)m / 4.0, -14);
+    else
+        v = ldexp(1.0 + (double)m / 4.0, e - 15);
+    return s ? -v : v;
+}
+
+/* The 124 non-negative finite E5M2 values in increasing order (code 0..0x7B). */
+static double e5m2_pos[124];
+static int e5m2_ready = 0;
+
+static void e5m2_init(void)
+{
+    if (e5m2_ready)
+        return;
+    for (int c = 0; c < 124; ++c)
+        e5m2_pos[c] = orc_e5m2_value((uint8_t)c);
+    e5m2_ready = 1;
+}
+
+/* Same rule as the E4M3 encoder over the E5M2 value set. */
+uint8_t orc_e5m2_encode(float x)
+{
+    e5m2_init();
+    if (isnan(x))
+        return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= e5m2_pos[123])
+        return sign | 123;
+    int lo = 0, hi = 123;
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (e5m2_pos[mid] <= a)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    double vlo = e5m2_pos[lo], vhi = e5m2_pos[hi];
+    double midpoint = 0.5 * (vlo + vhi);
+    int code;
+    if (a < midpoint)
+        code = lo;
+    else if (a > midpoint)
+        code = hi;
+    else
+        code = (lo & 1) ? hi : lo;
+    return sign | (uint8_t)code;
+}
+
+void orc_e5m2_encode_array(const float* x, uint8_t* codes, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        codes[i] = orc_e5m2_encode(x[i]);
+}
+
+static int is_fp8(int dtype) { return dtype == ORC_E4M3 || dtype == ORC_E5M2; }
+
 static double elem(const void* base, int dtype, size_t i, double scale)
 {
     switch (dtype) {
@@ -137,6 +211,8 @@ static double elem(const void* base, int dtype, size_t i, double scale)
         return bf16_value(((const uint16_t*)base)[i]);
     case ORC_E4M3:
         return orc_e4m3_value(((const uint8_t*)base)[i]) * scale;
+    case ORC_E5M2:
+        return orc_e5m2_value(((const uint8_t*)base)[i]) * scale;
     default:
         return NAN;
     }
@@ -160,7 +236,7 @@ int orc_paged_decode(double* out,
 {
     if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
         return ORC_ERR_SHAPE;
-    if (q_dtype == ORC_E4M3 || q_dtype < 0 || q_dtype > 2 || kv_dtype < 0 || kv_dtype > 2)
+    if (is_fp8(q_dtype) || q_dtype < 0 || q_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
         return ORC_ERR_DTYPE;
     const int group = num_heads / num_kv_heads;
     const int count = seqs ? n_seqs : num_seqs;
@@ -242,9 +318,9 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                           int num_tokens, int num_kv_heads, int head_dim,
                           int block_size, int num_blocks, float k_scale, float v_scale)
 {
-    if (in_dtype == ORC_E4M3 || in_dtype < 0 || in_dtype > 2 || kv_dtype < 0 || kv_dtype > 2)
+    if (is_fp8(in_dtype) || in_dtype < 0 || in_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
         return ORC_ERR_DTYPE;
-    if (kv_dtype != ORC_E4M3 && kv_dtype != in_dtype)
+    if (!is_fp8(kv_dtype) && kv_dtype != in_dtype)
         return ORC_ERR_DTYPE;
     const size_t isz = dtype_size(in_dtype), csz = dtype_size(kv_dtype);
     const int64_t capacity = (int64_t)num_blocks * block_size;
@@ -275,8 +351,8 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                 const float vx = (float)elem(v, in_dtype, src + i, 1.0);
                 const float ky = kx / k_scale; /* binary32 division */
                 const float vy = vx / v_scale;
-                ((uint8_t*)k_cache)[dst + i] = orc_e4m3_encode(ky);
-                ((uint8_t*)v_cache)[dst + i] = orc_e4m3_encode(vy);
+                ((uint8_t*)k_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(ky) : orc_e5m2_encode(ky);
+                ((uint8_t*)v_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(vy) : orc_e5m2_encode(vy);
             }
         }
     }

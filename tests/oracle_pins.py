@@ -328,10 +328,106 @@ def check_fp8_attention_dequant(lib):
         assert np.allclose(got[s], ref, rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------ E5M2 format
+
+def e5m2_library_values():
+    """All 256 E5M2 codes decoded by torch's float8_e5m2 (an independent implementation)."""
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).to(torch.float64).numpy()
+
+
+def check_e5m2_decode_table(lib):
+    ref = e5m2_library_values()
+    got = np.array([oracle.e5m2_value(c, lib) for c in range(256)])
+    nan_ref, nan_got = np.isnan(ref), np.isnan(got)
+    assert np.array_equal(nan_ref, nan_got)
+    assert np.array_equal(ref[~nan_ref], got[~nan_got])
+    assert np.array_equal(np.signbit(ref[~nan_ref]), np.signbit(got[~nan_got]))
+
+
+def check_e5m2_spot_values(lib):
+    # OCP 8-bit floating point spec: bias 15, subnormal step 2^-16, max 57344, S.11111.00 inf
+    expect = {0x00: 0.0, 0x01: 2.0 ** -16, 0x03: 3 * 2.0 ** -16, 0x04: 2.0 ** -14, 0x3C: 1.0,
+              0x3E: 1.5, 0x7B: 57344.0, 0xFB: -57344.0, 0x7C: np.inf, 0xFC: -np.inf, 0xBC: -1.0}
+    for c, v in expect.items():
+        assert oracle.e5m2_value(c, lib) == v, hex(c)
+    for c in (0x7D, 0x7E, 0x7F, 0xFD, 0xFE, 0xFF):
+        assert math.isnan(oracle.e5m2_value(c, lib))
+
+
+def check_e5m2_encode_vs_library(lib, n=200_000, seed=8):
+    rng = np.random.default_rng(seed)
+    mag = np.exp2(rng.uniform(-20.0, np.log2(57343.0), size=n)).astype(np.float32)
+    x = np.where(rng.random(n) < 0.5, -mag, mag).astype(np.float32)
+    x = np.concatenate([x, rng.standard_normal(n).astype(np.float32) * 100]).astype(np.float32)
+    x = x[np.abs(x) < 57344]
+    ref = torch.from_numpy(x).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    got = oracle.e5m2_encode(x, lib)
+    bad = np.nonzero(ref != got)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, e.g. x={x[bad[:3]]} ref={ref[bad[:3]]} got={got[bad[:3]]}"
+
+
+def check_e5m2_ties_saturation_roundtrip(lib):
+    finite = [oracle.e5m2_value(c, lib) for c in range(124)]
+    for c in range(123):
+        lo, hi = finite[c], finite[c + 1]
+        mid = np.float32((lo + hi) / 2)
+        assert float(mid) == (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        got = oracle.e5m2_encode([mid, np.nextafter(mid, np.float32(np.inf)), np.nextafter(mid, np.float32(0)),
+                                  -mid], lib)
+        assert got[0] == even and got[1] == c + 1 and got[2] == c and got[3] == (0x80 | even), (c, got)
+    big = np.array([57344.0, 60000.0, 61440.0, 1e9, np.inf], dtype=np.float32)
+    assert np.all(oracle.e5m2_encode(big, lib) == 0x7B) and np.all(oracle.e5m2_encode(-big, lib) == 0xFB)
+    assert oracle.e5m2_encode([np.nan], lib)[0] == 0x7F
+    codes = [c for c in range(256) if np.isfinite(oracle.e5m2_value(c, lib))]
+    vals = np.array([oracle.e5m2_value(c, lib) for c in codes], dtype=np.float32)
+    assert np.array_equal(oracle.e5m2_encode(vals, lib), np.array(codes, dtype=np.uint8))
+
+
+def check_append_e5m2_vs_library(lib):
+    rng = np.random.default_rng(22)
+    T, Hkv, d, bs, nb = 40, 2, 32, 8, 8
+    k = rng.standard_normal((T, Hkv, d)).astype(np.float32) * 3
+    v = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    ks = np.float32(np.abs(k).max() / np.float32(57344)); vs = np.float32(np.abs(v).max() / np.float32(57344))
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    kc = oracle.empty_cache(nb, Hkv, bs, d, "e5m2"); vc = oracle.empty_cache(nb, Hkv, bs, d, "e5m2")
+    oracle.reshape_and_cache(k, v, "f32", kc, vc, "e5m2", slots, Hkv, d, bs, nb, ks, vs, lib=lib)
+    for t in range(T):
+        b, o = divmod(int(slots[t]), bs)
+        ek = torch.from_numpy((k[t] / ks).astype(np.float32)).to(torch.float8_e5m2).view(torch.uint8).numpy()
+        ev = torch.from_numpy((v[t] / vs).astype(np.float32)).to(torch.float8_e5m2).view(torch.uint8).numpy()
+        assert np.array_equal(kc[b, :, o, :], ek) and np.array_equal(vc[b, :, o, :], ev)
+
+
+def check_e5m2_attention_dequant(lib):
+    """Attention over an E5M2 cache equals attention over the library-decoded values times the scale."""
+    rng = np.random.default_rng(23)
+    nb, Hkv, bs, d, Hq = 6, 2, 8, 16, 4
+    kc = rng.integers(0, 256, (nb, Hkv, bs, d), dtype=np.uint8)
+    vc = rng.integers(0, 256, (nb, Hkv, bs, d), dtype=np.uint8)
+    kc[(kc & 0x7C) == 0x7C] = 0x31; vc[(vc & 0x7C) == 0x7C] = 0x2A     # no inf / NaN codes
+    ks, vs = np.float32(2.0 ** -12), np.float32(2.0 ** -14)
+    lut = e5m2_library_values()
+    kf = (lut[kc] * float(ks)); vf = (lut[vc] * float(vs))
+    q = rng.standard_normal((2, Hq, d)).astype(np.float32)
+    bt = np.array([[3, 1, 4], [0, 5, -1]], np.int32)
+    sl = np.array([20, 11], np.int32)
+    got = oracle.paged_decode(q, "f32", kc, vc, "e5m2", bt, sl, Hq, Hkv, d, bs, nb, 0.25, ks, vs, lib=lib)
+    for s in range(2):
+        L = int(sl[s])
+        K = np.concatenate([np.transpose(kf[bt[s, j]], (1, 0, 2)) for j in range(-(-L // bs))])[:L]
+        V = np.concatenate([np.transpose(vf[bt[s, j]], (1, 0, 2)) for j in range(-(-L // bs))])[:L]
+        ref = sdpa_fp64(q[s], K, V, 0.25)
+        assert np.allclose(got[s], ref, rtol=0, atol=1e-12)
+
+
 ALL_CHECKS = [
     check_e4m3_decode_table, check_e4m3_spot_values, check_e4m3_encode_vs_library, check_e4m3_ties_to_even,
     check_e4m3_saturation_and_roundtrip, check_length_one_is_v, check_length_two_closed_form,
     check_equal_keys_give_mean, check_large_scores_pick_argmax, check_matches_library_sdpa, check_gqa_grouping,
     check_permutation_invariance, check_block_size_invariance, check_worked_block_table, check_zero_length,
     check_append_golden, check_append_fp8_vs_library, check_fp8_attention_dequant,
+    check_e5m2_decode_table, check_e5m2_spot_values, check_e5m2_encode_vs_library,
+    check_e5m2_ties_saturation_roundtrip, check_append_e5m2_vs_library, check_e5m2_attention_dequant,
 ]

@@ -22,8 +22,27 @@ MUTANTS = {
     "last_token_dropped": ("const int L = seq_lens[s];", "const int L = seq_lens[s] > 1 ? seq_lens[s] - 1 : seq_lens[s];"),
     "no_normalisation": ("o[i] /= denom;", "o[i] /= 1.0;"),
     "no_max_subtraction": ("const double w = exp(x[t] - m);", "const double w = exp(x[t]);"),
-    "e4m3_sign_dropped": ("return s ? -v : v;", "return v;"),
-    "e4m3_ties_to_odd": ("code = (lo & 1) ? hi : lo;", "code = (lo & 1) ? lo : hi;"),
+    "e4m3_sign_dropped": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);\n    return s ? -v : v;",
+                          "v = ldexp(1.0 + (double)m / 8.0, e - 7);\n    return v;"),
+    "e4m3_ties_to_odd": ("double vlo = e4m3_pos[lo], vhi = e4m3_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi); "
+                         "/* exact: both are short binary fractions */\n    int code;\n    if (a < midpoint)\n"
+                         "        code = lo;\n    else if (a > midpoint)\n        code = hi;\n    else\n"
+                         "        code = (lo & 1) ? hi : lo;",
+                         "double vlo = e4m3_pos[lo], vhi = e4m3_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi); "
+                         "/* exact: both are short binary fractions */\n    int code;\n    if (a < midpoint)\n"
+                         "        code = lo;\n    else if (a > midpoint)\n        code = hi;\n    else\n"
+                         "        code = (lo & 1) ? lo : hi;"),
+    "e5m2_sign_dropped": ("v = ldexp(1.0 + (double)m / 4.0, e - 15);\n    return s ? -v : v;",
+                          "v = ldexp(1.0 + (double)m / 4.0, e - 15);\n    return v;"),
+    "e5m2_bias_off_by_one": ("v = ldexp(1.0 + (double)m / 4.0, e - 15);", "v = ldexp(1.0 + (double)m / 4.0, e - 14);"),
+    "e5m2_ties_to_odd": ("double vlo = e5m2_pos[lo], vhi = e5m2_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi);\n"
+                         "    int code;\n    if (a < midpoint)\n        code = lo;\n    else if (a > midpoint)\n"
+                         "        code = hi;\n    else\n        code = (lo & 1) ? hi : lo;",
+                         "double vlo = e5m2_pos[lo], vhi = e5m2_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi);\n"
+                         "    int code;\n    if (a < midpoint)\n        code = lo;\n    else if (a > midpoint)\n"
+                         "        code = hi;\n    else\n        code = (lo & 1) ? lo : hi;"),
+    "e5m2_saturates_to_infinity": ("if (a >= e5m2_pos[123])\n        return sign | 123;",
+                                   "if (a >= e5m2_pos[123])\n        return sign | 124;"),
     "e4m3_bias_off_by_one": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "fp8_scale_multiplied": ("const float ky = kx / k_scale;", "const float ky = kx * k_scale;"),
     "append_offset_wrong": ("const int64_t blk = slot / block_size, off = slot % block_size;",
