@@ -80,7 +80,10 @@ typedef enum {
     PKV_ERR_DEVICE = 6       /* device query failed (no device, bad context) */
 } pkv_status;
 
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
+/* PKV_FP8_E5M2: OCP E5M2 codes (bias 15, largest finite 57344), per-tensor
+ * scales like E4M3; decoded by the tensor-core kernel only (bf16 q, head_dim
+ * 128, block 16 or 32); other shapes return PKV_ERR_SHAPE / PKV_ERR_DTYPE. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3 } pkv_dtype;
 
 /* Bits of the device error word. */
 #define PKV_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks): block skipped */
@@ -207,7 +210,8 @@ PKV_API int paged_attention_decode_static(void* out, const void* q, const void* 
  * k[t][h][:] to k_cache[slot / block_size][h][slot % block_size][:] (and v the
  * same way) for every kv head h. Same dtype: a bit copy. FP8_E4M3 cache from
  * F32 or BF16 rows: code = E4M3(x / k_scale) with an IEEE fp32 division and
- * round-to-nearest-even, saturating to +-448 (v with v_scale).
+ * round-to-nearest-even, saturating to +-448 (v with v_scale); FP8_E5M2 the
+ * same with E5M2 codes, saturating to +-57344.
  * Duplicate non-negative slots in one call give an unspecified winner.
  * device_error: optional int32 device word that receives PKV_DEVERR_SLOT.
  */

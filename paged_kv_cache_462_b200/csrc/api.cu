@@ -66,6 +66,8 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool is_fp8(int dtype) { return dtype == PKV_FP8_E4M3 || dtype == PKV_FP8_E5M2; }
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -258,7 +260,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
         (block_size != 8 && block_size != 16 && block_size != 32))
         return PKV_ERR_SHAPE;
     if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
-          (q_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3)))
+          (q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2))))
         return PKV_ERR_DTYPE;
     if (num_seqs == 0)
         return PKV_OK;
@@ -297,7 +299,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     if (workspace_bytes < lay.bytes)
         return PKV_ERR_WORKSPACE;
 
-    const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+    const bool fp8 = kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2;
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
     p.out = out;
@@ -371,7 +373,7 @@ int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, co
 {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
         return PKV_ERR_SHAPE;
-    if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) && (kv_dtype == in_dtype || kv_dtype == PKV_FP8_E4M3)))
+    if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) && (kv_dtype == in_dtype || is_fp8(kv_dtype))))
         return PKV_ERR_DTYPE;
     if (num_seqs == 0)
         return PKV_OK;
@@ -381,7 +383,7 @@ int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, co
         return PKV_ERR_WORKSPACE;
     if (!aligned16(new_k) || !aligned16(new_v))
         return PKV_ERR_SHAPE;
-    if (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.0f && v_scale > 0.0f))
+    if (is_fp8(kv_dtype) && !(k_scale > 0.0f && v_scale > 0.0f))
         return PKV_ERR_SHAPE;
     const int group = num_heads / num_kv_heads;
     if (q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)) {
@@ -409,7 +411,7 @@ int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache
         (block_size != 8 && block_size != 16 && block_size != 32))
         return PKV_ERR_SHAPE;
     if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) &&
-          (kv_dtype == in_dtype || kv_dtype == PKV_FP8_E4M3)))
+          (kv_dtype == in_dtype || is_fp8(kv_dtype))))
         return PKV_ERR_DTYPE;
     if (num_tokens == 0)
         return PKV_OK;
@@ -417,7 +419,7 @@ int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache
         return PKV_ERR_NULL;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
         return PKV_ERR_SHAPE;
-    if (kv_dtype == PKV_FP8_E4M3 && !(k_scale > 0.0f && v_scale > 0.0f))
+    if (is_fp8(kv_dtype) && !(k_scale > 0.0f && v_scale > 0.0f))
         return PKV_ERR_SHAPE;
     return cache_dispatch(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
                           num_blocks, in_dtype, kv_dtype, k_scale, v_scale, device_error,

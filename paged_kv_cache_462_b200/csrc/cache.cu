@@ -21,8 +21,8 @@ namespace pkv {
 
 namespace {
 
-// TIN: float or bf16 input rows; TC: cache element (same as TIN, or uint8_t E4M3 codes).
-template <class TIN, class TC>
+// TIN: float or bf16 input rows; TC: cache element (same as TIN, or uint8_t FP8 codes of format FMT).
+template <class TIN, class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const TIN* __restrict__ k, const TIN* __restrict__ v, TC* __restrict__ kc, TC* __restrict__ vc,
     const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads, int head_dim, int block_size,
@@ -50,13 +50,13 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
         const TIN* src = (is_v ? v : k) + ((long long)t * num_kv_heads + h) * head_dim + c * 8;
         TC* dst = (is_v ? vc : kc) + ((blk * num_kv_heads + h) * block_size + off) * head_dim + c * 8;
         if constexpr (sizeof(TC) == 1)
-            quant8(src, reinterpret_cast<uint8_t*>(dst), is_v ? v_scale : k_scale);
+            quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? v_scale : k_scale);
         else
             copy8(src, dst);
     }
 }
 
-template <class TIN, class TC>
+template <class TIN, class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
 int launch_cache(const void* k, const void* v, void* kc, void* vc, const int64_t* slots, int num_tokens,
                  int num_kv_heads, int head_dim, int block_size, int num_blocks, float k_scale, float v_scale,
                  int32_t* err, cudaStream_t stream)
@@ -67,7 +67,7 @@ int launch_cache(const void* k, const void* v, void* kc, void* vc, const int64_t
         blocks = 148ll * 16;
     if (blocks < 1)
         blocks = 1;
-    reshape_and_cache_kernel<TIN, TC><<<(unsigned)blocks, 256, 0, stream>>>(
+    reshape_and_cache_kernel<TIN, TC, FMT><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const TIN*>(k), static_cast<const TIN*>(v), static_cast<TC*>(kc), static_cast<TC*>(vc), slots,
         num_tokens, num_kv_heads, head_dim, block_size, (long long)num_blocks * block_size, k_scale, v_scale, err);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
@@ -92,6 +92,14 @@ int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, c
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3)
         return launch_cache<__nv_bfloat16, uint8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
                                                     head_dim, block_size, num_blocks, k_scale, v_scale, err, stream);
+    if (in_dtype == PKV_F32 && kv_dtype == PKV_FP8_E5M2)
+        return launch_cache<float, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                                       num_kv_heads, head_dim, block_size, num_blocks, k_scale,
+                                                       v_scale, err, stream);
+    if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E5M2)
+        return launch_cache<__nv_bfloat16, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                                               num_kv_heads, head_dim, block_size, num_blocks,
+                                                               k_scale, v_scale, err, stream);
     return PKV_ERR_DTYPE;
 }
 

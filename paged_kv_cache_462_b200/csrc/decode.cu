@@ -1,6 +1,7 @@
 // Dispatch of paged_attention_decode: the warp-MMA kernel (decode_mma.cuh) for
-// bf16 / E4M3 caches of the shapes it covers, the CUDA-core kernel
-// (decode_kernel.cuh) for fp32 caches and every other supported shape.
+// bf16 / E4M3 / E5M2 caches of the shapes it covers, the CUDA-core kernel
+// (decode_kernel.cuh) for fp32 caches and the other bf16 / E4M3 shapes (E5M2
+// has no CUDA-core form).
 #include "decode_kernel.cuh"
 
 namespace pkv {
@@ -12,6 +13,8 @@ int decode_mma_dispatch_bf16(int D, int BS, int G, int HG, const DecodeParams& p
                              int* occ);
 int decode_mma_dispatch_e4m3(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
                              int* occ);
+int decode_mma_dispatch_e5m2(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
+                             int* occ);
 
 int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
                         cudaStream_t st, int* occ)
@@ -20,12 +23,14 @@ int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const Decode
         return decode_mma_dispatch_bf16(D, BS, G, HG, p, nruns, st, occ);
     if (kv_dtype == PKV_FP8_E4M3)
         return decode_mma_dispatch_e4m3(D, BS, G, HG, p, nruns, st, occ);
+    if (kv_dtype == PKV_FP8_E5M2)
+        return decode_mma_dispatch_e5m2(D, BS, G, HG, p, nruns, st, occ);
     return PKV_ERR_DTYPE;
 }
 
 bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)
 {
-    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3)
+    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3 && kv_dtype != PKV_FP8_E5M2)
         return false;
     if (block_size != 16 && block_size != 32)
         return false;

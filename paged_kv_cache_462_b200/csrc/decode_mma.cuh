@@ -85,12 +85,16 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
     }
 }
 
-// two E4M3 codes (low byte first) -> f16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes)
+// two FP8 codes (low byte first) -> f16x2, exact for both formats
+template <class KV>
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two_codes)
 {
     uint32_t r;
     const uint16_t v = static_cast<uint16_t>(two_codes);
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    if constexpr (KV::kFmt == __NV_E5M2)
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(r) : "h"(v));
+    else
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
     return r;
 }
 
@@ -123,7 +127,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
 // Decode-step append fused into the producer warp: write the new token of sequence s (row s of
 // new_k / new_v) for KV heads h0 .. h0+nh-1 into its slot, with the conversion reshape_and_cache
 // uses, then order those writes before this warp's later TMA reads of the same block.
-template <class TC>
+template <class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
 __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0, int nh, int D, int BS, int lane,
                                             long long slot)
 {
@@ -140,11 +144,11 @@ __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0
         if (p.in_dtype == PKV_F32) {
             const float* src = static_cast<const float*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
         } else {
             const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
             else
                 copy8(src, reinterpret_cast<__nv_bfloat16*>(dst));
         }
@@ -158,7 +162,7 @@ __device__ __forceinline__ void fence_proxy_async_global()
 
 // `last_phys`: physical block the sequence's last position maps to (-1 when its id was bad);
 // a slot outside it is still written but flagged, since the decode may not see it
-template <int KVBYTES>
+template <class KV>
 __device__ __forceinline__ void append_new_token_impl(const DecodeParams& p, int s, int h0, int nh, int D, int BS,
                                                       int lane, int last_phys)
 {
@@ -169,8 +173,8 @@ __device__ __forceinline__ void append_new_token_impl(const DecodeParams& p, int
         if (slot >= (long long)p.num_blocks * BS) {
             if (lane == 0)
                 atomicOr(p.err, PKV_DEVERR_SLOT);
-        } else if constexpr (KVBYTES == 1) {
-            append_rows<uint8_t>(p, s, h0, nh, D, BS, lane, slot);
+        } else if constexpr (KV::kBytes == 1) {
+            append_rows<uint8_t, KV::kFmt>(p, s, h0, nh, D, BS, lane, slot);
         } else {
             append_rows<__nv_bfloat16>(p, s, h0, nh, D, BS, lane, slot);
         }
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                 const int row = __shfl_sync(kFullMask, cur, i);
                 const int app = __shfl_sync(kFullMask, cur_app, i);
                 if (app >= 0)   // the decode-step append of this stream, before its last block is read
-                    append_new_token_impl<KV::kBytes>(p, app / NHG, (app % NHG) * HG, HG, D, BS, lane,
+                    append_new_token_impl<KV>(p, app / NHG, (app % NHG) * HG, HG, D, BS, lane,
                                                       row < 0 ? -1 : row / (Hkv * BS));
                 if (lane == 0 && !aborted) {
                     const int k = k0 + i;
@@ -472,8 +476,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
                                 const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
-                                const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi),
-                                                       e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi >> 16)};
+                                const uint32_t a[4] = {fp8x2_to_f16x2<KV>(lo), fp8x2_to_f16x2<KV>(hi),
+                                                       fp8x2_to_f16x2<KV>(lo >> 16), fp8x2_to_f16x2<KV>(hi >> 16)};
                                 mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
                             }
                         }
@@ -585,10 +589,10 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                                     hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
                                 }
                                 // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1)
-                                const uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0020)),
-                                                       e4m3x2_to_f16x2(__byte_perm(lo, 0u, 0x0031)),
-                                                       e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0020)),
-                                                       e4m3x2_to_f16x2(__byte_perm(hi, 0u, 0x0031))};
+                                const uint32_t a[4] = {fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0020)),
+                                                       fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0031)),
+                                                       fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0020)),
+                                                       fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0031))};
                                 mma_16816<true>(o[dt + h2], a, pb0, pb1);
                             }
                         }
@@ -880,7 +884,9 @@ struct MmaLauncher {
         if (S < 2)
             return PKV_ERR_SHAPE;
         const long long rows = (long long)p.num_blocks * p.num_kv_heads * BS;
-        const int kvdt = KV::kBytes == 1 ? PKV_FP8_E4M3 : PKV_BF16;
+        int kvdt = PKV_BF16;
+        if constexpr (KV::kBytes == 1)
+            kvdt = KV::kFmt == __NV_E5M2 ? PKV_FP8_E5M2 : PKV_FP8_E4M3;
         CUtensorMap kmap, vmap;
         if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, D, rows, C::kRows) ||
             !make_cache_tensormap(&vmap, p.v_cache, kvdt, D, rows, C::kRows))

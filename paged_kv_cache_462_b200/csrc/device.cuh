@@ -148,6 +148,13 @@ struct KvE4M3 {
     using T = uint8_t;
     static constexpr int kBytes = 1;
     static constexpr float kUnbias = kE4M3Unbias;
+    static constexpr __nv_fp8_interpretation_t kFmt = __NV_E4M3;
+};
+// OCP E5M2 codes (tensor-core kernel only: widened exactly to f16 there)
+struct KvE5M2 {
+    using T = uint8_t;
+    static constexpr int kBytes = 1;
+    static constexpr __nv_fp8_interpretation_t kFmt = __NV_E5M2;
 };
 
 __device__ __forceinline__ void widen_word(KvF32, uint32_t w, float* f) { f[0] = __uint_as_float(w); }
@@ -294,7 +301,9 @@ __device__ __forceinline__ void copy8(const T* src, T* dst)
     }
 }
 
-template <class TIN>
+// 8 values -> 8 codes of format FMT: x / scale (IEEE fp32 division), round to nearest even,
+// saturated to the largest finite value
+template <__nv_fp8_interpretation_t FMT = __NV_E4M3, class TIN>
 __device__ __forceinline__ void quant8(const TIN* src, uint8_t* dst, float scale)
 {
     float f[8];
@@ -306,7 +315,7 @@ __device__ __forceinline__ void quant8(const TIN* src, uint8_t* dst, float scale
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const float2 y = make_float2(__fdiv_rn(f[4 * h + 2 * i], scale), __fdiv_rn(f[4 * h + 2 * i + 1], scale));
-            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, FMT);
             packed |= static_cast<uint32_t>(c) << (16 * i);
         }
         w[h] = packed;

@@ -7,8 +7,8 @@ import torch
 import oracle
 import paged_kv_cache_462_b200 as pkv
 
-TOL = {"f32": 1e-5, "bf16": 1e-2, "e4m3": 3e-2}   # max |gpu - oracle| per cache dtype
-TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}
+TOL = {"f32": 1e-5, "bf16": 1e-2, "e4m3": 3e-2, "e5m2": 3e-2}   # max |gpu - oracle| per cache dtype
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8, "e5m2": torch.float8_e5m2}
 
 
 def to_dev(a: np.ndarray, name: str, device="cuda") -> torch.Tensor:
@@ -16,6 +16,8 @@ def to_dev(a: np.ndarray, name: str, device="cuda") -> torch.Tensor:
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
     if name == "f32":
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    if name == "e5m2":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).to(device).view(torch.float8_e5m2)
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).to(device)
 
 
@@ -28,6 +30,8 @@ def cache_bytes(t: torch.Tensor) -> np.ndarray:
     c = t.detach().cpu()
     if c.dtype == torch.bfloat16:
         return c.view(torch.int16).numpy().view(np.uint16)
+    if c.dtype in (torch.float8_e5m2, torch.float8_e4m3fn):
+        return c.view(torch.uint8).numpy()
     return c.numpy()
 
 

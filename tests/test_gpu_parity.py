@@ -342,3 +342,82 @@ def test_guard_regions_untouched(cfg, parts):
     assert bool((wbig[wbytes:] == 0xA5).all())
     ref, _, _ = oracle.run_step(b)
     assert max_err(g.out, ref) <= TOL[sp.kv_dtype]
+
+
+# ------------------------------------------------------------------ E5M2 caches
+
+def test_append_e5m2_special_values():
+    """Saturation at 57344, ties, subnormals, signed zero through the hardware E5M2 conversion;
+    NaN inputs must give a NaN code (which NaN code is not fixed by the format)."""
+    vals = np.array([0.0, -0.0, 57344.0, 60000.0, 61440.0, 1e9, -1e9, np.inf, -np.inf, 2.0 ** -16, -(2.0 ** -17),
+                     3 * 2.0 ** -18, 1.125, 1.375, 20.0, 28.0, 12288.0, 2.0 ** -14, 1e-30, 0.3, np.nan],
+                    dtype=np.float32)
+    D = 64
+    rows = np.resize(vals, (3, 1, D)).astype(np.float32)
+    rows[1] *= -1.5
+    rows[2] = np.random.default_rng(4).standard_normal((1, D)).astype(np.float32) * 1000
+    slots = np.array([3, 17, 40], np.int64)
+    okc = oracle.empty_cache(4, 1, 16, D, "e5m2"); ovc = oracle.empty_cache(4, 1, 16, D, "e5m2")
+    oracle.reshape_and_cache(rows, rows, "f32", okc, ovc, "e5m2", slots, 1, D, 16, 4, 1.0, 0.5)
+    kc = torch.zeros(4, 1, 16, D, dtype=torch.float8_e5m2, device="cuda"); vc = torch.zeros_like(kc)
+    t = torch.from_numpy(rows).cuda()
+    pkv.reshape_and_cache(t, t.clone(), kc, vc, torch.from_numpy(slots).cuda(), 1.0, 0.5)
+    for got, ref in ((cache_bytes(kc), okc), (cache_bytes(vc), ovc)):
+        nan_ref = (ref & 0x7C) == 0x7C
+        nan_ref &= (ref & 0x03) != 0
+        nan_got = ((got & 0x7C) == 0x7C) & ((got & 0x03) != 0)
+        assert np.array_equal(nan_ref, nan_got)
+        assert np.array_equal(got[~nan_ref], ref[~nan_ref])
+
+
+@pytest.mark.parametrize("inp", ["bf16", "f32"])
+def test_append_e5m2_bit_exact(inp):
+    rng = np.random.default_rng(6)
+    T, Hkv, D, BS, NB = 300, 4, 128, 16, 40
+    rows_k = rng.standard_normal((T, Hkv, D)).astype(np.float32) * 3
+    rows_v = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+    if inp == "bf16":
+        rows_k, rows_v = W.f32_to_bf16_bits(rows_k), W.f32_to_bf16_bits(rows_v)
+    slots = rng.permutation(NB * BS)[:T].astype(np.int64)
+    slots[::7] = -1
+    ks, vs = np.float32(3 * 4.5 / 57344), np.float32(4.5 / 57344)
+    okc = oracle.empty_cache(NB, Hkv, BS, D, "e5m2"); ovc = oracle.empty_cache(NB, Hkv, BS, D, "e5m2")
+    oracle.reshape_and_cache(rows_k, rows_v, inp, okc, ovc, "e5m2", slots, Hkv, D, BS, NB, ks, vs)
+    kc = torch.zeros(okc.shape, dtype=torch.float8_e5m2, device="cuda"); vc = torch.zeros_like(kc)
+    pkv.reshape_and_cache(to_dev(rows_k, inp), to_dev(rows_v, inp), kc, vc, torch.from_numpy(slots).cuda(),
+                          float(ks), float(vs))
+    assert np.array_equal(cache_bytes(kc), okc) and np.array_equal(cache_bytes(vc), ovc)
+
+
+@pytest.mark.parametrize("BS", [16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 5, 8])
+def test_e5m2_shapes(BS, G):
+    Hkv = 2
+    lengths = [0, 1, BS, BS + 1, 3 * BS - 1, 97, 200]
+    b = W.build_batch(_spec(f"e5m2_{BS}_{G}", len(lengths), G * Hkv, Hkv, 128, BS, "e5m2", lengths,
+                            seed=5000 + BS * 10 + G))
+    g, _ = _check_step(b, partitions=(0, 5))
+    assert np.all(g.out.float().cpu().numpy()[0] == 0)
+
+
+@pytest.mark.parametrize("cfg,over", [(1, dict(num_seqs=6)), (4, dict(num_seqs=5)), (3, dict(num_seqs=16)),
+                                      (2, dict(num_seqs=2, lengths=("fixed", 2000)))])
+def test_e5m2_workloads_fused_step(cfg, over):
+    b = W.config_batch(cfg, kv_dtype="e5m2", **over)
+    ref, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    out = g.fused_step(0)
+    assert g.device_errors() == 0
+    assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
+    assert max_err(out, ref) <= TOL["e5m2"]
+
+
+def test_e5m2_uncovered_shapes_are_rejected():
+    """E5M2 is decoded by the tensor-core kernel only: head_dim 64 or block 8 is refused before any launch."""
+    for D, BS in ((64, 16), (128, 8)):
+        q = torch.zeros(2, 4, D, dtype=torch.bfloat16, device="cuda")
+        kc = torch.zeros(4, 2, BS, D, dtype=torch.float8_e5m2, device="cuda")
+        bt = torch.zeros(2, 2, dtype=torch.int32, device="cuda")
+        sl = torch.ones(2, dtype=torch.int32, device="cuda")
+        with pytest.raises(pkv.PkvError):
+            pkv.paged_attention_decode(torch.empty_like(q), q, kc, kc.clone(), bt, sl, 0.1, 1.0, 1.0)
