@@ -50,7 +50,7 @@ def _bind(lib):
     lib.orc_e5m2_encode_array.argtypes = [P, P, i64]
     lib.orc_e5m2_encode_array.restype = None
     lib.orc_paged_decode.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
-                                     f64, f64, f64, P, i32]
+                                     f64, f64, f64, P, i32, i32]
     lib.orc_paged_decode.restype = i32
     lib.orc_reshape_and_cache.argtypes = [P, P, i32, P, P, i32, P, P, i64, i32, i32, i32, i32, i32, f32, f32]
     lib.orc_reshape_and_cache.restype = i32
@@ -101,8 +101,10 @@ def e5m2_encode(x, lib=None) -> np.ndarray:
 
 def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
                  num_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                 scale, k_scale=1.0, v_scale=1.0, seqs=None, lib=None) -> np.ndarray:
-    """fp64 attention output [len(seqs) or num_seqs, num_heads, head_dim]."""
+                 scale, k_scale=1.0, v_scale=1.0, seqs=None, lib=None, q_len=1) -> np.ndarray:
+    """fp64 attention output [len(seqs) or num_seqs, num_heads, head_dim]; with q_len > 1,
+    q is [num_seqs, q_len, num_heads, head_dim] (query j at position seq_len - q_len + j,
+    causal) and the output [rows, q_len, num_heads, head_dim]."""
     lib = lib or load()
     q = np.ascontiguousarray(q, dtype=NP_DT[q_dtype])
     k_cache = np.ascontiguousarray(k_cache, dtype=NP_DT[kv_dtype])
@@ -113,11 +115,12 @@ def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
     MB = bt.shape[1] if bt.ndim == 2 else 0
     sub = None if seqs is None else np.ascontiguousarray(seqs, dtype=np.int32)
     rows = S if sub is None else sub.size
-    out = np.zeros((rows, num_heads, head_dim), dtype=np.float64)
+    out = np.zeros((rows, num_heads, head_dim) if q_len == 1 else (rows, q_len, num_heads, head_dim),
+                   dtype=np.float64)
     st = lib.orc_paged_decode(_ptr(out), _ptr(q), DT[q_dtype], _ptr(k_cache), _ptr(v_cache), DT[kv_dtype],
                               _ptr(bt), _ptr(sl), S, num_heads, num_kv_heads, head_dim, block_size, MB,
                               num_blocks, float(scale), float(k_scale), float(v_scale),
-                              _ptr(sub), 0 if sub is None else int(sub.size))
+                              _ptr(sub), 0 if sub is None else int(sub.size), int(q_len))
     if st != 0:
         raise OracleError(f"orc_paged_decode status {st}")
     return out

@@ -232,9 +232,9 @@ int orc_paged_decode(double* out,
                      int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                      int block_size, int max_blocks_per_seq, int num_blocks,
                      double scale, double k_scale, double v_scale,
-                     const int32_t* seqs, int n_seqs)
+                     const int32_t* seqs, int n_seqs, int q_len)
 {
-    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0)
+    if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 || q_len < 1)
         return ORC_ERR_SHAPE;
     if (is_fp8(q_dtype) || q_dtype < 0 || q_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
         return ORC_ERR_DTYPE;
@@ -264,16 +264,20 @@ int orc_paged_decode(double* out,
                 goto done;
             }
         }
-        for (int g = 0; g < num_heads; ++g) {
-            double* o = out + ((size_t)r * num_heads + g) * head_dim;
+        /* query j of the q_len new tokens sits at position L - q_len + j and sees the
+         * tokens up to and including itself: Lq = L - q_len + 1 + j of them */
+        for (int gq = 0; gq < q_len * num_heads; ++gq) {
+            const int j = gq / num_heads, g = gq % num_heads;
+            const int Lq = L - q_len + 1 + j;
+            double* o = out + ((size_t)r * q_len * num_heads + gq) * head_dim;
             const int h = g / group;
             for (int i = 0; i < head_dim; ++i)
                 o[i] = 0.0;
-            if (L == 0)
+            if (Lq <= 0)
                 continue;
-            const size_t qoff = ((size_t)s * num_heads + g) * head_dim;
+            const size_t qoff = ((size_t)s * q_len * num_heads + gq) * head_dim;
             /* scores x_t = scale * q . K_t */
-            for (int t = 0; t < L; ++t) {
+            for (int t = 0; t < Lq; ++t) {
                 const int32_t p = block_tables[(size_t)s * max_blocks_per_seq + t / block_size];
                 const int off = t % block_size;
                 if (p < 0 || p >= num_blocks) {
@@ -288,11 +292,11 @@ int orc_paged_decode(double* out,
             }
             /* softmax weights w_t = exp(x_t - max x) and the weighted sum of V_t */
             double m = x[0];
-            for (int t = 1; t < L; ++t)
+            for (int t = 1; t < Lq; ++t)
                 if (x[t] > m)
                     m = x[t];
             double denom = 0.0;
-            for (int t = 0; t < L; ++t) {
+            for (int t = 0; t < Lq; ++t) {
                 const int32_t p = block_tables[(size_t)s * max_blocks_per_seq + t / block_size];
                 const int off = t % block_size;
                 const size_t voff = (((size_t)p * num_kv_heads + h) * block_size + off) * head_dim;

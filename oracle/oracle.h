@@ -13,8 +13,10 @@ double orc_e5m2_value(uint8_t code);
 uint8_t orc_e5m2_encode(float x);
 void orc_e5m2_encode_array(const float* x, uint8_t* codes, int64_t n);
 
-/* out: [len(seqs) or num_seqs][num_heads][head_dim] doubles, rows in the order of
- * `seqs` (all sequences when seqs == NULL). */
+/* out: [len(seqs) or num_seqs][q_len][num_heads][head_dim] doubles, rows in the order
+ * of `seqs` (all sequences when seqs == NULL); q: [num_seqs][q_len][num_heads][head_dim].
+ * Query j of sequence s sits at position seq_lens[s] - q_len + j and attends the
+ * tokens up to and including it (q_len = 1: plain decode). */
 int orc_paged_decode(double* out,
                      const void* q, int q_dtype,
                      const void* k_cache, const void* v_cache, int kv_dtype,
@@ -22,7 +24,7 @@ int orc_paged_decode(double* out,
                      int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                      int block_size, int max_blocks_per_seq, int num_blocks,
                      double scale, double k_scale, double v_scale,
-                     const int32_t* seqs, int n_seqs);
+                     const int32_t* seqs, int n_seqs, int q_len);
 
 /* Writes rows `rows` (all num_tokens rows when rows == NULL) of k/v into the caches. */
 int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,

@@ -422,6 +422,48 @@ def check_e5m2_attention_dequant(lib):
         assert np.allclose(got[s], ref, rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------- several queries per sequence
+
+def check_multi_query_matches_causal_sdpa(lib):
+    """q_len new tokens per sequence: torch SDPA (fp64) with an explicit causal mask over the
+    contiguous K/V equals the paged oracle; query j sees tokens 0 .. L - q_len + j."""
+    rng = np.random.default_rng(31)
+    Hq, Hkv, d, bs, q_len = 8, 2, 16, 4, 3
+    lengths = [3, 5, 9, 14]
+    _, Ks, Vs = _random_case(rng, lengths, Hq, Hkv, d)
+    q = rng.standard_normal((len(lengths), q_len, Hq, d))
+    kc, vc, bt, sl = page_sequences(Ks, Vs, bs, sum(-(-L // bs) for L in lengths) + 3, rng)
+    got = oracle.paged_decode(q.astype(np.float32), "f32", kc, vc, "f32", bt, sl, Hq, Hkv, d, bs, kc.shape[0], 0.3,
+                              lib=lib, q_len=q_len)
+    for s, L in enumerate(lengths):
+        qt = torch.from_numpy(q[s].astype(np.float32).astype(np.float64)).permute(1, 0, 2)[None]   # [1, Hq, q_len, d]
+        kt = torch.from_numpy(Ks[s].astype(np.float64)).permute(1, 0, 2)[None]
+        vt = torch.from_numpy(Vs[s].astype(np.float64)).permute(1, 0, 2)[None]
+        pos = torch.arange(L - q_len, L)[:, None]
+        mask = torch.arange(L)[None, :] <= pos                                                  # [q_len, L]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3,
+                                                                enable_gqa=True)[0].permute(1, 0, 2).numpy()
+        assert np.allclose(got[s], ref, rtol=0, atol=1e-12), s
+
+
+def check_multi_query_is_decode_at_each_position(lib):
+    """Query j of a q_len chunk equals the single-query decode of a sequence cut at length
+    L - q_len + 1 + j (bit for bit: the same definition, the same order)."""
+    rng = np.random.default_rng(32)
+    Hq, Hkv, d, bs, q_len = 4, 1, 8, 8, 4
+    lengths = [4, 7, 20]
+    _, Ks, Vs = _random_case(rng, lengths, Hq, Hkv, d)
+    q = rng.standard_normal((len(lengths), q_len, Hq, d)).astype(np.float32)
+    kc, vc, bt, sl = page_sequences(Ks, Vs, bs, sum(-(-L // bs) for L in lengths) + 3, rng)
+    got = oracle.paged_decode(q, "f32", kc, vc, "f32", bt, sl, Hq, Hkv, d, bs, kc.shape[0], 0.5, lib=lib,
+                              q_len=q_len)
+    for j in range(q_len):
+        cut = (sl - q_len + 1 + j).astype(np.int32)
+        one = oracle.paged_decode(np.ascontiguousarray(q[:, j]), "f32", kc, vc, "f32", bt, cut, Hq, Hkv, d, bs,
+                                  kc.shape[0], 0.5, lib=lib)
+        assert np.array_equal(got[:, j], one), j
+
+
 ALL_CHECKS = [
     check_e4m3_decode_table, check_e4m3_spot_values, check_e4m3_encode_vs_library, check_e4m3_ties_to_even,
     check_e4m3_saturation_and_roundtrip, check_length_one_is_v, check_length_two_closed_form,
@@ -430,4 +472,5 @@ ALL_CHECKS = [
     check_append_golden, check_append_fp8_vs_library, check_fp8_attention_dequant,
     check_e5m2_decode_table, check_e5m2_spot_values, check_e5m2_encode_vs_library,
     check_e5m2_ties_saturation_roundtrip, check_append_e5m2_vs_library, check_e5m2_attention_dequant,
+    check_multi_query_matches_causal_sdpa, check_multi_query_is_decode_at_each_position,
 ]

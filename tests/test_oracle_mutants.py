@@ -41,6 +41,7 @@ MUTANTS = {
                          "double vlo = e5m2_pos[lo], vhi = e5m2_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi);\n"
                          "    int code;\n    if (a < midpoint)\n        code = lo;\n    else if (a > midpoint)\n"
                          "        code = hi;\n    else\n        code = (lo & 1) ? lo : hi;"),
+    "causal_limit_off_by_one": ("const int Lq = L - q_len + 1 + j;", "const int Lq = L - q_len + j;"),
     "e5m2_saturates_to_infinity": ("if (a >= e5m2_pos[123])\n        return sign | 123;",
                                    "if (a >= e5m2_pos[123])\n        return sign | 124;"),
     "e4m3_bias_off_by_one": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
