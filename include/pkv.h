@@ -160,6 +160,29 @@ PKV_API int paged_decode_step(void* out, const void* q, void* k_cache, void* v_c
                               const int64_t* slot_mapping, int in_dtype, void* stream);
 
 /*
+ * Several new tokens per sequence (chunked prefill, speculative-decoding
+ * verification): q_len queries per sequence, causal within the chunk. Query j
+ * of sequence s is the token at position seq_lens[s] - q_len + j (seq_lens
+ * counts the q_len new tokens, already appended with reshape_and_cache) and
+ * attends the cached tokens 0 .. seq_lens[s] - q_len + j, i.e. all earlier
+ * tokens and itself; a query whose position is negative gets a zero row.
+ *
+ *   q, out       [num_seqs][q_len][num_heads][head_dim], q_dtype BF16
+ *   q_len        1 .. 8 with q_len * (num_heads / num_kv_heads) in {1, 2, 4, 5, 8}
+ *   workspace    >= paged_attention_workspace_size(num_seqs, q_len * num_heads,
+ *                num_kv_heads, head_dim, num_partitions) bytes
+ * Other arguments as paged_attention_decode. Runs on the tensor-core kernel
+ * (bf16 / E4M3 / E5M2 caches, block size 16 or 32, head_dim 128, or 64 for
+ * bf16); other shapes return PKV_ERR_SHAPE. q_len = 1 is paged_attention_decode.
+ */
+PKV_API int paged_attention_decode_mq(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                      int q_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                      float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                                      int kv_dtype, float k_scale, float v_scale, int num_partitions,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Test hook for the failure path (no counterpart in the pages). The same call
  * as paged_attention_decode, except that the producer warp that owns unit
  * `withheld_unit` (units = (sequence, KV-head group, block) in order) never

@@ -59,6 +59,9 @@ def load_library():
     lib.paged_decode_step.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                       f32, f32, i32, P, sz, P, P, P, i32, P]
     lib.paged_decode_step.restype = i32
+    lib.paged_attention_decode_mq.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, i32,
+                                              i32, f32, f32, i32, P, sz, P]
+    lib.paged_attention_decode_mq.restype = i32
     lib.pkv_test_decode_timeout.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                             f32, f32, i32, P, sz, i32, P]
     lib.pkv_test_decode_timeout.restype = i32
@@ -164,6 +167,31 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scal
             _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
             block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
             int(num_partitions), _cuda("workspace", workspace), workspace.numel())
+
+
+def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale=1.0, v_scale=1.0,
+                              num_partitions=0, workspace=None, stream=None) -> None:
+    """q_len new tokens per sequence, causal within the chunk: q, out [num_seqs, q_len, num_heads, head_dim]
+    (bf16); query j of sequence s sits at position seq_lens[s] - q_len + j and attends every token
+    up to itself. The new tokens' K/V must already be in the cache."""
+    S, QL, Hq, D = q.shape
+    NB, Hkv, BS, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q/out and the caches")
+    if out.dtype != q.dtype or v_cache.dtype != k_cache.dtype:
+        raise TypeError("out must match q's dtype and v_cache k_cache's")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
+    if workspace is None:
+        workspace = _cached_workspace(S, Hq * QL, Hkv, D, num_partitions, q.device)
+    st = load_library().paged_attention_decode_mq(
+        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, QL, Hq, Hkv, D, BS, float(scale),
+        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
+        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _stream_handle(stream))
+    _check("paged_attention_decode_mq", st)
 
 
 def withheld_unit_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, withheld_unit, workspace,

@@ -250,15 +250,19 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                 float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
                 float v_scale, int num_partitions, void* workspace, size_t workspace_bytes, void* stream,
-                const AppendArgs* app, int withheld_unit = -1)
+                const AppendArgs* app, int withheld_unit = -1, int q_len = 1)
 {
     if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
-        num_heads % num_kv_heads != 0 || num_partitions < 0)
+        num_heads % num_kv_heads != 0 || num_partitions < 0 || q_len < 1 || q_len > 8)
         return PKV_ERR_SHAPE;
-    const int group = num_heads / num_kv_heads;
+    // query columns per KV head: q_len new tokens x the GQA group (the kernels' "group")
+    const int group = num_heads / num_kv_heads * q_len;
     if (!group_supported(group) || (head_dim != 64 && head_dim != 128) ||
         (block_size != 8 && block_size != 16 && block_size != 32))
         return PKV_ERR_SHAPE;
+    if (q_len > 1 && (app || !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group,
+                                                                       num_kv_heads))))
+        return PKV_ERR_SHAPE;   // several new tokens: tensor-core kernel only, no fused append
     if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
           (q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2))))
         return PKV_ERR_DTYPE;
@@ -321,6 +325,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
+    p.q_len = q_len;
     if (withheld_unit >= 0) {
         if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
             return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
@@ -349,6 +354,18 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
                        block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
                        num_partitions, workspace, workspace_bytes, stream, nullptr);
+}
+
+int paged_attention_decode_mq(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int q_len,
+                              int num_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                              int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
+                              float v_scale, int num_partitions, void* workspace, size_t workspace_bytes,
+                              void* stream)
+{
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                       block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
+                       num_partitions, workspace, workspace_bytes, stream, nullptr, -1, q_len);
 }
 
 int pkv_test_decode_timeout(void* out, const void* q, const void* k_cache, const void* v_cache,

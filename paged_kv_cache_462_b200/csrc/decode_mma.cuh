@@ -183,6 +183,17 @@ __device__ __forceinline__ void append_new_token_impl(const DecodeParams& p, int
     __syncwarp();
 }
 
+// Row of `q` / `out` ([num_seqs][q_len][num_heads][d]) of query column c of KV head `head` of
+// sequence s: column c is new token c / Gq of the sequence and query head head * Gq + c % Gq,
+// Gq = num_heads / num_kv_heads (q_len = 1: column c is query head head * G + c).
+__device__ __forceinline__ size_t query_row(const DecodeParams& p, int s, int head, int c)
+{
+    const int QL = p.q_len > 1 ? p.q_len : 1;
+    const int Gq = p.num_heads / p.num_kv_heads;
+    const int j = c / Gq, gh = c - j * Gq;
+    return ((size_t)s * QL + j) * p.num_heads + (size_t)head * Gq + gh;
+}
+
 // ------------------------------------------------------------------ configuration
 
 template <class KV, int D, int BS, int G, int HG>
@@ -307,8 +318,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
             // a new token needs a position in the sequence: seq_lens[s] >= 1
             if (tid == 0 && p.new_k != nullptr && __ldg(p.new_slots + s) >= 0)
                 atomicOr(p.err, PKV_DEVERR_SLOT);
-            QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * p.num_heads * D;
-            for (int i = tid; i < p.num_heads * D; i += C::kThreads)
+            const int rows = p.num_heads * (p.q_len > 1 ? p.q_len : 1);
+            QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * rows * D;
+            for (int i = tid; i < rows * D; i += C::kThreads)
                 from_float(0.f, o + i);
         }
     }
@@ -413,11 +425,17 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         const int head = hg * HG + warp;           // this warp's KV head
         int L = p.seq_lens[s];
         L = L < 0 ? 0 : (L > capacity ? capacity : L);
+        // causal limits of this lane's two query columns 2t, 2t+1: column c (new token c / Gq of
+        // q_len) sees the tokens before position L - q_len + 1 + c / Gq (all L when q_len = 1)
+        const int QL = p.q_len > 1 ? p.q_len : 1;
+        const int Gq = p.num_heads / p.num_kv_heads;
+        const int lim0 = 2 * t < G ? L - QL + 1 + (2 * t) / Gq : 0;           // padding columns: none
+        const int lim1 = 2 * t + 1 < G ? L - QL + 1 + (2 * t + 1) / Gq : 0;
 
-        // Q^T as the B operand: b0 = (k: d pair, n: query head g); rows g >= G are zero.
+        // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
         uint32_t qb[C::kKS][2];
         {
-            const QT* qp = reinterpret_cast<const QT*>(p.q) + ((size_t)s * p.num_heads + (size_t)head * G + g) * D;
+            const QT* qp = reinterpret_cast<const QT*>(p.q) + (g < G ? query_row(p, s, head, g) : 0) * D;
 #pragma unroll
             for (int ks = 0; ks < C::kKS; ++ks) {
                 if (g < G) {
@@ -529,11 +547,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                         released = true;
                     }
                     // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
-                    const int tok0 = tt * 16 + g;
-                    sc[0] = (tok0 < valid) ? sc[0] * qk_scale : -INFINITY;
-                    sc[1] = (tok0 < valid) ? sc[1] * qk_scale : -INFINITY;
-                    sc[2] = (tok0 + 8 < valid) ? sc[2] * qk_scale : -INFINITY;
-                    sc[3] = (tok0 + 8 < valid) ? sc[3] * qk_scale : -INFINITY;
+                    const int tok0 = jb * BS + tt * 16 + g;   // position in the sequence
+                    sc[0] = (tok0 < lim0) ? sc[0] * qk_scale : -INFINITY;
+                    sc[1] = (tok0 < lim1) ? sc[1] * qk_scale : -INFINITY;
+                    sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk_scale : -INFINITY;
+                    sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk_scale : -INFINITY;
                     // The reference moves only when some score passes it by the slack; each lane
                     // tests its own scores first, so the butterfly max runs only when one does
                     // (same result as reducing first: the tile max passes iff some lane's does).
@@ -635,7 +653,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
             return F16 ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
         };
         if (first_run == last_run) {
-            QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
+            QT* out0 = reinterpret_cast<QT*>(p.out) + (2 * t < G ? query_row(p, s, head, 2 * t) : 0) * D;
+            QT* out1 = reinterpret_cast<QT*>(p.out) + (2 * t + 1 < G ? query_row(p, s, head, 2 * t + 1) : 0) * D;
             const float inv0 = l[0] > 0.f ? p.v_scale / l[0] : 0.f;
             const float inv1 = l[1] > 0.f ? p.v_scale / l[1] : 0.f;
 #pragma unroll
@@ -644,9 +663,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                 for (int half = 0; half < 2; ++half) {
                     const int d = d_of(dt, half);
                     if (2 * t < G)
-                        from_float(o[dt][2 * half] * inv0, out + (2 * t) * D + d);
+                        from_float(o[dt][2 * half] * inv0, out0 + d);
                     if (2 * t + 1 < G)
-                        from_float(o[dt][2 * half + 1] * inv1, out + (2 * t + 1) * D + d);
+                        from_float(o[dt][2 * half + 1] * inv1, out1 + d);
                 }
         } else {
             float* part = p.partials + ((size_t)(blockIdx.x + stream) * HG + warp) * p.slot_floats;
@@ -681,7 +700,7 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
                                            int warp, int lane)
 {
     const int head = (stream - s * NHG) * HG + warp;
-    QT* out = reinterpret_cast<QT*>(p.out) + ((size_t)s * p.num_heads + (size_t)head * G) * D;
+    QT* out = reinterpret_cast<QT*>(p.out);
     auto slot = [&](int c) -> const float* {
         return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
     };
@@ -789,10 +808,11 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
             for (int gq = 0; gq < G; ++gq)
                 L = (gq == gv) ? Lsum[gq] : L;
             const float inv = L > 0.f ? p.v_scale / L : 0.f;
-            from_float(acc[v].x * inv, out + idx);
-            from_float(acc[v].y * inv, out + idx + 1);
-            from_float(acc[v].z * inv, out + idx + 2);
-            from_float(acc[v].w * inv, out + idx + 3);
+            QT* dst = out + query_row(p, s, head, gv) * D + (idx - gv * D);
+            from_float(acc[v].x * inv, dst);
+            from_float(acc[v].y * inv, dst + 1);
+            from_float(acc[v].z * inv, dst + 2);
+            from_float(acc[v].w * inv, dst + 3);
         }
     }
 }

@@ -45,6 +45,9 @@ struct DecodeParams {
     const void* new_v;
     const int64_t* new_slots;
     int in_dtype;
+    // new tokens per sequence (tensor-core kernel; 0 or 1: one): the G query columns of a KV head
+    // are q_len tokens x (num_heads / num_kv_heads) heads, token-major, causal within the chunk
+    int q_len;
     // failure-path test hook (tensor-core kernel): 1 + the unit whose stage the producer never
     // hands to its consumers, so their bounded wait runs out; 0 = none
     int withheld_unit;

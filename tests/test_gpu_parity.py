@@ -421,3 +421,59 @@ def test_e5m2_uncovered_shapes_are_rejected():
         sl = torch.ones(2, dtype=torch.int32, device="cuda")
         with pytest.raises(pkv.PkvError):
             pkv.paged_attention_decode(torch.empty_like(q), q, kc, kc.clone(), bt, sl, 0.1, 1.0, 1.0)
+
+
+# ------------------------------------------------------------------ several new tokens per sequence
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+@pytest.mark.parametrize("BS", [16, 32])
+@pytest.mark.parametrize("q_len,Hq,Hkv", [(2, 8, 2), (4, 4, 2), (8, 2, 2), (2, 4, 2), (5, 2, 2)])
+def test_multi_query_causal(kv, BS, q_len, Hq, Hkv):
+    """q_len new tokens per sequence against the oracle's causal definition, every output element;
+    lengths include sequences shorter than the chunk (their early queries see nothing)."""
+    lengths = [1, q_len - 1 if q_len > 1 else 1, q_len, BS + 3, 3 * BS - 1, 97, 300]
+    b = W.build_batch(_spec(f"mq_{kv}_{BS}_{q_len}_{Hq}", len(lengths), Hq, Hkv, 128, BS, kv, lengths,
+                            seed=900 + BS + q_len * 10 + Hq))
+    sp = b.spec
+    _, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    g.append()
+    rng = np.random.default_rng(q_len * 100 + Hq)
+    qm = W.f32_to_bf16_bits(rng.standard_normal((b.num_seqs, q_len, Hq, 128)).astype(np.float32))
+    ref = oracle.paged_decode(qm, "bf16", okc, ovc, kv, b.block_tables, b.seq_lens, Hq, Hkv, 128, BS, b.num_blocks,
+                              b.scale, b.k_scale, b.v_scale, q_len=q_len)
+    q = to_dev(qm, "bf16")
+    for parts in (0, 3):
+        out = torch.full_like(q, float("nan"))
+        ws = pkv.new_workspace(b.num_seqs, Hq * q_len, Hkv, 128, parts)
+        pkv.paged_attention_decode_mq(out, q, g.kc, g.vc, g.bt, g.sl, float(b.scale), float(b.k_scale),
+                                      float(b.v_scale), parts, ws)
+        torch.cuda.synchronize()
+        assert pkv.read_device_error(ws) == 0
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert np.max(np.abs(got - ref)) <= TOL[kv], parts
+
+
+def test_multi_query_one_token_is_decode():
+    b = W.config_batch(1, num_seqs=6)
+    g = GpuStep(b)
+    g.append()
+    out1 = g.decode(0).clone()
+    out2 = torch.empty_like(out1)
+    sp = b.spec
+    ws = pkv.new_workspace(b.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, 0)
+    pkv.paged_attention_decode_mq(out2.view(b.num_seqs, 1, sp.num_heads, sp.head_dim),
+                                  g.q.view(b.num_seqs, 1, sp.num_heads, sp.head_dim), g.kc, g.vc, g.bt, g.sl,
+                                  float(b.scale), 1.0, 1.0, 0, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+def test_multi_query_unsupported_shapes_are_rejected():
+    q = torch.zeros(2, 3, 4, 128, dtype=torch.bfloat16, device="cuda")      # 3 tokens x G 2 = 6 columns
+    kc = torch.zeros(8, 2, 16, 128, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(2, 2, dtype=torch.int32, device="cuda")
+    sl = torch.full((2,), 5, dtype=torch.int32, device="cuda")
+    with pytest.raises(pkv.PkvError):
+        pkv.paged_attention_decode_mq(torch.empty_like(q), q, kc, kc.clone(), bt, sl, 0.1)
