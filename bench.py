@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--config", type=int, default=1, help="workload 0..4 (default 1, Llama-3-8B bf16)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partitions", type=int, default=0, help="decode runs (0 = automatic)")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="new tokens per sequence: > 1 times the causal multi-query decode instead of the step")
     ap.add_argument("--kv-dtype", choices=["bf16", "e4m3", "e5m2"], default=None,
                     help="run the workload with this cache dtype instead of its own (configs 1-4)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
@@ -76,11 +78,14 @@ def describe(b: W.DecodeBatch) -> str:
             + (f", prefix groups of {sp.share_group} sharing <= {sp.share_blocks} blocks" if sp.share_group else ""))
 
 
-def step_bytes(b: W.DecodeBatch):
+def step_bytes(b: W.DecodeBatch, q_len: int = 1):
+    """Algorithmic bytes of the step: decode (q/out rows scale with q_len), and the append (none
+    in the multi-query form, whose new tokens are already in the cache)."""
     sp = b.spec
-    dec = acct.decode_bytes(b.seq_lens, b.block_tables, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+    dec = acct.decode_bytes(b.seq_lens, b.block_tables, sp.num_heads * q_len, sp.num_kv_heads, sp.head_dim,
                             sp.block_size, sp.kv_dtype, sp.q_dtype)
-    app = acct.append_bytes(int((b.new_slots >= 0).sum()), sp.num_kv_heads, sp.head_dim, sp.in_dtype, sp.kv_dtype)
+    app = 0 if q_len > 1 else acct.append_bytes(int((b.new_slots >= 0).sum()), sp.num_kv_heads, sp.head_dim,
+                                                sp.in_dtype, sp.kv_dtype)
     return dec, app
 
 
@@ -223,6 +228,7 @@ class DeviceState:
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
         self.out = torch.empty_like(self.q)
         self.partitions = partitions
+        self.q_len = 1
         self.ws = pkv.new_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, partitions, device)
         for i in range(0, b.hist_slots.size, 1 << 16):      # history already in the cache before the step
             pkv.reshape_and_cache(self._dev(b.hist_k[i:i + (1 << 16)], sp.in_dtype),
@@ -248,15 +254,35 @@ class DeviceState:
                                         float(b.k_scale), float(b.v_scale), self.partitions, self.ws)
 
     def step(self):
-        """append + decode through paged_decode_step (one launch where the fused kernel applies)"""
+        """append + decode through paged_decode_step (one launch where the fused kernel applies);
+        with q_len > 1 the causal multi-query decode of the last q_len tokens of every sequence"""
         b = self.b
+        if self.q_len > 1:
+            self.pkv.paged_attention_decode_mq(self.out_mq, self.q_mq, self.kc, self.vc, self.bt, self.sl,
+                                               float(b.scale), float(b.k_scale), float(b.v_scale), self.partitions,
+                                               self.ws_mq)
+            return
         self.pkv.paged_decode_step(self.out, self.q, self.kc, self.vc, self.bt, self.sl, self.new_k, self.new_v,
                                    self.new_slots, float(b.scale), float(b.k_scale), float(b.v_scale),
                                    self.partitions, self.ws)
 
+    def set_q_len(self, q_len: int):
+        """Multi-query mode: the history plus the appended token stand for the last q_len tokens."""
+        self.q_len = q_len
+        if q_len > 1:
+            sp, t = self.b.spec, self.torch
+            g = t.Generator(device="cpu").manual_seed(462)
+            self.q_mq = t.randn((self.b.num_seqs, q_len, sp.num_heads, sp.head_dim), generator=g).to(
+                t.bfloat16).to(self.dev)
+            self.out_mq = t.empty_like(self.q_mq)
+            self.ws_mq = self.pkv.new_workspace(sp.num_seqs, sp.num_heads * q_len, sp.num_kv_heads, sp.head_dim,
+                                                self.partitions, self.dev)
+            self.append()
+
     def errors(self):
         self.torch.cuda.synchronize(self.dev)
-        return int(self.err.item()) | self.pkv.read_device_error(self.ws)
+        e = int(self.err.item()) | self.pkv.read_device_error(self.ws)
+        return e | (self.pkv.read_device_error(self.ws_mq) if self.q_len > 1 else 0)
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
@@ -361,7 +387,8 @@ def ours_arm(args):
     spec = workload_spec(args)
     b = W.build_batch(spec, seed=spec.seed + 1000 * rank)
     state = DeviceState(torch, pkv, b, dev, args.partitions)
-    dec, app = step_bytes(b)
+    state.set_q_len(args.q_len)
+    dec, app = step_bytes(b, args.q_len)
     bytes_step = dec["total"] + app
     # a read (not a write) of a buffer twice the size of L2: the L2 ends up holding clean lines of
     # another buffer, as after the weight-streaming GEMMs that precede attention in a decode step
@@ -406,8 +433,10 @@ def ours_arm(args):
     # end to end: per-step inputs from pinned host memory, output back to pinned host memory
     e2e = None
     if not args.no_e2e:
-        host = {n: getattr(state, n).detach().cpu().pin_memory() for n in ("q", "new_k", "new_v", "new_slots", "sl", "bt")}
-        out_h = torch.empty(state.out.shape, dtype=state.out.dtype).pin_memory()
+        names = ("q_mq", "sl", "bt") if args.q_len > 1 else ("q", "new_k", "new_v", "new_slots", "sl", "bt")
+        host = {n: getattr(state, n).detach().cpu().pin_memory() for n in names}
+        dev_out = state.out_mq if args.q_len > 1 else state.out
+        out_h = torch.empty(dev_out.shape, dtype=dev_out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_h.numel() * out_h.element_size()
         Ke = K
@@ -420,7 +449,7 @@ def ours_arm(args):
             for n, t in host.items():
                 getattr(state, n).copy_(t, non_blocking=True)
             state.step()
-            out_h.copy_(state.out, non_blocking=True)
+            out_h.copy_(dev_out, non_blocking=True)
             if rec:
                 ee[i - args.warmup][1].record(stream)
         torch.cuda.synchronize(dev)
@@ -456,7 +485,9 @@ def ours_arm(args):
                 "kv_storage": spec.kv_dtype, "partitions": args.partitions or pkv.default_partitions(
                     spec.head_dim, spec.block_size, spec.num_heads, spec.num_kv_heads,
                     {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3}[spec.kv_dtype]),
-                "step": ("paged_decode_step: append of one new token per sequence fused into the paged "
+                "step": (f"paged_attention_decode_mq: the last {args.q_len} tokens of every sequence as queries, "
+                         "causal within the chunk (their K/V already cached)" if args.q_len > 1 else
+                         "paged_decode_step: append of one new token per sequence fused into the paged "
                          "decode launch" if fused else
                          "paged_decode_step: reshape_and_cache then paged_attention_decode (two launches)"),
                 "l2": "cold: a 256 MiB read before every step, outside the step's CUDA events",
