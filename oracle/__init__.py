@@ -50,9 +50,9 @@ def _bind(lib):
     lib.orc_e5m2_encode_array.argtypes = [P, P, i64]
     lib.orc_e5m2_encode_array.restype = None
     lib.orc_paged_decode.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
-                                     f64, f64, f64, P, i32, i32]
+                                     f64, f64, f64, P, i32, i32, P, P]
     lib.orc_paged_decode.restype = i32
-    lib.orc_reshape_and_cache.argtypes = [P, P, i32, P, P, i32, P, P, i64, i32, i32, i32, i32, i32, f32, f32]
+    lib.orc_reshape_and_cache.argtypes = [P, P, i32, P, P, i32, P, P, i64, i32, i32, i32, i32, i32, f32, f32, P, P]
     lib.orc_reshape_and_cache.restype = i32
     return lib
 
@@ -101,7 +101,8 @@ def e5m2_encode(x, lib=None) -> np.ndarray:
 
 def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
                  num_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                 scale, k_scale=1.0, v_scale=1.0, seqs=None, lib=None, q_len=1) -> np.ndarray:
+                 scale, k_scale=1.0, v_scale=1.0, seqs=None, lib=None, q_len=1, k_head_scales=None,
+                 v_head_scales=None) -> np.ndarray:
     """fp64 attention output [len(seqs) or num_seqs, num_heads, head_dim]; with q_len > 1,
     q is [num_seqs, q_len, num_heads, head_dim] (query j at position seq_len - q_len + j,
     causal) and the output [rows, q_len, num_heads, head_dim]."""
@@ -114,13 +115,15 @@ def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
     S = sl.shape[0]
     MB = bt.shape[1] if bt.ndim == 2 else 0
     sub = None if seqs is None else np.ascontiguousarray(seqs, dtype=np.int32)
+    khs = None if k_head_scales is None else np.ascontiguousarray(k_head_scales, dtype=np.float32)
+    vhs = None if v_head_scales is None else np.ascontiguousarray(v_head_scales, dtype=np.float32)
     rows = S if sub is None else sub.size
     out = np.zeros((rows, num_heads, head_dim) if q_len == 1 else (rows, q_len, num_heads, head_dim),
                    dtype=np.float64)
     st = lib.orc_paged_decode(_ptr(out), _ptr(q), DT[q_dtype], _ptr(k_cache), _ptr(v_cache), DT[kv_dtype],
                               _ptr(bt), _ptr(sl), S, num_heads, num_kv_heads, head_dim, block_size, MB,
                               num_blocks, float(scale), float(k_scale), float(v_scale),
-                              _ptr(sub), 0 if sub is None else int(sub.size), int(q_len))
+                              _ptr(sub), 0 if sub is None else int(sub.size), int(q_len), _ptr(khs), _ptr(vhs))
     if st != 0:
         raise OracleError(f"orc_paged_decode status {st}")
     return out
@@ -128,8 +131,10 @@ def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
 
 def reshape_and_cache(k, v, in_dtype, k_cache, v_cache, kv_dtype, slot_mapping,
                       num_kv_heads, head_dim, block_size, num_blocks,
-                      k_scale=1.0, v_scale=1.0, rows=None, lib=None) -> None:
-    """Write rows of k/v ([T, Hkv, d]) into the numpy caches in place."""
+                      k_scale=1.0, v_scale=1.0, rows=None, lib=None, k_head_scales=None,
+                      v_head_scales=None) -> None:
+    """Write rows of k/v ([T, Hkv, d]) into the numpy caches in place (FP8: per-tensor scales, or
+    one per KV head when k_head_scales / v_head_scales are given)."""
     lib = lib or load()
     k = np.ascontiguousarray(k, dtype=NP_DT[in_dtype])
     v = np.ascontiguousarray(v, dtype=NP_DT[in_dtype])
@@ -137,10 +142,12 @@ def reshape_and_cache(k, v, in_dtype, k_cache, v_cache, kv_dtype, slot_mapping,
     assert k_cache.dtype == NP_DT[kv_dtype] and v_cache.dtype == NP_DT[kv_dtype]
     sm = np.ascontiguousarray(slot_mapping, dtype=np.int64)
     r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    khs = None if k_head_scales is None else np.ascontiguousarray(k_head_scales, dtype=np.float32)
+    vhs = None if v_head_scales is None else np.ascontiguousarray(v_head_scales, dtype=np.float32)
     st = lib.orc_reshape_and_cache(_ptr(k), _ptr(v), DT[in_dtype], _ptr(k_cache), _ptr(v_cache), DT[kv_dtype],
                                    _ptr(sm), _ptr(r), 0 if r is None else int(r.size), int(sm.size),
                                    num_kv_heads, head_dim, block_size, num_blocks,
-                                   float(np.float32(k_scale)), float(np.float32(v_scale)))
+                                   float(np.float32(k_scale)), float(np.float32(v_scale)), _ptr(khs), _ptr(vhs))
     if st != 0:
         raise OracleError(f"orc_reshape_and_cache status {st}")
 

@@ -232,7 +232,8 @@ int orc_paged_decode(double* out,
                      int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                      int block_size, int max_blocks_per_seq, int num_blocks,
                      double scale, double k_scale, double v_scale,
-                     const int32_t* seqs, int n_seqs, int q_len)
+                     const int32_t* seqs, int n_seqs, int q_len,
+                     const float* k_head_scales, const float* v_head_scales)
 {
     if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 || q_len < 1)
         return ORC_ERR_SHAPE;
@@ -271,6 +272,9 @@ int orc_paged_decode(double* out,
             const int Lq = L - q_len + 1 + j;
             double* o = out + ((size_t)r * q_len * num_heads + gq) * head_dim;
             const int h = g / group;
+            /* FP8 dequantisation scale: one per tensor, or one per KV head when given */
+            const double ksc = k_head_scales ? (double)k_head_scales[h] : k_scale;
+            const double vsc = v_head_scales ? (double)v_head_scales[h] : v_scale;
             for (int i = 0; i < head_dim; ++i)
                 o[i] = 0.0;
             if (Lq <= 0)
@@ -287,7 +291,7 @@ int orc_paged_decode(double* out,
                 const size_t koff = (((size_t)p * num_kv_heads + h) * block_size + off) * head_dim;
                 double dot = 0.0;
                 for (int i = 0; i < head_dim; ++i)
-                    dot += elem(q, q_dtype, qoff + i, 1.0) * elem(k_cache, kv_dtype, koff + i, k_scale);
+                    dot += elem(q, q_dtype, qoff + i, 1.0) * elem(k_cache, kv_dtype, koff + i, ksc);
                 x[t] = scale * dot;
             }
             /* softmax weights w_t = exp(x_t - max x) and the weighted sum of V_t */
@@ -303,7 +307,7 @@ int orc_paged_decode(double* out,
                 const double w = exp(x[t] - m);
                 denom += w;
                 for (int i = 0; i < head_dim; ++i)
-                    o[i] += w * elem(v_cache, kv_dtype, voff + i, v_scale);
+                    o[i] += w * elem(v_cache, kv_dtype, voff + i, vsc);
             }
             for (int i = 0; i < head_dim; ++i)
                 o[i] /= denom;
@@ -320,7 +324,8 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                           void* k_cache, void* v_cache, int kv_dtype,
                           const int64_t* slot_mapping, const int64_t* rows, int64_t n_rows,
                           int num_tokens, int num_kv_heads, int head_dim,
-                          int block_size, int num_blocks, float k_scale, float v_scale)
+                          int block_size, int num_blocks, float k_scale, float v_scale,
+                          const float* k_head_scales, const float* v_head_scales)
 {
     if (is_fp8(in_dtype) || in_dtype < 0 || in_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
         return ORC_ERR_DTYPE;
@@ -353,8 +358,8 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
             for (int i = 0; i < head_dim; ++i) {
                 const float kx = (float)elem(k, in_dtype, src + i, 1.0);
                 const float vx = (float)elem(v, in_dtype, src + i, 1.0);
-                const float ky = kx / k_scale; /* binary32 division */
-                const float vy = vx / v_scale;
+                const float ky = kx / (k_head_scales ? k_head_scales[h] : k_scale); /* binary32 division */
+                const float vy = vx / (v_head_scales ? v_head_scales[h] : v_scale);
                 ((uint8_t*)k_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(ky) : orc_e5m2_encode(ky);
                 ((uint8_t*)v_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(vy) : orc_e5m2_encode(vy);
             }

@@ -24,12 +24,16 @@ int orc_paged_decode(double* out,
                      int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                      int block_size, int max_blocks_per_seq, int num_blocks,
                      double scale, double k_scale, double v_scale,
-                     const int32_t* seqs, int n_seqs, int q_len);
+                     const int32_t* seqs, int n_seqs, int q_len,
+                     const float* k_head_scales, const float* v_head_scales);
 
-/* Writes rows `rows` (all num_tokens rows when rows == NULL) of k/v into the caches. */
+/* Writes rows `rows` (all num_tokens rows when rows == NULL) of k/v into the caches.
+ * FP8 caches: per-tensor k_scale / v_scale, or one scale per KV head when
+ * k_head_scales / v_head_scales ([num_kv_heads]) are given (the same in attention). */
 int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                           void* k_cache, void* v_cache, int kv_dtype,
                           const int64_t* slot_mapping, const int64_t* rows, int64_t n_rows,
                           int num_tokens, int num_kv_heads, int head_dim,
-                          int block_size, int num_blocks, float k_scale, float v_scale);
+                          int block_size, int num_blocks, float k_scale, float v_scale,
+                          const float* k_head_scales, const float* v_head_scales);
 #endif

@@ -464,6 +464,43 @@ def check_multi_query_is_decode_at_each_position(lib):
         assert np.array_equal(got[:, j], one), j
 
 
+# ------------------------------------------------------------- per-KV-head FP8 scales
+
+def check_head_scales_equal_per_head_runs(lib):
+    """One scale per KV head: appending and attending with head scales (s0, s1) equals, head by
+    head, the per-tensor oracle run with that head's scale (bit for bit); equal head scales
+    equal the per-tensor run."""
+    rng = np.random.default_rng(41)
+    T, Hkv, d, bs, nb, Hq = 24, 2, 16, 8, 6, 4
+    k = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    v = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    k[:, 1] *= 20; v[:, 1] *= 0.05                                  # heads of very different ranges
+    khs = (np.abs(k).max(axis=(0, 2)) / 448).astype(np.float32)
+    vhs = (np.abs(v).max(axis=(0, 2)) / 448).astype(np.float32)
+    blocks = [int(b) for b in rng.permutation(nb)[: T // bs]]          # T is a multiple of bs
+    slots = np.array([blocks[t // bs] * bs + t % bs for t in range(T)], np.int64)
+    bt = np.array([blocks], np.int32); sl = np.array([T], np.int32)
+    q = rng.standard_normal((1, Hq, d)).astype(np.float32)
+    kc = oracle.empty_cache(nb, Hkv, bs, d, "e4m3"); vc = oracle.empty_cache(nb, Hkv, bs, d, "e4m3")
+    oracle.reshape_and_cache(k, v, "f32", kc, vc, "e4m3", slots, Hkv, d, bs, nb, lib=lib,
+                             k_head_scales=khs, v_head_scales=vhs)
+    got = oracle.paged_decode(q, "f32", kc, vc, "e4m3", bt, sl, Hq, Hkv, d, bs, nb, 0.25, lib=lib,
+                              k_head_scales=khs, v_head_scales=vhs)
+    G = Hq // Hkv
+    for h in range(Hkv):
+        kc1 = oracle.empty_cache(nb, 1, bs, d, "e4m3"); vc1 = oracle.empty_cache(nb, 1, bs, d, "e4m3")
+        oracle.reshape_and_cache(np.ascontiguousarray(k[:, h:h + 1]), np.ascontiguousarray(v[:, h:h + 1]), "f32",
+                                 kc1, vc1, "e4m3", slots, 1, d, bs, nb, khs[h], vhs[h], lib=lib)
+        assert np.array_equal(kc[:, h], kc1[:, 0]) and np.array_equal(vc[:, h], vc1[:, 0])
+        one = oracle.paged_decode(np.ascontiguousarray(q[:, h * G:(h + 1) * G]), "f32", kc1, vc1, "e4m3", bt, sl,
+                                  G, 1, d, bs, nb, 0.25, khs[h], vhs[h], lib=lib)
+        assert np.array_equal(got[:, h * G:(h + 1) * G], one), h
+    same = oracle.paged_decode(q, "f32", kc, vc, "e4m3", bt, sl, Hq, Hkv, d, bs, nb, 0.25, 0.5, 0.25, lib=lib)
+    same_h = oracle.paged_decode(q, "f32", kc, vc, "e4m3", bt, sl, Hq, Hkv, d, bs, nb, 0.25, lib=lib,
+                                 k_head_scales=[0.5, 0.5], v_head_scales=[0.25, 0.25])
+    assert np.array_equal(same, same_h)
+
+
 ALL_CHECKS = [
     check_e4m3_decode_table, check_e4m3_spot_values, check_e4m3_encode_vs_library, check_e4m3_ties_to_even,
     check_e4m3_saturation_and_roundtrip, check_length_one_is_v, check_length_two_closed_form,
@@ -473,4 +510,5 @@ ALL_CHECKS = [
     check_e5m2_decode_table, check_e5m2_spot_values, check_e5m2_encode_vs_library,
     check_e5m2_ties_saturation_roundtrip, check_append_e5m2_vs_library, check_e5m2_attention_dequant,
     check_multi_query_matches_causal_sdpa, check_multi_query_is_decode_at_each_position,
+    check_head_scales_equal_per_head_runs,
 ]

@@ -17,8 +17,10 @@ MUTANTS = {
     "block_index_swapped": ("block_tables[(size_t)s * max_blocks_per_seq + t / block_size];\n                const int off = t % block_size;\n                if",
                             "block_tables[(size_t)s * max_blocks_per_seq + t % block_size];\n                const int off = t / block_size;\n                if"),
     "scale_dropped": ("x[t] = scale * dot;", "x[t] = dot;"),
-    "v_read_from_k": ("o[i] += w * elem(v_cache, kv_dtype, voff + i, v_scale);",
-                      "o[i] += w * elem(k_cache, kv_dtype, voff + i, v_scale);"),
+    "v_read_from_k": ("o[i] += w * elem(v_cache, kv_dtype, voff + i, vsc);",
+                      "o[i] += w * elem(k_cache, kv_dtype, voff + i, vsc);"),
+    "head_scale_of_wrong_head": ("const double ksc = k_head_scales ? (double)k_head_scales[h] : k_scale;",
+                                 "const double ksc = k_head_scales ? (double)k_head_scales[0] : k_scale;"),
     "last_token_dropped": ("const int L = seq_lens[s];", "const int L = seq_lens[s] > 1 ? seq_lens[s] - 1 : seq_lens[s];"),
     "no_normalisation": ("o[i] /= denom;", "o[i] /= 1.0;"),
     "no_max_subtraction": ("const double w = exp(x[t] - m);", "const double w = exp(x[t]);"),
@@ -45,7 +47,8 @@ MUTANTS = {
     "e5m2_saturates_to_infinity": ("if (a >= e5m2_pos[123])\n        return sign | 123;",
                                    "if (a >= e5m2_pos[123])\n        return sign | 124;"),
     "e4m3_bias_off_by_one": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
-    "fp8_scale_multiplied": ("const float ky = kx / k_scale;", "const float ky = kx * k_scale;"),
+    "fp8_scale_multiplied": ("const float ky = kx / (k_head_scales ? k_head_scales[h] : k_scale);",
+                             "const float ky = kx * (k_head_scales ? k_head_scales[h] : k_scale);"),
     "append_offset_wrong": ("const int64_t blk = slot / block_size, off = slot % block_size;",
                             "const int64_t blk = slot / block_size, off = (slot + 1) % block_size;"),
     "negative_slot_written": ("if (slot < 0)\n            continue;", "if (slot < -1000)\n            continue;"),
