@@ -160,6 +160,31 @@ PKV_API int paged_decode_step(void* out, const void* q, void* k_cache, void* v_c
                               const int64_t* slot_mapping, int in_dtype, void* stream);
 
 /*
+ * FP8 caches with one scale per KV head (the promptx.wiki inference tutorial,
+ * quantisation section, sets per-tensor against per-attention-head KV
+ * quantisation): k_head_scales / v_head_scales are device arrays of
+ * num_kv_heads floats > 0 (caller-owned, read during the call), used where the
+ * per-tensor calls use k_scale / v_scale — the append encodes
+ * code = FP8(x / k_head_scales[h]) for KV head h, the decode dequantises with
+ * the same scale. kv_dtype must be FP8_E4M3 or FP8_E5M2; the decode runs on
+ * the tensor-core kernel only (the shapes paged_attention_decode lists for
+ * it), others return PKV_ERR_SHAPE; a null scale array returns PKV_ERR_NULL.
+ * Otherwise the same as reshape_and_cache and paged_attention_decode.
+ */
+PKV_API int reshape_and_cache_head_scales(const void* k, const void* v, void* k_cache, void* v_cache,
+                                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                                          int head_dim, int block_size, int num_blocks, int in_dtype, int kv_dtype,
+                                          const float* k_head_scales, const float* v_head_scales,
+                                          int32_t* device_error, void* stream);
+PKV_API int paged_attention_decode_head_scales(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                               const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                               int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                               float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                                               int kv_dtype, const float* k_head_scales,
+                                               const float* v_head_scales, int num_partitions, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
+/*
  * Several new tokens per sequence (chunked prefill, speculative-decoding
  * verification): q_len queries per sequence, causal within the chunk. Query j
  * of sequence s is the token at position seq_lens[s] - q_len + j (seq_lens

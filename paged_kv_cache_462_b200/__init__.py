@@ -59,6 +59,11 @@ def load_library():
     lib.paged_decode_step.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                       f32, f32, i32, P, sz, P, P, P, i32, P]
     lib.paged_decode_step.restype = i32
+    lib.reshape_and_cache_head_scales.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P]
+    lib.reshape_and_cache_head_scales.restype = i32
+    lib.paged_attention_decode_head_scales.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32,
+                                                       i32, i32, P, P, i32, P, sz, P]
+    lib.paged_attention_decode_head_scales.restype = i32
     lib.paged_attention_decode_mq.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, i32,
                                               i32, f32, f32, i32, P, sz, P]
     lib.paged_attention_decode_mq.restype = i32
@@ -248,6 +253,42 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=1.0, v_scale
         _cuda("slot_mapping", slot_mapping), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
         float(k_scale), float(v_scale), err, _stream_handle(stream))
     _check("reshape_and_cache", st)
+
+
+def _head_scales(name, t, Hkv):
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or t.shape != (Hkv,):
+        raise TypeError(f"{name} must be a float32 tensor of num_kv_heads scales")
+    return _cuda(name, t)
+
+
+def reshape_and_cache_head_scales(k, v, k_cache, v_cache, slot_mapping, k_head_scales, v_head_scales,
+                                  device_error=None, stream=None) -> None:
+    """reshape_and_cache into an FP8 cache with one scale per KV head (float32 [num_kv_heads] tensors)."""
+    T, Hkv, D = k.shape
+    NB, Hkv2, BS, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between rows and caches")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
+        raise TypeError("slot_mapping must be int64 [num_tokens]")
+    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error)
+    st = load_library().reshape_and_cache_head_scales(
+        _cuda("k", k), _cuda("v", v), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
+        _cuda("slot_mapping", slot_mapping), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
+        _head_scales("k_head_scales", k_head_scales, Hkv), _head_scales("v_head_scales", v_head_scales, Hkv), err,
+        _stream_handle(stream))
+    _check("reshape_and_cache_head_scales", st)
+
+
+def paged_attention_decode_head_scales(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_head_scales,
+                                       v_head_scales, num_partitions=0, workspace=None, stream=None) -> None:
+    """paged_attention_decode over an FP8 cache with one scale per KV head."""
+    args = list(_decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, 1.0, 1.0, num_partitions,
+                             workspace))
+    Hkv = k_cache.shape[1]
+    args[16:18] = [_head_scales("k_head_scales", k_head_scales, Hkv), _head_scales("v_head_scales", v_head_scales,
+                                                                                    Hkv)]
+    st = load_library().paged_attention_decode_head_scales(*args, _stream_handle(stream))
+    _check("paged_attention_decode_head_scales", st)
 
 
 def read_device_error(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:

@@ -250,7 +250,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                 float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
                 float v_scale, int num_partitions, void* workspace, size_t workspace_bytes, void* stream,
-                const AppendArgs* app, int withheld_unit = -1, int q_len = 1)
+                const AppendArgs* app, int withheld_unit = -1, int q_len = 1, const float* k_head_scales = nullptr,
+                const float* v_head_scales = nullptr)
 {
     if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
         num_heads % num_kv_heads != 0 || num_partitions < 0 || q_len < 1 || q_len > 8)
@@ -263,6 +264,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     if (q_len > 1 && (app || !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group,
                                                                        num_kv_heads))))
         return PKV_ERR_SHAPE;   // several new tokens: tensor-core kernel only, no fused append
+    if ((k_head_scales || v_head_scales) &&
+        (!k_head_scales || !v_head_scales || !is_fp8(kv_dtype) ||
+         !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads))))
+        return PKV_ERR_SHAPE;   // per-head scales: both arrays, FP8 caches, tensor-core kernel
     if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
           (q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2))))
         return PKV_ERR_DTYPE;
@@ -326,6 +331,8 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
     p.q_len = q_len;
+    p.k_head_scales = k_head_scales;
+    p.v_head_scales = v_head_scales;
     if (withheld_unit >= 0) {
         if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
             return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
@@ -354,6 +361,21 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
                        block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale, v_scale,
                        num_partitions, workspace, workspace_bytes, stream, nullptr);
+}
+
+int paged_attention_decode_head_scales(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                       int num_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                                       int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                                       const float* k_head_scales, const float* v_head_scales, int num_partitions,
+                                       void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!k_head_scales || !v_head_scales)
+        return PKV_ERR_NULL;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                       block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, 1.0f, 1.0f,
+                       num_partitions, workspace, workspace_bytes, stream, nullptr, -1, 1, k_head_scales,
+                       v_head_scales);
 }
 
 int paged_attention_decode_mq(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -420,9 +442,14 @@ int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, co
                                   k_scale, v_scale, num_partitions, workspace, workspace_bytes, stream);
 }
 
-int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
-                      int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
-                      int kv_dtype, float k_scale, float v_scale, int32_t* device_error, void* stream)
+}  // extern "C"
+
+namespace {
+
+int cache_impl(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+               int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
+               int kv_dtype, float k_scale, float v_scale, const float* k_head_scales, const float* v_head_scales,
+               int32_t* device_error, void* stream)
 {
     if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || (head_dim != 64 && head_dim != 128) ||
         (block_size != 8 && block_size != 16 && block_size != 32))
@@ -436,11 +463,38 @@ int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache
         return PKV_ERR_NULL;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
         return PKV_ERR_SHAPE;
-    if (is_fp8(kv_dtype) && !(k_scale > 0.0f && v_scale > 0.0f))
+    if (is_fp8(kv_dtype) && !k_head_scales && !(k_scale > 0.0f && v_scale > 0.0f))
         return PKV_ERR_SHAPE;
     return cache_dispatch(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
-                          num_blocks, in_dtype, kv_dtype, k_scale, v_scale, device_error,
-                          static_cast<cudaStream_t>(stream));
+                          num_blocks, in_dtype, kv_dtype, k_scale, v_scale, k_head_scales, v_head_scales,
+                          device_error, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                      int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
+                      int kv_dtype, float k_scale, float v_scale, int32_t* device_error, void* stream)
+{
+    return cache_impl(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                      num_blocks, in_dtype, kv_dtype, k_scale, v_scale, nullptr, nullptr, device_error, stream);
+}
+
+int reshape_and_cache_head_scales(const void* k, const void* v, void* k_cache, void* v_cache,
+                                  const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, int in_dtype, int kv_dtype,
+                                  const float* k_head_scales, const float* v_head_scales, int32_t* device_error,
+                                  void* stream)
+{
+    if (!is_fp8(kv_dtype))
+        return PKV_ERR_DTYPE;
+    if (num_tokens > 0 && (!k_head_scales || !v_head_scales))
+        return PKV_ERR_NULL;
+    return cache_impl(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                      num_blocks, in_dtype, kv_dtype, 1.0f, 1.0f, k_head_scales, v_head_scales, device_error,
+                      stream);
 }
 
 }  // extern "C"

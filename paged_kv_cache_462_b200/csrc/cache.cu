@@ -26,7 +26,8 @@ template <class TIN, class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const TIN* __restrict__ k, const TIN* __restrict__ v, TC* __restrict__ kc, TC* __restrict__ vc,
     const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads, int head_dim, int block_size,
-    long long capacity, float k_scale, float v_scale, int32_t* err)
+    long long capacity, float k_scale, float v_scale, const float* __restrict__ k_head_scales,
+    const float* __restrict__ v_head_scales, int32_t* err)
 {
     const int pieces = head_dim / 8;                 // 8-element pieces per row
     const long long per_token = (long long)num_kv_heads * pieces;
@@ -50,7 +51,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
         const TIN* src = (is_v ? v : k) + ((long long)t * num_kv_heads + h) * head_dim + c * 8;
         TC* dst = (is_v ? vc : kc) + ((blk * num_kv_heads + h) * block_size + off) * head_dim + c * 8;
         if constexpr (sizeof(TC) == 1)
-            quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? v_scale : k_scale);
+            quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst),
+                        is_v ? (v_head_scales ? __ldg(v_head_scales + h) : v_scale)
+                             : (k_head_scales ? __ldg(k_head_scales + h) : k_scale));
         else
             copy8(src, dst);
     }
@@ -59,7 +62,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
 template <class TIN, class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
 int launch_cache(const void* k, const void* v, void* kc, void* vc, const int64_t* slots, int num_tokens,
                  int num_kv_heads, int head_dim, int block_size, int num_blocks, float k_scale, float v_scale,
-                 int32_t* err, cudaStream_t stream)
+                 const float* k_head_scales, const float* v_head_scales, int32_t* err, cudaStream_t stream)
 {
     const long long items = 2ll * num_tokens * num_kv_heads * (head_dim / 8);
     long long blocks = (items + 255) / 256;
@@ -69,7 +72,8 @@ int launch_cache(const void* k, const void* v, void* kc, void* vc, const int64_t
         blocks = 1;
     reshape_and_cache_kernel<TIN, TC, FMT><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const TIN*>(k), static_cast<const TIN*>(v), static_cast<TC*>(kc), static_cast<TC*>(vc), slots,
-        num_tokens, num_kv_heads, head_dim, block_size, (long long)num_blocks * block_size, k_scale, v_scale, err);
+        num_tokens, num_kv_heads, head_dim, block_size, (long long)num_blocks * block_size, k_scale, v_scale,
+        k_head_scales, v_head_scales, err);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
 }
 
@@ -77,29 +81,30 @@ int launch_cache(const void* k, const void* v, void* kc, void* vc, const int64_t
 
 int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                    int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
-                   int kv_dtype, float k_scale, float v_scale, int32_t* err, cudaStream_t stream)
+                   int kv_dtype, float k_scale, float v_scale, const float* k_head_scales,
+                   const float* v_head_scales, int32_t* err, cudaStream_t stream)
 {
     if (in_dtype == PKV_F32 && kv_dtype == PKV_F32)
         return launch_cache<float, float>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                          block_size, num_blocks, k_scale, v_scale, err, stream);
+                                          block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_BF16)
         return launch_cache<__nv_bfloat16, __nv_bfloat16>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
                                                           num_kv_heads, head_dim, block_size, num_blocks, k_scale,
-                                                          v_scale, err, stream);
+                                                          v_scale, k_head_scales, v_head_scales, err, stream);
     if (in_dtype == PKV_F32 && kv_dtype == PKV_FP8_E4M3)
         return launch_cache<float, uint8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                            block_size, num_blocks, k_scale, v_scale, err, stream);
+                                            block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3)
         return launch_cache<__nv_bfloat16, uint8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
-                                                    head_dim, block_size, num_blocks, k_scale, v_scale, err, stream);
+                                                    head_dim, block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
     if (in_dtype == PKV_F32 && kv_dtype == PKV_FP8_E5M2)
         return launch_cache<float, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
                                                        num_kv_heads, head_dim, block_size, num_blocks, k_scale,
-                                                       v_scale, err, stream);
+                                                       v_scale, k_head_scales, v_head_scales, err, stream);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E5M2)
         return launch_cache<__nv_bfloat16, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
                                                                num_kv_heads, head_dim, block_size, num_blocks,
-                                                               k_scale, v_scale, err, stream);
+                                                               k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
     return PKV_ERR_DTYPE;
 }
 

@@ -144,11 +144,13 @@ __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0
         if (p.in_dtype == PKV_F32) {
             const float* src = static_cast<const float*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
+                                                         : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
         } else {
             const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? p.v_scale_in : p.k_scale);
+                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
+                                                         : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
             else
                 copy8(src, reinterpret_cast<__nv_bfloat16*>(dst));
         }
@@ -410,7 +412,6 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
     // =========================== consumer warps ==============================
     const int g = lane >> 2;   // MMA row group
     const int t = lane & 3;    // MMA column pair
-    const float qk_scale = p.q_scale;
 
 
     int x = run_begin;
@@ -429,6 +430,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         // q_len) sees the tokens before position L - q_len + 1 + c / Gq (all L when q_len = 1)
         const int QL = p.q_len > 1 ? p.q_len : 1;
         const int Gq = p.num_heads / p.num_kv_heads;
+        // FP8 per-head scales (when given): this head's into the score and output factors
+        const float qk_scale = p.k_head_scales ? p.q_scale * __ldg(p.k_head_scales + head) : p.q_scale;
+        const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
         const int lim0 = 2 * t < G ? L - QL + 1 + (2 * t) / Gq : 0;           // padding columns: none
         const int lim1 = 2 * t + 1 < G ? L - QL + 1 + (2 * t + 1) / Gq : 0;
 
@@ -655,8 +659,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         if (first_run == last_run) {
             QT* out0 = reinterpret_cast<QT*>(p.out) + (2 * t < G ? query_row(p, s, head, 2 * t) : 0) * D;
             QT* out1 = reinterpret_cast<QT*>(p.out) + (2 * t + 1 < G ? query_row(p, s, head, 2 * t + 1) : 0) * D;
-            const float inv0 = l[0] > 0.f ? p.v_scale / l[0] : 0.f;
-            const float inv1 = l[1] > 0.f ? p.v_scale / l[1] : 0.f;
+            const float inv0 = l[0] > 0.f ? out_scale / l[0] : 0.f;
+            const float inv1 = l[1] > 0.f ? out_scale / l[1] : 0.f;
 #pragma unroll
             for (int dt = 0; dt < C::kDT; ++dt)
 #pragma unroll
@@ -700,6 +704,7 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
                                            int warp, int lane)
 {
     const int head = (stream - s * NHG) * HG + warp;
+    const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
     QT* out = reinterpret_cast<QT*>(p.out);
     auto slot = [&](int c) -> const float* {
         return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
@@ -807,7 +812,7 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
 #pragma unroll
             for (int gq = 0; gq < G; ++gq)
                 L = (gq == gv) ? Lsum[gq] : L;
-            const float inv = L > 0.f ? p.v_scale / L : 0.f;
+            const float inv = L > 0.f ? out_scale / L : 0.f;
             QT* dst = out + query_row(p, s, head, gv) * D + (idx - gv * D);
             from_float(acc[v].x * inv, dst);
             from_float(acc[v].y * inv, dst + 1);
@@ -917,8 +922,8 @@ struct MmaLauncher {
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
         // E4M3 -> f16 widening is exact: only the per-tensor scales remain
-        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 ? p.k_scale : 1.0f);
-        p.v_scale = KV::kBytes == 1 ? p.v_scale_in : 1.0f;
+        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
+        p.v_scale = KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f;
         kern<<<nruns, C::kThreads, smem, stream>>>(kmap, vmap, p);
         if (cudaGetLastError() != cudaSuccess)
             return PKV_ERR_LAUNCH;

@@ -48,6 +48,10 @@ struct DecodeParams {
     // new tokens per sequence (tensor-core kernel; 0 or 1: one): the G query columns of a KV head
     // are q_len tokens x (num_heads / num_kv_heads) heads, token-major, causal within the chunk
     int q_len;
+    // FP8 caches: one dequantisation scale per KV head ([num_kv_heads], device; null: the
+    // per-tensor k_scale / v_scale_in)
+    const float* k_head_scales;
+    const float* v_head_scales;
     // failure-path test hook (tensor-core kernel): 1 + the unit whose stage the producer never
     // hands to its consumers, so their bounded wait runs out; 0 = none
     int withheld_unit;
@@ -67,7 +71,8 @@ bool step_fusable(int q_dtype, int kv_dtype, int head_dim, int block_size, int g
 
 int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                    int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                   int in_dtype, int kv_dtype, float k_scale, float v_scale, int32_t* err, cudaStream_t stream);
+                   int in_dtype, int kv_dtype, float k_scale, float v_scale, const float* k_head_scales,
+                   const float* v_head_scales, int32_t* err, cudaStream_t stream);
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device (cached).
 bool ensure_smem_attribute(const void* kernel, size_t bytes);

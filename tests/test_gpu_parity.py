@@ -11,7 +11,7 @@ import torch
 import oracle
 import paged_kv_cache_462_b200 as pkv
 import workloads as W
-from gpu_harness import TOL, GpuStep, cache_bytes, max_err, to_dev
+from gpu_harness import TOL, TORCH_DT, GpuStep, cache_bytes, max_err, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -477,3 +477,46 @@ def test_multi_query_unsupported_shapes_are_rejected():
     sl = torch.full((2,), 5, dtype=torch.int32, device="cuda")
     with pytest.raises(pkv.PkvError):
         pkv.paged_attention_decode_mq(torch.empty_like(q), q, kc, kc.clone(), bt, sl, 0.1)
+
+
+# ------------------------------------------------------------------ per-KV-head FP8 scales
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("parts", [0, 5])
+def test_head_scales_append_and_decode(kv, parts):
+    """FP8 caches with one scale per KV head (heads of very different ranges): appends bit-exact
+    and outputs within tolerance of the oracle using the same head scales."""
+    b = W.config_batch(1, num_seqs=6, kv_dtype=kv)
+    sp = b.spec
+    Hkv, D, BS, NB = sp.num_kv_heads, sp.head_dim, sp.block_size, b.num_blocks
+    gain = np.geomspace(0.05, 40.0, Hkv).astype(np.float32)           # per-head magnitude
+    def rows(x):
+        f = W.bf16_bits_to_f32(x) * gain[None, :, None]
+        return W.f32_to_bf16_bits(f.astype(np.float32))
+    hk, hv, nk, nv = rows(b.hist_k), rows(b.hist_v), rows(b.new_k), rows(b.new_v)
+    top = 448.0 if kv == "e4m3" else 57344.0
+    def head_absmax(*xs):
+        return np.max([np.abs(W.bf16_bits_to_f32(x)).max(axis=(0, 2)) for x in xs], axis=0)
+    khs = (head_absmax(hk, nk) / np.float32(top)).astype(np.float32)
+    vhs = (head_absmax(hv, nv) / np.float32(top)).astype(np.float32)
+    okc = oracle.empty_cache(NB, Hkv, BS, D, kv); ovc = oracle.empty_cache(NB, Hkv, BS, D, kv)
+    for k_, v_, sl_ in ((hk, hv, b.hist_slots), (nk, nv, b.new_slots)):
+        oracle.reshape_and_cache(k_, v_, "bf16", okc, ovc, kv, sl_, Hkv, D, BS, NB,
+                                 k_head_scales=khs, v_head_scales=vhs)
+    ref = oracle.paged_decode(b.q, "bf16", okc, ovc, kv, b.block_tables, b.seq_lens, sp.num_heads, Hkv, D, BS, NB,
+                              b.scale, k_head_scales=khs, v_head_scales=vhs)
+    kc = torch.zeros((NB, Hkv, BS, D), dtype=TORCH_DT[kv], device="cuda"); vc = torch.zeros_like(kc)
+    tk, tv = torch.from_numpy(khs).cuda(), torch.from_numpy(vhs).cuda()
+    for k_, v_, sl_ in ((hk, hv, b.hist_slots), (nk, nv, b.new_slots)):
+        pkv.reshape_and_cache_head_scales(to_dev(k_, "bf16"), to_dev(v_, "bf16"), kc, vc,
+                                          torch.from_numpy(sl_).cuda(), tk, tv)
+    out = torch.empty((b.num_seqs, sp.num_heads, D), dtype=torch.bfloat16, device="cuda")
+    ws = pkv.new_workspace(b.num_seqs, sp.num_heads, Hkv, D, parts)
+    pkv.paged_attention_decode_head_scales(out, to_dev(b.q, "bf16"), kc, vc, torch.from_numpy(b.block_tables).cuda(),
+                                           torch.from_numpy(b.seq_lens).cuda(), float(b.scale), tk, tv, parts, ws)
+    torch.cuda.synchronize()
+    assert pkv.read_device_error(ws) == 0
+    assert np.array_equal(cache_bytes(kc), okc) and np.array_equal(cache_bytes(vc), ovc)
+    G = sp.num_heads // Hkv
+    err = np.abs(to_f64(out) - ref).max(axis=(0, 2))                   # per query head
+    assert np.all(err <= TOL[kv] * np.repeat(gain, G)), err            # outputs scale with the head's V range
