@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
-DT = {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3}
-NP_DT = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8, "e5m2": np.uint8}
+DT = {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3, "int8": 4}
+NP_DT = {"f32": np.float32, "bf16": np.uint16, "e4m3": np.uint8, "e5m2": np.uint8, "int8": np.int8}
 
 _lib = None
 
@@ -45,6 +45,8 @@ def _bind(lib):
     lib.orc_e4m3_encode.restype = ctypes.c_uint8
     lib.orc_e4m3_encode_array.argtypes = [P, P, i64]
     lib.orc_e4m3_encode_array.restype = None
+    lib.orc_int8_encode.argtypes = [f32]
+    lib.orc_int8_encode.restype = ctypes.c_int8
     lib.orc_e5m2_value.argtypes = [ctypes.c_uint8]
     lib.orc_e5m2_value.restype = f64
     lib.orc_e5m2_encode_array.argtypes = [P, P, i64]

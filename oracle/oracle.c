@@ -40,6 +40,11 @@
  *               (xx != 0) = NaN, largest finite 57344; the same encode rule
  *               (round to nearest even, magnitudes at or above 57344 saturate
  *               to it, NaN stays NaN).
+ *   INT8 KV     the promptx.wiki tutorial's quantisation section also names
+ *               8-bit integer KV caches. Reading: symmetric, one scale per
+ *               tensor (or per KV head), code = clamp(round-half-even(x /
+ *               scale), -127, 127) with the division in binary32, value =
+ *               code * scale; NaN encodes to 0.
  *
  * Layouts (a reading: the pages give none):
  *   cache     [num_blocks][num_kv_heads][block_size][head_dim]
@@ -200,7 +205,24 @@ void orc_e5m2_encode_array(const float* x, uint8_t* codes, int64_t n)
         codes[i] = orc_e5m2_encode(x[i]);
 }
 
-static int is_fp8(int dtype) { return dtype == ORC_E4M3 || dtype == ORC_E5M2; }
+/* Symmetric 8-bit integer code: nearest integer to x (ties to even), clamped to +-127. */
+int8_t orc_int8_encode(float x)
+{
+    if (isnan(x))
+        return 0;
+    if (x >= 127.0f)
+        return 127;
+    if (x <= -127.0f)
+        return -127;
+    double r = floor((double)x);
+    double frac = (double)x - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))
+        r += 1.0;
+    return (int8_t)r;
+}
+
+/* the 8-bit caches: quantised with a scale */
+static int is_fp8(int dtype) { return dtype == ORC_E4M3 || dtype == ORC_E5M2 || dtype == ORC_INT8; }
 
 static double elem(const void* base, int dtype, size_t i, double scale)
 {
@@ -213,6 +235,8 @@ static double elem(const void* base, int dtype, size_t i, double scale)
         return orc_e4m3_value(((const uint8_t*)base)[i]) * scale;
     case ORC_E5M2:
         return orc_e5m2_value(((const uint8_t*)base)[i]) * scale;
+    case ORC_INT8:
+        return (double)((const int8_t*)base)[i] * scale;
     default:
         return NAN;
     }
@@ -237,7 +261,7 @@ int orc_paged_decode(double* out,
 {
     if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 || q_len < 1)
         return ORC_ERR_SHAPE;
-    if (is_fp8(q_dtype) || q_dtype < 0 || q_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
+    if (is_fp8(q_dtype) || q_dtype < 0 || q_dtype > 4 || kv_dtype < 0 || kv_dtype > 4)
         return ORC_ERR_DTYPE;
     const int group = num_heads / num_kv_heads;
     const int count = seqs ? n_seqs : num_seqs;
@@ -327,7 +351,7 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                           int block_size, int num_blocks, float k_scale, float v_scale,
                           const float* k_head_scales, const float* v_head_scales)
 {
-    if (is_fp8(in_dtype) || in_dtype < 0 || in_dtype > 3 || kv_dtype < 0 || kv_dtype > 3)
+    if (is_fp8(in_dtype) || in_dtype < 0 || in_dtype > 4 || kv_dtype < 0 || kv_dtype > 4)
         return ORC_ERR_DTYPE;
     if (!is_fp8(kv_dtype) && kv_dtype != in_dtype)
         return ORC_ERR_DTYPE;
@@ -360,6 +384,11 @@ int orc_reshape_and_cache(const void* k, const void* v, int in_dtype,
                 const float vx = (float)elem(v, in_dtype, src + i, 1.0);
                 const float ky = kx / (k_head_scales ? k_head_scales[h] : k_scale); /* binary32 division */
                 const float vy = vx / (v_head_scales ? v_head_scales[h] : v_scale);
+                if (kv_dtype == ORC_INT8) {
+                    ((int8_t*)k_cache)[dst + i] = orc_int8_encode(ky);
+                    ((int8_t*)v_cache)[dst + i] = orc_int8_encode(vy);
+                    continue;
+                }
                 ((uint8_t*)k_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(ky) : orc_e5m2_encode(ky);
                 ((uint8_t*)v_cache)[dst + i] = kv_dtype == ORC_E4M3 ? orc_e4m3_encode(vy) : orc_e5m2_encode(vy);
             }

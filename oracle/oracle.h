@@ -3,7 +3,7 @@
 #define PKV_ORACLE_H
 #include <stdint.h>
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2, ORC_E5M2 = 3 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2, ORC_E5M2 = 3, ORC_INT8 = 4 };
 enum { ORC_OK = 0, ORC_ERR_SHAPE = 1, ORC_ERR_DTYPE = 2, ORC_ERR_INDEX = 3, ORC_ERR_ALLOC = 4 };
 
 double orc_e4m3_value(uint8_t code);
@@ -12,6 +12,7 @@ void orc_e4m3_encode_array(const float* x, uint8_t* codes, int64_t n);
 double orc_e5m2_value(uint8_t code);
 uint8_t orc_e5m2_encode(float x);
 void orc_e5m2_encode_array(const float* x, uint8_t* codes, int64_t n);
+int8_t orc_int8_encode(float x);
 
 /* out: [len(seqs) or num_seqs][q_len][num_heads][head_dim] doubles, rows in the order
  * of `seqs` (all sequences when seqs == NULL); q: [num_seqs][q_len][num_heads][head_dim].

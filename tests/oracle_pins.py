@@ -501,6 +501,52 @@ def check_head_scales_equal_per_head_runs(lib):
     assert np.array_equal(same, same_h)
 
 
+# ------------------------------------------------------------- INT8 caches
+
+def check_int8_encode_vs_library(lib, n=200_000, seed=9):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal(n) * 60).astype(np.float32)
+    x = np.concatenate([x, np.arange(-130, 131, 0.5, dtype=np.float32)])        # every tie, both clamps
+    ref = np.clip(np.rint(x), -127, 127).astype(np.int8)                          # numpy rounds ties to even
+    got = np.array([lib.orc_int8_encode(float(v)) for v in x], dtype=np.int8)
+    assert np.array_equal(ref, got)
+    assert lib.orc_int8_encode(float("nan")) == 0
+
+
+def check_append_int8_vs_library(lib):
+    rng = np.random.default_rng(24)
+    T, Hkv, d, bs, nb = 40, 2, 32, 8, 8
+    k = rng.standard_normal((T, Hkv, d)).astype(np.float32) * 3
+    v = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    ks = np.float32(np.abs(k).max() / np.float32(127)); vs = np.float32(np.abs(v).max() / np.float32(127))
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    kc = oracle.empty_cache(nb, Hkv, bs, d, "int8"); vc = oracle.empty_cache(nb, Hkv, bs, d, "int8")
+    oracle.reshape_and_cache(k, v, "f32", kc, vc, "int8", slots, Hkv, d, bs, nb, ks, vs, lib=lib)
+    for t in range(T):
+        b, o = divmod(int(slots[t]), bs)
+        ek = np.clip(np.rint((k[t] / ks).astype(np.float32)), -127, 127).astype(np.int8)
+        ev = np.clip(np.rint((v[t] / vs).astype(np.float32)), -127, 127).astype(np.int8)
+        assert np.array_equal(kc[b, :, o, :], ek) and np.array_equal(vc[b, :, o, :], ev)
+
+
+def check_int8_attention_dequant(lib):
+    rng = np.random.default_rng(25)
+    nb, Hkv, bs, d, Hq = 6, 2, 8, 16, 4
+    kc = rng.integers(-127, 128, (nb, Hkv, bs, d), dtype=np.int8)
+    vc = rng.integers(-127, 128, (nb, Hkv, bs, d), dtype=np.int8)
+    ks, vs = np.float32(0.01), np.float32(0.003)
+    kf = kc.astype(np.float64) * float(ks); vf = vc.astype(np.float64) * float(vs)
+    q = rng.standard_normal((2, Hq, d)).astype(np.float32)
+    bt = np.array([[3, 1, 4], [0, 5, -1]], np.int32)
+    sl = np.array([20, 11], np.int32)
+    got = oracle.paged_decode(q, "f32", kc, vc, "int8", bt, sl, Hq, Hkv, d, bs, nb, 0.25, ks, vs, lib=lib)
+    for s in range(2):
+        L = int(sl[s])
+        K = np.concatenate([np.transpose(kf[bt[s, j]], (1, 0, 2)) for j in range(-(-L // bs))])[:L]
+        V = np.concatenate([np.transpose(vf[bt[s, j]], (1, 0, 2)) for j in range(-(-L // bs))])[:L]
+        assert np.allclose(got[s], sdpa_fp64(q[s], K, V, 0.25), rtol=0, atol=1e-12)
+
+
 ALL_CHECKS = [
     check_e4m3_decode_table, check_e4m3_spot_values, check_e4m3_encode_vs_library, check_e4m3_ties_to_even,
     check_e4m3_saturation_and_roundtrip, check_length_one_is_v, check_length_two_closed_form,
@@ -510,5 +556,6 @@ ALL_CHECKS = [
     check_e5m2_decode_table, check_e5m2_spot_values, check_e5m2_encode_vs_library,
     check_e5m2_ties_saturation_roundtrip, check_append_e5m2_vs_library, check_e5m2_attention_dequant,
     check_multi_query_matches_causal_sdpa, check_multi_query_is_decode_at_each_position,
-    check_head_scales_equal_per_head_runs,
+    check_head_scales_equal_per_head_runs, check_int8_encode_vs_library, check_append_int8_vs_library,
+    check_int8_attention_dequant,
 ]

@@ -43,6 +43,8 @@ MUTANTS = {
                          "double vlo = e5m2_pos[lo], vhi = e5m2_pos[hi];\n    double midpoint = 0.5 * (vlo + vhi);\n"
                          "    int code;\n    if (a < midpoint)\n        code = lo;\n    else if (a > midpoint)\n"
                          "        code = hi;\n    else\n        code = (lo & 1) ? lo : hi;"),
+    "int8_ties_away_from_zero": ("if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))", "if (frac >= 0.5)"),
+    "int8_clamps_at_128": ("    if (x >= 127.0f)\n        return 127;", "    if (x >= 128.0f)\n        return 127;"),
     "causal_limit_off_by_one": ("const int Lq = L - q_len + 1 + j;", "const int Lq = L - q_len + j;"),
     "e5m2_saturates_to_infinity": ("if (a >= e5m2_pos[123])\n        return sign | 123;",
                                    "if (a >= e5m2_pos[123])\n        return sign | 124;"),
