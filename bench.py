@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--partitions", type=int, default=0, help="decode runs (0 = automatic)")
     ap.add_argument("--q-len", type=int, default=1,
                     help="new tokens per sequence: > 1 times the causal multi-query decode instead of the step")
-    ap.add_argument("--kv-dtype", choices=["bf16", "e4m3", "e5m2"], default=None,
+    ap.add_argument("--kv-dtype", choices=["bf16", "e4m3", "e5m2", "int8"], default=None,
                     help="run the workload with this cache dtype instead of its own (configs 1-4)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -221,7 +221,8 @@ class DeviceState:
         self.new_k = self._dev(b.new_k, sp.in_dtype)
         self.new_v = self._dev(b.new_v, sp.in_dtype)
         self.new_slots = torch.from_numpy(b.new_slots).to(device)
-        cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8, "e5m2": torch.float8_e5m2}[sp.kv_dtype]
+        cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8, "e5m2": torch.float8_e5m2,
+               "int8": torch.int8}[sp.kv_dtype]
         shape = (b.num_blocks, sp.num_kv_heads, sp.block_size, sp.head_dim)
         self.kc = torch.zeros(shape, dtype=cdt, device=device)
         self.vc = torch.zeros(shape, dtype=cdt, device=device)
@@ -478,13 +479,13 @@ def ours_arm(args):
             "scaling": "weak",
             "vs_baseline": None,
             # arithmetic: tensor-core products in bf16 (E4M3 codes widened exactly to f16), fp32 sums
-            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "f16", "e5m2": "f16"}[spec.kv_dtype],
+            "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "f16", "e5m2": "f16", "int8": "f16"}[spec.kv_dtype],
             "data": "synthetic",
             "config": {
                 "workload": describe(b), "config_index": args.config,
                 "kv_storage": spec.kv_dtype, "partitions": args.partitions or pkv.default_partitions(
                     spec.head_dim, spec.block_size, spec.num_heads, spec.num_kv_heads,
-                    {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3}[spec.kv_dtype]),
+                    {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3, "int8": 4}[spec.kv_dtype]),
                 "step": (f"paged_attention_decode_mq: the last {args.q_len} tokens of every sequence as queries, "
                          "causal within the chunk (their K/V already cached)" if args.q_len > 1 else
                          "paged_decode_step: append of one new token per sequence fused into the paged "

@@ -83,7 +83,10 @@ typedef enum {
 /* PKV_FP8_E5M2: OCP E5M2 codes (bias 15, largest finite 57344), per-tensor
  * scales like E4M3; decoded by the tensor-core kernel only (bf16 q, head_dim
  * 128, block 16 or 32); other shapes return PKV_ERR_SHAPE / PKV_ERR_DTYPE. */
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3 } pkv_dtype;
+/* PKV_INT8: symmetric 8-bit integer codes, code = clamp(round-half-even(x /
+ * scale), -127, 127), value = code * scale; per-tensor or per-KV-head scales
+ * like the FP8 formats, same shapes as PKV_FP8_E5M2. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3, PKV_INT8 = 4 } pkv_dtype;
 
 /* Bits of the device error word. */
 #define PKV_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks): block skipped */

@@ -24,12 +24,12 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpagedkv.so")
 
-F32, BF16, FP8_E4M3, FP8_E5M2 = 0, 1, 2, 3
+F32, BF16, FP8_E4M3, FP8_E5M2, INT8 = 0, 1, 2, 3, 4
 DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 # uint8 caches hold E4M3 codes; E5M2 caches are passed as torch.float8_e5m2 tensors
 _TORCH_DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3,
-                torch.float8_e5m2: FP8_E5M2}
+                torch.float8_e5m2: FP8_E5M2, torch.int8: INT8}
 
 _lib = None
 

@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import numpy as np
 
-ELT = {"f32": 4, "bf16": 2, "e4m3": 1, "e5m2": 1}
+ELT = {"f32": 4, "bf16": 2, "e4m3": 1, "e5m2": 1, "int8": 1}
 
 
 def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, elt_bytes: int) -> int:

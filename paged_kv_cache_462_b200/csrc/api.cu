@@ -66,7 +66,8 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool is_fp8(int dtype) { return dtype == PKV_FP8_E4M3 || dtype == PKV_FP8_E5M2; }
+// 8-bit caches quantised with scales (FP8 formats and INT8)
+bool is_fp8(int dtype) { return dtype == PKV_FP8_E4M3 || dtype == PKV_FP8_E5M2 || dtype == PKV_INT8; }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -269,7 +270,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
          !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads))))
         return PKV_ERR_SHAPE;   // per-head scales: both arrays, FP8 caches, tensor-core kernel
     if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
-          (q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2))))
+          (q_dtype == PKV_BF16 && is_fp8(kv_dtype))))
         return PKV_ERR_DTYPE;
     if (num_seqs == 0)
         return PKV_OK;
@@ -308,7 +309,7 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
     if (workspace_bytes < lay.bytes)
         return PKV_ERR_WORKSPACE;
 
-    const bool fp8 = kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2;
+    const bool fp8 = is_fp8(kv_dtype);
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
     p.out = out;

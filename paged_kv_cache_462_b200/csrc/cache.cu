@@ -13,8 +13,10 @@
 // division) is converted with the hardware round-to-nearest-even, saturating
 // conversion (cuda_fp8.h), 8 codes per 8-byte store.
 #include <cstdint>
+#include <type_traits>
 
 #include "device.cuh"
+
 #include "pkv_internal.h"
 
 namespace pkv {
@@ -50,10 +52,12 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
         const long long blk = slot / block_size, off = slot - blk * block_size;
         const TIN* src = (is_v ? v : k) + ((long long)t * num_kv_heads + h) * head_dim + c * 8;
         TC* dst = (is_v ? vc : kc) + ((blk * num_kv_heads + h) * block_size + off) * head_dim + c * 8;
-        if constexpr (sizeof(TC) == 1)
-            quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst),
-                        is_v ? (v_head_scales ? __ldg(v_head_scales + h) : v_scale)
-                             : (k_head_scales ? __ldg(k_head_scales + h) : k_scale));
+        const float sc = is_v ? (v_head_scales ? __ldg(v_head_scales + h) : v_scale)
+                              : (k_head_scales ? __ldg(k_head_scales + h) : k_scale);
+        if constexpr (std::is_same<TC, int8_t>::value)
+            quant8_i8(src, reinterpret_cast<uint8_t*>(dst), sc);
+        else if constexpr (sizeof(TC) == 1)
+            quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), sc);
         else
             copy8(src, dst);
     }
@@ -105,6 +109,14 @@ int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, c
         return launch_cache<__nv_bfloat16, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
                                                                num_kv_heads, head_dim, block_size, num_blocks,
                                                                k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
+    if (in_dtype == PKV_F32 && kv_dtype == PKV_INT8)
+        return launch_cache<float, int8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                           block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales,
+                                           err, stream);
+    if (in_dtype == PKV_BF16 && kv_dtype == PKV_INT8)
+        return launch_cache<__nv_bfloat16, int8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
+                                                   head_dim, block_size, num_blocks, k_scale, v_scale,
+                                                   k_head_scales, v_head_scales, err, stream);
     return PKV_ERR_DTYPE;
 }
 

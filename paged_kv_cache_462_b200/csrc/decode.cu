@@ -15,6 +15,8 @@ int decode_mma_dispatch_e4m3(int D, int BS, int G, int HG, const DecodeParams& p
                              int* occ);
 int decode_mma_dispatch_e5m2(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
                              int* occ);
+int decode_mma_dispatch_i8(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
+                           int* occ);
 
 int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
                         cudaStream_t st, int* occ)
@@ -25,12 +27,14 @@ int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const Decode
         return decode_mma_dispatch_e4m3(D, BS, G, HG, p, nruns, st, occ);
     if (kv_dtype == PKV_FP8_E5M2)
         return decode_mma_dispatch_e5m2(D, BS, G, HG, p, nruns, st, occ);
+    if (kv_dtype == PKV_INT8)
+        return decode_mma_dispatch_i8(D, BS, G, HG, p, nruns, st, occ);
     return PKV_ERR_DTYPE;
 }
 
 bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)
 {
-    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3 && kv_dtype != PKV_FP8_E5M2)
+    if (kv_dtype != PKV_BF16 && kv_dtype != PKV_FP8_E4M3 && kv_dtype != PKV_FP8_E5M2 && kv_dtype != PKV_INT8)
         return false;
     if (block_size != 16 && block_size != 32)
         return false;

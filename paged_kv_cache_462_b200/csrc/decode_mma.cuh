@@ -85,11 +85,18 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
     }
 }
 
-// two FP8 codes (low byte first) -> f16x2, exact for both formats
+// two 8-bit codes (low byte first) -> f16x2, exact for E4M3, E5M2 and INT8
 template <class KV>
 __device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two_codes)
 {
     uint32_t r;
+    if constexpr (KV::kInt8) {
+        // the offset byte x + 128 as the mantissa of 1024.0: f16 value 1152 + x, less 1152 (exact)
+        r = __byte_perm(two_codes ^ 0x8080u, 0x64646464u, 0x4140);
+        const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&r), __halves2half2(__ushort_as_half(0x6480),
+                                                                                      __ushort_as_half(0x6480)));
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
     const uint16_t v = static_cast<uint16_t>(two_codes);
     if constexpr (KV::kFmt == __NV_E5M2)
         asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(r) : "h"(v));
@@ -127,7 +134,16 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map)
 // Decode-step append fused into the producer warp: write the new token of sequence s (row s of
 // new_k / new_v) for KV heads h0 .. h0+nh-1 into its slot, with the conversion reshape_and_cache
 // uses, then order those writes before this warp's later TMA reads of the same block.
-template <class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3>
+template <__nv_fp8_interpretation_t FMT, bool INT8, class TIN>
+__device__ __forceinline__ void quant8_any(const TIN* src, uint8_t* dst, float scale)
+{
+    if constexpr (INT8)
+        quant8_i8(src, dst, scale);
+    else
+        quant8<FMT>(src, dst, scale);
+}
+
+template <class TC, __nv_fp8_interpretation_t FMT = __NV_E4M3, bool INT8 = false>
 __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0, int nh, int D, int BS, int lane,
                                             long long slot)
 {
@@ -144,12 +160,12 @@ __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0
         if (p.in_dtype == PKV_F32) {
             const float* src = static_cast<const float*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
+                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
                                                          : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
         } else {
             const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8<FMT>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
+                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
                                                          : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
             else
                 copy8(src, reinterpret_cast<__nv_bfloat16*>(dst));
@@ -176,7 +192,7 @@ __device__ __forceinline__ void append_new_token_impl(const DecodeParams& p, int
             if (lane == 0)
                 atomicOr(p.err, PKV_DEVERR_SLOT);
         } else if constexpr (KV::kBytes == 1) {
-            append_rows<uint8_t, KV::kFmt>(p, s, h0, nh, D, BS, lane, slot);
+            append_rows<uint8_t, KV::kFmt, KV::kInt8>(p, s, h0, nh, D, BS, lane, slot);
         } else {
             append_rows<__nv_bfloat16>(p, s, h0, nh, D, BS, lane, slot);
         }
@@ -911,7 +927,7 @@ struct MmaLauncher {
         const long long rows = (long long)p.num_blocks * p.num_kv_heads * BS;
         int kvdt = PKV_BF16;
         if constexpr (KV::kBytes == 1)
-            kvdt = KV::kFmt == __NV_E5M2 ? PKV_FP8_E5M2 : PKV_FP8_E4M3;
+            kvdt = KV::kInt8 ? PKV_INT8 : KV::kFmt == __NV_E5M2 ? PKV_FP8_E5M2 : PKV_FP8_E4M3;
         CUtensorMap kmap, vmap;
         if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, D, rows, C::kRows) ||
             !make_cache_tensormap(&vmap, p.v_cache, kvdt, D, rows, C::kRows))

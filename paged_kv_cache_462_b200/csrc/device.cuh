@@ -136,16 +136,19 @@ constexpr float kE4M3Unbias = 1.329227995784915872903807060280344576e36f;  // 2^
 
 struct KvF32 {
     using T = float;
+    static constexpr bool kInt8 = false;
     static constexpr int kBytes = 4;
     static constexpr float kUnbias = 1.0f;
 };
 struct KvBF16 {
     using T = __nv_bfloat16;
+    static constexpr bool kInt8 = false;
     static constexpr int kBytes = 2;
     static constexpr float kUnbias = 1.0f;
 };
 struct KvE4M3 {
     using T = uint8_t;
+    static constexpr bool kInt8 = false;
     static constexpr int kBytes = 1;
     static constexpr float kUnbias = kE4M3Unbias;
     static constexpr __nv_fp8_interpretation_t kFmt = __NV_E4M3;
@@ -153,8 +156,16 @@ struct KvE4M3 {
 // OCP E5M2 codes (tensor-core kernel only: widened exactly to f16 there)
 struct KvE5M2 {
     using T = uint8_t;
+    static constexpr bool kInt8 = false;
     static constexpr int kBytes = 1;
     static constexpr __nv_fp8_interpretation_t kFmt = __NV_E5M2;
+};
+// symmetric INT8 codes (tensor-core kernel only: widened exactly to f16 there)
+struct KvI8 {
+    using T = uint8_t;
+    static constexpr bool kInt8 = true;
+    static constexpr int kBytes = 1;
+    static constexpr __nv_fp8_interpretation_t kFmt = __NV_E4M3;   // unused for integers
 };
 
 __device__ __forceinline__ void widen_word(KvF32, uint32_t w, float* f) { f[0] = __uint_as_float(w); }
@@ -323,6 +334,28 @@ __device__ __forceinline__ void quant8(const TIN* src, uint8_t* dst, float scale
     *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
 }
 
+
+// 8 values -> 8 symmetric INT8 codes: x / scale (IEEE fp32 division), nearest integer with ties
+// to even, clamped to +-127; NaN -> 0
+template <class TIN>
+__device__ __forceinline__ void quant8_i8(const TIN* src, uint8_t* dst, float scale)
+{
+    float f[8];
+    load8(src, f);
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float y = __fdiv_rn(f[4 * h + i], scale);
+            const int c = (y != y) ? 0 : __float2int_rn(fminf(fmaxf(y, -127.0f), 127.0f));
+            packed |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * i);
+        }
+        w[h] = packed;
+    }
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+}
 
 __device__ __forceinline__ float to_float(float x) { return x; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }

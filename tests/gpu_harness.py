@@ -7,8 +7,9 @@ import torch
 import oracle
 import paged_kv_cache_462_b200 as pkv
 
-TOL = {"f32": 1e-5, "bf16": 1e-2, "e4m3": 3e-2, "e5m2": 3e-2}   # max |gpu - oracle| per cache dtype
-TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8, "e5m2": torch.float8_e5m2}
+TOL = {"f32": 1e-5, "bf16": 1e-2, "e4m3": 3e-2, "e5m2": 3e-2, "int8": 3e-2}   # max |gpu - oracle| per cache dtype
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8, "e5m2": torch.float8_e5m2,
+            "int8": torch.int8}
 
 
 def to_dev(a: np.ndarray, name: str, device="cuda") -> torch.Tensor:
@@ -16,6 +17,8 @@ def to_dev(a: np.ndarray, name: str, device="cuda") -> torch.Tensor:
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
     if name == "f32":
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+    if name == "int8":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int8)).to(device)
     if name == "e5m2":
         return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).to(device).view(torch.float8_e5m2)
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).to(device)

@@ -481,7 +481,7 @@ def test_multi_query_unsupported_shapes_are_rejected():
 
 # ------------------------------------------------------------------ per-KV-head FP8 scales
 
-@pytest.mark.parametrize("kv", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
 @pytest.mark.parametrize("parts", [0, 5])
 def test_head_scales_append_and_decode(kv, parts):
     """FP8 caches with one scale per KV head (heads of very different ranges): appends bit-exact
@@ -494,7 +494,7 @@ def test_head_scales_append_and_decode(kv, parts):
         f = W.bf16_bits_to_f32(x) * gain[None, :, None]
         return W.f32_to_bf16_bits(f.astype(np.float32))
     hk, hv, nk, nv = rows(b.hist_k), rows(b.hist_v), rows(b.new_k), rows(b.new_v)
-    top = 448.0 if kv == "e4m3" else 57344.0
+    top = {"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[kv]
     def head_absmax(*xs):
         return np.max([np.abs(W.bf16_bits_to_f32(x)).max(axis=(0, 2)) for x in xs], axis=0)
     khs = (head_absmax(hk, nk) / np.float32(top)).astype(np.float32)
@@ -520,3 +520,50 @@ def test_head_scales_append_and_decode(kv, parts):
     G = sp.num_heads // Hkv
     err = np.abs(to_f64(out) - ref).max(axis=(0, 2))                   # per query head
     assert np.all(err <= TOL[kv] * np.repeat(gain, G)), err            # outputs scale with the head's V range
+
+
+# ------------------------------------------------------------------ INT8 caches
+
+@pytest.mark.parametrize("inp", ["bf16", "f32"])
+def test_append_int8_bit_exact(inp):
+    rng = np.random.default_rng(7)
+    T, Hkv, D, BS, NB = 300, 4, 128, 16, 40
+    rows_k = rng.standard_normal((T, Hkv, D)).astype(np.float32) * 3
+    rows_v = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+    if inp == "f32":                                        # ties, clamps, NaN and infinities too
+        rows_k[0, 0, :12] = [0.5, 1.5, 2.5, -0.5, -2.5, 126.5, 127.5, 300.0, -300.0, np.nan, np.inf, -np.inf]
+    if inp == "bf16":
+        rows_k, rows_v = W.f32_to_bf16_bits(rows_k), W.f32_to_bf16_bits(rows_v)
+    slots = rng.permutation(NB * BS)[:T].astype(np.int64)
+    slots[::7] = -1
+    slots[0] = 5
+    ks = np.float32(1.0) if inp == "f32" else np.float32(3 * 4.5 / 127)
+    vs = np.float32(4.5 / 127)
+    okc = oracle.empty_cache(NB, Hkv, BS, D, "int8"); ovc = oracle.empty_cache(NB, Hkv, BS, D, "int8")
+    oracle.reshape_and_cache(rows_k, rows_v, inp, okc, ovc, "int8", slots, Hkv, D, BS, NB, ks, vs)
+    kc = torch.zeros(okc.shape, dtype=torch.int8, device="cuda"); vc = torch.zeros_like(kc)
+    pkv.reshape_and_cache(to_dev(rows_k, inp), to_dev(rows_v, inp), kc, vc, torch.from_numpy(slots).cuda(),
+                          float(ks), float(vs))
+    assert np.array_equal(cache_bytes(kc), okc) and np.array_equal(cache_bytes(vc), ovc)
+
+
+@pytest.mark.parametrize("BS", [16, 32])
+@pytest.mark.parametrize("G", [1, 4, 5, 8])
+def test_int8_shapes(BS, G):
+    Hkv = 2
+    lengths = [0, 1, BS, BS + 1, 3 * BS - 1, 97, 200]
+    b = W.build_batch(_spec(f"int8_{BS}_{G}", len(lengths), G * Hkv, Hkv, 128, BS, "int8", lengths,
+                            seed=7000 + BS * 10 + G))
+    g, _ = _check_step(b, partitions=(0, 5))
+    assert np.all(g.out.float().cpu().numpy()[0] == 0)
+
+
+@pytest.mark.parametrize("cfg,over", [(1, dict(num_seqs=6)), (4, dict(num_seqs=5)), (3, dict(num_seqs=16))])
+def test_int8_workloads_fused_step(cfg, over):
+    b = W.config_batch(cfg, kv_dtype="int8", **over)
+    ref, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    out = g.fused_step(0)
+    assert g.device_errors() == 0
+    assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
+    assert max_err(out, ref) <= TOL["int8"]

@@ -40,7 +40,7 @@ import numpy as np
 
 BASE_SEED = 462_000
 
-DTYPES = ("f32", "bf16", "e4m3", "e5m2")
+DTYPES = ("f32", "bf16", "e4m3", "e5m2", "int8")
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -73,7 +73,7 @@ class Spec:
     block_size: int
     q_dtype: str            # "f32" | "bf16"
     in_dtype: str           # dtype of appended k/v rows: "f32" | "bf16"
-    kv_dtype: str           # cache dtype: "f32" | "bf16" | "e4m3" | "e5m2"
+    kv_dtype: str           # cache dtype: "f32" | "bf16" | "e4m3" | "e5m2" | "int8"
     lengths: tuple          # ("uniform", lo, hi) | ("fixed", L) | ("lognormal", median, sigma, lo, hi) | ("list", (...))
     pool: tuple             # ("fixed", num_blocks) | ("double_unique", round_to)
     share_group: int = 0    # sequences per prefix-sharing group (0 = none)
@@ -256,10 +256,10 @@ def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
             pos = L - 1
             new_slots[s] = int(tables[s, pos // bs]) * bs + pos % bs
 
-    if spec.kv_dtype in ("e4m3", "e5m2"):
+    if spec.kv_dtype in ("e4m3", "e5m2", "int8"):
         # per-tensor scales: absmax of every K (V) value written to the cache maps to the format's
-        # largest finite value (448 for E4M3, 57344 for E5M2)
-        top = np.float32(448.0 if spec.kv_dtype == "e4m3" else 57344.0)
+        # largest finite value (448 for E4M3, 57344 for E5M2, 127 for INT8)
+        top = np.float32({"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[spec.kv_dtype])
         k_scale = np.float32(max(_absmax(hist_k, spec.in_dtype), _absmax(new_k, spec.in_dtype)) / top)
         v_scale = np.float32(max(_absmax(hist_v, spec.in_dtype), _absmax(new_v, spec.in_dtype)) / top)
     else:
