@@ -88,35 +88,27 @@ int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, c
                    int kv_dtype, float k_scale, float v_scale, const float* k_head_scales,
                    const float* v_head_scales, int32_t* err, cudaStream_t stream)
 {
+#define PKV_CACHE(TIN, TC, ...)                                                                               \
+    return launch_cache<TIN, TC, ##__VA_ARGS__>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, \
+                                                head_dim, block_size, num_blocks, k_scale, v_scale,            \
+                                                k_head_scales, v_head_scales, err, stream)
     if (in_dtype == PKV_F32 && kv_dtype == PKV_F32)
-        return launch_cache<float, float>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                          block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(float, float);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_BF16)
-        return launch_cache<__nv_bfloat16, __nv_bfloat16>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
-                                                          num_kv_heads, head_dim, block_size, num_blocks, k_scale,
-                                                          v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(__nv_bfloat16, __nv_bfloat16);
     if (in_dtype == PKV_F32 && kv_dtype == PKV_FP8_E4M3)
-        return launch_cache<float, uint8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                            block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(float, uint8_t);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3)
-        return launch_cache<__nv_bfloat16, uint8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
-                                                    head_dim, block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(__nv_bfloat16, uint8_t);
     if (in_dtype == PKV_F32 && kv_dtype == PKV_FP8_E5M2)
-        return launch_cache<float, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
-                                                       num_kv_heads, head_dim, block_size, num_blocks, k_scale,
-                                                       v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(float, uint8_t, __NV_E5M2);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E5M2)
-        return launch_cache<__nv_bfloat16, uint8_t, __NV_E5M2>(k, v, k_cache, v_cache, slot_mapping, num_tokens,
-                                                               num_kv_heads, head_dim, block_size, num_blocks,
-                                                               k_scale, v_scale, k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(__nv_bfloat16, uint8_t, __NV_E5M2);
     if (in_dtype == PKV_F32 && kv_dtype == PKV_INT8)
-        return launch_cache<float, int8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                           block_size, num_blocks, k_scale, v_scale, k_head_scales, v_head_scales,
-                                           err, stream);
+        PKV_CACHE(float, int8_t);
     if (in_dtype == PKV_BF16 && kv_dtype == PKV_INT8)
-        return launch_cache<__nv_bfloat16, int8_t>(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
-                                                   head_dim, block_size, num_blocks, k_scale, v_scale,
-                                                   k_head_scales, v_head_scales, err, stream);
+        PKV_CACHE(__nv_bfloat16, int8_t);
+#undef PKV_CACHE
     return PKV_ERR_DTYPE;
 }
 

@@ -157,16 +157,16 @@ __device__ __forceinline__ void append_rows(const DecodeParams& p, int s, int h0
         const int h = h0 + r / pieces, c = r % pieces;
         const long long src_off = ((long long)s * p.num_kv_heads + h) * D + c * 8;
         TC* dst = (is_v ? vc : kc) + ((blk * p.num_kv_heads + h) * BS + off) * D + c * 8;
+        const float sc = is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
+                              : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale);
         if (p.in_dtype == PKV_F32) {
             const float* src = static_cast<const float*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
-                                                         : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
+                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), sc);
         } else {
             const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(is_v ? p.new_v : p.new_k) + src_off;
             if constexpr (sizeof(TC) == 1)
-                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), is_v ? (p.v_head_scales ? __ldg(p.v_head_scales + h) : p.v_scale_in)
-                                                         : (p.k_head_scales ? __ldg(p.k_head_scales + h) : p.k_scale));
+                quant8_any<FMT, INT8>(src, reinterpret_cast<uint8_t*>(dst), sc);
             else
                 copy8(src, reinterpret_cast<__nv_bfloat16*>(dst));
         }
