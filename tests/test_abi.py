@@ -95,3 +95,32 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         pkv.paged_attention_decode(q.clone(), q, kc, kc.clone(), torch.zeros(1, 4, dtype=torch.int32),
                                    torch.ones(1, dtype=torch.int32), 0.125, workspace=torch.zeros(1 << 20, dtype=torch.uint8))
+
+
+def test_multi_query_and_head_scale_host_validation(lib):
+    mq = lib.paged_attention_decode_mq
+    args = lambda **kw: [kw.get(n, d) for n, d in (
+        ("out", FAKE), ("q", FAKE), ("k", FAKE), ("v", FAKE), ("bt", FAKE), ("sl", FAKE), ("S", 4), ("QL", 2),
+        ("Hq", 8), ("Hkv", 2), ("D", 128), ("BS", 16), ("scale", 0.1), ("MB", 4), ("NB", 32), ("qdt", 1),
+        ("kvdt", 1), ("ks", 1.0), ("vs", 1.0), ("parts", 0), ("ws", FAKE), ("wsb", 1 << 20), ("stream", None))]
+    assert mq(*args(QL=0)) == 2 and mq(*args(QL=9)) == 2      # 1 <= q_len <= 8
+    assert mq(*args(QL=3, Hq=4)) == 2                          # 3 tokens x 2 heads = 6 columns
+    assert mq(*args(QL=2, BS=8)) == 2                          # tensor-core shapes only
+    assert mq(*args(QL=2, qdt=0, kvdt=0)) == 2                 # f32: no multi-query form
+    hs = lib.paged_attention_decode_head_scales
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8, 2, 128, 16, 0.1, 4, 32, 1]
+    assert hs(*base, 2, None, FAKE, 0, FAKE, 1 << 20, None) == 1             # a scale array missing
+    assert hs(*base, 1, FAKE, FAKE, 0, FAKE, 1 << 20, None) == 2             # bf16 cache: no head scales
+    rc = lib.reshape_and_cache_head_scales
+    assert rc(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 1, FAKE, FAKE, None, None) == 3   # bf16 cache
+    assert rc(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 4, None, FAKE, None, None) == 1   # null scales
+
+
+def test_int8_and_e5m2_dtype_pairs(lib):
+    ptrs = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, ws=FAKE, wsb=1 << 20)
+    assert _decode(lib, **ptrs, qdt=0, kvdt=4) == 3            # f32 q with an INT8 cache
+    assert _decode(lib, **ptrs, qdt=4, kvdt=4) == 3            # INT8 q
+    assert _decode(lib, **ptrs, qdt=3, kvdt=3) == 3            # E5M2 q
+    f = lib.reshape_and_cache
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 4, 0.0, 1.0, None, None) == 2   # zero INT8 scale
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 4, 4, 1.0, 1.0, None, None) == 3   # INT8 input rows
