@@ -85,6 +85,41 @@ PKV_API int pkv_bm_step(pkv_block_manager* bm, const int64_t* seq_ids, int n, in
 PKV_API int pkv_bm_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n, int32_t* block_tables,
                           int32_t* seq_lens);
 
+/*
+ * Shared-prefix plan of one decode batch (host buffers in, host buffers out,
+ * all caller-owned; no device access). The pages' prefix caching reuses whole
+ * blocks (wzjinhao.cn vLLM write-up, section 2.3; "vLLM inference cost
+ * optimisation", section 11): sequences whose tables hold the same physical
+ * block hold the same tokens there, so one pass over that block can serve the
+ * queries of all of them. This call finds those blocks; the decode of a group
+ * then reads each one once and merges it with every member's own remainder.
+ *
+ * Rule (a reading; the pages give no grouping procedure): only full blocks
+ * count (block j of sequence s when (j + 1) * block_size <= seq_lens[s] and
+ * the entry is >= 0). Candidates are the sequences whose first block is full,
+ * bucketed by its id (buckets in order of their first sequence), each bucket
+ * cut into chunks of max_group sequences in index order; a chunk of one stays
+ * alone. In a chunk, for j = 0, 1, ...: among the members still sharing, take
+ * the id that most of them hold at j (ties: the first such member's id); stop
+ * when no id is held by two; the members holding it keep sharing.
+ *
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq], -1 padded (the decode's tables)
+ *   seq_lens       int32 [num_seqs]
+ *   group_members  int32 [num_seqs]   out: member sequence indices, group after group
+ *   group_offsets  int32 [num_seqs + 1] out: group g = members [offsets[g], offsets[g + 1])
+ *   group_tables   int32 [num_seqs][max_blocks_per_seq] out: row g = the group's shared
+ *                  blocks, -1 padded (rows >= *num_groups untouched)
+ *   group_lens     int32 [num_seqs]   out: tokens in row g's blocks (blocks x block_size)
+ *   shared_blocks  int32 [num_seqs]   out: leading blocks of sequence s read through its
+ *                  group's row (they equal its own table's); 0 = outside every group
+ * Returns PKV_OK, PKV_ERR_NULL, or PKV_ERR_SHAPE (num_seqs < 0, a size <= 0 or
+ * max_group < 1). max_group 1 makes no groups.
+ */
+PKV_API int pkv_prefix_plan(const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int max_group, int32_t* group_members,
+                            int32_t* group_offsets, int32_t* group_tables, int32_t* group_lens,
+                            int32_t* shared_blocks, int* num_groups);
+
 #ifdef __cplusplus
 }
 #endif

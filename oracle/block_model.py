@@ -102,3 +102,52 @@ class BlockModel:
                 cows.append((src, dst))
         tables = [self.seqs[s][1] + [-1] * (self.max_blocks - len(self.seqs[s][1])) for s in ids]
         return OK, slots, tables, [self.seqs[s][0] for s in ids], cows, len(ids)
+
+
+def prefix_plan(tables, lens, bs: int, max_group: int):
+    """Shared-prefix groups of one decode batch: [(members, group_table, shared)], where
+    ``shared[i]`` = leading blocks member i reads through ``group_table`` instead of its own.
+
+    Reading of the pages' block-granular prefix sharing (wzjinhao.cn write-up, section 2.3;
+    "vLLM inference cost optimisation", section 11): sequences whose tables hold the same
+    physical block hold the same tokens there, so one pass over that block can serve all of
+    them. Only full blocks count (j + 1 <= len / bs). Candidates: sequences whose first block
+    is full, bucketed by its id (buckets in order of first appearance), each bucket cut into
+    chunks of max_group in index order; a chunk of one is left alone. Within a chunk, walk
+    j = 0, 1, ...: among the members still sharing, take the id held at j by the most of
+    them (ties: the first such member's id); stop when no id is held by two; the members
+    holding it stay. No arithmetic of the attention lives here."""
+    def full(s, j):
+        return j < len(tables[s]) and (j + 1) * bs <= lens[s] and tables[s][j] >= 0
+
+    buckets, order = {}, []
+    for s in range(len(lens)):
+        if full(s, 0):
+            b = int(tables[s][0])
+            if b not in buckets:
+                buckets[b] = []
+                order.append(b)
+            buckets[b].append(s)
+    groups = []
+    for b in order:
+        members = buckets[b]
+        for c0 in range(0, len(members), max(1, max_group)):
+            chunk = members[c0:c0 + max(1, max_group)]
+            if len(chunk) < 2:
+                continue
+            active, shared, table, j = list(chunk), {s: 0 for s in chunk}, [], 0
+            while True:
+                ids = [int(tables[s][j]) for s in active if full(s, j)]
+                best, best_n = None, 1
+                for x in ids:
+                    if ids.count(x) > best_n:
+                        best, best_n = x, ids.count(x)
+                if best is None:
+                    break
+                table.append(best)
+                active = [s for s in active if full(s, j) and tables[s][j] == best]
+                for s in active:
+                    shared[s] = j + 1
+                j += 1
+            groups.append((chunk, table, [shared[s] for s in chunk]))
+    return groups

@@ -31,8 +31,9 @@ def _lib():
         lib.pkv_bm_ref_count.argtypes = [P, i32]
         lib.pkv_bm_step.argtypes = [P, P, i32, P, P, P, P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         lib.pkv_bm_tables.argtypes = [P, P, i32, P, P]
+        lib.pkv_prefix_plan.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, ctypes.POINTER(ctypes.c_int)]
         for n in ("pkv_bm_add", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_num_free", "pkv_bm_seq_len",
-                  "pkv_bm_ref_count", "pkv_bm_step", "pkv_bm_tables"):
+                  "pkv_bm_ref_count", "pkv_bm_step", "pkv_bm_tables", "pkv_prefix_plan"):
             getattr(lib, n).restype = i32
         _bound = True
     return lib
@@ -107,3 +108,42 @@ class BlockManager:
         lens = np.zeros(ids.size, dtype=np.int32)
         st = self._lib.pkv_bm_tables(self._h, ids.ctypes.data, ids.size, tables.ctypes.data, lens.ctypes.data)
         return st, tables, lens
+
+
+class PrefixPlan:
+    """Output of pkv_prefix_plan: ``members[offsets[g]:offsets[g + 1]]`` share row g of
+    ``tables`` (``lens[g]`` tokens); sequence s reads its first ``shared[s]`` blocks there."""
+
+    def __init__(self, members, offsets, tables, lens, shared, num_groups):
+        self.num_groups = num_groups
+        self.members, self.offsets = members, offsets[: num_groups + 1]
+        self.tables, self.lens, self.shared = tables[:num_groups], lens[:num_groups], shared
+
+    def groups(self):
+        """[(members, shared block ids, per-member shared counts)] in group order."""
+        out = []
+        for g in range(self.num_groups):
+            m = self.members[self.offsets[g]:self.offsets[g + 1]].tolist()
+            t = self.tables[g][self.tables[g] >= 0].tolist()
+            out.append((m, t, [int(self.shared[s]) for s in m]))
+        return out
+
+
+def prefix_plan(block_tables, seq_lens, block_size: int, max_group: int) -> PrefixPlan:
+    """Group the sequences of one decode batch by the full physical blocks they share
+    (host arrays: block_tables int32 [n, max_blocks], seq_lens int32 [n])."""
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    n, mb = bt.shape
+    members = np.zeros(n, dtype=np.int32)
+    offsets = np.zeros(n + 1, dtype=np.int32)
+    tables = np.full((max(n, 1), mb), -1, dtype=np.int32)
+    lens = np.zeros(max(n, 1), dtype=np.int32)
+    shared = np.zeros(n, dtype=np.int32)
+    ng = ctypes.c_int(0)
+    st = _lib().pkv_prefix_plan(bt.ctypes.data, sl.ctypes.data, n, mb, block_size, max_group, members.ctypes.data,
+                                offsets.ctypes.data, tables.ctypes.data, lens.ctypes.data, shared.ctypes.data,
+                                ctypes.byref(ng))
+    if st != 0:
+        raise PkvError("pkv_prefix_plan", st)
+    return PrefixPlan(members, offsets, tables, lens, shared, ng.value)

@@ -178,12 +178,18 @@ def _absmax(x: np.ndarray, dtype_name: str) -> np.float32:
     return np.float32(np.abs(x).max())
 
 
-def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
-    """Draw one batch. Draw order: lengths, pool permutation, q, K, V, new k, new v."""
-    rng = np.random.default_rng(spec.seed if seed is None else seed)
-    S, Hq, Hkv, d, bs = spec.num_seqs, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
-    assert Hq % Hkv == 0
+@dataclass
+class Layout:
+    """Lengths and block tables of a batch, before any tensor is drawn."""
+    seq_lens: np.ndarray          # int32 [S]
+    block_tables: np.ndarray      # int32 [S, MB], -1 padded
+    num_blocks: int
+    shared_n: np.ndarray          # int64 [S]: leading blocks taken from the group's shared prefix
+    groups: list                  # [(members, blocks in the group's shared prefix)]
 
+
+def _layout(spec: Spec, rng: np.random.Generator) -> Layout:
+    S, bs = spec.num_seqs, spec.block_size
     seq_lens = _draw_lengths(spec, rng)
     nb = (seq_lens.astype(np.int64) + bs - 1) // bs
     MB = spec.max_blocks_per_seq or int(max(1, nb.max()))
@@ -229,6 +235,23 @@ def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
             tables[s, :n] = perm[nxt:nxt + n]
             nxt += n
     assert nxt == unique
+    return Layout(seq_lens, tables, num_blocks, shared_n, groups)
+
+
+def batch_layout(spec: Spec, seed: int | None = None) -> Layout:
+    """The lengths and tables ``build_batch`` draws for ``spec`` (same seed, same values)."""
+    return _layout(spec, np.random.default_rng(spec.seed if seed is None else seed))
+
+
+def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
+    """Draw one batch. Draw order: lengths, pool permutation, q, K, V, new k, new v."""
+    rng = np.random.default_rng(spec.seed if seed is None else seed)
+    S, Hq, Hkv, d, bs = spec.num_seqs, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
+    assert Hq % Hkv == 0
+    lay = _layout(spec, rng)
+    seq_lens, tables, num_blocks, groups = lay.seq_lens, lay.block_tables, lay.num_blocks, lay.groups
+    MB = tables.shape[1]
+    nb = (seq_lens.astype(np.int64) + bs - 1) // bs
 
     # referenced physical blocks in first-use order (shared ones once)
     ref = []
