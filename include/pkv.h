@@ -33,7 +33,9 @@
  * Grouped-query attention: query head g reads KV head g / (num_heads / num_kv_heads)
  * (a group of query heads shares one KV head: Aliyun article, GQA/MQA section).
  *
- * dtypes: q_dtype/kv_dtype pairs (F32, F32), (BF16, BF16), (BF16, FP8_E4M3).
+ * dtypes: q_dtype/kv_dtype pairs (F32, F32), (BF16, BF16), (BF16, FP8_E4M3),
+ * (BF16, FP8_E5M2), (BF16, INT8); the append writes F32 or BF16 rows into any
+ * of them (into a cache of another dtype only when it is an 8-bit one).
  * FP8 caches hold OCP E4M3 codes of x / scale with per-tensor fp32 scales
  * (Aliyun article, section 15 "the KV cache itself can be quantized";
  * promptx.wiki tutorial, per-tensor KV scales). Arithmetic is fp32 throughout.
@@ -140,9 +142,9 @@ PKV_API int paged_attention_decode(void* out, const void* q, const void* k_cache
 /*
  * One whole decode step: the append of each sequence's new token (reshape_and_cache of
  * new_k/new_v row s at slot_mapping[s], one new token per sequence) followed by
- * paged_attention_decode over the cache that includes it. For bf16 and E4M3 caches of
+ * paged_attention_decode over the cache that includes it. For bf16 and 8-bit caches of
  * the shapes the tensor-core decode kernel covers (block_size 16 or 32, group <= 8,
- * head_dim 64/128 for bf16, 128 for E4M3) both happen in ONE launch: the warp that
+ * head_dim 64/128 for bf16, 128 for E4M3, E5M2 and INT8) both happen in ONE launch: the warp that
  * streams a sequence's last block first writes the new rows into it. Other shapes run
  * the two calls in stream order. Results are those of the two calls.
  *
@@ -169,7 +171,7 @@ PKV_API int paged_decode_step(void* out, const void* q, void* k_cache, void* v_c
  * num_kv_heads floats > 0 (caller-owned, read during the call), used where the
  * per-tensor calls use k_scale / v_scale — the append encodes
  * code = FP8(x / k_head_scales[h]) for KV head h, the decode dequantises with
- * the same scale. kv_dtype must be FP8_E4M3 or FP8_E5M2; the decode runs on
+ * the same scale. kv_dtype must be FP8_E4M3, FP8_E5M2 or INT8; the decode runs on
  * the tensor-core kernel only (the shapes paged_attention_decode lists for
  * it), others return PKV_ERR_SHAPE; a null scale array returns PKV_ERR_NULL.
  * Otherwise the same as reshape_and_cache and paged_attention_decode.
@@ -200,7 +202,7 @@ PKV_API int paged_attention_decode_head_scales(void* out, const void* q, const v
  *   workspace    >= paged_attention_workspace_size(num_seqs, q_len * num_heads,
  *                num_kv_heads, head_dim, num_partitions) bytes
  * Other arguments as paged_attention_decode. Runs on the tensor-core kernel
- * (bf16 / E4M3 / E5M2 caches, block size 16 or 32, head_dim 128, or 64 for
+ * (bf16 / E4M3 / E5M2 / INT8 caches, block size 16 or 32, head_dim 128, or 64 for
  * bf16); other shapes return PKV_ERR_SHAPE. q_len = 1 is paged_attention_decode.
  */
 PKV_API int paged_attention_decode_mq(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -262,7 +264,8 @@ PKV_API int paged_attention_decode_static(void* out, const void* q, const void* 
  * same way) for every kv head h. Same dtype: a bit copy. FP8_E4M3 cache from
  * F32 or BF16 rows: code = E4M3(x / k_scale) with an IEEE fp32 division and
  * round-to-nearest-even, saturating to +-448 (v with v_scale); FP8_E5M2 the
- * same with E5M2 codes, saturating to +-57344.
+ * same with E5M2 codes, saturating to +-57344; INT8 code =
+ * clamp(round-half-even(x / scale), -127, 127), NaN -> 0.
  * Duplicate non-negative slots in one call give an unspecified winner.
  * device_error: optional int32 device word that receives PKV_DEVERR_SLOT.
  */

@@ -1,4 +1,4 @@
-// Paged decode attention for bf16 and E4M3 caches on sm_100a: whole-block TMA
+// Paged decode attention for bf16 and 8-bit (E4M3, E5M2, INT8) caches on sm_100a: whole-block TMA
 // tiles, one warp per KV head, warp-level tensor-core MMA with fp32 accumulation.
 //
 // Same result as the CUDA-core kernel (decode_kernel.cuh): for every sequence s
@@ -13,13 +13,13 @@
 // well below the HBM rate. Here one tile costs ~100 instructions.
 //
 // Layout of the work:
-//  * Unit = (sequence, head group of HG <= 8 KV heads, logical block). The K
+//  * Unit = (sequence, head group of HG in {1, 2, 4} KV heads, logical block). The K
 //    rows of a unit are HG*block_size consecutive rows of the pool
-//    ([block][kv head][token][d]), i.e. one contiguous run (32 KB for bf16, 8
+//    ([block][kv head][token][d]), i.e. one contiguous run (16 KB for bf16, 4
 //    heads, block 16, d 128), fetched with 2-D TMA tensor copies whose 128-byte
 //    swizzle makes the ldmatrix reads below bank-conflict free. Same for V.
 //  * Units in (sequence, head group, block) order are cut into gridDim.x equal
-//    runs (one CTA per SM). Warp HG is the producer (block-table lookups, one
+//    runs (two or three CTAs per SM). Warp HG is the producer (block-table lookups, one
 //    TMA copy per 128-byte-wide box, a ring of stages with full/empty
 //    mbarriers); warps 0..HG-1 are consumers, warp w owning KV head
 //    hg*HG + w of every unit, so a run's segment of one (sequence, head)
@@ -28,9 +28,10 @@
 //    heads of the group, k = head_dim), scale, mask, online softmax with a lazy
 //    running max (moved only when a tile max passes it by 8, in log2 units),
 //    P^T re-laid out with 4 shuffles into the B operand of O^T += V^T P^T
-//    (head_dim x 8 heads, k = 16 tokens). bf16 caches use bf16 MMA; E4M3 codes
-//    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2) and use f16 MMA, the
-//    per-tensor scales applied to the fp32 scores and outputs.
+//    (head_dim x 8 heads, k = 16 tokens). bf16 caches use bf16 MMA; 8-bit codes
+//    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2 / .e5m2x2; for INT8 a byte
+//    permute and one f16 subtraction) and use f16 MMA, the per-tensor or
+//    per-head scales applied to the fp32 scores and outputs.
 //  * Split streams (a stream cut by a run boundary): each run's warp stores its
 //    piece's fp32 partial (o, m, l) and moves on. A second, small kernel
 //    launched as a programmatic dependent launch merges them (log-sum-exp, a
