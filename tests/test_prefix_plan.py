@@ -159,6 +159,15 @@ def test_mixed_prefix_workload_plan():
         shared[m] = p
     nb = np.asarray(nblocks(lens, bs))
     assert (int(nb.sum()), sum(len(r) for _, r, _ in plan) + int((nb - shared).sum())) == (47514, 33743)
+    reads = {}
+    for mg in (2, 4):
+        smaller = prefix_plan(tables, lens, bs, mg)
+        check_plan(smaller, tables, lens, bs, mg)
+        sh = np.zeros(len(lens), np.int64)
+        for m, _, p in smaller:
+            sh[m] = p
+        reads[mg] = sum(len(r) for _, r, _ in smaller) + int((nb - sh).sum())
+    assert reads == {2: 39865, 4: 35791}
 
 
 # ------------------------------------------------------------------ planted mistakes
