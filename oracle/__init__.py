@@ -54,6 +54,9 @@ def _bind(lib):
     lib.orc_paged_decode.argtypes = [P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
                                      f64, f64, f64, P, i32, i32, P, P]
     lib.orc_paged_decode.restype = i32
+    lib.orc_paged_decode_lse.argtypes = [P, P, P, i32, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                         f64, f64, f64, P, i32, i32, P, P]
+    lib.orc_paged_decode_lse.restype = i32
     lib.orc_reshape_and_cache.argtypes = [P, P, i32, P, P, i32, P, P, i64, i32, i32, i32, i32, i32, f32, f32, P, P]
     lib.orc_reshape_and_cache.restype = i32
     return lib
@@ -104,10 +107,11 @@ def e5m2_encode(x, lib=None) -> np.ndarray:
 def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
                  num_heads, num_kv_heads, head_dim, block_size, num_blocks,
                  scale, k_scale=1.0, v_scale=1.0, seqs=None, lib=None, q_len=1, k_head_scales=None,
-                 v_head_scales=None) -> np.ndarray:
+                 v_head_scales=None, return_lse=False):
     """fp64 attention output [len(seqs) or num_seqs, num_heads, head_dim]; with q_len > 1,
     q is [num_seqs, q_len, num_heads, head_dim] (query j at position seq_len - q_len + j,
-    causal) and the output [rows, q_len, num_heads, head_dim]."""
+    causal) and the output [rows, q_len, num_heads, head_dim]. With ``return_lse`` also the
+    natural log of every row's softmax denominator (shape of the output without head_dim)."""
     lib = lib or load()
     q = np.ascontiguousarray(q, dtype=NP_DT[q_dtype])
     k_cache = np.ascontiguousarray(k_cache, dtype=NP_DT[kv_dtype])
@@ -122,13 +126,14 @@ def paged_decode(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
     rows = S if sub is None else sub.size
     out = np.zeros((rows, num_heads, head_dim) if q_len == 1 else (rows, q_len, num_heads, head_dim),
                    dtype=np.float64)
-    st = lib.orc_paged_decode(_ptr(out), _ptr(q), DT[q_dtype], _ptr(k_cache), _ptr(v_cache), DT[kv_dtype],
-                              _ptr(bt), _ptr(sl), S, num_heads, num_kv_heads, head_dim, block_size, MB,
-                              num_blocks, float(scale), float(k_scale), float(v_scale),
-                              _ptr(sub), 0 if sub is None else int(sub.size), int(q_len), _ptr(khs), _ptr(vhs))
+    lse = np.zeros(out.shape[:-1], dtype=np.float64) if return_lse else None
+    st = lib.orc_paged_decode_lse(_ptr(out), _ptr(lse), _ptr(q), DT[q_dtype], _ptr(k_cache), _ptr(v_cache),
+                                  DT[kv_dtype], _ptr(bt), _ptr(sl), S, num_heads, num_kv_heads, head_dim,
+                                  block_size, MB, num_blocks, float(scale), float(k_scale), float(v_scale),
+                                  _ptr(sub), 0 if sub is None else int(sub.size), int(q_len), _ptr(khs), _ptr(vhs))
     if st != 0:
         raise OracleError(f"orc_paged_decode status {st}")
-    return out
+    return (out, lse) if return_lse else out
 
 
 def reshape_and_cache(k, v, in_dtype, k_cache, v_cache, kv_dtype, slot_mapping,

@@ -249,15 +249,15 @@ static size_t dtype_size(int dtype)
 
 /* ------------------------------------------------------------- attention */
 
-int orc_paged_decode(double* out,
-                     const void* q, int q_dtype,
-                     const void* k_cache, const void* v_cache, int kv_dtype,
-                     const int32_t* block_tables, const int32_t* seq_lens,
-                     int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                     int block_size, int max_blocks_per_seq, int num_blocks,
-                     double scale, double k_scale, double v_scale,
-                     const int32_t* seqs, int n_seqs, int q_len,
-                     const float* k_head_scales, const float* v_head_scales)
+int orc_paged_decode_lse(double* out, double* lse,
+                         const void* q, int q_dtype,
+                         const void* k_cache, const void* v_cache, int kv_dtype,
+                         const int32_t* block_tables, const int32_t* seq_lens,
+                         int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                         int block_size, int max_blocks_per_seq, int num_blocks,
+                         double scale, double k_scale, double v_scale,
+                         const int32_t* seqs, int n_seqs, int q_len,
+                         const float* k_head_scales, const float* v_head_scales)
 {
     if (num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 || q_len < 1)
         return ORC_ERR_SHAPE;
@@ -301,6 +301,8 @@ int orc_paged_decode(double* out,
             const double vsc = v_head_scales ? (double)v_head_scales[h] : v_scale;
             for (int i = 0; i < head_dim; ++i)
                 o[i] = 0.0;
+            if (lse)
+                lse[(size_t)r * q_len * num_heads + gq] = -INFINITY;
             if (Lq <= 0)
                 continue;
             const size_t qoff = ((size_t)s * q_len * num_heads + gq) * head_dim;
@@ -335,11 +337,30 @@ int orc_paged_decode(double* out,
             }
             for (int i = 0; i < head_dim; ++i)
                 o[i] /= denom;
+            /* log of the softmax denominator: log sum_t exp(x_t) = m + log sum_t exp(x_t - m) */
+            if (lse)
+                lse[(size_t)r * q_len * num_heads + gq] = m + log(denom);
         }
     }
 done:
     free(x);
     return status;
+}
+
+int orc_paged_decode(double* out,
+                     const void* q, int q_dtype,
+                     const void* k_cache, const void* v_cache, int kv_dtype,
+                     const int32_t* block_tables, const int32_t* seq_lens,
+                     int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                     int block_size, int max_blocks_per_seq, int num_blocks,
+                     double scale, double k_scale, double v_scale,
+                     const int32_t* seqs, int n_seqs, int q_len,
+                     const float* k_head_scales, const float* v_head_scales)
+{
+    return orc_paged_decode_lse(out, NULL, q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, seq_lens,
+                                num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                                num_blocks, scale, k_scale, v_scale, seqs, n_seqs, q_len, k_head_scales,
+                                v_head_scales);
 }
 
 /* ---------------------------------------------------------------- append */

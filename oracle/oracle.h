@@ -28,6 +28,20 @@ int orc_paged_decode(double* out,
                      const int32_t* seqs, int n_seqs, int q_len,
                      const float* k_head_scales, const float* v_head_scales);
 
+/* orc_paged_decode that also writes, when lse != NULL, the natural log of each query
+ * row's softmax denominator, log sum_t exp(scale * q . K_t) ([rows][q_len][num_heads];
+ * -inf for a row that sees no token): what two disjoint parts of a sequence need to
+ * be combined into the attention over both. */
+int orc_paged_decode_lse(double* out, double* lse,
+                         const void* q, int q_dtype,
+                         const void* k_cache, const void* v_cache, int kv_dtype,
+                         const int32_t* block_tables, const int32_t* seq_lens,
+                         int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                         int block_size, int max_blocks_per_seq, int num_blocks,
+                         double scale, double k_scale, double v_scale,
+                         const int32_t* seqs, int n_seqs, int q_len,
+                         const float* k_head_scales, const float* v_head_scales);
+
 /* Writes rows `rows` (all num_tokens rows when rows == NULL) of k/v into the caches.
  * FP8 caches: per-tensor k_scale / v_scale, or one scale per KV head when
  * k_head_scales / v_head_scales ([num_kv_heads]) are given (the same in attention). */

@@ -547,6 +547,73 @@ def check_int8_attention_dequant(lib):
         assert np.allclose(got[s], sdpa_fp64(q[s], K, V, 0.25), rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------------ log-sum-exp of the scores
+
+def check_lse_matches_library_logsumexp(lib):
+    """The row's log softmax denominator against torch.logsumexp of the scores (fp64 matmul
+    on the contiguous K); equal keys give score + log L; a row that sees nothing gives -inf."""
+    rng = np.random.default_rng(21)
+    lengths = [1, 2, 15, 16, 17, 40, 0]
+    q, Ks, Vs = _random_case(rng, lengths, Hq=8, Hkv=2, d=16)
+    kc, vc, bt, sl = page_sequences(Ks, Vs, 16, 40, rng)
+    _, lse = oracle.paged_decode(q, "f32", kc, vc, "f32", bt, sl, 8, 2, 16, 16, kc.shape[0], 0.25, lib=lib,
+                                 return_lse=True)
+    for s, L in enumerate(lengths):
+        for g in range(8):
+            if L == 0:
+                assert lse[s, g] == -np.inf
+                continue
+            K = torch.from_numpy(Ks[s][:, g // 4, :].astype(np.float64))
+            x = 0.25 * (K @ torch.from_numpy(q[s, g].astype(np.float64)))
+            assert abs(lse[s, g] - float(torch.logsumexp(x, 0))) <= 1e-12, (s, g)
+    L = 23
+    K = np.repeat(rng.standard_normal((1, 1, 16)).astype(np.float32), L, axis=0)
+    V = rng.standard_normal((L, 1, 16)).astype(np.float32)
+    q1 = rng.standard_normal((1, 1, 16)).astype(np.float32)
+    kc, vc, bt, sl = page_sequences([K], [V], 4, 8, rng)
+    _, lse = oracle.paged_decode(q1, "f32", kc, vc, "f32", bt, sl, 1, 1, 16, 4, 8, 0.5, lib=lib, return_lse=True)
+    score = 0.5 * float(np.dot(q1[0, 0].astype(np.float64), K[0, 0].astype(np.float64)))
+    assert abs(lse[0, 0] - (score + math.log(L))) <= 1e-12
+
+
+def check_lse_splits_combine(lib):
+    """A sequence cut after its first a blocks: attention over the first part (its table
+    cut to a blocks) and over the rest (the table shifted by a blocks, length L - a*bs)
+    combine, weighted by exp(lse), into the attention over the whole sequence. This is the
+    decomposition a shared-prefix decode relies on (a shared head of the table plus each
+    sequence's own tail)."""
+    rng = np.random.default_rng(22)
+    bs, Hq, Hkv, d = 8, 8, 2, 16
+    lengths = [9, 16, 17, 40, 57]
+    q, Ks, Vs = _random_case(rng, lengths, Hq=Hq, Hkv=Hkv, d=d)
+    for kv in ("f32", "e4m3"):
+        kc, vc, bt, sl = page_sequences(Ks, Vs, bs, 40, rng)
+        ks = vs = 1.0
+        if kv == "e4m3":
+            ks, vs = 0.01, 0.02
+            kc = oracle.e4m3_encode(kc / np.float32(ks), lib=lib).reshape(kc.shape)
+            vc = oracle.e4m3_encode(vc / np.float32(vs), lib=lib).reshape(vc.shape)
+        nb = kc.shape[0]
+        full, lse = oracle.paged_decode(q, "f32", kc, vc, kv, bt, sl, Hq, Hkv, d, bs, nb, 0.25, ks, vs, lib=lib,
+                                        return_lse=True)
+        for s, L in enumerate(lengths):
+            for a in range(1, -(-L // bs) + 1):
+                head_t = np.full_like(bt[s:s + 1], -1)
+                head_t[0, :a] = bt[s, :a]
+                tail_t = np.full_like(bt[s:s + 1], -1)
+                tail_t[0, :bt.shape[1] - a] = bt[s, a:]
+                n1, n2 = min(L, a * bs), max(0, L - a * bs)
+                o1, l1 = oracle.paged_decode(q[s:s + 1], "f32", kc, vc, kv, head_t, np.array([n1], np.int32), Hq,
+                                             Hkv, d, bs, nb, 0.25, ks, vs, lib=lib, return_lse=True)
+                o2, l2 = oracle.paged_decode(q[s:s + 1], "f32", kc, vc, kv, tail_t, np.array([n2], np.int32), Hq,
+                                             Hkv, d, bs, nb, 0.25, ks, vs, lib=lib, return_lse=True)
+                M = np.maximum(l1, l2)
+                w1, w2 = np.exp(l1 - M), np.exp(l2 - M)
+                comb = (w1[..., None] * o1 + w2[..., None] * o2) / (w1 + w2)[..., None]
+                assert np.allclose(comb[0], full[s], rtol=0, atol=1e-12), (kv, s, a)
+                assert np.allclose(M + np.log(w1 + w2), lse[s:s + 1], rtol=0, atol=1e-12), (kv, s, a)
+
+
 ALL_CHECKS = [
     check_e4m3_decode_table, check_e4m3_spot_values, check_e4m3_encode_vs_library, check_e4m3_ties_to_even,
     check_e4m3_saturation_and_roundtrip, check_length_one_is_v, check_length_two_closed_form,
@@ -557,5 +624,5 @@ ALL_CHECKS = [
     check_e5m2_ties_saturation_roundtrip, check_append_e5m2_vs_library, check_e5m2_attention_dequant,
     check_multi_query_matches_causal_sdpa, check_multi_query_is_decode_at_each_position,
     check_head_scales_equal_per_head_runs, check_int8_encode_vs_library, check_append_int8_vs_library,
-    check_int8_attention_dequant,
+    check_int8_attention_dequant, check_lse_matches_library_logsumexp, check_lse_splits_combine,
 ]

@@ -54,6 +54,8 @@ MUTANTS = {
     "append_offset_wrong": ("const int64_t blk = slot / block_size, off = slot % block_size;",
                             "const int64_t blk = slot / block_size, off = (slot + 1) % block_size;"),
     "negative_slot_written": ("if (slot < 0)\n            continue;", "if (slot < -1000)\n            continue;"),
+    "lse_without_max": ("= m + log(denom);", "= log(denom);"),
+    "lse_of_weights_not_scores": ("= m + log(denom);", "= m + log(denom / Lq);"),
     "dequant_scale_ignored": ("return orc_e4m3_value(((const uint8_t*)base)[i]) * scale;",
                               "return orc_e4m3_value(((const uint8_t*)base)[i]);"),
 }
