@@ -104,11 +104,22 @@ def _dtype_code(t: torch.Tensor) -> int:
         raise TypeError(f"unsupported dtype {t.dtype}") from None
 
 
-def _cuda(name, t: torch.Tensor):
+def _launch_device(name, t) -> int:
+    """The current CUDA device (where the library launches), once `t` is known to be a CUDA tensor."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return torch.cuda.current_device()
+
+
+def _cuda(name, t: torch.Tensor, dev: int | None = None):
+    """Device pointer of a contiguous CUDA tensor on device `dev` (the current device, where the
+    library launches; a tensor elsewhere would be read through a pointer this device cannot use)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if dev is not None and t.device.index != dev:
+        raise ValueError(f"{name} is on {t.device}, the current CUDA device is cuda:{dev}")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -144,18 +155,20 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
 
     q, out: [num_seqs, num_heads, head_dim] (float32 or bfloat16);
     k_cache, v_cache: [num_blocks, num_kv_heads, block_size, head_dim]
-    (float32, bfloat16, or uint8/float8_e4m3fn E4M3 codes with k_scale/v_scale);
+    (float32, bfloat16, uint8/float8_e4m3fn E4M3 codes, float8_e5m2 codes or int8 codes, the
+    8-bit ones with k_scale/v_scale);
     block_tables: int32 [num_seqs, max_blocks_per_seq]; seq_lens: int32 [num_seqs].
     """
     args = _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale,
-                        num_partitions, workspace)
+                        num_partitions, workspace, stream)
     st = load_library().paged_attention_decode(*args, _stream_handle(stream))
     _check("paged_attention_decode", st)
 
 
 def _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale, num_partitions,
-                 workspace):
+                 workspace, stream=None):
     """Checked C arguments of a decode call, up to (not including) the stream."""
+    dev = _launch_device("q", q)
     S, Hq, D = q.shape
     NB, Hkv, BS, D2 = k_cache.shape
     if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
@@ -167,11 +180,12 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scal
     if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
     if workspace is None:
-        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, q.device)
-    return (_cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-            _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
+        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, dev, stream)
+    return (_cuda("out", out, dev), _cuda("q", q, dev), _cuda("k_cache", k_cache, dev),
+            _cuda("v_cache", v_cache, dev), _cuda("block_tables", block_tables, dev),
+            _cuda("seq_lens", seq_lens, dev), S, Hq, Hkv, D, BS, float(scale),
             block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
-            int(num_partitions), _cuda("workspace", workspace), workspace.numel())
+            int(num_partitions), _cuda("workspace", workspace, dev), workspace.numel())
 
 
 def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale=1.0, v_scale=1.0,
@@ -179,6 +193,7 @@ def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, seq_lens, 
     """q_len new tokens per sequence, causal within the chunk: q, out [num_seqs, q_len, num_heads, head_dim]
     (bf16); query j of sequence s sits at position seq_lens[s] - q_len + j and attends every token
     up to itself. The new tokens' K/V must already be in the cache."""
+    dev = _launch_device("q", q)
     S, QL, Hq, D = q.shape
     NB, Hkv, BS, D2 = k_cache.shape
     if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
@@ -190,12 +205,13 @@ def paged_attention_decode_mq(out, q, k_cache, v_cache, block_tables, seq_lens, 
     if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
     if workspace is None:
-        workspace = _cached_workspace(S, Hq * QL, Hkv, D, num_partitions, q.device)
+        workspace = _cached_workspace(S, Hq * QL, Hkv, D, num_partitions, dev, stream)
     st = load_library().paged_attention_decode_mq(
-        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, QL, Hq, Hkv, D, BS, float(scale),
-        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
-        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _stream_handle(stream))
+        _cuda("out", out, dev), _cuda("q", q, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("block_tables", block_tables, dev), _cuda("seq_lens", seq_lens, dev), S, QL, Hq, Hkv, D, BS,
+        float(scale), block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale),
+        float(v_scale), int(num_partitions), _cuda("workspace", workspace, dev), workspace.numel(),
+        _stream_handle(stream))
     _check("paged_attention_decode_mq", st)
 
 
@@ -205,7 +221,7 @@ def withheld_unit_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale
     to its consumers, so their bounded wait runs out and the workspace error word gets
     DEVERR_TIMEOUT (read it with read_device_error, then workspace_init before reuse)."""
     args = _decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale, v_scale,
-                        num_partitions, workspace)
+                        num_partitions, workspace, stream)
     st = load_library().pkv_test_decode_timeout(*args, int(withheld_unit), _stream_handle(stream))
     _check("pkv_test_decode_timeout", st)
 
@@ -215,6 +231,7 @@ def paged_decode_step(out, q, k_cache, v_cache, block_tables, seq_lens, new_k, n
     """One decode step: append new_k/new_v row s at slot_mapping[s] (one new token per sequence,
     in its last block), then paged_attention_decode over the cache. One launch where the
     tensor-core decode kernel applies."""
+    dev = _launch_device("q", q)
     S, Hq, D = q.shape
     NB, Hkv, BS, D2 = k_cache.shape
     if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
@@ -228,65 +245,68 @@ def paged_decode_step(out, q, k_cache, v_cache, block_tables, seq_lens, new_k, n
     if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
         raise ValueError("block_tables must be [num_seqs, max_blocks] and seq_lens [num_seqs]")
     if workspace is None:
-        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, q.device)
+        workspace = _cached_workspace(S, Hq, Hkv, D, num_partitions, dev, stream)
     st = load_library().paged_decode_step(
-        _cuda("out", out), _cuda("q", q), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-        _cuda("block_tables", block_tables), _cuda("seq_lens", seq_lens), S, Hq, Hkv, D, BS, float(scale),
-        block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale), float(v_scale),
-        int(num_partitions), _cuda("workspace", workspace), workspace.numel(), _cuda("new_k", new_k),
-        _cuda("new_v", new_v), _cuda("slot_mapping", slot_mapping), _dtype_code(new_k), _stream_handle(stream))
+        _cuda("out", out, dev), _cuda("q", q, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("block_tables", block_tables, dev), _cuda("seq_lens", seq_lens, dev), S, Hq, Hkv, D, BS,
+        float(scale), block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale),
+        float(v_scale), int(num_partitions), _cuda("workspace", workspace, dev), workspace.numel(),
+        _cuda("new_k", new_k, dev), _cuda("new_v", new_v, dev), _cuda("slot_mapping", slot_mapping, dev),
+        _dtype_code(new_k), _stream_handle(stream))
     _check("paged_decode_step", st)
 
 
 def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, k_scale=1.0, v_scale=1.0,
                       device_error=None, stream=None) -> None:
     """Write k[t], v[t] ([num_tokens, num_kv_heads, head_dim]) into slot slot_mapping[t] of the caches."""
+    dev = _launch_device("k", k)
     T, Hkv, D = k.shape
     NB, Hkv2, BS, D2 = k_cache.shape
     if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("shape mismatch between rows and caches")
     if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
         raise TypeError("slot_mapping must be int64 [num_tokens]")
-    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error)
+    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error, dev)
     st = load_library().reshape_and_cache(
-        _cuda("k", k), _cuda("v", v), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-        _cuda("slot_mapping", slot_mapping), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
+        _cuda("k", k, dev), _cuda("v", v, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("slot_mapping", slot_mapping, dev), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
         float(k_scale), float(v_scale), err, _stream_handle(stream))
     _check("reshape_and_cache", st)
 
 
-def _head_scales(name, t, Hkv):
+def _head_scales(name, t, Hkv, dev):
     if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or t.shape != (Hkv,):
         raise TypeError(f"{name} must be a float32 tensor of num_kv_heads scales")
-    return _cuda(name, t)
+    return _cuda(name, t, dev)
 
 
 def reshape_and_cache_head_scales(k, v, k_cache, v_cache, slot_mapping, k_head_scales, v_head_scales,
                                   device_error=None, stream=None) -> None:
-    """reshape_and_cache into an FP8 cache with one scale per KV head (float32 [num_kv_heads] tensors)."""
+    """reshape_and_cache into an 8-bit cache with one scale per KV head (float32 [num_kv_heads] tensors)."""
+    dev = _launch_device("k", k)
     T, Hkv, D = k.shape
     NB, Hkv2, BS, D2 = k_cache.shape
     if (Hkv2, D2) != (Hkv, D) or tuple(v.shape) != tuple(k.shape) or tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("shape mismatch between rows and caches")
     if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (T,):
         raise TypeError("slot_mapping must be int64 [num_tokens]")
-    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error)
+    err = ctypes.c_void_p(None) if device_error is None else _cuda("device_error", device_error, dev)
     st = load_library().reshape_and_cache_head_scales(
-        _cuda("k", k), _cuda("v", v), _cuda("k_cache", k_cache), _cuda("v_cache", v_cache),
-        _cuda("slot_mapping", slot_mapping), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
-        _head_scales("k_head_scales", k_head_scales, Hkv), _head_scales("v_head_scales", v_head_scales, Hkv), err,
-        _stream_handle(stream))
+        _cuda("k", k, dev), _cuda("v", v, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("slot_mapping", slot_mapping, dev), T, Hkv, D, BS, NB, _dtype_code(k), _dtype_code(k_cache),
+        _head_scales("k_head_scales", k_head_scales, Hkv, dev), _head_scales("v_head_scales", v_head_scales, Hkv, dev),
+        err, _stream_handle(stream))
     _check("reshape_and_cache_head_scales", st)
 
 
 def paged_attention_decode_head_scales(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_head_scales,
                                        v_head_scales, num_partitions=0, workspace=None, stream=None) -> None:
-    """paged_attention_decode over an FP8 cache with one scale per KV head."""
+    """paged_attention_decode over an 8-bit cache with one scale per KV head."""
     args = list(_decode_args(out, q, k_cache, v_cache, block_tables, seq_lens, scale, 1.0, 1.0, num_partitions,
-                             workspace))
-    Hkv = k_cache.shape[1]
-    args[16:18] = [_head_scales("k_head_scales", k_head_scales, Hkv), _head_scales("v_head_scales", v_head_scales,
-                                                                                    Hkv)]
+                             workspace, stream))
+    Hkv, dev = k_cache.shape[1], _launch_device("q", q)
+    args[16:18] = [_head_scales("k_head_scales", k_head_scales, Hkv, dev),
+                   _head_scales("v_head_scales", v_head_scales, Hkv, dev)]
     st = load_library().paged_attention_decode_head_scales(*args, _stream_handle(stream))
     _check("paged_attention_decode_head_scales", st)
 
@@ -302,18 +322,25 @@ def read_device_error(workspace: torch.Tensor, clear: bool = False, stream=None)
 _ws_cache: dict = {}
 
 
-def _cached_workspace(S, Hq, Hkv, D, parts, device):
+def _cached_workspace(S, Hq, Hkv, D, parts, dev, stream):
+    """A workspace kept per (device, partitions, stream), so calls on different streams never share
+    one; a new one is zeroed by the library on the stream that will use it."""
     n = workspace_size(S, Hq, Hkv, D, parts)
-    key = (str(device), parts)
+    handle = _stream_handle(stream)
+    key = (dev, parts, handle.value)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < n:
-        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        if ws is not None:
+            torch.cuda.synchronize(dev)   # the smaller one may still be in use on its stream
+        ws = torch.empty(n, dtype=torch.uint8, device=torch.device("cuda", dev))
+        _check("pkv_workspace_init", load_library().pkv_workspace_init(_cuda("workspace", ws), n, handle))
         _ws_cache[key] = ws
     return ws
 
 
 __all__ = [
-    "paged_attention_decode", "paged_decode_step", "reshape_and_cache", "workspace_size", "new_workspace", "workspace_init",
+    "paged_attention_decode", "paged_decode_step", "paged_attention_decode_mq", "paged_attention_decode_head_scales",
+    "reshape_and_cache", "reshape_and_cache_head_scales", "workspace_size", "new_workspace", "workspace_init",
     "read_device_error", "default_partitions", "status_string", "load_library", "PkvError",
-    "F32", "BF16", "FP8_E4M3",
+    "F32", "BF16", "FP8_E4M3", "FP8_E5M2", "INT8",
 ]
