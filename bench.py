@@ -291,8 +291,9 @@ class DeviceState:
 def oracle_pair_sampler(b: W.DecodeBatch):
     """Single (sequence, KV head 0) attention problems cut from the batch, for timing the oracle.
 
-    Returns a list of (callable, bytes). The data preparation (history fill through
-    the oracle's own append, slicing of KV head 0) is done here, outside the timing.
+    Returns a list of (callable, bytes, seq_len, attention-only callable, its bytes). The
+    data preparation (history fill through the oracle's own append, slicing of KV head 0)
+    is done here, outside the timing.
     """
     import oracle
     sp = b.spec
@@ -308,29 +309,54 @@ def oracle_pair_sampler(b: W.DecodeBatch):
     items = []
     for s in seqs:
         L = int(b.seq_lens[s])
-        nbytes = (acct.decode_bytes(b.seq_lens[s:s + 1], b.block_tables[s:s + 1], G, 1, sp.head_dim,
-                                    sp.block_size, sp.kv_dtype, sp.q_dtype)["total"]
-                  + acct.append_bytes(1, 1, sp.head_dim, sp.in_dtype, sp.kv_dtype))
+        attn_bytes = acct.decode_bytes(b.seq_lens[s:s + 1], b.block_tables[s:s + 1], G, 1, sp.head_dim,
+                                       sp.block_size, sp.kv_dtype, sp.q_dtype)["total"]
+        nbytes = attn_bytes + acct.append_bytes(1, 1, sp.head_dim, sp.in_dtype, sp.kv_dtype)
+
+        def attend(s=s):
+            oracle.paged_decode(q0, sp.q_dtype, kc0, vc0, sp.kv_dtype, b.block_tables, b.seq_lens, G, 1,
+                                sp.head_dim, sp.block_size, b.num_blocks, b.scale, b.k_scale, b.v_scale, seqs=[s])
 
         def run(s=s):
             oracle.reshape_and_cache(nk0, nv0, sp.in_dtype, kc0, vc0, sp.kv_dtype, b.new_slots, 1, sp.head_dim,
                                      sp.block_size, b.num_blocks, b.k_scale, b.v_scale, rows=[s])
-            oracle.paged_decode(q0, sp.q_dtype, kc0, vc0, sp.kv_dtype, b.block_tables, b.seq_lens, G, 1,
-                                sp.head_dim, sp.block_size, b.num_blocks, b.scale, b.k_scale, b.v_scale, seqs=[s])
-        items.append((run, nbytes, L))
+            attend(s)
+        items.append((run, nbytes, L, attend, attn_bytes))
     return items
 
 
 def time_oracle(items, seconds: float):
     done_bytes, n, t0 = 0, 0, time.perf_counter()
     while True:
-        run, nbytes, _ = items[n % len(items)]
+        run, nbytes = items[n % len(items)][:2]
         run()
         done_bytes += nbytes
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             return done_bytes / el / 1e9, n, el
+
+
+def time_oracle_threads(items, seconds: float, threads: int):
+    """The attention-only problems on `threads` host threads at once (the C oracle runs with
+    the interpreter lock released, and the problems only read shared arrays): aggregate
+    GB/s, problems done, elapsed seconds."""
+    import concurrent.futures as cf
+    t0 = time.perf_counter()
+
+    def worker(i):
+        done, n = 0, 0
+        while time.perf_counter() - t0 < seconds:
+            _, _, _, attend, nbytes = items[(i + n) % len(items)]
+            attend()
+            done += nbytes
+            n += 1
+        return done, n
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        res = list(ex.map(worker, range(threads)))
+    el = time.perf_counter() - t0
+    return sum(r[0] for r in res) / el / 1e9, sum(r[1] for r in res), el
 
 
 # ----------------------------------------------------------------------------- arms
@@ -346,7 +372,7 @@ def reference_arm(args):
         items[i % len(items)][0]()
     times, nbytes = [], 0
     for i in range(args.steps):
-        run, nb, _ = items[i % len(items)]
+        run, nb = items[i % len(items)][:2]
         t0 = time.perf_counter()
         run()
         times.append(time.perf_counter() - t0)
@@ -526,6 +552,12 @@ def ours_arm(args):
                 "value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
                 "sample": f"{n} single (sequence, KV head 0) problems of this workload cycled for {el:.1f} s "
                           f"(append + attention each), fp64 C oracle, one thread"}
+            threads = os.cpu_count() or 1
+            v, n, el = time_oracle_threads(items, args.cpu_seconds, threads)
+            line["cpu_baseline_all_cores"] = {
+                "value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                "sample": f"{n} attention-only problems of the same sample on {threads} threads for {el:.1f} s, "
+                          f"fp64 C oracle"}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()

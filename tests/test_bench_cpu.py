@@ -43,3 +43,18 @@ def test_reference_arm_json_line():
     assert line["steps"] == 5 and line["higher_is_better"] is True
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_timing_on_all_cores():
+    """The all-cores oracle sample: every thread does work, the attention-only bytes are the
+    decode accounting of that sequence, and the same problems run on one or more threads."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    b = W.config_batch(0)
+    items = bench.oracle_pair_sampler(b)
+    run, nbytes, L, attend, attn_bytes = items[0]
+    assert nbytes > attn_bytes > 0
+    one = bench.time_oracle_threads(items, 0.3, 1)
+    many = bench.time_oracle_threads(items, 0.3, 4)
+    assert one[0] > 0 and one[1] > 0 and many[1] >= 4
