@@ -120,6 +120,27 @@ PKV_API int pkv_prefix_plan(const int32_t* block_tables, const int32_t* seq_lens
                             int32_t* group_offsets, int32_t* group_tables, int32_t* group_lens,
                             int32_t* shared_blocks, int* num_groups);
 
+/*
+ * Inputs of the two passes of a shared-prefix decode, from a pkv_prefix_plan result (host
+ * buffers, caller-owned). The prefix pass runs over the plan's group rows with 8 query
+ * columns per KV head: member i of group g takes columns i * Gq .. i * Gq + Gq - 1
+ * (Gq = query heads per KV head) and sees its own shared blocks only; the suffix pass runs
+ * every sequence over the rest of its own table.
+ *
+ *   col_seq       int32 [num_groups][8] out: sequence of each column, -1 = unused
+ *   col_limit     int32 [num_groups][8] out: tokens that column sees (shared blocks x block_size)
+ *   suffix_tables int32 [num_seqs][max_blocks_per_seq] out: row s = block_tables[s] shifted left
+ *                 by shared_blocks[s], -1 padded
+ *   suffix_lens   int32 [num_seqs] out: seq_lens[s] - shared_blocks[s] * block_size
+ * Returns PKV_OK, PKV_ERR_NULL, or PKV_ERR_SHAPE (a group with more than 8 / Gq members,
+ * Gq not dividing 8, a shared count beyond the table or the length, bad sizes).
+ */
+PKV_API int pkv_prefix_pass_inputs(const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                   int max_blocks_per_seq, int block_size, const int32_t* group_members,
+                                   const int32_t* group_offsets, int num_groups, const int32_t* shared_blocks,
+                                   int query_heads_per_kv_head, int32_t* col_seq, int32_t* col_limit,
+                                   int32_t* suffix_tables, int32_t* suffix_lens);
+
 #ifdef __cplusplus
 }
 #endif

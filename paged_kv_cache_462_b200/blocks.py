@@ -32,8 +32,9 @@ def _lib():
         lib.pkv_bm_step.argtypes = [P, P, i32, P, P, P, P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
         lib.pkv_bm_tables.argtypes = [P, P, i32, P, P]
         lib.pkv_prefix_plan.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, ctypes.POINTER(ctypes.c_int)]
+        lib.pkv_prefix_pass_inputs.argtypes = [P, P, i32, i32, i32, P, P, i32, P, i32, P, P, P, P]
         for n in ("pkv_bm_add", "pkv_bm_fork", "pkv_bm_append", "pkv_bm_free", "pkv_bm_num_free", "pkv_bm_seq_len",
-                  "pkv_bm_ref_count", "pkv_bm_step", "pkv_bm_tables", "pkv_prefix_plan"):
+                  "pkv_bm_ref_count", "pkv_bm_step", "pkv_bm_tables", "pkv_prefix_plan", "pkv_prefix_pass_inputs"):
             getattr(lib, n).restype = i32
         _bound = True
     return lib
@@ -147,3 +148,26 @@ def prefix_plan(block_tables, seq_lens, block_size: int, max_group: int) -> Pref
     if st != 0:
         raise PkvError("pkv_prefix_plan", st)
     return PrefixPlan(members, offsets, tables, lens, shared, ng.value)
+
+
+def prefix_pass_inputs(block_tables, seq_lens, block_size: int, plan: PrefixPlan, query_heads_per_kv_head: int):
+    """(col_seq int32 [groups, 8], col_limit int32 [groups, 8], suffix_tables, suffix_lens) for the
+    two passes of a shared-prefix decode (pkv_prefix_pass_inputs)."""
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    n, mb = bt.shape
+    g = plan.num_groups
+    col_seq = np.full((max(g, 1), 8), -1, dtype=np.int32)
+    col_limit = np.zeros((max(g, 1), 8), dtype=np.int32)
+    suf_t = np.full((n, mb), -1, dtype=np.int32)
+    suf_l = np.zeros(n, dtype=np.int32)
+    members = np.ascontiguousarray(plan.members, dtype=np.int32)
+    offsets = np.ascontiguousarray(plan.offsets, dtype=np.int32)
+    shared = np.ascontiguousarray(plan.shared, dtype=np.int32)
+    st = _lib().pkv_prefix_pass_inputs(bt.ctypes.data, sl.ctypes.data, n, mb, block_size, members.ctypes.data,
+                                       offsets.ctypes.data, g, shared.ctypes.data, query_heads_per_kv_head,
+                                       col_seq.ctypes.data, col_limit.ctypes.data, suf_t.ctypes.data,
+                                       suf_l.ctypes.data)
+    if st != 0:
+        raise PkvError("pkv_prefix_pass_inputs", st)
+    return col_seq[:g], col_limit[:g], suf_t, suf_l

@@ -106,3 +106,48 @@ extern "C" int pkv_prefix_plan(const int32_t* block_tables, const int32_t* seq_l
     *num_groups = ng;
     return PKV_OK;
 }
+
+extern "C" int pkv_prefix_pass_inputs(const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                      int max_blocks_per_seq, int block_size, const int32_t* group_members,
+                                      const int32_t* group_offsets, int num_groups, const int32_t* shared_blocks,
+                                      int query_heads_per_kv_head, int32_t* col_seq, int32_t* col_limit,
+                                      int32_t* suffix_tables, int32_t* suffix_lens)
+{
+    const int Gq = query_heads_per_kv_head;
+    if (num_seqs < 0 || num_groups < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || Gq <= 0 || 8 % Gq != 0)
+        return PKV_ERR_SHAPE;
+    if (num_seqs == 0 && num_groups == 0)
+        return PKV_OK;
+    if (!block_tables || !seq_lens || !shared_blocks || !suffix_tables || !suffix_lens)
+        return PKV_ERR_NULL;
+    if (num_groups > 0 && (!group_members || !group_offsets || !col_seq || !col_limit))
+        return PKV_ERR_NULL;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int sh = shared_blocks[s];
+        if (sh < 0 || sh > max_blocks_per_seq || (long long)sh * block_size > seq_lens[s])
+            return PKV_ERR_SHAPE;
+    }
+    for (int g = 0; g < num_groups; ++g) {
+        const int m0 = group_offsets[g], m1 = group_offsets[g + 1];
+        if (m0 < 0 || m1 < m0 || m1 > num_seqs || (m1 - m0) * Gq > 8)
+            return PKV_ERR_SHAPE;
+        for (int c = 0; c < 8; ++c) {
+            const int i = c / Gq;
+            const bool used = m0 + i < m1;
+            const int s = used ? group_members[m0 + i] : -1;
+            if (used && (s < 0 || s >= num_seqs))
+                return PKV_ERR_SHAPE;
+            col_seq[g * 8 + c] = s;
+            col_limit[g * 8 + c] = used ? shared_blocks[s] * block_size : 0;
+        }
+    }
+    for (int s = 0; s < num_seqs; ++s) {
+        const int sh = shared_blocks[s];
+        const int32_t* row = block_tables + (size_t)s * max_blocks_per_seq;
+        int32_t* dst = suffix_tables + (size_t)s * max_blocks_per_seq;
+        std::copy(row + sh, row + max_blocks_per_seq, dst);
+        std::fill(dst + (max_blocks_per_seq - sh), dst + max_blocks_per_seq, -1);
+        suffix_lens[s] = seq_lens[s] - sh * block_size;
+    }
+    return PKV_OK;
+}

@@ -245,3 +245,69 @@ def test_cpp_planner_on_workload_and_guards(cplan):
         cplan(lay.block_tables, lay.seq_lens, 16, 0)
     with pytest.raises(PkvError):
         cplan(lay.block_tables, lay.seq_lens, 0, 8)
+
+
+# ------------------------------------------------------------------ the two passes' inputs
+
+@pytest.fixture(scope="module")
+def pass_inputs():
+    from paged_kv_cache_462_b200 import build
+    build.build()
+    from paged_kv_cache_462_b200.blocks import prefix_pass_inputs
+    return prefix_pass_inputs
+
+
+def test_pass_inputs_layout(cplan, pass_inputs):
+    tables = np.array([[5, 6, 7, -1], [5, 6, 9, 3], [5, 8, -1, -1], [2, 3, -1, -1]], np.int32)
+    lens = np.array([40, 60, 20, 30], np.int32)
+    plan = cplan(tables, lens, 16, 4)                    # Gq = 2: at most 4 members per group
+    assert plan.groups() == [([0, 1, 2], [5, 6], [2, 2, 1])]
+    col_seq, col_limit, suf_t, suf_l = pass_inputs(tables, lens, 16, plan, 2)
+    assert col_seq.tolist() == [[0, 0, 1, 1, 2, 2, -1, -1]]
+    assert col_limit.tolist() == [[32, 32, 32, 32, 16, 16, 0, 0]]
+    assert suf_t.tolist() == [[7, -1, -1, -1], [9, 3, -1, -1], [8, -1, -1, -1], [2, 3, -1, -1]]
+    assert suf_l.tolist() == [8, 28, 4, 30]
+    from paged_kv_cache_462_b200 import PkvError
+    with pytest.raises(PkvError):                        # 3 members x 4 heads > 8 columns
+        pass_inputs(tables, lens, 16, plan, 4)
+    with pytest.raises(PkvError):                        # Gq must divide 8
+        pass_inputs(tables, lens, 16, plan, 3)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_prefix_passes_recombine_to_the_decode(cplan, pass_inputs, kv):
+    """Plan a mixed batch with shared prefixes, build both passes' inputs, run each pass through
+    the oracle (prefix: the group row, each member limited to its shared tokens; suffix: the
+    shifted table), combine by log-sum-exp weights: every row equals the plain decode."""
+    import oracle
+    b = W.config_batch(3, num_seqs=12, num_heads=8, num_kv_heads=2, head_dim=32, kv_dtype=kv,
+                       lengths=("lognormal", 300, 0.6, 20, 900), share_group=4, share_blocks=12,
+                       max_blocks_per_seq=60)
+    sp, bs = b.spec, b.spec.block_size
+    Gq = sp.num_heads // sp.num_kv_heads
+    _, kc, vc = oracle.run_step(b)
+    dec = lambda q, bt, sl: oracle.paged_decode(q, sp.q_dtype, kc, vc, kv, bt, sl, sp.num_heads, sp.num_kv_heads,
+                                                sp.head_dim, bs, b.num_blocks, b.scale, b.k_scale, b.v_scale,
+                                                return_lse=True)
+    full, full_lse = dec(b.q, b.block_tables, b.seq_lens)
+    plan = cplan(b.block_tables, b.seq_lens, bs, 8 // Gq)
+    assert plan.num_groups >= 2
+    col_seq, col_limit, suf_t, suf_l = pass_inputs(b.block_tables, b.seq_lens, bs, plan, Gq)
+    o2, l2 = dec(b.q, suf_t, suf_l)
+    o1 = np.zeros_like(o2)
+    l1 = np.full(l2.shape, -np.inf)
+    for g in range(plan.num_groups):
+        for c in range(0, 8, Gq):
+            s = int(col_seq[g, c])
+            if s < 0:
+                continue
+            o, l = dec(b.q[s:s + 1], plan.tables[g:g + 1], np.array([col_limit[g, c]], np.int32))
+            o1[s], l1[s] = o[0], l[0]
+    M = np.maximum(l1, l2)
+    w1 = np.where(l1 == -np.inf, 0.0, np.exp(l1 - M))
+    w2 = np.where(l2 == -np.inf, 0.0, np.exp(l2 - M))
+    comb = (w1[..., None] * o1 + w2[..., None] * o2) / (w1 + w2)[..., None]
+    assert np.allclose(comb, full, rtol=0, atol=1e-12)
+    assert np.allclose(M + np.log(w1 + w2), full_lse, rtol=0, atol=1e-12)
+    saved = sum(len(r) for _, r, _ in plan.groups())
+    assert int(plan.shared.sum()) > saved           # the shared blocks are read fewer times
