@@ -311,3 +311,36 @@ def test_prefix_passes_recombine_to_the_decode(cplan, pass_inputs, kv):
     assert np.allclose(M + np.log(w1 + w2), full_lse, rtol=0, atol=1e-12)
     saved = sum(len(r) for _, r, _ in plan.groups())
     assert int(plan.shared.sum()) > saved           # the shared blocks are read fewer times
+
+
+def test_cpp_planner_on_cpp_block_manager(cplan, blocks_cpp):
+    """Tables from the C++ block manager (forks, appends with copy on write): every block the
+    C++ plan shares has a count of two or more in the C++ manager."""
+    rng = np.random.default_rng(44)
+    for trial in range(10):
+        bs = int(rng.choice([4, 16]))
+        c = blocks_cpp.BlockManager(300, bs, 40)
+        live = []
+        for sid in range(int(rng.integers(3, 12))):
+            if live and rng.random() < 0.6:
+                assert c.fork(live[int(rng.integers(len(live)))], sid) == 0
+            else:
+                assert c.add(sid, int(rng.integers(1, 5 * bs))) == 0
+            live.append(sid)
+            for _ in range(int(rng.integers(0, 2 * bs))):
+                c.append(live[int(rng.integers(len(live)))])
+        st, tables, lens = c.tables(live)
+        assert st == 0
+        refs = [c.ref_count(blk) for blk in range(300)]
+        for mg in (2, 8):
+            plan = cplan(tables, lens, bs, mg)
+            check_plan(plan.groups(), tables.tolist(), lens.tolist(), bs, mg, refs=refs)
+        c.close()
+
+
+@pytest.fixture(scope="module")
+def blocks_cpp():
+    from paged_kv_cache_462_b200 import build
+    build.build()
+    from paged_kv_cache_462_b200 import blocks
+    return blocks
