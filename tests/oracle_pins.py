@@ -574,6 +574,19 @@ def check_lse_matches_library_logsumexp(lib):
     _, lse = oracle.paged_decode(q1, "f32", kc, vc, "f32", bt, sl, 1, 1, 16, 4, 8, 0.5, lib=lib, return_lse=True)
     score = 0.5 * float(np.dot(q1[0, 0].astype(np.float64), K[0, 0].astype(np.float64)))
     assert abs(lse[0, 0] - (score + math.log(L))) <= 1e-12
+    # several new tokens: row (j, g) covers the tokens up to position L - q_len + j
+    QL, lengths = 3, [5, 19]
+    qm, Ks, Vs = _random_case(rng, lengths, Hq=4, Hkv=2, d=16)
+    qm = rng.standard_normal((len(lengths), QL, 4, 16)).astype(np.float32)
+    kc, vc, bt, sl = page_sequences(Ks, Vs, 8, 8, rng)
+    _, lse = oracle.paged_decode(qm, "f32", kc, vc, "f32", bt, sl, 4, 2, 16, 8, 8, 0.25, lib=lib, q_len=QL,
+                                 return_lse=True)
+    for s, L in enumerate(lengths):
+        for j in range(QL):
+            for g in range(4):
+                K = torch.from_numpy(Ks[s][: L - QL + 1 + j, g // 2, :].astype(np.float64))
+                x = 0.25 * (K @ torch.from_numpy(qm[s, j, g].astype(np.float64)))
+                assert abs(lse[s, j, g] - float(torch.logsumexp(x, 0))) <= 1e-12, (s, j, g)
 
 
 def check_lse_splits_combine(lib):
