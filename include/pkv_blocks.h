@@ -45,6 +45,7 @@ extern "C" {
 #define PKV_BM_UNKNOWN_SEQ 21 /* no sequence with this id */
 #define PKV_BM_DUPLICATE_SEQ 22
 #define PKV_BM_TABLE_FULL 23  /* the sequence would need more than max_blocks_per_seq blocks */
+#define PKV_BM_HOST_ALLOC 24  /* a host allocation failed (the call may have been partly applied) */
 
 typedef struct pkv_block_manager pkv_block_manager;
 

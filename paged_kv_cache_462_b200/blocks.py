@@ -7,7 +7,7 @@ import numpy as np
 
 from . import PkvError, load_library
 
-NO_BLOCKS, UNKNOWN_SEQ, DUPLICATE_SEQ, TABLE_FULL = 20, 21, 22, 23
+NO_BLOCKS, UNKNOWN_SEQ, DUPLICATE_SEQ, TABLE_FULL, HOST_ALLOC = 20, 21, 22, 23, 24
 
 _bound = False
 

@@ -107,7 +107,7 @@ pkv_block_manager* pkv_bm_create(int num_blocks, int block_size, int max_blocks_
 void pkv_bm_destroy(pkv_block_manager* bm) { delete bm; }
 
 int pkv_bm_add(pkv_block_manager* bm, int64_t seq_id, int prompt_len)
-{
+try {
     if (!bm)
         return PKV_ERR_NULL;
     if (prompt_len < 0)
@@ -126,10 +126,12 @@ int pkv_bm_add(pkv_block_manager* bm, int64_t seq_id, int prompt_len)
         q.table.push_back(bm->take());
     bm->seqs.emplace(seq_id, std::move(q));
     return PKV_OK;
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 int pkv_bm_fork(pkv_block_manager* bm, int64_t parent_id, int64_t child_id)
-{
+try {
     if (!bm)
         return PKV_ERR_NULL;
     auto it = bm->seqs.find(parent_id);
@@ -142,17 +144,21 @@ int pkv_bm_fork(pkv_block_manager* bm, int64_t parent_id, int64_t child_id)
         bm->refs[b] += 1;
     bm->seqs.emplace(child_id, std::move(child));
     return PKV_OK;
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 int pkv_bm_append(pkv_block_manager* bm, int64_t seq_id, int64_t* slot, int32_t* cow_src, int32_t* cow_dst)
-{
+try {
     if (!bm || !slot || !cow_src || !cow_dst)
         return PKV_ERR_NULL;
     return bm->append(seq_id, slot, cow_src, cow_dst);
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 int pkv_bm_free(pkv_block_manager* bm, int64_t seq_id)
-{
+try {
     if (!bm)
         return PKV_ERR_NULL;
     auto it = bm->seqs.find(seq_id);
@@ -162,6 +168,8 @@ int pkv_bm_free(pkv_block_manager* bm, int64_t seq_id)
         bm->release(b);
     bm->seqs.erase(it);
     return PKV_OK;
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 int pkv_bm_num_free(const pkv_block_manager* bm) { return bm ? (int)bm->free_list.size() : -1; }
@@ -183,7 +191,7 @@ int pkv_bm_ref_count(const pkv_block_manager* bm, int block)
 
 int pkv_bm_step(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* slot_mapping, int32_t* block_tables,
                 int32_t* seq_lens, int32_t* cow_pairs, int* n_cow, int* n_done)
-{
+try {
     if (!bm || !n_cow || !n_done)
         return PKV_ERR_NULL;
     *n_cow = 0;
@@ -206,6 +214,8 @@ int pkv_bm_step(pkv_block_manager* bm, const int64_t* seq_ids, int n, int64_t* s
     }
     bm->write_tables(seq_ids, n, block_tables, seq_lens);
     return PKV_OK;
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 int pkv_bm_tables(const pkv_block_manager* bm, const int64_t* seq_ids, int n, int32_t* block_tables,

@@ -29,7 +29,7 @@ extern "C" int pkv_prefix_plan(const int32_t* block_tables, const int32_t* seq_l
                                int max_blocks_per_seq, int block_size, int max_group, int32_t* group_members,
                                int32_t* group_offsets, int32_t* group_tables, int32_t* group_lens,
                                int32_t* shared_blocks, int* num_groups)
-{
+try {
     if (!num_groups)
         return PKV_ERR_NULL;
     *num_groups = 0;
@@ -105,6 +105,8 @@ extern "C" int pkv_prefix_plan(const int32_t* block_tables, const int32_t* seq_l
     }
     *num_groups = ng;
     return PKV_OK;
+} catch (...) {
+    return PKV_BM_HOST_ALLOC;
 }
 
 extern "C" int pkv_prefix_pass_inputs(const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
