@@ -39,7 +39,10 @@ int sm_count(int dev)
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 0;
-    g_sm_count[dev] = n;
+    try {
+        g_sm_count[dev] = n;
+    } catch (...) {
+    }
     return n;
 }
 
@@ -121,7 +124,10 @@ bool ensure_smem_attribute(const void* kernel, size_t bytes)
         return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return false;
-    g_smem_set[key] = bytes;
+    try {   // only a cache of the attribute: a failed insert just means it is set again next time
+        g_smem_set[key] = bytes;
+    } catch (...) {
+    }
     return true;
 }
 
