@@ -558,6 +558,9 @@ def check_lse_matches_library_logsumexp(lib):
     kc, vc, bt, sl = page_sequences(Ks, Vs, 16, 40, rng)
     _, lse = oracle.paged_decode(q, "f32", kc, vc, "f32", bt, sl, 8, 2, 16, 16, kc.shape[0], 0.25, lib=lib,
                                  return_lse=True)
+    _, sub = oracle.paged_decode(q, "f32", kc, vc, "f32", bt, sl, 8, 2, 16, 16, kc.shape[0], 0.25, seqs=[4, 0],
+                                 lib=lib, return_lse=True)
+    assert np.array_equal(sub, lse[[4, 0]])          # rows follow `seqs`
     for s, L in enumerate(lengths):
         for g in range(8):
             if L == 0:
