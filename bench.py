@@ -552,7 +552,7 @@ def ours_arm(args):
                 "value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
                 "sample": f"{n} single (sequence, KV head 0) problems of this workload cycled for {el:.1f} s "
                           f"(append + attention each), fp64 C oracle, one thread"}
-            threads = os.cpu_count() or 1
+            threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
             v, n, el = time_oracle_threads(items, args.cpu_seconds, threads)
             line["cpu_baseline_all_cores"] = {
                 "value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
