@@ -80,3 +80,13 @@ def test_fp8_scales_map_absmax_to_448():
     absk = max(np.abs(W.bf16_bits_to_f32(b.hist_k)).max(), np.abs(W.bf16_bits_to_f32(b.new_k)).max())
     assert b.k_scale == np.float32(absk / np.float32(448))
     _check_structure(b)
+
+
+def test_batch_layout_is_build_batch_tables():
+    """The tables-only draw gives exactly the lengths, tables and pool of the full batch."""
+    import workloads as W
+    for i, kw in ((0, {}), (3, dict(num_seqs=24)), (1, dict(num_seqs=5))):
+        b = W.config_batch(i, **kw)
+        lay = W.batch_layout(b.spec)
+        assert np.array_equal(lay.seq_lens, b.seq_lens) and np.array_equal(lay.block_tables, b.block_tables)
+        assert lay.num_blocks == b.num_blocks
