@@ -3,7 +3,7 @@
 append (reshape_and_cache) followed by paged decode attention over every
 running sequence, on a seeded synthetic batch resident in HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--impl ours|reference]
 
 Prints ONE JSON line (rank 0). ``value`` is the step's algorithmic bytes
 (K/V tiles of every distinct referenced block, q, out, block tables and
@@ -12,6 +12,8 @@ over ranks (each rank runs its own replica: the path has no exchange step).
 ``roofline`` reports the decode kernel alone against the measured HBM copy
 bandwidth. ``e2e`` repeats the step with every per-step input copied in from
 pinned host memory and the output copied back inside the timed region.
+``targets`` times the other points of the throughput target (long-context and
+mixed-batch workloads with bf16 and E4M3 caches) the same way in the same run.
 ``--impl reference`` times the CPU oracle (fp64, one core) on the same
 workload, a bounded sample per step.
 """
@@ -46,7 +48,8 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=1, help="workload 0..4 (default 1, Llama-3-8B bf16)")
+    ap.add_argument("--config", type=int, default=3,
+                    help="workload 0..4 (default 3: the mixed batch with shared prefixes, bf16, the largest)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--partitions", type=int, default=0, help="decode runs (0 = automatic)")
     ap.add_argument("--q-len", type=int, default=1,
@@ -56,7 +59,15 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the extra target points (long-context and mixed batch, bf16 and E4M3 caches)")
     return ap.parse_args()
+
+
+# The throughput target names two workloads (long context: config 2; mixed batch with shared
+# prefixes: config 3) with bf16 and FP8 E4M3 caches; the points other than the main line's are
+# timed in the same run, with the same step count, and reported under "targets".
+TARGET_POINTS = ((2, "bf16"), (2, "e4m3"), (3, "bf16"), (3, "e4m3"))
 
 
 def workload_spec(args) -> W.Spec:
@@ -121,59 +132,91 @@ def kernel_sha() -> str:
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock, power and throttle reasons during the timed region."""
+    """SM clock, power and throttle reasons sampled during the timed region (read-only queries).
 
+    NVML is polled every ~1 ms from a thread (nvidia-smi's 20 ms loop saw no sample at all in a
+    timed region of a few milliseconds); without NVML, ``nvidia-smi -lms 20`` is read instead.
+    Every sample carries its time, and ``summary(t0, t1)`` keeps those inside [t0, t1]."""
+
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.samples = []
+    def __init__(self, device_index: str, period_s: float = 0.001):
+        self.samples = []          # (time, sm MHz, max sm MHz, set of active reason names)
+        self.source = None
         self.proc = None
-        self.on = False
+        self._stop = threading.Event()
+        self.period = period_s
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
-                 "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(int(device_index))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.source = "nvml"
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
         except Exception:
-            self.proc = None
-            return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                     "-i", str(device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+                self.t = threading.Thread(target=self._read_smi, daemon=True)
+            except Exception:
+                self.t = None
+        if self.t is not None:
+            self.t.start()
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv, h = self.nv, self.h
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((time.perf_counter(), mhz, self.max_mhz,
+                                     {n for n, b in self.bits.items() if r & b}))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            if self.on:
-                self.samples.append([x.strip() for x in line.split(",")])
-
-    def start(self):
-        self.on = True
+            f = [x.strip() for x in line.split(",")]
+            try:
+                self.samples.append((time.perf_counter(), float(f[1]), float(f[2]),
+                                     {n for n, v in zip(self.REASONS, f[5:9]) if v.lower() == "active"}))
+            except (ValueError, IndexError):
+                continue
 
     def stop(self):
-        self.on = False
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for s in self.samples:
-            try:
-                sm.append(float(s[1]))
-                mx.append(float(s[2]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, s[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+    def summary(self, t0: float, t1: float):
+        """Median SM clock, max clock and the union of active reasons over samples in [t0, t1]."""
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source,
+                    "window_ms": 1e3 * (t1 - t0)}
+        reasons = set()
+        for x in inside:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "source": self.source,
+                "window_ms": 1e3 * (t1 - t0)}
 
 
 def smi_index(torch, dev: int) -> str:
@@ -393,6 +436,29 @@ def reference_arm(args):
     return 0
 
 
+def time_steps(torch, state, K: int, warmup: int, flush_l2, stream, dev):
+    """W untimed steps, then K steps each bracketed by CUDA events on the launching stream, with
+    the L2 flush between steps outside the events. Returns (per-step ms, wall start, wall end of
+    the timed region)."""
+    for _ in range(warmup):
+        flush_l2()
+        state.step()
+    torch.cuda.synchronize(dev)
+    if state.errors():
+        raise SystemExit(f"device error word {state.errors()} after warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for i in range(K):
+        flush_l2()                        # cold L2 for every step (outside the step's events)
+        ev[i][0].record(stream)
+        state.step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    return [e[0].elapsed_time(e[1]) for e in ev], t0, t1
+
+
 def ours_arm(args):
     import torch
     import paged_kv_cache_462_b200 as pkv
@@ -426,33 +492,13 @@ def ours_arm(args):
         torch.sum(flush_buf, dim=0, out=flush_out)
 
     stream = torch.cuda.current_stream(dev)
-
-    for _ in range(args.warmup):
-        flush_l2()
-        state.step()
-    torch.cuda.synchronize(dev)
-    if state.errors():
-        raise SystemExit(f"device error word {state.errors()} after warm-up")
-
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = ClockSampler(smi_index(torch, local)) if rank == 0 else None
     if dist:
         dist.barrier()
-    torch.cuda.synchronize(dev)
-    if clocks:
-        clocks.start()
-    for i in range(K):
-        flush_l2()                        # cold L2 for every step (outside the step's events)
-        ev[i][0].record(stream)
-        state.step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    if clocks:
-        clocks.stop()
+    step_ms, t_on, t_off = time_steps(torch, state, K, args.warmup, flush_l2, stream, dev)
     if dist:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
     ms = sum(step_ms) / K
     fused = pkv.load_library() is not None and spec.kv_dtype != "f32" and spec.block_size in (16, 32)
     errs = state.errors()
@@ -483,6 +529,40 @@ def ours_arm(args):
         e2e_ms = sum(a.elapsed_time(c) for a, c in ee) / Ke
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
+    # the other points of the throughput target, timed the same way (same K and W), one at a time
+    targets = []
+    if not args.no_targets and args.q_len == 1 and args.kv_dtype is None and args.partitions == 0:
+        main_kv = spec.kv_dtype
+        del state
+        torch.cuda.empty_cache()
+        batches = {args.config: b}
+        for cfg, kv in TARGET_POINTS:
+            if cfg == args.config and kv == main_kv:
+                continue
+            if cfg not in batches:
+                batches = {args.config: b, cfg: W.build_batch(W.config_spec(cfg),
+                                                              seed=W.config_spec(cfg).seed + 1000 * rank)}
+            tb = W.with_cache_dtype(batches[cfg], kv)
+            ts = DeviceState(torch, pkv, tb, dev, 0)
+            tdec, tapp = step_bytes(tb)
+            tbytes = tdec["total"] + tapp
+            if dist:
+                dist.barrier()
+            tms, t0, t1 = time_steps(torch, ts, K, args.warmup, flush_l2, stream, dev)
+            terr = ts.errors()
+            agg_t = aggregate_ranks(torch, dist, dev, ms=sum(tms) / K, step_bytes=float(tbytes), errors=float(terr))
+            targets.append({"config_index": cfg, "kv_storage": kv, "workload": describe(tb),
+                            "ms_per_step": agg_t["ms"], "value": agg_t["step_bytes"] / (agg_t["ms"] * 1e-3) / 1e9,
+                            "unit": "GB/s", "algorithmic_bytes": tbytes,
+                            "kv_logical_gbs": tdec["kv_logical"] / (sum(tms) / K * 1e-3) / 1e9,
+                            "seq_steps_per_s": world * tb.spec.num_seqs / (agg_t["ms"] * 1e-3),
+                            "device_errors": int(agg_t["errors"]),
+                            "clocks": clocks.summary(t0, t1) if clocks else None})
+            del ts
+            torch.cuda.empty_cache()
+    if clocks:
+        clocks.stop()
+
     # aggregate over ranks: max time, summed bytes
     agg = aggregate_ranks(torch, dist, dev, ms=ms, decode_ms=ms,
                           e2e_ms=e2e["ms"] if e2e else 0.0, step_bytes=float(bytes_step), errors=float(errs))
@@ -493,6 +573,8 @@ def ours_arm(args):
         peak, peak_kind = measured_peak()
         kern_bytes = dec["total"] + app          # the step kernel: decode plus the fused append
         kern_gbs = kern_bytes / (ms * 1e-3) / 1e9
+        for t in targets:
+            t["frac"] = t["value"] / world / peak
         line = {
             "metric": METRIC,
             "value": bytes_all / (ms_max * 1e-3) / 1e9,
@@ -504,7 +586,7 @@ def ours_arm(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            # arithmetic: tensor-core products in bf16 (E4M3 codes widened exactly to f16), fp32 sums
+            # arithmetic of the products: bf16 for bf16 caches; 8-bit codes widened exactly to f16
             "dtype": {"f32": "f32", "bf16": "bf16", "e4m3": "f16", "e5m2": "f16", "int8": "f16"}[spec.kv_dtype],
             "data": "synthetic",
             "config": {
@@ -539,9 +621,11 @@ def ours_arm(args):
             },
             # fused: the decode kernel (append inside) + the merge kernel; else append + decode
             "gpu_launches": 2 * K,
-            "clocks": clocks.summary() if clocks else None,
+            "clocks": clocks.summary(t_on, t_off) if clocks else None,
             "device_errors": errs_all,
         }
+        if targets:
+            line["targets"] = targets
         if e2e:
             line["e2e"] = {"value": bytes_all / (e2e_max * 1e-3) / 1e9, "unit": "GB/s",
                            "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_max}

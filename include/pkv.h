@@ -114,14 +114,18 @@ PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int n
 PKV_API int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Paged decode attention. One launch: the total work, sum over (sequence,
- * kv head) of ceil(seq_len / block_size) blocks, is cut into num_partitions
- * equal runs of blocks (0 = one or more per SM, from the occupancy); a run
- * may cover several (sequence, kv head) pairs and a pair may be split across
- * runs. Each run streams its K/V tiles through shared memory and keeps an
- * online softmax; a pair split across runs is finished by whichever run
- * arrives last, which merges the fp32 partials from the workspace (the
- * log-sum-exp combination), so no run ever waits for another.
+ * Paged decode attention. The total work, sum over (sequence, kv head) of
+ * ceil(seq_len / block_size) blocks, is cut into num_partitions equal runs of
+ * blocks (0 = one or more per SM, from the occupancy); a run may cover several
+ * (sequence, kv head) pairs and a pair may be split across runs. Each run
+ * streams its K/V tiles through shared memory and keeps an online softmax; no
+ * run ever waits for another. A pair split across runs leaves one fp32 partial
+ * (o, m, l) per run in the workspace, and the log-sum-exp merge of those
+ * partials writes its output: for the tensor-core kernel (bf16 and 8-bit
+ * caches of the shapes paged_decode_step lists) a second, small kernel
+ * launched right behind the decode kernel on `stream` does the merge; for the
+ * CUDA-core kernel (F32 caches and the other shapes) the run that finishes a
+ * pair last merges it inside the same launch.
  *
  *   out          [num_seqs][num_heads][head_dim], q_dtype
  *   q            [num_seqs][num_heads][head_dim], q_dtype
@@ -234,10 +238,12 @@ PKV_API int pkv_test_decode_timeout(void* out, const void* q, const void* k_cach
 
 /*
  * paged_attention_decode without a caller workspace, for callers that cannot
- * allocate device memory: code running while a CUDA graph is captured,
- * plug-ins whose host framework owns every allocation, hosts that reserve all
- * memory at start-up. (The pages have no counterpart; this is an interface
- * convenience, same arithmetic as paged_attention_decode.)
+ * allocate device memory: plug-ins and custom operators whose host framework
+ * owns every allocation and forbids allocating while they run, hosts that
+ * reserve all device memory at start-up, and latency-bound serving loops that
+ * cannot afford cudaMalloc's implicit device synchronisation. (The pages have
+ * no counterpart; this is an interface convenience, same arithmetic as
+ * paged_attention_decode.)
  *
  * Arguments are those of paged_attention_decode minus the workspace. The
  * scratch is a fixed 32 MiB array inside the library, present on every GPU
@@ -246,10 +252,13 @@ PKV_API int pkv_test_decode_timeout(void* out, const void* q, const void* k_cach
  * num_partitions) exceeds 32 MiB returns PKV_ERR_WORKSPACE without launching.
  * Nothing is allocated. The first call on each device looks up the array's
  * device address (with that device current), so make that first call before
- * any stream capture. Every call clears the array's counters and error word on
- * `stream` and then shares the array: calls that overlap on the GPU (other
- * streams, other threads) race and must be serialised by the caller. The
- * device error word is not readable through this entry point.
+ * any stream capture; the address is looked up again when the device's
+ * context changes (for instance after cudaDeviceReset). The call runs every
+ * host check of paged_attention_decode before it queues anything; then it
+ * clears the array's counters and error word on `stream` and launches. Every
+ * call shares the array: calls that overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller. The device error word
+ * is not readable through this entry point.
  */
 PKV_API int paged_attention_decode_static(void* out, const void* q, const void* k_cache, const void* v_cache,
                                           const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,

@@ -131,6 +131,111 @@ bool ensure_smem_attribute(const void* kernel, size_t bytes)
     return true;
 }
 
+// Host checks, partition count and launch parameters of a decode call; nothing is queued. On
+// PKV_OK, *runs = 0 means there is nothing to launch (no sequences).
+int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                   const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                   int block_size, float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                   float k_scale, float v_scale, int num_partitions, void* workspace, size_t workspace_bytes,
+                   const AppendArgs* app, int withheld_unit, int q_len, const float* k_head_scales,
+                   const float* v_head_scales, DecodeParams* p_out, int* runs_out)
+{
+    *runs_out = 0;
+    if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads != 0 || num_partitions < 0 || q_len < 1 || q_len > 8)
+        return PKV_ERR_SHAPE;
+    // query columns per KV head: q_len new tokens x the GQA group (the kernels' "group")
+    const int group = num_heads / num_kv_heads * q_len;
+    if (!group_supported(group) || (head_dim != 64 && head_dim != 128) ||
+        (block_size != 8 && block_size != 16 && block_size != 32))
+        return PKV_ERR_SHAPE;
+    if (q_len > 1 && (app || !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group,
+                                                                       num_kv_heads))))
+        return PKV_ERR_SHAPE;   // several new tokens: tensor-core kernel only, no fused append
+    if ((k_head_scales || v_head_scales) &&
+        (!k_head_scales || !v_head_scales || !is_fp8(kv_dtype) ||
+         !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads))))
+        return PKV_ERR_SHAPE;   // per-head scales: both arrays, FP8 caches, tensor-core kernel
+    if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
+          (q_dtype == PKV_BF16 && is_fp8(kv_dtype))))
+        return PKV_ERR_DTYPE;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
+        return PKV_ERR_NULL;
+    if (!workspace)
+        return PKV_ERR_WORKSPACE;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return PKV_ERR_SHAPE;
+    if ((long long)num_seqs * max_blocks_per_seq * num_kv_heads >= (1ll << 31) ||
+        (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
+        (long long)num_blocks * num_kv_heads * block_size >= (1ll << 31))
+        return PKV_ERR_SHAPE;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
+        return PKV_ERR_SHAPE;
+
+    int runs = num_partitions;
+    if (runs == 0) {
+        const int dev = current_device();
+        const int sms = dev >= 0 ? sm_count(dev) : 0;
+        if (sms <= 0)
+            return PKV_ERR_DEVICE;
+        DecodeParams probe;
+        std::memset(&probe, 0, sizeof probe);
+        probe.num_seqs = num_seqs;
+        probe.num_kv_heads = num_kv_heads;
+        int occ = 0;
+        const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, probe, 0, nullptr, &occ);
+        if (st != PKV_OK)
+            return st;
+        if (occ < 1)
+            return PKV_ERR_SHAPE;
+        runs = sms * (occ > kMaxRunsPerSM ? kMaxRunsPerSM : occ);
+    }
+    const WorkspaceLayout lay = layout_for(num_seqs, num_kv_heads, group, head_dim, runs);
+    if (workspace_bytes < lay.bytes)
+        return PKV_ERR_WORKSPACE;
+
+    const bool fp8 = is_fp8(kv_dtype);
+    DecodeParams& p = *p_out;
+    std::memset(&p, 0, sizeof p);
+    p.out = out;
+    p.q = q;
+    p.k_cache = static_cast<const uint8_t*>(k_cache);
+    p.v_cache = static_cast<const uint8_t*>(v_cache);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.scale = scale;
+    p.k_scale = fp8 ? k_scale : 1.0f;
+    p.v_scale_in = fp8 ? v_scale : 1.0f;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.err = reinterpret_cast<int32_t*>(ws);
+    p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
+    p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
+    p.slot_floats = slot_floats_for(group, head_dim);
+    p.q_len = q_len;
+    p.k_head_scales = k_head_scales;
+    p.v_head_scales = v_head_scales;
+    if (withheld_unit >= 0) {
+        if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
+            return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
+        p.withheld_unit = withheld_unit + 1;
+    }
+    if (app) {
+        p.new_k = app->k;
+        p.new_v = app->v;
+        p.new_slots = app->slots;
+        p.in_dtype = app->in_dtype;
+    }
+    *runs_out = runs;
+    return PKV_OK;
+}
+
 }  // namespace pkv
 
 using namespace pkv;
@@ -246,13 +351,6 @@ int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_
 
 namespace {
 
-struct AppendArgs {
-    const void* k;
-    const void* v;
-    const int64_t* slots;
-    int in_dtype;
-};
-
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                 const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                 float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
@@ -260,98 +358,15 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const AppendArgs* app, int withheld_unit = -1, int q_len = 1, const float* k_head_scales = nullptr,
                 const float* v_head_scales = nullptr)
 {
-    if (num_seqs < 0 || num_seqs > kMaxSeqs || num_heads <= 0 || num_kv_heads <= 0 ||
-        num_heads % num_kv_heads != 0 || num_partitions < 0 || q_len < 1 || q_len > 8)
-        return PKV_ERR_SHAPE;
-    // query columns per KV head: q_len new tokens x the GQA group (the kernels' "group")
-    const int group = num_heads / num_kv_heads * q_len;
-    if (!group_supported(group) || (head_dim != 64 && head_dim != 128) ||
-        (block_size != 8 && block_size != 16 && block_size != 32))
-        return PKV_ERR_SHAPE;
-    if (q_len > 1 && (app || !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group,
-                                                                       num_kv_heads))))
-        return PKV_ERR_SHAPE;   // several new tokens: tensor-core kernel only, no fused append
-    if ((k_head_scales || v_head_scales) &&
-        (!k_head_scales || !v_head_scales || !is_fp8(kv_dtype) ||
-         !(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads))))
-        return PKV_ERR_SHAPE;   // per-head scales: both arrays, FP8 caches, tensor-core kernel
-    if (!((q_dtype == PKV_F32 && kv_dtype == PKV_F32) || (q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
-          (q_dtype == PKV_BF16 && is_fp8(kv_dtype))))
-        return PKV_ERR_DTYPE;
-    if (num_seqs == 0)
-        return PKV_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
-        return PKV_ERR_NULL;
-    if (!workspace)
-        return PKV_ERR_WORKSPACE;
-    if (max_blocks_per_seq <= 0 || num_blocks <= 0)
-        return PKV_ERR_SHAPE;
-    if ((long long)num_seqs * max_blocks_per_seq * num_kv_heads >= (1ll << 31) ||
-        (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
-        (long long)num_blocks * num_kv_heads * block_size >= (1ll << 31))
-        return PKV_ERR_SHAPE;
-    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
-        return PKV_ERR_SHAPE;
-
-    int runs = num_partitions;
-    if (runs == 0) {
-        const int dev = current_device();
-        const int sms = dev >= 0 ? sm_count(dev) : 0;
-        if (sms <= 0)
-            return PKV_ERR_DEVICE;
-        DecodeParams probe;
-        std::memset(&probe, 0, sizeof probe);
-        probe.num_seqs = num_seqs;
-        probe.num_kv_heads = num_kv_heads;
-        int occ = 0;
-        const int st = decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, probe, 0, nullptr, &occ);
-        if (st != PKV_OK)
-            return st;
-        if (occ < 1)
-            return PKV_ERR_SHAPE;
-        runs = sms * (occ > kMaxRunsPerSM ? kMaxRunsPerSM : occ);
-    }
-    const WorkspaceLayout lay = layout_for(num_seqs, num_kv_heads, group, head_dim, runs);
-    if (workspace_bytes < lay.bytes)
-        return PKV_ERR_WORKSPACE;
-
-    const bool fp8 = is_fp8(kv_dtype);
     DecodeParams p;
-    std::memset(&p, 0, sizeof p);
-    p.out = out;
-    p.q = q;
-    p.k_cache = static_cast<const uint8_t*>(k_cache);
-    p.v_cache = static_cast<const uint8_t*>(v_cache);
-    p.block_tables = block_tables;
-    p.seq_lens = seq_lens;
-    p.num_seqs = num_seqs;
-    p.num_heads = num_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.max_blocks_per_seq = max_blocks_per_seq;
-    p.num_blocks = num_blocks;
-    p.scale = scale;
-    p.k_scale = fp8 ? k_scale : 1.0f;
-    p.v_scale_in = fp8 ? v_scale : 1.0f;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    p.err = reinterpret_cast<int32_t*>(ws);
-    p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
-    p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
-    p.slot_floats = slot_floats_for(group, head_dim);
-    p.q_len = q_len;
-    p.k_head_scales = k_head_scales;
-    p.v_head_scales = v_head_scales;
-    if (withheld_unit >= 0) {
-        if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
-            return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
-        p.withheld_unit = withheld_unit + 1;
-    }
-    if (app) {
-        p.new_k = app->k;
-        p.new_v = app->v;
-        p.new_slots = app->slots;
-        p.in_dtype = app->in_dtype;
-    }
-    return decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, group, p, runs,
+    int runs = 0;
+    const int st = decode_prepare(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                                  head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype,
+                                  k_scale, v_scale, num_partitions, workspace, workspace_bytes, app, withheld_unit,
+                                  q_len, k_head_scales, v_head_scales, &p, &runs);
+    if (st != PKV_OK || runs == 0)
+        return st;
+    return decode_dispatch(q_dtype, kv_dtype, head_dim, block_size, num_heads / num_kv_heads * q_len, p, runs,
                            static_cast<cudaStream_t>(stream), nullptr);
 }
 

@@ -74,6 +74,24 @@ int cache_dispatch(const void* k, const void* v, void* k_cache, void* v_cache, c
                    int in_dtype, int kv_dtype, float k_scale, float v_scale, const float* k_head_scales,
                    const float* v_head_scales, int32_t* err, cudaStream_t stream);
 
+// Rows of the decode-step append (paged_decode_step): row s of k / v goes to slots[s].
+struct AppendArgs {
+    const void* k;
+    const void* v;
+    const int64_t* slots;
+    int in_dtype;
+};
+
+// Host checks of a decode call (what paged_attention_decode validates before launching), the
+// partition count and the kernels' parameters; queues nothing. Returns a pkv_status; on PKV_OK,
+// *runs is the partition count to launch with, or 0 when there is nothing to launch.
+int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                   const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                   int block_size, float scale, int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                   float k_scale, float v_scale, int num_partitions, void* workspace, size_t workspace_bytes,
+                   const AppendArgs* app, int withheld_unit, int q_len, const float* k_head_scales,
+                   const float* v_head_scales, DecodeParams* p_out, int* runs);
+
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device (cached).
 bool ensure_smem_attribute(const void* kernel, size_t bytes);
 

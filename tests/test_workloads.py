@@ -90,3 +90,16 @@ def test_batch_layout_is_build_batch_tables():
         lay = W.batch_layout(b.spec)
         assert np.array_equal(lay.seq_lens, b.seq_lens) and np.array_equal(lay.block_tables, b.block_tables)
         assert lay.num_blocks == b.num_blocks
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+def test_with_cache_dtype_equals_a_fresh_draw(kv):
+    """Re-typing a drawn batch gives exactly what build_batch draws with the cache dtype replaced."""
+    spec = W.config_spec(1)
+    spec.num_seqs = 6
+    a = W.with_cache_dtype(W.build_batch(spec), kv)
+    spec.kv_dtype = kv
+    b = W.build_batch(spec)
+    assert a.spec.kv_dtype == kv and a.k_scale == b.k_scale and a.v_scale == b.v_scale
+    for f in ("seq_lens", "block_tables", "q", "hist_k", "hist_v", "hist_slots", "new_k", "new_v", "new_slots"):
+        assert np.array_equal(getattr(a, f), getattr(b, f)), f

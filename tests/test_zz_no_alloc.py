@@ -1,8 +1,8 @@
 """paged_attention_decode_static: the decode entry point that allocates nothing.
 
-It serves callers that cannot allocate device memory (graph capture, plug-ins
-whose host owns all allocations); its scratch is a fixed array inside the
-library. Called through the C ABI, twice in a row, it must give the output of
+It serves callers that cannot allocate device memory (plug-ins whose host
+framework owns every allocation, hosts that reserve all memory at start-up);
+its scratch is a fixed array inside the library. Called through the C ABI, twice in a row, it must give the output of
 paged_attention_decode with a caller workspace, within the parity tolerance.
 This file is collected last so that a failure here comes after every other test.
 """

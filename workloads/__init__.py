@@ -178,6 +178,18 @@ def _absmax(x: np.ndarray, dtype_name: str) -> np.float32:
     return np.float32(np.abs(x).max())
 
 
+def _cache_scales(kv_dtype, in_dtype, hist_k, hist_v, new_k, new_v):
+    """Per-tensor scales of an 8-bit cache: the absmax of every K (V) value written to the cache
+    maps to the format's largest finite value (448 for E4M3, 57344 for E5M2, 127 for INT8);
+    1 for f32 / bf16 caches."""
+    if kv_dtype in ("e4m3", "e5m2", "int8"):
+        top = np.float32({"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[kv_dtype])
+        k_scale = np.float32(max(_absmax(hist_k, in_dtype), _absmax(new_k, in_dtype)) / top)
+        v_scale = np.float32(max(_absmax(hist_v, in_dtype), _absmax(new_v, in_dtype)) / top)
+        return k_scale, v_scale
+    return np.float32(1.0), np.float32(1.0)
+
+
 @dataclass
 class Layout:
     """Lengths and block tables of a batch, before any tensor is drawn."""
@@ -279,15 +291,7 @@ def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
             pos = L - 1
             new_slots[s] = int(tables[s, pos // bs]) * bs + pos % bs
 
-    if spec.kv_dtype in ("e4m3", "e5m2", "int8"):
-        # per-tensor scales: absmax of every K (V) value written to the cache maps to the format's
-        # largest finite value (448 for E4M3, 57344 for E5M2, 127 for INT8)
-        top = np.float32({"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[spec.kv_dtype])
-        k_scale = np.float32(max(_absmax(hist_k, spec.in_dtype), _absmax(new_k, spec.in_dtype)) / top)
-        v_scale = np.float32(max(_absmax(hist_v, spec.in_dtype), _absmax(new_v, spec.in_dtype)) / top)
-    else:
-        k_scale = np.float32(1.0)
-        v_scale = np.float32(1.0)
+    k_scale, v_scale = _cache_scales(spec.kv_dtype, spec.in_dtype, hist_k, hist_v, new_k, new_v)
 
     scale = np.float32(1.0 / math.sqrt(d))
     shared = int(sum(n for members, n in groups if len(members) > 1)) if groups else 0
@@ -313,3 +317,22 @@ def subset_tokens(batch: DecodeBatch, seqs) -> np.ndarray:
         blocks.update(int(p) for p in batch.block_tables[s, :nb[s]])
     blk = batch.hist_slots // bs
     return np.nonzero(np.isin(blk, np.fromiter(blocks, dtype=np.int64, count=len(blocks))))[0]
+
+
+def with_cache_dtype(batch: DecodeBatch, kv_dtype: str) -> DecodeBatch:
+    """The same batch (lengths, tables, q, K, V, new rows: the arrays are shared, not copied) with
+    another cache dtype and that dtype's per-tensor scales: what ``build_batch`` draws for the spec
+    with ``kv_dtype`` replaced, without drawing the tensors again."""
+    import copy
+    sp = copy.copy(batch.spec)
+    if kv_dtype != sp.kv_dtype:
+        if sp.in_dtype != "bf16" or kv_dtype not in ("bf16", "e4m3", "e5m2", "int8"):
+            raise ValueError(f"cannot re-type a {sp.in_dtype}-row batch to a {kv_dtype} cache")
+        sp.kv_dtype = kv_dtype
+        sp.name = f"{sp.name}_{kv_dtype}kv"
+    b = copy.copy(batch)
+    b.spec = sp
+    b.k_scale, b.v_scale = _cache_scales(kv_dtype, sp.in_dtype, batch.hist_k, batch.hist_v, batch.new_k,
+                                         batch.new_v)
+    b.extra = dict(batch.extra)
+    return b
