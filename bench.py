@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle sample length for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefix-sharing", choices=["auto", "on", "off"], default="auto",
+                    help="shared-prefix decode (blocks a plan shares read once per group): auto = on for "
+                         "workloads whose sequences share prefix blocks (config 3)")
     ap.add_argument("--no-targets", action="store_true",
                     help="skip the extra target points (long-context and mixed batch, bf16 and E4M3 caches)")
     return ap.parse_args()
@@ -89,12 +92,17 @@ def describe(b: W.DecodeBatch) -> str:
             + (f", prefix groups of {sp.share_group} sharing <= {sp.share_blocks} blocks" if sp.share_group else ""))
 
 
-def step_bytes(b: W.DecodeBatch, q_len: int = 1):
-    """Algorithmic bytes of the step: decode (q/out rows scale with q_len), and the append (none
-    in the multi-query form, whose new tokens are already in the cache)."""
+def step_bytes(b: W.DecodeBatch, q_len: int = 1, plan=None):
+    """Algorithmic bytes of the step: decode (q/out rows scale with q_len; with a shared-prefix
+    plan the table entries of shared blocks are replaced by the plan's arrays), and the append
+    (none in the multi-query form, whose new tokens are already in the cache)."""
     sp = b.spec
     dec = acct.decode_bytes(b.seq_lens, b.block_tables, sp.num_heads * q_len, sp.num_kv_heads, sp.head_dim,
                             sp.block_size, sp.kv_dtype, sp.q_dtype)
+    if plan is not None:
+        pb = acct.plan_bytes(b.seq_lens, sp.block_size, plan)
+        dec["tables"] += pb["plan"] - pb["tables_saved"]
+        dec["total"] += pb["plan"] - pb["tables_saved"]
     app = 0 if q_len > 1 else acct.append_bytes(int((b.new_slots >= 0).sum()), sp.num_kv_heads, sp.head_dim,
                                                 sp.in_dtype, sp.kv_dtype)
     return dec, app
@@ -273,6 +281,7 @@ class DeviceState:
         self.out = torch.empty_like(self.q)
         self.partitions = partitions
         self.q_len = 1
+        self.plan = None
         self.ws = pkv.new_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim, partitions, device)
         for i in range(0, b.hist_slots.size, 1 << 16):      # history already in the cache before the step
             pkv.reshape_and_cache(self._dev(b.hist_k[i:i + (1 << 16)], sp.in_dtype),
@@ -297,10 +306,31 @@ class DeviceState:
         self.pkv.paged_attention_decode(self.out, self.q, self.kc, self.vc, self.bt, self.sl, float(b.scale),
                                         float(b.k_scale), float(b.v_scale), self.partitions, self.ws)
 
+    def use_prefix_plan(self, max_group: int = 8):
+        """Decode with the shared-prefix kernels: the plan of the batch's tables (pkv_prefix_plan,
+        computed once on the host: the sharing structure changes when sequences fork or finish,
+        not every step) copied to the device, and a workspace sized for its groups."""
+        from paged_kv_cache_462_b200 import blocks
+        t0 = time.perf_counter()
+        plan = blocks.prefix_plan(self.b.block_tables, self.b.seq_lens, self.b.spec.block_size, max_group)
+        self.plan_host_ms = 1e3 * (time.perf_counter() - t0)
+        self.plan = self.pkv.DevicePrefixPlan(plan, max_group, self.dev)
+        sp = self.b.spec
+        self.ws = self.pkv.new_shared_prefix_workspace(sp.num_seqs, sp.num_heads, sp.num_kv_heads, sp.head_dim,
+                                                       self.plan.num_groups, self.partitions, self.dev)
+        return plan
+
     def step(self):
         """append + decode through paged_decode_step (one launch where the fused kernel applies);
-        with q_len > 1 the causal multi-query decode of the last q_len tokens of every sequence"""
+        with a prefix plan paged_decode_step_shared_prefix (prefix pass, suffix pass with the
+        append, merge); with q_len > 1 the causal multi-query decode of the last q_len tokens of
+        every sequence"""
         b = self.b
+        if self.plan is not None:
+            self.pkv.paged_decode_step_shared_prefix(self.out, self.q, self.kc, self.vc, self.bt, self.sl, self.plan,
+                                                     self.new_k, self.new_v, self.new_slots, float(b.scale),
+                                                     float(b.k_scale), float(b.v_scale), self.partitions, self.ws)
+            return
         if self.q_len > 1:
             self.pkv.paged_attention_decode_mq(self.out_mq, self.q_mq, self.kc, self.vc, self.bt, self.sl,
                                                float(b.scale), float(b.k_scale), float(b.v_scale), self.partitions,
@@ -436,6 +466,13 @@ def reference_arm(args):
     return 0
 
 
+def use_prefix_plan(args, spec) -> bool:
+    """The shared-prefix decode for workloads whose sequences share prefix blocks (or when asked)."""
+    if args.q_len != 1 or args.prefix_sharing == "off" or spec.kv_dtype == "f32":
+        return False
+    return args.prefix_sharing == "on" or spec.share_group > 1
+
+
 def time_steps(torch, state, K: int, warmup: int, flush_l2, stream, dev):
     """W untimed steps, then K steps each bracketed by CUDA events on the launching stream, with
     the L2 flush between steps outside the events. Returns (per-step ms, wall start, wall end of
@@ -481,7 +518,8 @@ def ours_arm(args):
     b = W.build_batch(spec, seed=spec.seed + 1000 * rank)
     state = DeviceState(torch, pkv, b, dev, args.partitions)
     state.set_q_len(args.q_len)
-    dec, app = step_bytes(b, args.q_len)
+    plan = state.use_prefix_plan(spec.share_group) if use_prefix_plan(args, spec) else None
+    dec, app = step_bytes(b, args.q_len, plan)
     bytes_step = dec["total"] + app
     # a read (not a write) of a buffer twice the size of L2: the L2 ends up holding clean lines of
     # another buffer, as after the weight-streaming GEMMs that precede attention in a decode step
@@ -507,7 +545,11 @@ def ours_arm(args):
     e2e = None
     if not args.no_e2e:
         names = ("q_mq", "sl", "bt") if args.q_len > 1 else ("q", "new_k", "new_v", "new_slots", "sl", "bt")
-        host = {n: getattr(state, n).detach().cpu().pin_memory() for n in names}
+        dev_in = {n: getattr(state, n) for n in names}
+        if state.plan is not None:   # the plan's arrays travel with the tables they come from
+            dev_in.update({f"plan_{n}": getattr(state.plan, n) for n in ("members", "offsets", "tables", "lens",
+                                                                          "shared")})
+        host = {n: t.detach().cpu().pin_memory() for n, t in dev_in.items()}
         dev_out = state.out_mq if args.q_len > 1 else state.out
         out_h = torch.empty(dev_out.shape, dtype=dev_out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -520,7 +562,7 @@ def ours_arm(args):
             if rec:
                 ee[i - args.warmup][0].record(stream)
             for n, t in host.items():
-                getattr(state, n).copy_(t, non_blocking=True)
+                dev_in[n].copy_(t, non_blocking=True)
             state.step()
             out_h.copy_(dev_out, non_blocking=True)
             if rec:
@@ -544,7 +586,8 @@ def ours_arm(args):
                                                               seed=W.config_spec(cfg).seed + 1000 * rank)}
             tb = W.with_cache_dtype(batches[cfg], kv)
             ts = DeviceState(torch, pkv, tb, dev, 0)
-            tdec, tapp = step_bytes(tb)
+            tplan = ts.use_prefix_plan(tb.spec.share_group) if use_prefix_plan(args, tb.spec) else None
+            tdec, tapp = step_bytes(tb, 1, tplan)
             tbytes = tdec["total"] + tapp
             if dist:
                 dist.barrier()
@@ -552,6 +595,7 @@ def ours_arm(args):
             terr = ts.errors()
             agg_t = aggregate_ranks(torch, dist, dev, ms=sum(tms) / K, step_bytes=float(tbytes), errors=float(terr))
             targets.append({"config_index": cfg, "kv_storage": kv, "workload": describe(tb),
+                            "prefix_groups": tplan.num_groups if tplan is not None else 0,
                             "ms_per_step": agg_t["ms"], "value": agg_t["step_bytes"] / (agg_t["ms"] * 1e-3) / 1e9,
                             "unit": "GB/s", "algorithmic_bytes": tbytes,
                             "kv_logical_gbs": tdec["kv_logical"] / (sum(tms) / K * 1e-3) / 1e9,
@@ -596,6 +640,9 @@ def ours_arm(args):
                     {"f32": 0, "bf16": 1, "e4m3": 2, "e5m2": 3, "int8": 4}[spec.kv_dtype]),
                 "step": (f"paged_attention_decode_mq: the last {args.q_len} tokens of every sequence as queries, "
                          "causal within the chunk (their K/V already cached)" if args.q_len > 1 else
+                         f"paged_decode_step_shared_prefix: prefix pass over the {plan.num_groups} groups' shared "
+                         f"blocks (plan made once on the host in {state.plan_host_ms:.2f} ms, outside the timed "
+                         "region), suffix pass with the append fused, merge" if plan is not None else
                          "paged_decode_step: append of one new token per sequence fused into the paged "
                          "decode launch" if fused else
                          "paged_decode_step: reshape_and_cache then paged_attention_decode (two launches)"),
@@ -609,7 +656,9 @@ def ours_arm(args):
             "roofline": {
                 "bound": "hbm",
                 # events bracket the whole step: the decode kernel (append fused) and its merge kernel
-                "kernel": ("paged_decode_mma_kernel (append fused) + paged_decode_merge_kernel" if fused
+                "kernel": ("paged_decode_mma_kernel prefix pass + suffix pass (append fused) + "
+                           "paged_decode_prefix_merge_kernel" if plan is not None and plan.num_groups > 0 else
+                           "paged_decode_mma_kernel (append fused) + paged_decode_merge_kernel" if fused
                            else "reshape_and_cache_kernel + paged_decode_kernel"),
                 "achieved": kern_gbs,
                 "peak": peak,
@@ -620,7 +669,7 @@ def ours_arm(args):
                 "algorithmic_bytes": kern_bytes,
             },
             # fused: the decode kernel (append inside) + the merge kernel; else append + decode
-            "gpu_launches": 2 * K,
+            "gpu_launches": (3 if plan is not None and plan.num_groups > 0 else 2) * K,
             "clocks": clocks.summary(t_on, t_off) if clocks else None,
             "device_errors": errs_all,
         }

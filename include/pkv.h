@@ -95,6 +95,7 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3, PK
 #define PKV_DEVERR_SEQ_LEN 2   /* seq_len < 0 or > max_blocks_per_seq * block_size: clamped */
 #define PKV_DEVERR_SLOT 4      /* append slot >= num_blocks * block_size: row skipped */
 #define PKV_DEVERR_TIMEOUT 8   /* a bounded pipeline wait gave up (output incomplete) */
+#define PKV_DEVERR_PLAN 16     /* a shared-prefix plan entry out of range: that sequence's output is unspecified */
 
 /*
  * Bytes of device workspace paged_attention_decode needs: an error word, one
@@ -215,6 +216,70 @@ PKV_API int paged_attention_decode_mq(void* out, const void* q, const void* k_ca
                                       float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
                                       int kv_dtype, float k_scale, float v_scale, int num_partitions,
                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Shared-prefix decode. Prefix caching reuses whole blocks: sequences whose
+ * tables hold the same physical block hold the same tokens there (wzjinhao.cn
+ * vLLM write-up, section 2.3 "Chunked Prefill and Prefix Caching";
+ * "vLLM inference cost optimisation", section 11). Given a plan of such
+ * sharing (pkv_prefix_plan in pkv_blocks.h, on the same tables), this call
+ * reads every shared block once for all the sequences of its group: a prefix
+ * pass attends the queries of up to max_group members (max_group *
+ * num_heads / num_kv_heads <= 32 query columns per KV head) against each
+ * shared block, each member seeing only its own shared blocks; a suffix pass
+ * attends each sequence over the rest of its table; a merge combines the two
+ * by their log-sum-exp weights. The output equals paged_attention_decode's
+ * (same softmax over the same tokens, up to the order of the fp32 sums).
+ *
+ * The plan (device arrays, caller-owned, pkv_prefix_plan's outputs):
+ *   group_members  int32, members of group g at [group_offsets[g], group_offsets[g + 1])
+ *   group_offsets  int32 [num_groups + 1]
+ *   group_tables   int32 [num_groups][max_blocks_per_seq]: row g = the group's shared blocks
+ *   group_lens     int32 [num_groups]: tokens in row g (its blocks x block_size)
+ *   shared_blocks  int32 [num_seqs]: leading (full) blocks of sequence s read through its
+ *                  group's row; > 0 only for members of a group
+ *   num_groups     0 .. num_seqs (0: the plain decode, bit for bit)
+ * Tensor-core shapes only (bf16 q; bf16, E4M3, E5M2 or INT8 caches; block 16 or
+ * 32; head_dim 128, or 64 for bf16); no per-head scales, one query per sequence.
+ * workspace >= paged_attention_shared_prefix_workspace_size(num_seqs, num_heads,
+ * num_kv_heads, head_dim, num_groups, num_partitions) bytes, zeroed once.
+ * Errors: host checks as paged_attention_decode (PKV_ERR_SHAPE also for
+ * max_group * num_heads / num_kv_heads > 32); a group with more than max_group
+ * members, a member index outside [0, num_seqs) or a shared count beyond a
+ * sequence's full blocks or its group's row sets PKV_DEVERR_PLAN, and the
+ * outputs of the sequences concerned are unspecified. Launches: the prefix pass
+ * (when num_groups > 0), the suffix pass and the merge, in order on `stream`.
+ */
+PKV_API size_t paged_attention_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                                            int head_dim, int num_groups, int num_partitions);
+PKV_API int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                                 const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                                 float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                                                 int kv_dtype, float k_scale, float v_scale,
+                                                 const int32_t* group_members, const int32_t* group_offsets,
+                                                 const int32_t* group_tables, const int32_t* group_lens,
+                                                 const int32_t* shared_blocks, int num_groups, int max_group,
+                                                 int num_partitions, void* workspace, size_t workspace_bytes,
+                                                 void* stream);
+/*
+ * The decode step of paged_decode_step with the shared-prefix decode: the append
+ * of each sequence's new token rides in the suffix pass's launch (the block
+ * holding position seq_lens[s] - 1 must be the sequence's own, i.e. past its
+ * shared blocks; otherwise PKV_DEVERR_SLOT). Arguments as
+ * paged_attention_decode_shared_prefix plus those of paged_decode_step.
+ */
+PKV_API int paged_decode_step_shared_prefix(void* out, const void* q, void* k_cache, void* v_cache,
+                                            const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                            int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                            float scale, int max_blocks_per_seq, int num_blocks, int q_dtype,
+                                            int kv_dtype, float k_scale, float v_scale,
+                                            const int32_t* group_members, const int32_t* group_offsets,
+                                            const int32_t* group_tables, const int32_t* group_lens,
+                                            const int32_t* shared_blocks, int num_groups, int max_group,
+                                            int num_partitions, void* workspace, size_t workspace_bytes,
+                                            const void* new_k, const void* new_v, const int64_t* slot_mapping,
+                                            int in_dtype, void* stream);
 
 /*
  * Test hook for the failure path (no counterpart in the pages). The same call

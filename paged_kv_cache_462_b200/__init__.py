@@ -25,7 +25,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libpagedkv.so")
 
 F32, BF16, FP8_E4M3, FP8_E5M2, INT8 = 0, 1, 2, 3, 4
-DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_PLAN = 1, 2, 4, 8, 16
 
 # uint8 caches hold E4M3 codes; E5M2 caches are passed as torch.float8_e5m2 tensors
 _TORCH_DTYPE = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3,
@@ -76,6 +76,16 @@ def load_library():
     lib.pkv_read_device_error.restype = i32
     lib.pkv_default_partitions.argtypes = [i32, i32, i32, i32, i32]
     lib.pkv_default_partitions.restype = i32
+    lib.paged_attention_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.paged_attention_shared_prefix_workspace_size.restype = sz
+    lib.paged_attention_decode_shared_prefix.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32,
+                                                         i32, i32, f32, f32, P, P, P, P, P, i32, i32, i32, P, sz,
+                                                         P]
+    lib.paged_attention_decode_shared_prefix.restype = i32
+    lib.paged_decode_step_shared_prefix.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32,
+                                                    i32, f32, f32, P, P, P, P, P, i32, i32, i32, P, sz, P, P, P,
+                                                    i32, P]
+    lib.paged_decode_step_shared_prefix.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -319,6 +329,109 @@ def read_device_error(workspace: torch.Tensor, clear: bool = False, stream=None)
     return int(v.value)
 
 
+class DevicePrefixPlan:
+    """A shared-prefix plan (``blocks.prefix_plan``'s result) copied to the device as the
+    shared-prefix decode reads it: int32 members, offsets [groups + 1], tables [groups, max_blocks],
+    lens [groups], shared [num_seqs]; ``max_group`` is the planner's group-size limit."""
+
+    def __init__(self, plan, max_group: int, device=None):
+        import numpy as np
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        self.num_groups = int(plan.num_groups)
+        self.max_group = int(max_group)
+        self.members = t(plan.members)
+        self.offsets = t(plan.offsets[: self.num_groups + 1])
+        self.tables = t(plan.tables[: self.num_groups])
+        self.lens = t(plan.lens[: self.num_groups])
+        self.shared = t(plan.shared)
+
+    def tensors(self):
+        return (self.members, self.offsets, self.tables, self.lens, self.shared)
+
+
+def shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_groups, num_partitions=0) -> int:
+    n = load_library().paged_attention_shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim,
+                                                                    num_groups, num_partitions)
+    if n == 0:
+        raise PkvError("paged_attention_shared_prefix_workspace_size", 2)
+    return int(n)
+
+
+def new_shared_prefix_workspace(num_seqs, num_heads, num_kv_heads, head_dim, num_groups, num_partitions=0,
+                                device=None) -> torch.Tensor:
+    """A zeroed workspace for the shared-prefix decode."""
+    n = shared_prefix_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_groups, num_partitions)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _plan_args(plan: DevicePrefixPlan, dev, S, MB):
+    if not isinstance(plan, DevicePrefixPlan):
+        raise TypeError("plan must be a DevicePrefixPlan")
+    if plan.shared.shape != (S,) or (plan.num_groups and plan.tables.shape[1] != MB):
+        raise ValueError("plan does not match the batch (shared [num_seqs], tables [groups, max_blocks])")
+    ptr = lambda name, t: _cuda(name, t, dev) if t.numel() else ctypes.c_void_p(None)
+    return (ptr("plan.members", plan.members), ptr("plan.offsets", plan.offsets), ptr("plan.tables", plan.tables),
+            ptr("plan.lens", plan.lens), _cuda("plan.shared", plan.shared, dev), plan.num_groups, plan.max_group)
+
+
+def _shared_prefix_workspace(workspace, S, Hq, Hkv, D, plan, num_partitions, dev):
+    if workspace is not None:
+        return workspace
+    n = shared_prefix_workspace_size(S, Hq, Hkv, D, plan.num_groups, num_partitions)
+    return torch.zeros(n, dtype=torch.uint8, device=torch.device("cuda", dev))
+
+
+def paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, plan, scale,
+                                         k_scale=1.0, v_scale=1.0, num_partitions=0, workspace=None,
+                                         stream=None) -> None:
+    """paged_attention_decode with the blocks a plan shares read once per group (a prefix pass over
+    the groups' shared rows, a suffix pass over each sequence's own blocks, a log-sum-exp merge)."""
+    dev = _launch_device("q", q)
+    S, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape) or k_cache.shape[3] != D:
+        raise ValueError("shape mismatch between q/out and the caches")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or block_tables.dim() != 2 \
+            or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be int32 [num_seqs, max_blocks] and seq_lens int32 [num_seqs]")
+    ws = _shared_prefix_workspace(workspace, S, Hq, Hkv, D, plan, num_partitions, dev)
+    st = load_library().paged_attention_decode_shared_prefix(
+        _cuda("out", out, dev), _cuda("q", q, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("block_tables", block_tables, dev), _cuda("seq_lens", seq_lens, dev), S, Hq, Hkv, D, BS,
+        float(scale), block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale),
+        float(v_scale), *_plan_args(plan, dev, S, block_tables.shape[1]), int(num_partitions),
+        _cuda("workspace", ws, dev), ws.numel(), _stream_handle(stream))
+    _check("paged_attention_decode_shared_prefix", st)
+
+
+def paged_decode_step_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens, plan, new_k, new_v,
+                                    slot_mapping, scale, k_scale=1.0, v_scale=1.0, num_partitions=0, workspace=None,
+                                    stream=None) -> None:
+    """paged_decode_step with the shared-prefix decode (the append rides in the suffix pass)."""
+    dev = _launch_device("q", q)
+    S, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape) or k_cache.shape[3] != D:
+        raise ValueError("shape mismatch between q/out and the caches")
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or block_tables.dim() != 2 \
+            or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be int32 [num_seqs, max_blocks] and seq_lens int32 [num_seqs]")
+    if tuple(new_k.shape) != (S, Hkv, D) or tuple(new_v.shape) != (S, Hkv, D) or new_v.dtype != new_k.dtype:
+        raise ValueError("new_k/new_v must be [num_seqs, num_kv_heads, head_dim] of one dtype")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.shape != (S,):
+        raise TypeError("slot_mapping must be int64 [num_seqs]")
+    ws = _shared_prefix_workspace(workspace, S, Hq, Hkv, D, plan, num_partitions, dev)
+    st = load_library().paged_decode_step_shared_prefix(
+        _cuda("out", out, dev), _cuda("q", q, dev), _cuda("k_cache", k_cache, dev), _cuda("v_cache", v_cache, dev),
+        _cuda("block_tables", block_tables, dev), _cuda("seq_lens", seq_lens, dev), S, Hq, Hkv, D, BS,
+        float(scale), block_tables.shape[1], NB, _dtype_code(q), _dtype_code(k_cache), float(k_scale),
+        float(v_scale), *_plan_args(plan, dev, S, block_tables.shape[1]), int(num_partitions),
+        _cuda("workspace", ws, dev), ws.numel(), _cuda("new_k", new_k, dev), _cuda("new_v", new_v, dev),
+        _cuda("slot_mapping", slot_mapping, dev), _dtype_code(new_k), _stream_handle(stream))
+    _check("paged_decode_step_shared_prefix", st)
+
+
 _ws_cache: dict = {}
 
 
@@ -342,5 +455,7 @@ __all__ = [
     "paged_attention_decode", "paged_decode_step", "paged_attention_decode_mq", "paged_attention_decode_head_scales",
     "reshape_and_cache", "reshape_and_cache_head_scales", "workspace_size", "new_workspace", "workspace_init",
     "read_device_error", "default_partitions", "status_string", "load_library", "PkvError",
+    "paged_attention_decode_shared_prefix", "paged_decode_step_shared_prefix", "DevicePrefixPlan",
+    "shared_prefix_workspace_size", "new_shared_prefix_workspace",
     "F32", "BF16", "FP8_E4M3", "FP8_E5M2", "INT8",
 ]

@@ -40,6 +40,19 @@ def decode_bytes(seq_lens, block_tables, num_heads, num_kv_heads, head_dim, bloc
                 unique_blocks=unique_blocks, total=kv_unique + q_out + tables)
 
 
+def plan_bytes(seq_lens, block_size, plan) -> dict:
+    """Change in the bytes a shared-prefix decode reads besides K/V, q and out: the block-table
+    entries of the shared blocks are not read (their group's row is, once per group), and the
+    plan's arrays are (members, offsets, row lengths, per-sequence shared counts). Returns
+    {"tables_saved": bytes, "plan": bytes}."""
+    shared = np.asarray(plan.shared, dtype=np.int64)
+    groups = int(plan.num_groups)
+    members = int(np.asarray(plan.offsets)[groups]) if groups else 0
+    group_blocks = int((np.asarray(plan.lens[:groups], dtype=np.int64) // block_size).sum()) if groups else 0
+    return {"tables_saved": 4 * int(shared.sum()),
+            "plan": 4 * (group_blocks + members + (groups + 1) + groups + shared.size)}
+
+
 def append_bytes(num_tokens, num_kv_heads, head_dim, in_dtype, kv_dtype) -> int:
     """reshape_and_cache: read the K and V rows and their slot, write the cache rows."""
     rows = 2 * num_tokens * num_kv_heads * head_dim

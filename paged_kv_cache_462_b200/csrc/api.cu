@@ -468,6 +468,166 @@ int paged_decode_step(void* out, const void* q, void* k_cache, void* v_cache, co
 
 namespace {
 
+// Bytes of the prefix pass's partials: a slot of 8 columns x (head_dim + 2) floats for every
+// (run + stream) x column tile, streams = groups x KV heads.
+size_t prefix_partials_bytes(int num_groups, int num_kv_heads, int head_dim, long long runs_p)
+{
+    if (num_groups <= 0)
+        return 0;   // no prefix pass
+    const size_t slot = round_up((size_t)8 * (head_dim + 2), 4) * 4;
+    return (size_t)(runs_p + (long long)num_groups * num_kv_heads) * 4 * slot;
+}
+
+int shared_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
+                       int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                       int num_blocks, int q_dtype, int kv_dtype, float k_scale, float v_scale,
+                       const int32_t* group_members, const int32_t* group_offsets, const int32_t* group_tables,
+                       const int32_t* group_lens, const int32_t* shared_blocks, int num_groups, int max_group,
+                       int num_partitions, void* workspace, size_t workspace_bytes, const AppendArgs* app,
+                       void* stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+        num_groups < 0 || num_groups > num_seqs || max_group < 1)
+        return PKV_ERR_SHAPE;
+    const int Gq = num_heads / num_kv_heads;
+    if (max_group * Gq > 32)
+        return PKV_ERR_SHAPE;   // a group's queries of one KV head fill at most 4 column tiles of 8
+    if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, Gq, num_kv_heads)))
+        return q_dtype == PKV_BF16 && (kv_dtype == PKV_BF16 || is_fp8(kv_dtype)) ? PKV_ERR_SHAPE : PKV_ERR_DTYPE;
+    if (num_seqs == 0)
+        return PKV_OK;
+    if (!shared_blocks || (num_groups > 0 && (!group_members || !group_offsets || !group_tables || !group_lens)))
+        return PKV_ERR_NULL;
+    DecodeParams ps;
+    int runs_s = 0;
+    int st = decode_prepare(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                            head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                            v_scale, num_partitions, workspace, workspace_bytes, app, -1, 1, nullptr, nullptr, &ps,
+                            &runs_s);
+    if (st != PKV_OK || runs_s == 0)
+        return st;
+    ps.skip_blocks = shared_blocks;
+
+    int runs_p = num_partitions;
+    const int HG = mma_head_group(kv_dtype, head_dim, block_size, num_kv_heads);
+    if (runs_p == 0) {
+        const int dev = current_device();
+        const int sms = dev >= 0 ? sm_count(dev) : 0;
+        if (sms <= 0)
+            return PKV_ERR_DEVICE;
+        DecodeParams probe;
+        std::memset(&probe, 0, sizeof probe);
+        probe.num_seqs = num_groups;
+        probe.num_kv_heads = num_kv_heads;
+        int occ = 0;
+        MmaOp op{};
+        op.kind = MmaOp::kPrefixOccupancy;
+        op.p = &probe;
+        op.occ = &occ;
+        st = decode_mma_op(kv_dtype, head_dim, block_size, Gq, HG, op);
+        if (st != PKV_OK)
+            return st;
+        if (occ < 1)
+            return PKV_ERR_SHAPE;
+        runs_p = sms * (occ > kMaxRunsPerSM ? kMaxRunsPerSM : occ);
+    }
+    const size_t suffix_bytes = layout_for(num_seqs, num_kv_heads, Gq, head_dim, runs_s).bytes;
+    const size_t prefix_off = round_up(suffix_bytes, 256);
+    if (workspace_bytes < prefix_off + prefix_partials_bytes(num_groups, num_kv_heads, head_dim, runs_p))
+        return PKV_ERR_WORKSPACE;
+
+    DecodeParams pp = ps;
+    pp.num_seqs = num_groups;
+    pp.seq_lens = group_lens;
+    pp.block_tables = group_tables;
+    pp.skip_blocks = nullptr;
+    pp.new_k = pp.new_v = nullptr;
+    pp.new_slots = nullptr;
+    pp.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + prefix_off);
+    pp.slot_floats = (int)round_up((size_t)8 * (head_dim + 2), 4);
+    pp.pfx_members = group_members;
+    pp.pfx_offsets = group_offsets;
+    pp.pfx_shared = shared_blocks;
+    pp.pfx_max_group = max_group;
+    pp.pfx_num_seqs = num_seqs;
+
+    MmaOp op{};
+    op.kind = MmaOp::kLaunchSharedPrefix;
+    op.p = &ps;
+    op.pp = &pp;
+    op.nruns = runs_s;
+    op.runs_p = runs_p;
+    op.stream = static_cast<cudaStream_t>(stream);
+    return decode_mma_op(kv_dtype, head_dim, block_size, Gq, HG, op);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t paged_attention_shared_prefix_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                                    int num_groups, int num_partitions)
+{
+    const size_t base = paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions);
+    if (base == 0 || num_groups < 0)
+        return 0;
+    long long runs = num_partitions;
+    if (runs == 0) {
+        const int dev = current_device();
+        const int sms = dev >= 0 ? sm_count(dev) : 0;
+        if (sms <= 0)
+            return 0;
+        runs = (long long)sms * kMaxRunsPerSM;
+    }
+    return round_up(base, 256) + prefix_partials_bytes(num_groups, num_kv_heads, head_dim, runs);
+}
+
+int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                         int num_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                                         int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype,
+                                         float k_scale, float v_scale, const int32_t* group_members,
+                                         const int32_t* group_offsets, const int32_t* group_tables,
+                                         const int32_t* group_lens, const int32_t* shared_blocks, int num_groups,
+                                         int max_group, int num_partitions, void* workspace, size_t workspace_bytes,
+                                         void* stream)
+{
+    return shared_prefix_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                              head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                              v_scale, group_members, group_offsets, group_tables, group_lens, shared_blocks,
+                              num_groups, max_group, num_partitions, workspace, workspace_bytes, nullptr, stream);
+}
+
+int paged_decode_step_shared_prefix(void* out, const void* q, void* k_cache, void* v_cache,
+                                    const int32_t* block_tables, const int32_t* seq_lens, int num_seqs, int num_heads,
+                                    int num_kv_heads, int head_dim, int block_size, float scale,
+                                    int max_blocks_per_seq, int num_blocks, int q_dtype, int kv_dtype, float k_scale,
+                                    float v_scale, const int32_t* group_members, const int32_t* group_offsets,
+                                    const int32_t* group_tables, const int32_t* group_lens,
+                                    const int32_t* shared_blocks, int num_groups, int max_group, int num_partitions,
+                                    void* workspace, size_t workspace_bytes, const void* new_k, const void* new_v,
+                                    const int64_t* slot_mapping, int in_dtype, void* stream)
+{
+    if (!((in_dtype == PKV_F32 || in_dtype == PKV_BF16) && (kv_dtype == in_dtype || is_fp8(kv_dtype))))
+        return PKV_ERR_DTYPE;
+    if (num_seqs > 0 && (!new_k || !new_v || !slot_mapping))
+        return PKV_ERR_NULL;
+    if (num_seqs > 0 && (!aligned16(new_k) || !aligned16(new_v)))
+        return PKV_ERR_SHAPE;
+    if (is_fp8(kv_dtype) && !(k_scale > 0.0f && v_scale > 0.0f))
+        return PKV_ERR_SHAPE;
+    const AppendArgs app{new_k, new_v, slot_mapping, in_dtype};
+    return shared_prefix_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads, num_kv_heads,
+                              head_dim, block_size, scale, max_blocks_per_seq, num_blocks, q_dtype, kv_dtype, k_scale,
+                              v_scale, group_members, group_offsets, group_tables, group_lens, shared_blocks,
+                              num_groups, max_group, num_partitions, workspace, workspace_bytes, &app, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
 int cache_impl(const void* k, const void* v, void* k_cache, void* v_cache, const int64_t* slot_mapping,
                int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int in_dtype,
                int kv_dtype, float k_scale, float v_scale, const float* k_head_scales, const float* v_head_scales,

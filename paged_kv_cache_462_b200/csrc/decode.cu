@@ -9,27 +9,34 @@ namespace pkv {
 int decode_dispatch_f32(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
 int decode_dispatch_bf16(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
 int decode_dispatch_e4m3(int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st, int* occ);
-int decode_mma_dispatch_bf16(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
-                             int* occ);
-int decode_mma_dispatch_e4m3(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
-                             int* occ);
-int decode_mma_dispatch_e5m2(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
-                             int* occ);
-int decode_mma_dispatch_i8(int D, int BS, int G, int HG, const DecodeParams& p, int nruns, cudaStream_t st,
-                           int* occ);
+int decode_mma_dispatch_bf16(int D, int BS, int G, int HG, const MmaOp& op);
+int decode_mma_dispatch_e4m3(int D, int BS, int G, int HG, const MmaOp& op);
+int decode_mma_dispatch_e5m2(int D, int BS, int G, int HG, const MmaOp& op);
+int decode_mma_dispatch_i8(int D, int BS, int G, int HG, const MmaOp& op);
+
+int decode_mma_op(int kv_dtype, int D, int BS, int G, int HG, const MmaOp& op)
+{
+    if (kv_dtype == PKV_BF16)
+        return decode_mma_dispatch_bf16(D, BS, G, HG, op);
+    if (kv_dtype == PKV_FP8_E4M3)
+        return decode_mma_dispatch_e4m3(D, BS, G, HG, op);
+    if (kv_dtype == PKV_FP8_E5M2)
+        return decode_mma_dispatch_e5m2(D, BS, G, HG, op);
+    if (kv_dtype == PKV_INT8)
+        return decode_mma_dispatch_i8(D, BS, G, HG, op);
+    return PKV_ERR_DTYPE;
+}
 
 int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
                         cudaStream_t st, int* occ)
 {
-    if (kv_dtype == PKV_BF16)
-        return decode_mma_dispatch_bf16(D, BS, G, HG, p, nruns, st, occ);
-    if (kv_dtype == PKV_FP8_E4M3)
-        return decode_mma_dispatch_e4m3(D, BS, G, HG, p, nruns, st, occ);
-    if (kv_dtype == PKV_FP8_E5M2)
-        return decode_mma_dispatch_e5m2(D, BS, G, HG, p, nruns, st, occ);
-    if (kv_dtype == PKV_INT8)
-        return decode_mma_dispatch_i8(D, BS, G, HG, p, nruns, st, occ);
-    return PKV_ERR_DTYPE;
+    MmaOp op{};
+    op.kind = occ ? MmaOp::kOccupancy : MmaOp::kLaunch;
+    op.p = &p;
+    op.nruns = nruns;
+    op.stream = st;
+    op.occ = occ;
+    return decode_mma_op(kv_dtype, D, BS, G, HG, op);
 }
 
 bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)

@@ -86,6 +86,40 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
     }
 }
 
+// D += A B with A 16x32 and B 32x8 of 8-bit floats (A: the cache's format, B: E4M3), fp32 sums
+template <__nv_fp8_interpretation_t AFMT>
+__device__ __forceinline__ void mma_16832_f8(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    if constexpr (AFMT == __NV_E5M2) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+            "{%0, %1, %2, %3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+}
+
+// Two values (f16x2, low half first) as E4M3 hi and lo codes with hi + lo ~ x: hi = E4M3(x) and
+// lo = E4M3(x - hi), the difference exact in f16 (hi is x rounded to 4 significant bits). Each
+// result holds its two codes in bits 0-15, low half's code first. |x| must stay below 448.
+__device__ __forceinline__ void split_e4m3x2(uint32_t x, uint32_t& hi, uint32_t& lo)
+{
+    uint16_t h, l;
+    uint32_t hv;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h) : "r"(x));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hv) : "h"(h));
+    const __half2 d = __hsub2(*reinterpret_cast<const __half2*>(&x), *reinterpret_cast<const __half2*>(&hv));
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l) : "r"(*reinterpret_cast<const uint32_t*>(&d)));
+    hi = h;
+    lo = l;
+}
+
 // two 8-bit codes (low byte first) -> f16x2, exact for E4M3, E5M2 and INT8
 template <class KV>
 __device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two_codes)
@@ -215,9 +249,15 @@ __device__ __forceinline__ size_t query_row(const DecodeParams& p, int s, int he
 
 // ------------------------------------------------------------------ configuration
 
-template <class KV, int D, int BS, int G, int HG>
+// PFX: the prefix pass of a shared-prefix decode. A unit is one KV head of one shared block of a
+// group (HG = 1) and the kNT = 4 consumer warps take its 32 query columns (the group's members x
+// their query heads), 8 each, against the same staged K/V tile.
+template <class KV, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaCfg {
-    static constexpr bool kF16 = KV::kBytes == 1;            // E4M3 widened to f16; bf16 stays bf16
+    // products: bf16 caches in bf16 MMA; E4M3 / E5M2 codes straight into FP8 MMA (q and p as E4M3
+    // hi + lo pairs); INT8 codes widened exactly to f16 for f16 MMA
+    static constexpr bool kF8 = KV::kBytes == 1 && !KV::kInt8;
+    static constexpr bool kF16 = KV::kInt8;
     static constexpr int kRowBytes = D * KV::kBytes;          // one token row of one head
     static constexpr int kBoxCols = 128 / KV::kBytes;         // elements per 128-byte box row
     static constexpr int kBoxes = kRowBytes / 128;            // boxes across head_dim
@@ -228,7 +268,8 @@ struct MmaCfg {
     static constexpr int kTT = BS / 16;                       // 16-token tiles per block
     static constexpr int kKS = D / 16;                        // q.K k-steps (16 d each)
     static constexpr int kDT = D / 16;                        // p.V m-tiles (16 d each)
-    static constexpr int W = HG;                              // consumer warps
+    static constexpr int kNT = PFX ? 4 : 1;                   // column tiles (warps) per KV head
+    static constexpr int W = HG * kNT;                        // consumer warps
     static constexpr int kThreads = (W + 1) * 32;
     // CTAs per SM: E4M3 tiles (16 KB stages) take three, for 12 consumer warps per SM to hide the
     // widening chain's latency; the same ~192 KB of stages per SM stay in flight either way
@@ -236,29 +277,50 @@ struct MmaCfg {
     static_assert(kRowBytes % 128 == 0, "rows are whole 128-byte swizzle spans");
     static_assert(BS % 16 == 0 && G <= 8 && HG <= 8, "tile shape");
     static_assert(kRows <= 256, "TMA box height");
+    static_assert(!kF8 || D == 128, "FP8 MMA tiles: one 128-byte box across head_dim");
+    static_assert(!PFX || (HG == 1 && G == 8), "prefix pass: one KV head per unit, 8 columns per warp");
 };
 
 // Byte offset of the 16-byte chunk `c` (0..7) of box row `r` in a 128B-swizzled box.
 __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// Tokens of sequence s this pass streams: seq_lens[s] clamped to [0, capacity], less the
+// skip_blocks[s] leading blocks of a shared-prefix suffix pass (at most the full blocks). `err`
+// collects PKV_DEVERR_SEQ_LEN / PKV_DEVERR_PLAN for values that needed clamping.
+__device__ __forceinline__ int stream_tokens(const DecodeParams& p, int s, int BS, int capacity, int& skip, int& err)
+{
+    int L = p.seq_lens[s];
+    if (L < 0 || L > capacity) {
+        err |= PKV_DEVERR_SEQ_LEN;
+        L = L < 0 ? 0 : capacity;
+    }
+    skip = 0;
+    if (p.skip_blocks != nullptr) {
+        skip = p.skip_blocks[s];
+        if (skip < 0 || skip > L / BS) {
+            err |= PKV_DEVERR_PLAN;
+            skip = skip < 0 ? 0 : L / BS;
+        }
+    }
+    return L - skip * BS;
+}
+
 // prefix[s] = units (head group x logical block) of sequences before s, units of a sequence =
-// ceil(L / block_size) * groups with L clamped to [0, capacity]. All threads of the CTA; ends
-// with a barrier. False if some seq_len needed clamping.
-__device__ __forceinline__ bool build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity)
+// ceil(L / block_size) * groups with L the tokens the pass streams (stream_tokens). All threads
+// of the CTA; ends with a barrier. Returns the PKV_DEVERR_* bits of clamped lengths or skips.
+__device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity)
 {
     const int tid = threadIdx.x, lane = tid & 31;
-    bool bad_len = false;
+    int bad = 0;
     for (int s = tid; s < p.num_seqs; s += blockDim.x) {
-        int L = p.seq_lens[s];
-        if (L < 0 || L > capacity) {
-            bad_len = true;
-            L = L < 0 ? 0 : capacity;
-        }
+        int skip;
+        const int L = stream_tokens(p, s, BS, capacity, skip, bad);
         prefix[s + 1] = ((L + BS - 1) / BS) * NHG;
     }
     if (tid == 0)
         prefix[0] = 0;
-    const bool any_bad = __syncthreads_or(bad_len);
+    const int any_bad = __syncthreads_or(bad & PKV_DEVERR_SEQ_LEN) ? PKV_DEVERR_SEQ_LEN : 0;
+    const int any_plan = __syncthreads_or(bad & PKV_DEVERR_PLAN) ? PKV_DEVERR_PLAN : 0;
     if (tid < 32) {
         int carry = 0;
         for (int base = 0; base < p.num_seqs; base += 32) {
@@ -277,19 +339,25 @@ __device__ __forceinline__ bool build_unit_prefix(const DecodeParams& p, int* pr
         }
     }
     __syncthreads();
-    return !any_bad;
+    return any_bad | any_plan;
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <class KV, class QT, int D, int BS, int G, int HG>
-__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV, D, BS, G, HG>::kCtasPerSM)
+template <class KV, class QT, int D, int BS, int G, int HG, bool PFX = false>
+__global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCfg<KV, D, BS, G, HG, PFX>::kCtasPerSM)
     paged_decode_mma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                             const DecodeParams p)
 {
-    using C = MmaCfg<KV, D, BS, G, HG>;
+    using C = MmaCfg<KV, D, BS, G, HG, PFX>;
     constexpr int W = C::W;
     constexpr bool F16 = C::kF16;
+    constexpr bool F8 = C::kF8;
+    // lazy running max: moved when a tile max passes it by kSlack (log2 units). FP8 products take
+    // p * 2^kPOff <= 2^(kSlack + kPOff) = 256 (E4M3 holds up to 448), which keeps small weights in
+    // E4M3's normal range; the factor cancels between o and l.
+    constexpr float kSlack = F8 ? 2.0f : kMmaRescaleSlack;
+    constexpr float kPOff = F8 ? 6.0f : 0.0f;
     const int S = p.stages_per_warp;   // ring depth (stages of the CTA)
     const int Hkv = p.num_kv_heads;
     const int NHG = Hkv / HG;          // head groups per sequence
@@ -308,8 +376,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
     // the merge kernel that follows may be scheduled now; it waits for this grid before reading
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if ((smem_addr(smem) & 1023u) != 0u) {   // the 128-byte swizzle needs 1024-byte aligned stages
-        if (tid == 0)
+        if (tid == 0) {
             atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+            if (p.wait_prior_at_exit)
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
         return;
     }
 
@@ -321,8 +392,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (!build_unit_prefix(p, prefix, BS, NHG, capacity) && blockIdx.x == 0 && tid == 0)
-        atomicOr(p.err, PKV_DEVERR_SEQ_LEN);
+    {
+        const int bad = build_unit_prefix(p, prefix, BS, NHG, capacity);
+        if (bad && blockIdx.x == 0 && tid == 0)
+            atomicOr(p.err, bad);
+    }
 
     const int total = prefix[p.num_seqs];
     const int nruns = gridDim.x;
@@ -331,12 +405,20 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
     const int run_end = min(total, run_begin + per_run);
     const int nunits = run_end - run_begin;
 
-    // zero rows of empty sequences (one run per sequence)
-    for (int s = blockIdx.x; s < p.num_seqs; s += nruns) {
+    // zero rows of empty sequences (one run per sequence); a prefix pass writes no rows, and a
+    // suffix pass leaves the rows of sequences with shared blocks to the merge
+    for (int s = blockIdx.x; !PFX && s < p.num_seqs; s += nruns) {
         if (prefix[s + 1] == prefix[s]) {
-            // a new token needs a position in the sequence: seq_lens[s] >= 1
+            // a new token needs a position in the sequence: seq_lens[s] >= 1 (and, in a suffix pass,
+            // a block of its own)
             if (tid == 0 && p.new_k != nullptr && __ldg(p.new_slots + s) >= 0)
                 atomicOr(p.err, PKV_DEVERR_SLOT);
+            if (p.skip_blocks != nullptr) {
+                int skipb, e = 0;
+                (void)stream_tokens(p, s, BS, capacity, skipb, e);
+                if (skipb > 0)
+                    continue;
+            }
             const int rows = p.num_heads * (p.q_len > 1 ? p.q_len : 1);
             QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * rows * D;
             for (int i = tid; i < rows * D; i += C::kThreads)
@@ -366,7 +448,12 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
             const int hg = r / nb, j = r - hg * nb;
             if (p.new_k != nullptr && j == nb - 1)
                 app = s * NHG + hg;
-            const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + j);
+            int skipb = 0;
+            if (p.skip_blocks != nullptr) {   // a suffix pass starts past the shared blocks
+                int e = 0;
+                (void)stream_tokens(p, s, BS, capacity, skipb, e);
+            }
+            const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + skipb + j);
             if (phys < 0 || phys >= p.num_blocks) {
                 atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
                 return -1;
@@ -440,28 +527,110 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         const int stream_begin = prefix[s] + hg * nb;
         const int stream_end = stream_begin + nb;
         const int seg_end = min(run_end, stream_end);
-        const int head = hg * HG + warp;           // this warp's KV head
-        int L = p.seq_lens[s];
-        L = L < 0 ? 0 : (L > capacity ? capacity : L);
-        // causal limits of this lane's two query columns 2t, 2t+1: column c (new token c / Gq of
-        // q_len) sees the tokens before position L - q_len + 1 + c / Gq (all L when q_len = 1)
+        const int head = hg * HG + warp / C::kNT;   // this warp's KV head
+        const int tile = warp % C::kNT;             // prefix pass: this warp's 8 of the 32 columns
+        int skipb = 0, lerr = 0;
+        const int L = stream_tokens(p, s, BS, capacity, skipb, lerr);
         const int QL = p.q_len > 1 ? p.q_len : 1;
         const int Gq = p.num_heads / p.num_kv_heads;
         // FP8 per-head scales (when given): this head's into the score and output factors
         const float qk_scale = p.k_head_scales ? p.q_scale * __ldg(p.k_head_scales + head) : p.q_scale;
         const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
-        const int lim0 = 2 * t < G ? L - QL + 1 + (2 * t) / Gq : 0;           // padding columns: none
-        const int lim1 = 2 * t + 1 < G ? L - QL + 1 + (2 * t + 1) / Gq : 0;
+        // Query column c (0..7) of this warp: its row of q / out, and how many of the stream's
+        // tokens it sees. Decode: column c is new token c / Gq of q_len and sees the tokens before
+        // position L - q_len + 1 + c / Gq (all L when q_len = 1); columns >= G are padding.
+        // Prefix pass: column tile * 8 + c is query head (.. % Gq) of member (.. / Gq) of group s,
+        // which sees its own shared blocks of the group's row; columns past the members: padding.
+        auto column = [&](int c, size_t& row) -> int {
+            row = 0;
+            if constexpr (PFX) {
+                const int cg = tile * 8 + c, mem = cg / Gq;
+                const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
+                if (mem >= cnt || mem >= p.pfx_max_group)
+                    return 0;
+                const int seq = p.pfx_members[off + mem];
+                if (seq < 0 || seq >= p.pfx_num_seqs)
+                    return 0;
+                row = (size_t)seq * p.num_heads + (size_t)head * Gq + (cg - mem * Gq);
+                const int lim = p.pfx_shared[seq] * BS;
+                return lim < 0 ? 0 : (lim < L ? lim : L);
+            } else {
+                if (c >= G)
+                    return 0;
+                row = query_row(p, s, head, c);
+                return L - QL + 1 + c / Gq;
+            }
+        };
+        size_t row_g, row0, row1;
+        const int lim_g = column(g, row_g);
+        const int lim0 = column(2 * t, row0);
+        const int lim1 = column(2 * t + 1, row1);
+        const bool qcol = PFX ? lim_g > 0 : g < G;   // this lane holds a real column g of Q^T
+        if constexpr (PFX) {
+            if (tile == 0 && lane == 0) {
+                const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
+                bool bad = cnt > p.pfx_max_group;
+                for (int i = 0; i < cnt && i < p.pfx_max_group; ++i) {
+                    const int seq = p.pfx_members[off + i];
+                    bad |= seq < 0 || seq >= p.pfx_num_seqs || p.pfx_shared[seq] * BS > L;
+                }
+                if (bad)
+                    atomicOr(p.err, PKV_DEVERR_PLAN);
+            }
+        }
 
         // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
         uint32_t qb[C::kKS][2];
-        {
-            const QT* qp = reinterpret_cast<const QT*>(p.q) + (g < G ? query_row(p, s, head, g) : 0) * D;
+        float qk0 = qk_scale, qk1 = qk_scale;   // score factors of this lane's columns 2t, 2t+1
+        if constexpr (F8) {
+            // FP8 products: column g of Q^T times a power of two sigma_g (max |q| * sigma_g < 256),
+            // as E4M3 hi + lo codes (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3,
+            // b1 = d 32kk + 16 + 4t .. +3. 1 / sigma goes into the column's score factor.
+            constexpr int K8 = D / 32;
+            const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
+            float f[K8][2][4];
+            float mx = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < K8; ++kk)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (qcol)
+                        load_q<4>(qp + kk * 32 + hh * 16 + 4 * t, f[kk][hh]);
+                    else
+                        f[kk][hh][0] = f[kk][hh][1] = f[kk][hh][2] = f[kk][hh][3] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        mx = fmaxf(mx, fabsf(f[kk][hh][i]));
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
+            // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
+            int se = 127;
+            if (mx > 0.f) {
+                se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
+                se = se < 2 ? 2 : (se > 252 ? 252 : se);
+            }
+            const float sig = __uint_as_float((uint32_t)se << 23);
+            const float inv_sig = __uint_as_float((uint32_t)(254 - se) << 23);
+#pragma unroll
+            for (int kk = 0; kk < K8; ++kk)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t h01, l01, h23, l23;
+                    split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
+                    split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
+                    qb[kk][hh] = h01 | (h23 << 16);
+                    qb[K8 + kk][hh] = l01 | (l23 << 16);
+                }
+            qk0 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t) * 4);
+            qk1 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t + 1) * 4);
+        } else {
+            const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
 #pragma unroll
             for (int ks = 0; ks < C::kKS; ++ks) {
-                if (g < G) {
+                if (qcol) {
                     if constexpr (F16) {
-                        // k order permuted to match the E4M3 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
+                        // k order permuted to match the widened INT8 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
                         float f[4];
                         load_q<4>(qp + ks * 16 + 4 * t, f);
                         qb[ks][0] = pack2<true>(f[0], f[1]);
@@ -505,7 +674,18 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                     float sc[4] = {0.f, 0.f, 0.f, 0.f};
                     float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
                     const int mi = lane >> 3, rr = lane & 7;
-                    if constexpr (F16) {
+                    if constexpr (F8) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 32; ++kk) {
+                            // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment
+                            // of 16 tokens x d 32kk .. 32kk+31 as it lies in the stage, no conversion
+                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                            uint32_t a[4];
+                            ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
+                            mma_16832_f8<KV::kFmt>(sc, a, qb[kk][0], qb[kk][1]);                 // q hi
+                            mma_16832_f8<KV::kFmt>(sd, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);   // q lo
+                        }
+                    } else if constexpr (F16) {
 #pragma unroll
                         for (int ks = 0; ks < C::kKS; ks += 2) {
                             // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each
@@ -536,8 +716,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                         sc[i] += sd[i];
                     // V fragments of this tile into registers; after the block's last tile the
                     // stage goes back to the producer before the softmax and p.V arithmetic
-                    uint32_t vf[C::kDT * 4 / (F16 ? 2 : 1)];
-                    if constexpr (F16) {
+                    uint32_t vf[C::kDT * 4 / ((F16 || F8) ? 2 : 1)];
+                    if constexpr (F16 || F8) {
 #pragma unroll
                         for (int dt = 0; dt < C::kDT; dt += 2) {
                             // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
@@ -569,21 +749,21 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                     }
                     // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
                     const int tok0 = jb * BS + tt * 16 + g;   // position in the sequence
-                    sc[0] = (tok0 < lim0) ? sc[0] * qk_scale : -INFINITY;
-                    sc[1] = (tok0 < lim1) ? sc[1] * qk_scale : -INFINITY;
-                    sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk_scale : -INFINITY;
-                    sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk_scale : -INFINITY;
+                    sc[0] = (tok0 < lim0) ? sc[0] * qk0 : -INFINITY;
+                    sc[1] = (tok0 < lim1) ? sc[1] * qk1 : -INFINITY;
+                    sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk0 : -INFINITY;
+                    sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk1 : -INFINITY;
                     // The reference moves only when some score passes it by the slack; each lane
                     // tests its own scores first, so the butterfly max runs only when one does
                     // (same result as reducing first: the tile max passes iff some lane's does).
                     float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
-                    if (__any_sync(kFullMask, bm0 > m[0] + kMmaRescaleSlack || bm1 > m[1] + kMmaRescaleSlack)) {
+                    if (__any_sync(kFullMask, bm0 > m[0] + kSlack || bm1 > m[1] + kSlack)) {
 #pragma unroll
                         for (int off = 4; off < 32; off <<= 1) {
                             bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
                             bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
                         }
-                        const bool up0 = bm0 > m[0] + kMmaRescaleSlack, up1 = bm1 > m[1] + kMmaRescaleSlack;
+                        const bool up0 = bm0 > m[0] + kSlack, up1 = bm1 > m[1] + kSlack;
                         const float n0 = up0 ? bm0 : m[0], n1 = up1 ? bm1 : m[1];
                         const float a0 = up0 ? fast_exp2(m[0] - n0) : 1.f, a1 = up1 ? fast_exp2(m[1] - n1) : 1.f;
                         m[0] = n0;
@@ -599,24 +779,57 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                         }
                     }
                     float pr[4];
-                    pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - m[0]);
-                    pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - m[1]);
-                    pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - m[0]);
-                    pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - m[1]);
+                    const float mo0 = m[0] - kPOff, mo1 = m[1] - kPOff;
+                    pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - mo0);
+                    pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - mo1);
+                    pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - mo0);
+                    pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - mo1);
                     l[0] += pr[0] + pr[2];
                     l[1] += pr[1] + pr[3];
-                    // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
-                    const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
-                    const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
                     const int srcA = (2 * t) * 4 + (g >> 1), srcB = (2 * t + 1) * 4 + (g >> 1);
-                    const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
-                    const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
-                    const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
-                    const uint32_t pb0 = (g < G) ? __byte_perm(va, vb, 0x5410) : 0u;
-                    const uint32_t pb1 = (g < G) ? __byte_perm(va, vb, 0x7632) : 0u;
+                    uint32_t pb0, pb1;
+                    if constexpr (F8) {
+                        // ---- P^T as E4M3 hi (b0) and lo (b1) codes, k = tokens 2t, 2t+1, 2t+8, 2t+9 of column g
+                        uint32_t h0, l0, h1, l1;
+                        split_e4m3x2(pack2<true>(pr[0], pr[2]), h0, l0);   // column 2t:   tokens g, g+8
+                        split_e4m3x2(pack2<true>(pr[1], pr[3]), h1, l1);   // column 2t+1: tokens g, g+8
+                        const uint32_t wh = h0 | (h1 << 16), wl = l0 | (l1 << 16);
+                        const uint32_t ah = __shfl_sync(kFullMask, wh, srcA), bh = __shfl_sync(kFullMask, wh, srcB);
+                        const uint32_t al = __shfl_sync(kFullMask, wl, srcA), bl = __shfl_sync(kFullMask, wl, srcB);
+                        const uint32_t sel = (g & 1) ? 0x7362u : 0x5140u;
+                        pb0 = qcol ? __byte_perm(ah, bh, sel) : 0u;
+                        pb1 = qcol ? __byte_perm(al, bl, sel) : 0u;
+                    } else {
+                        // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
+                        const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
+                        const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
+                        const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
+                        const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
+                        const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
+                        pb0 = qcol ? __byte_perm(va, vb, 0x5410) : 0u;
+                        pb1 = qcol ? __byte_perm(va, vb, 0x7632) : 0u;
+                    }
                     // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
                     const bool partial = valid < tt * 16 + 16;
-                    if constexpr (F16) {
+                    if constexpr (F8) {
+#pragma unroll
+                        for (int dt = 0; dt < C::kDT; dt += 2) {
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
+                                if (partial) {
+                                    const int tk = tt * 16 + 2 * t;
+                                    lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                    hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                }
+                                // rows g / g+8 of the m-tile = d 2g / 2g+1 of chunk dt + h2; k = tokens
+                                // 2t, 2t+1, 2t+8, 2t+9 against P hi, then the same tokens against P lo
+                                const uint32_t a0 = __byte_perm(lo, hi, 0x6420), a1 = __byte_perm(lo, hi, 0x7531);
+                                const uint32_t a[4] = {a0, a1, a0, a1};
+                                mma_16832_f8<KV::kFmt>(o[dt + h2], a, pb0, pb1);
+                            }
+                        }
+                    } else if constexpr (F16) {
 #pragma unroll
                         for (int dt = 0; dt < C::kDT; dt += 2) {
 #pragma unroll
@@ -671,11 +884,13 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
         const int stream = s * NHG + hg;
         // element (head column c, row d) of this lane's accumulators
         auto d_of = [&](int dt, int half) -> int {
-            return F16 ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
+            return (F16 || F8) ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
         };
-        if (first_run == last_run) {
-            QT* out0 = reinterpret_cast<QT*>(p.out) + (2 * t < G ? query_row(p, s, head, 2 * t) : 0) * D;
-            QT* out1 = reinterpret_cast<QT*>(p.out) + (2 * t + 1 < G ? query_row(p, s, head, 2 * t + 1) : 0) * D;
+        // a whole stream writes `out`; pieces of split streams, every stream of a prefix pass and
+        // the suffix of a sequence with shared blocks leave (o, m, l) for the merge
+        if (first_run == last_run && !PFX && skipb == 0) {
+            QT* out0 = reinterpret_cast<QT*>(p.out) + row0 * D;
+            QT* out1 = reinterpret_cast<QT*>(p.out) + row1 * D;
             const float inv0 = l[0] > 0.f ? out_scale / l[0] : 0.f;
             const float inv1 = l[1] > 0.f ? out_scale / l[1] : 0.f;
 #pragma unroll
@@ -689,7 +904,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
                         from_float(o[dt][2 * half + 1] * inv1, out1 + d);
                 }
         } else {
-            float* part = p.partials + ((size_t)(blockIdx.x + stream) * HG + warp) * p.slot_floats;
+            float* part = p.partials + ((size_t)(blockIdx.x + stream) * W + warp) * p.slot_floats;
 #pragma unroll
             for (int dt = 0; dt < C::kDT; ++dt)
 #pragma unroll
@@ -712,6 +927,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG>::kThreads, MmaCfg<KV,
             }
         }
     }
+    // a suffix pass launched behind a prefix pass completes only after it (see the launcher)
+    if (p.wait_prior_at_exit && tid == 0)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Log-sum-exp merge of the nseg partials of KV head (stream's head group) * HG + warp of sequence
@@ -873,6 +1091,123 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     }
 }
 
+// Merge of a shared-prefix decode, launched behind the suffix pass as a programmatic dependent
+// launch (the suffix pass completes only after the prefix pass, so the wait covers both).
+// (a) Every (member of a group with shared blocks, KV head h, query head gq), one warp each: the
+//     prefix pass's pieces of column member * Gq + gq of stream (group, h) and the suffix pass's
+//     pieces of the member's stream, log-sum-exp combined into out.
+// (b) Sequences without shared blocks whose stream the suffix pass split: merge_split, as after a
+//     plain decode.
+// ps: the suffix pass's parameters (skip_blocks = the plan's shared blocks); pp: the prefix
+// pass's (its "sequences" are the groups). Shared memory: both unit prefixes.
+template <class QT, int D, int BS, int G, int HG>
+__global__ void __launch_bounds__(kMergeThreads)
+    paged_decode_prefix_merge_kernel(const DecodeParams ps, const DecodeParams pp, int runs_s, int runs_p)
+{
+    extern __shared__ int smem_prefix[];
+    int* prefix_s = smem_prefix;                     // [num_seqs + 1]
+    int* prefix_p = smem_prefix + ps.num_seqs + 1;   // [num_groups + 1]
+    const int Hkv = ps.num_kv_heads, NHG = Hkv / HG, Gq = ps.num_heads / Hkv;
+    const int capacity = ps.max_blocks_per_seq * BS;
+    (void)build_unit_prefix(ps, prefix_s, BS, NHG, capacity);
+    (void)build_unit_prefix(pp, prefix_p, BS, Hkv, capacity);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int total_s = prefix_s[ps.num_seqs], total_p = prefix_p[pp.num_seqs];
+    const int per_run_s = total_s > 0 ? (total_s + runs_s - 1) / runs_s : 1;
+    const int per_run_p = total_p > 0 ? (total_p + runs_p - 1) / runs_p : 1;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (kMergeThreads / 32);
+    const int wid = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
+
+    // (a) members of groups
+    const int members = pp.num_seqs > 0 ? pp.pfx_offsets[pp.num_seqs] : 0;   // no groups: no plan arrays
+    const int items_a = members * Hkv * Gq;
+    for (int it = wid; it < items_a; it += warps) {
+        const int mm = it / (Hkv * Gq), rem = it - mm * (Hkv * Gq);
+        const int h = rem / Gq, gq = rem - h * Gq;
+        int lo = 0, hi = pp.num_seqs;                 // group of member mm: offsets[gi] <= mm < offsets[gi + 1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pp.pfx_offsets[mid] <= mm)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int gi = lo, mi = mm - pp.pfx_offsets[gi];
+        const int seq = pp.pfx_members[mm];
+        if (mi >= pp.pfx_max_group || seq < 0 || seq >= ps.num_seqs)
+            continue;                                 // flagged by the prefix pass
+        int skipb = 0, e = 0;
+        (void)stream_tokens(ps, seq, BS, capacity, skipb, e);
+        if (skipb == 0)
+            continue;                                 // nothing shared: the suffix pass wrote it whole
+        float M = -INFINITY, Lsum = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool mine = 4 * lane < D;
+        auto add = [&](const float* o, float m, float l) {
+            if (m == -INFINITY)
+                return;
+            const float Mn = fmaxf(M, m);
+            const float a = M == -INFINITY ? 0.f : fast_exp2(M - Mn), b = fast_exp2(m - Mn);
+            Lsum = Lsum * a + l * b;
+            if (mine) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(o + 4 * lane));
+                acc.x = acc.x * a + b * v.x;
+                acc.y = acc.y * a + b * v.y;
+                acc.z = acc.z * a + b * v.z;
+                acc.w = acc.w * a + b * v.w;
+            }
+            M = Mn;
+        };
+        // prefix pieces: stream (gi, h) of the prefix pass, column mi * Gq + gq (tile cg / 8)
+        const int nb_p = (prefix_p[gi + 1] - prefix_p[gi]) / Hkv;
+        if (nb_p > 0) {
+            const int pstream = gi * Hkv + h, sb = prefix_p[gi] + h * nb_p;
+            const int cg = mi * Gq + gq, tile = cg >> 3, c = cg & 7;
+            for (int r = sb / per_run_p; r <= (sb + nb_p - 1) / per_run_p; ++r) {
+                const float* base = pp.partials + ((size_t)(r + pstream) * 4 + tile) * pp.slot_floats;
+                add(base + c * D, __ldcg(base + 8 * D + c), __ldcg(base + 8 * D + 8 + c));
+            }
+        }
+        // suffix pieces: stream (seq, h / HG) of the suffix pass, warp h % HG, column gq
+        const int nb_s = (prefix_s[seq + 1] - prefix_s[seq]) / NHG;
+        if (nb_s > 0) {
+            const int hg = h / HG, w = h - hg * HG, stream = seq * NHG + hg, sb = prefix_s[seq] + hg * nb_s;
+            for (int r = sb / per_run_s; r <= (sb + nb_s - 1) / per_run_s; ++r) {
+                const float* base = ps.partials + ((size_t)(r + stream) * HG + w) * ps.slot_floats;
+                add(base + gq * D, __ldcg(base + G * D + gq), __ldcg(base + G * D + G + gq));
+            }
+        }
+        const float out_scale = ps.v_head_scales ? ps.v_scale * __ldg(ps.v_head_scales + h) : ps.v_scale;
+        const float inv = Lsum > 0.f ? out_scale / Lsum : 0.f;
+        if (mine) {
+            QT* dst = reinterpret_cast<QT*>(ps.out) + ((size_t)seq * ps.num_heads + (size_t)h * Gq + gq) * D + 4 * lane;
+            from_float(acc.x * inv, dst);
+            from_float(acc.y * inv, dst + 1);
+            from_float(acc.z * inv, dst + 2);
+            from_float(acc.w * inv, dst + 3);
+        }
+    }
+
+    // (b) split streams of sequences without shared blocks
+    const int items_b = ps.num_seqs * NHG * HG;
+    for (int it = wid; it < items_b; it += warps) {
+        const int stream = it / HG, w = it - stream * HG;
+        const int s = stream / NHG, hg = stream - s * NHG;
+        const int nb = (prefix_s[s + 1] - prefix_s[s]) / NHG;
+        if (nb == 0)
+            continue;
+        int skipb = 0, e = 0;
+        (void)stream_tokens(ps, s, BS, capacity, skipb, e);
+        if (skipb > 0)
+            continue;
+        const int sb = prefix_s[s] + hg * nb;
+        const int first_run = sb / per_run_s, last_run = (sb + nb - 1) / per_run_s;
+        if (first_run != last_run)
+            merge_split<QT, D, G, HG>(ps, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 
 // Encode a 2-D tensor map over a cache: rows = num_blocks * num_kv_heads * block_size,
@@ -880,9 +1215,9 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
 bool make_cache_tensormap(CUtensorMap* map, const void* base, int kv_dtype, int head_dim, long long rows,
                           int box_rows);
 
-template <class KV, class QT, int D, int BS, int G, int HG>
+template <class KV, class QT, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaLauncher {
-    using C = MmaCfg<KV, D, BS, G, HG>;
+    using C = MmaCfg<KV, D, BS, G, HG, PFX>;
 
     static size_t smem_bytes(int num_seqs, int S)
     {
@@ -910,7 +1245,7 @@ struct MmaLauncher {
         const int S = stages(num_seqs);
         if (S < 2)
             return 0;
-        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG>;
+        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG, PFX>;
         const size_t smem = smem_bytes(num_seqs, S);
         if (!ensure_smem_attribute((const void*)kern, smem))
             return 0;
@@ -920,7 +1255,9 @@ struct MmaLauncher {
         return n;
     }
 
-    static int launch(DecodeParams p, int nruns, cudaStream_t stream)
+    // The decode kernel alone (p gets the launcher's fields); `pdl`: as a programmatic dependent
+    // launch behind the previous kernel on `stream`.
+    static int launch_decode(DecodeParams& p, int nruns, cudaStream_t stream, bool pdl)
     {
         const int S = stages(p.num_seqs);
         if (S < 2)
@@ -933,38 +1270,88 @@ struct MmaLauncher {
         if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, D, rows, C::kRows) ||
             !make_cache_tensormap(&vmap, p.v_cache, kvdt, D, rows, C::kRows))
             return PKV_ERR_LAUNCH;
-        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG>;
+        auto kern = paged_decode_mma_kernel<KV, QT, D, BS, G, HG, PFX>;
         const size_t smem = smem_bytes(p.num_seqs, S);
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
-        // E4M3 -> f16 widening is exact: only the per-tensor scales remain
+        // 8-bit codes enter the products as their format's values: only the per-tensor scales remain
         p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
         p.v_scale = KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f;
-        kern<<<nruns, C::kThreads, smem, stream>>>(kmap, vmap, p);
-        if (cudaGetLastError() != cudaSuccess)
-            return PKV_ERR_LAUNCH;
-        // the merge of split streams, allowed to start while the decode grid drains
-        auto merge = paged_decode_merge_kernel<QT, D, BS, G, HG>;
-        const size_t msmem = (size_t)(p.num_seqs + 1) * 4;
-        if (!ensure_smem_attribute((const void*)merge, msmem))
-            return PKV_ERR_LAUNCH;
-        const int items = p.num_seqs * p.num_kv_heads;
-        const int per_cta = kMergeThreads / 32;
-        int mgrid = (items + per_cta - 1) / per_cta;
-        if (mgrid > nruns)
-            mgrid = nruns;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(mgrid);
+        cfg.gridDim = dim3(nruns);
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, p) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+    }
+
+    static int launch_merge_pdl(const void* kern, void** args, int grid, size_t smem, cudaStream_t stream)
+    {
+        if (!ensure_smem_attribute(kern, smem))
+            return PKV_ERR_LAUNCH;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
         cfg.blockDim = dim3(kMergeThreads);
-        cfg.dynamicSmemBytes = msmem;
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, merge, p, nruns) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+        return cudaLaunchKernelExC(&cfg, kern, args) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+    }
+
+    static int launch(DecodeParams p, int nruns, cudaStream_t stream)
+    {
+        const int st = launch_decode(p, nruns, stream, false);
+        if (st != PKV_OK)
+            return st;
+        // the merge of split streams, allowed to start while the decode grid drains
+        const int items = p.num_seqs * p.num_kv_heads;
+        const int per_cta = kMergeThreads / 32;
+        int mgrid = (items + per_cta - 1) / per_cta;
+        if (mgrid > nruns)
+            mgrid = nruns;
+        void* args[] = {&p, &nruns};
+        return launch_merge_pdl((const void*)paged_decode_merge_kernel<QT, D, BS, G, HG>, args, mgrid,
+                                (size_t)(p.num_seqs + 1) * 4, stream);
+    }
+
+    // Shared-prefix decode: the prefix pass (pp: the plan's groups, one KV head per unit, 32 query
+    // columns), then the suffix pass (ps: every sequence past its shared blocks) as a programmatic
+    // dependent launch that may start while the prefix pass drains, then the merge of both.
+    static int launch_shared_prefix(DecodeParams ps, DecodeParams pp, int runs_s, int runs_p, cudaStream_t stream)
+    {
+        using PL = MmaLauncher<KV, QT, D, BS, 8, 1, true>;
+        const bool any_groups = pp.num_seqs > 0;
+        if (any_groups) {
+            const int st = PL::launch_decode(pp, runs_p, stream, false);
+            if (st != PKV_OK)
+                return st;
+        }
+        ps.wait_prior_at_exit = any_groups ? 1 : 0;
+        const int st = launch_decode(ps, runs_s, stream, any_groups);
+        if (st != PKV_OK)
+            return st;
+        const long long members_items = any_groups ? 1ll * ps.num_seqs * ps.num_heads : 0;
+        const long long items = members_items > 1ll * ps.num_seqs * ps.num_kv_heads
+                                    ? members_items : 1ll * ps.num_seqs * ps.num_kv_heads;
+        const int per_cta = kMergeThreads / 32;
+        long long mgrid = (items + per_cta - 1) / per_cta;
+        if (mgrid > runs_s)
+            mgrid = runs_s;
+        if (mgrid < 1)
+            mgrid = 1;
+        void* args[] = {&ps, &pp, &runs_s, &runs_p};
+        return launch_merge_pdl((const void*)paged_decode_prefix_merge_kernel<QT, D, BS, G, HG>, args, (int)mgrid,
+                                (size_t)(ps.num_seqs + 1 + pp.num_seqs + 1) * 4, stream);
     }
 };
 

@@ -55,6 +55,36 @@ struct DecodeParams {
     // failure-path test hook (tensor-core kernel): 1 + the unit whose stage the producer never
     // hands to its consumers, so their bounded wait runs out; 0 = none
     int withheld_unit;
+    // Shared-prefix decode, suffix pass (null: none): sequence s starts at logical block
+    // skip_blocks[s] of its table (the blocks before it are read by the prefix pass) and writes
+    // fp32 partials instead of `out` whenever skip_blocks[s] > 0.
+    const int32_t* skip_blocks;
+    // Shared-prefix decode, prefix pass (null: none): the kernel's "sequences" are the plan's
+    // groups (block_tables = group rows, seq_lens = their token counts, num_seqs = groups);
+    // column c of KV head h of group gi is query head h * Gq + c % Gq of member c / Gq, i.e. of
+    // sequence pfx_members[pfx_offsets[gi] + c / Gq], which sees pfx_shared[that sequence]
+    // blocks of the row. Gq = num_heads / num_kv_heads.
+    const int32_t* pfx_members;
+    const int32_t* pfx_offsets;
+    const int32_t* pfx_shared;
+    // members a group may hold (host-checked: pfx_max_group * Gq <= 32); larger groups are flagged
+    int pfx_max_group;
+    int pfx_num_seqs;   // sequences of the batch (members must lie in [0, pfx_num_seqs))
+    // 1: execute griddepcontrol.wait before the grid exits (a suffix pass launched behind the
+    // prefix pass, so that the merge's wait covers both)
+    int wait_prior_at_exit;
+};
+
+// One request to the warp-MMA kernels of a shape (decode_mma_dispatch.cuh).
+struct MmaOp {
+    enum Kind { kLaunch = 0, kOccupancy = 1, kLaunchSharedPrefix = 2, kPrefixOccupancy = 3 };
+    int kind;
+    const DecodeParams* p;    // the decode (or the shared-prefix suffix pass)
+    const DecodeParams* pp;   // the shared-prefix prefix pass (kLaunchSharedPrefix)
+    int nruns;                // runs of p
+    int runs_p;               // runs of pp
+    cudaStream_t stream;
+    int* occ;                 // out: CTAs per SM (occupancy kinds)
 };
 
 // Kernel selection: warp-MMA kernel for bf16 / E4M3 caches of supported shapes,
@@ -65,6 +95,8 @@ bool mma_supported(int kv_dtype, int head_dim, int block_size, int group, int nu
 int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads);
 int decode_mma_dispatch(int kv_dtype, int D, int BS, int G, int HG, const DecodeParams& p, int nruns,
                         cudaStream_t st, int* occ);
+// Any MmaOp on the warp-MMA kernels of a cache type and shape.
+int decode_mma_op(int kv_dtype, int D, int BS, int G, int HG, const MmaOp& op);
 
 // The fused step's append + decode in one launch (warp-MMA kernel only).
 bool step_fusable(int q_dtype, int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads);

@@ -124,3 +124,37 @@ def test_int8_and_e5m2_dtype_pairs(lib):
     f = lib.reshape_and_cache
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 1, 4, 0.0, 1.0, None, None) == 2   # zero INT8 scale
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 4, 4, 1.0, 1.0, None, None) == 3   # INT8 input rows
+
+
+def _shared(lib, **kw):
+    a = dict(S=4, Hq=8, Hkv=2, D=128, BS=16, MB=4, NB=32, qdt=1, kvdt=1, groups=1, max_group=4, parts=7,
+             ptr=ctypes.c_void_p(16), ws=ctypes.c_void_p(256), wsb=1 << 30)
+    a.update(kw)
+    p = a["ptr"]
+    return lib.paged_attention_decode_shared_prefix(p, p, p, p, p, p, a["S"], a["Hq"], a["Hkv"], a["D"], a["BS"],
+                                                    0.1, a["MB"], a["NB"], a["qdt"], a["kvdt"], 1.0, 1.0, p, p, p, p,
+                                                    a.get("shared", p), a["groups"], a["max_group"], a["parts"],
+                                                    a["ws"], a["wsb"], None)
+
+
+def test_shared_prefix_host_validation(lib):
+    """Shared-prefix decode: rejected before any device access."""
+    assert _shared(lib, max_group=9) == 2                  # 9 members x 4 query heads > 32 columns
+    assert _shared(lib, max_group=0) == 2
+    assert _shared(lib, groups=5) == 2                     # more groups than sequences
+    assert _shared(lib, groups=-1) == 2
+    assert _shared(lib, Hq=16, max_group=5) == 2           # 5 x 8 > 32
+    assert _shared(lib, qdt=0, kvdt=0) == 3                # f32 caches: no tensor-core kernel
+    assert _shared(lib, BS=8) == 2                         # block 8: no tensor-core kernel
+    assert _shared(lib, shared=ctypes.c_void_p(None)) == 1
+    assert _shared(lib, S=0, groups=0) == 0                # nothing to do
+
+
+def test_shared_prefix_workspace_size(lib):
+    base = lib.paged_attention_workspace_size(64, 32, 8, 128, 296)
+    n = lib.paged_attention_shared_prefix_workspace_size(64, 32, 8, 128, 8, 296)
+    slot = 4 * 8 * (128 + 2)                               # 8 columns x (d + 2) floats
+    assert n == (base + 255) // 256 * 256 + (296 + 8 * 8) * 4 * slot
+    assert lib.paged_attention_shared_prefix_workspace_size(64, 32, 8, 128, 0, 296) == (base + 255) // 256 * 256
+    assert lib.paged_attention_shared_prefix_workspace_size(64, 32, 8, 128, -1, 296) == 0
+    assert lib.paged_attention_shared_prefix_workspace_size(64, 24, 8, 128, 4, 296) == 0

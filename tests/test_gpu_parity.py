@@ -481,19 +481,17 @@ def test_multi_query_unsupported_shapes_are_rejected():
 
 # ------------------------------------------------------------------ per-KV-head FP8 scales
 
-@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
-@pytest.mark.parametrize("parts", [0, 5])
-def test_head_scales_append_and_decode(kv, parts):
-    """FP8 caches with one scale per KV head (heads of very different ranges): appends bit-exact
-    and outputs within tolerance of the oracle using the same head scales."""
+def _head_scale_case(kv, parts, gain_k, gain_v):
+    """Config 1 cut down with K and V rows of KV head h scaled by gain_k[h] / gain_v[h], 8-bit caches
+    with per-head absmax scales: GPU and oracle caches and outputs (GPU output, oracle output)."""
     b = W.config_batch(1, num_seqs=6, kv_dtype=kv)
     sp = b.spec
     Hkv, D, BS, NB = sp.num_kv_heads, sp.head_dim, sp.block_size, b.num_blocks
-    gain = np.geomspace(0.05, 40.0, Hkv).astype(np.float32)           # per-head magnitude
-    def rows(x):
+    def rows(x, gain):
         f = W.bf16_bits_to_f32(x) * gain[None, :, None]
         return W.f32_to_bf16_bits(f.astype(np.float32))
-    hk, hv, nk, nv = rows(b.hist_k), rows(b.hist_v), rows(b.new_k), rows(b.new_v)
+    hk, nk = rows(b.hist_k, gain_k), rows(b.new_k, gain_k)
+    hv, nv = rows(b.hist_v, gain_v), rows(b.new_v, gain_v)
     top = {"e4m3": 448.0, "e5m2": 57344.0, "int8": 127.0}[kv]
     def head_absmax(*xs):
         return np.max([np.abs(W.bf16_bits_to_f32(x)).max(axis=(0, 2)) for x in xs], axis=0)
@@ -517,9 +515,46 @@ def test_head_scales_append_and_decode(kv, parts):
     torch.cuda.synchronize()
     assert pkv.read_device_error(ws) == 0
     assert np.array_equal(cache_bytes(kc), okc) and np.array_equal(cache_bytes(vc), ovc)
-    G = sp.num_heads // Hkv
-    err = np.abs(to_f64(out) - ref).max(axis=(0, 2))                   # per query head
-    assert np.all(err <= TOL[kv] * np.repeat(gain, G)), err            # outputs scale with the head's V range
+    return to_f64(out), ref, sp.num_heads // Hkv
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+@pytest.mark.parametrize("parts", [0, 5])
+def test_head_scales_append_and_decode(kv, parts):
+    """FP8 caches with one scale per KV head (heads of very different ranges): appends bit-exact
+    and outputs within tolerance of the oracle using the same head scales, relative to each
+    head's V range (outputs scale with it)."""
+    gain = np.geomspace(0.05, 40.0, 8).astype(np.float32)           # per-head magnitude
+    out, ref, G = _head_scale_case(kv, parts, gain, gain)
+    err = np.abs(out - ref).max(axis=(0, 2))                          # per query head
+    assert np.all(err <= TOL[kv] * np.repeat(gain, G)), err
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+@pytest.mark.parametrize("parts", [0, 5])
+def test_head_scales_unit_range_values_absolute_tolerance(kv, parts):
+    """Per-head scales that differ widely for K (ranges 0.05x .. 40x) and moderately for V
+    (0.5x .. 2x, values of order one): every output within the plain absolute tolerance."""
+    gain_k = np.geomspace(0.05, 40.0, 8).astype(np.float32)
+    gain_v = np.geomspace(0.5, 2.0, 8).astype(np.float32)[::-1].copy()
+    out, ref, _ = _head_scale_case(kv, parts, gain_k, gain_v)
+    assert np.abs(out - ref).max() <= TOL[kv]
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+@pytest.mark.parametrize("qgain", [2.0 ** 8, 2.0 ** -16])
+def test_8bit_cache_query_magnitudes(kv, qgain):
+    """Queries far from unit size with 8-bit caches (q times 2^8: sharply peaked softmax; q times
+    2^-16: nearly uniform): the fused step against the oracle on the same bf16 q."""
+    b = W.config_batch(1, num_seqs=6, kv_dtype=kv)
+    q = W.bf16_bits_to_f32(b.q) * np.float32(qgain)        # a power of two: exact in bf16
+    b.q = W.f32_to_bf16_bits(q.astype(np.float32))
+    ref, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    out = g.fused_step(0)
+    assert g.device_errors() == 0
+    assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
+    assert max_err(out, ref) <= TOL[kv]
 
 
 # ------------------------------------------------------------------ INT8 caches

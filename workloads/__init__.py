@@ -258,10 +258,33 @@ def batch_layout(spec: Spec, seed: int | None = None) -> Layout:
 def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
     """Draw one batch. Draw order: lengths, pool permutation, q, K, V, new k, new v."""
     rng = np.random.default_rng(spec.seed if seed is None else seed)
-    S, Hq, Hkv, d, bs = spec.num_seqs, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
-    assert Hq % Hkv == 0
+    assert spec.num_heads % spec.num_kv_heads == 0
     lay = _layout(spec, rng)
-    seq_lens, tables, num_blocks, groups = lay.seq_lens, lay.block_tables, lay.num_blocks, lay.groups
+    groups = lay.groups
+    shared = int(sum(n for members, n in groups if len(members) > 1)) if groups else 0
+    return _draw_tensors(spec, rng, lay.seq_lens, lay.block_tables, lay.num_blocks, shared)
+
+
+def batch_from_tables(spec: Spec, block_tables: np.ndarray, seq_lens: np.ndarray, num_blocks: int,
+                      seed: int | None = None) -> DecodeBatch:
+    """A batch over given tables (e.g. a block manager's, with forks sharing blocks): q, the
+    history rows of every slot of every referenced block and the new token rows are drawn as in
+    ``build_batch`` (same order), the new token of sequence s at position seq_lens[s] - 1."""
+    rng = np.random.default_rng(spec.seed if seed is None else seed)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    assert sl.shape == (spec.num_seqs,) and bt.shape[0] == spec.num_seqs
+    nb = (sl.astype(np.int64) + spec.block_size - 1) // spec.block_size
+    counts = {}
+    for s in range(spec.num_seqs):
+        for j in range(int(nb[s])):
+            counts[int(bt[s, j])] = counts.get(int(bt[s, j]), 0) + 1
+    shared = sum(1 for c in counts.values() if c > 1)
+    return _draw_tensors(spec, rng, sl, bt, int(num_blocks), shared)
+
+
+def _draw_tensors(spec: Spec, rng, seq_lens, tables, num_blocks, shared) -> DecodeBatch:
+    S, Hq, Hkv, d, bs = spec.num_seqs, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.block_size
     MB = tables.shape[1]
     nb = (seq_lens.astype(np.int64) + bs - 1) // bs
 
@@ -292,9 +315,7 @@ def build_batch(spec: Spec, seed: int | None = None) -> DecodeBatch:
             new_slots[s] = int(tables[s, pos // bs]) * bs + pos % bs
 
     k_scale, v_scale = _cache_scales(spec.kv_dtype, spec.in_dtype, hist_k, hist_v, new_k, new_v)
-
     scale = np.float32(1.0 / math.sqrt(d))
-    shared = int(sum(n for members, n in groups if len(members) > 1)) if groups else 0
     return DecodeBatch(spec, num_blocks, MB, scale, k_scale, v_scale, seq_lens, tables, q,
                        hist_k, hist_v, hist_slots, new_k, new_v, new_slots, shared_blocks=shared)
 
