@@ -355,6 +355,26 @@ PKV_API int reshape_and_cache(const void* k, const void* v, void* k_cache, void*
 PKV_API int pkv_read_device_error(void* workspace, size_t workspace_bytes, int32_t* host_error, int clear,
                           void* stream);
 
+/*
+ * Host check of a decode batch's tables before they go to the device (host
+ * buffers, caller-owned; no device access). The kernels catch the same cases
+ * on the device and report them in the workspace error word; this call lets a
+ * scheduler find them first. Checks, per sequence s, the rules of the layouts
+ * above: seq_lens[s] in [0, max_blocks_per_seq * block_size] (else
+ * PKV_DEVERR_SEQ_LEN), entries j < ceil(seq_lens[s] / block_size) of row s in
+ * [0, num_blocks) (else PKV_DEVERR_BLOCK_ID), and, when slot_mapping is given
+ * (int64 [num_seqs], one new token per sequence as paged_decode_step takes
+ * it), every non-negative slot below num_blocks * block_size, inside the block
+ * that holds position seq_lens[s] - 1 and not also another sequence's slot
+ * (else PKV_DEVERR_SLOT). *bad_bits = the PKV_DEVERR_* bits found (0: clean),
+ * *first_bad = the first sequence with a problem or -1. Returns PKV_OK,
+ * PKV_ERR_NULL, PKV_ERR_SHAPE (num_seqs < 0, a size <= 0) or PKV_BM_HOST_ALLOC
+ * (host memory exhausted).
+ */
+PKV_API int pkv_validate_tables(const int32_t* block_tables, const int32_t* seq_lens, int num_seqs,
+                                int max_blocks_per_seq, int block_size, int num_blocks,
+                                const int64_t* slot_mapping, int32_t* bad_bits, int32_t* first_bad);
+
 /* Number of partitions num_partitions = 0 resolves to for this configuration on the current device. */
 PKV_API int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_kv_heads, int kv_dtype);
 

@@ -86,6 +86,9 @@ def load_library():
                                                     i32, f32, f32, P, P, P, P, P, i32, i32, i32, P, sz, P, P, P,
                                                     i32, P]
     lib.paged_decode_step_shared_prefix.restype = i32
+    lib.pkv_validate_tables.argtypes = [P, P, i32, i32, i32, i32, P, ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_int32)]
+    lib.pkv_validate_tables.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -432,6 +435,22 @@ def paged_decode_step_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_
     _check("paged_decode_step_shared_prefix", st)
 
 
+def validate_tables(block_tables, seq_lens, block_size: int, num_blocks: int, slot_mapping=None):
+    """Host check of a batch's tables (numpy or CPU tensors): (PKV_DEVERR_* bits found, first
+    offending sequence or -1). See pkv_validate_tables."""
+    import numpy as np
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    sm = None if slot_mapping is None else np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    if bt.ndim != 2 or bt.shape[0] != sl.shape[0] or (sm is not None and sm.shape != sl.shape):
+        raise ValueError("block_tables [n, max_blocks], seq_lens [n], slot_mapping [n]")
+    bits, first = ctypes.c_int32(0), ctypes.c_int32(-1)
+    _check("pkv_validate_tables", load_library().pkv_validate_tables(
+        bt.ctypes.data, sl.ctypes.data, sl.shape[0], max(1, bt.shape[1]), int(block_size), int(num_blocks),
+        None if sm is None else sm.ctypes.data, ctypes.byref(bits), ctypes.byref(first)))
+    return int(bits.value), int(first.value)
+
+
 _ws_cache: dict = {}
 
 
@@ -456,6 +475,6 @@ __all__ = [
     "reshape_and_cache", "reshape_and_cache_head_scales", "workspace_size", "new_workspace", "workspace_init",
     "read_device_error", "default_partitions", "status_string", "load_library", "PkvError",
     "paged_attention_decode_shared_prefix", "paged_decode_step_shared_prefix", "DevicePrefixPlan",
-    "shared_prefix_workspace_size", "new_shared_prefix_workspace",
+    "shared_prefix_workspace_size", "new_shared_prefix_workspace", "validate_tables",
     "F32", "BF16", "FP8_E4M3", "FP8_E5M2", "INT8",
 ]
