@@ -98,11 +98,13 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3, PK
 #define PKV_DEVERR_PLAN 16     /* a shared-prefix plan entry out of range: that sequence's output is unspecified */
 
 /*
- * Bytes of device workspace paged_attention_decode needs: an error word, one
- * arrival counter per (sequence, kv head) and fp32 split-KV partials
- * (o[G][head_dim], m[G], l[G]) for up to num_partitions + num_seqs*num_kv_heads
- * segments. num_partitions = 0 sizes it for the automatic partition count on
- * the current device. Returns 0 for unsupported sizes.
+ * Bytes of device workspace paged_attention_decode needs: a 256-byte header
+ * (error word, work-claim counters), one arrival counter per (sequence, kv
+ * head) and fp32 split-KV partials (o[G][head_dim], m[G], l[G]) for up to
+ * 4 * (5 * num_partitions) + num_seqs * num_kv_heads segments (a partition's
+ * share of the work is cut into at most 5 chunks). num_partitions = 0 sizes it
+ * for the automatic partition count on the current device. Returns 0 for
+ * unsupported sizes.
  */
 PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                       int num_partitions);
@@ -110,23 +112,28 @@ PKV_API size_t paged_attention_workspace_size(int num_seqs, int num_heads, int n
 /*
  * Zero a workspace (asynchronously on `stream`). Required once after the
  * workspace is allocated, and again after a call that reported
- * PKV_DEVERR_TIMEOUT; every normal call leaves the counters at zero.
+ * PKV_DEVERR_TIMEOUT or returned PKV_ERR_LAUNCH; every normal call leaves the
+ * workspace's counters at zero.
  */
 PKV_API int pkv_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Paged decode attention. The total work, sum over (sequence, kv head) of
- * ceil(seq_len / block_size) blocks, is cut into num_partitions equal runs of
- * blocks (0 = one or more per SM, from the occupancy); a run may cover several
- * (sequence, kv head) pairs and a pair may be split across runs. Each run
- * streams its K/V tiles through shared memory and keeps an online softmax; no
- * run ever waits for another. A pair split across runs leaves one fp32 partial
- * (o, m, l) per run in the workspace, and the log-sum-exp merge of those
- * partials writes its output: for the tensor-core kernel (bf16 and 8-bit
- * caches of the shapes paged_decode_step lists) a second, small kernel
- * launched right behind the decode kernel on `stream` does the merge; for the
- * CUDA-core kernel (F32 caches and the other shapes) the run that finishes a
- * pair last merges it inside the same launch.
+ * ceil(seq_len / block_size) blocks, taken in (sequence, kv head, block) order,
+ * is shared between num_partitions CTAs (0 = one or more per SM, from the
+ * occupancy); a piece of work may cover several (sequence, kv head) pairs and
+ * a pair may be split between pieces. Each piece streams its K/V tiles through
+ * shared memory and keeps an online softmax; no CTA ever waits for another. A
+ * pair split between pieces leaves one fp32 partial (o, m, l) per piece in the
+ * workspace, and the log-sum-exp merge of those partials writes its output.
+ * Tensor-core kernel (bf16 and 8-bit caches of the shapes paged_decode_step
+ * lists): every CTA takes an equal share of three quarters of the work, then
+ * claims small chunks of the last quarter from a workspace counter until none
+ * is left (the pieces are the same whichever CTA takes them, so the result
+ * does not depend on timing); a second, small kernel launched right behind the
+ * decode kernel on `stream` does the merge. CUDA-core kernel (F32 caches and
+ * the other shapes): equal runs, and the run that finishes a pair last merges
+ * it inside the same launch.
  *
  *   out          [num_seqs][num_heads][head_dim], q_dtype
  *   q            [num_seqs][num_heads][head_dim], q_dtype

@@ -62,8 +62,10 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
     const long long pairs = (long long)num_seqs * num_kv_heads;
     w.counters_off = kWorkspaceHeader;
     w.partials_off = w.counters_off + round_up((size_t)pairs * 4, 256);
-    // a run writes at most one partial per (stream it touches, head of the stream's group)
-    w.bytes = w.partials_off + (size_t)(runs * kMaxHeadGroup + pairs) * slot_floats_for(group, head_dim) * 4;
+    // a chunk (a run's own or a tail chunk, 1 + kTailChunksPerRun per run at most) writes at most
+    // one partial per (stream it touches, head of the stream's group)
+    w.bytes = w.partials_off +
+              (size_t)(runs * (1 + kTailChunksPerRun) * kMaxHeadGroup + pairs) * slot_floats_for(group, head_dim) * 4;
     return w;
 }
 
@@ -221,6 +223,8 @@ int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_
     p.q_len = q_len;
     p.k_head_scales = k_head_scales;
     p.v_head_scales = v_head_scales;
+    p.tail_chunks = kTailChunksPerRun;
+    p.chunk_ctr = reinterpret_cast<int32_t*>(ws) + 1;   // header word 1
     if (withheld_unit >= 0) {
         if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))
             return PKV_ERR_SHAPE;   // the hook lives in the tensor-core kernel only
@@ -475,7 +479,7 @@ size_t prefix_partials_bytes(int num_groups, int num_kv_heads, int head_dim, lon
     if (num_groups <= 0)
         return 0;   // no prefix pass
     const size_t slot = round_up((size_t)8 * (head_dim + 2), 4) * 4;
-    return (size_t)(runs_p + (long long)num_groups * num_kv_heads) * 4 * slot;
+    return (size_t)(runs_p * (1 + kTailChunksPerRun) + (long long)num_groups * num_kv_heads) * 4 * slot;
 }
 
 int shared_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -551,6 +555,7 @@ int shared_prefix_impl(void* out, const void* q, const void* k_cache, const void
     pp.pfx_shared = shared_blocks;
     pp.pfx_max_group = max_group;
     pp.pfx_num_seqs = num_seqs;
+    pp.chunk_ctr = reinterpret_cast<int32_t*>(workspace) + 2;   // header word 2: the prefix pass's claims
 
     MmaOp op{};
     op.kind = MmaOp::kLaunchSharedPrefix;

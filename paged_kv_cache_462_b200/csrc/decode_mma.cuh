@@ -51,6 +51,7 @@
 namespace pkv {
 
 constexpr float kMmaRescaleSlack = 8.0f;  // log2 units
+constexpr int kChunkRing = 16;             // chunk ids in flight between producer and consumers (> stages)
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -342,6 +343,43 @@ __device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* pre
     return any_bad | any_plan;
 }
 
+// The units of a launch, in (sequence, head group, block) order, cut into chunks. Chunk c < R (R =
+// the grid's CTAs) is CTA c's own: [c * P1, (c + 1) * P1), three quarters of the work shared out
+// evenly. The last quarter is cut into chunks of P2 >= kMinTailChunk units, about
+// tail_chunks per CTA, which CTAs claim from a counter as they finish: SMs that stream slower
+// take fewer of them, so the grid ends together. With tail_chunks = 0 (or too little work) the
+// R own chunks cover everything. Chunks are contiguous and in order: the pieces of a stream are
+// chunks of(begin) .. of(end - 1), the same for every schedule.
+struct Chunks {
+    int R, P1, P2, C, U;
+    __device__ __forceinline__ int begin(int c) const { return c < R ? c * P1 : R * P1 + (c - R) * P2; }
+    __device__ __forceinline__ int end(int c) const
+    {
+        return min(U, c < R ? (c + 1) * P1 : R * P1 + (c - R + 1) * P2);
+    }
+    __device__ __forceinline__ int of(int x) const { return x < R * P1 ? x / P1 : R + (x - R * P1) / P2; }
+};
+
+__device__ __forceinline__ Chunks make_chunks(int U, int R, int tail_chunks)
+{
+    Chunks ch;
+    ch.R = R;
+    ch.U = U;
+    const int per = (U + R - 1) / R;
+    if (tail_chunks <= 0 || U < 2 * R * kMinTailChunk) {   // static: one run per CTA
+        ch.P1 = per > 0 ? per : 1;
+        ch.P2 = 1;
+        ch.C = R;
+        return ch;
+    }
+    ch.P1 = (int)(3ll * U / (4ll * R));
+    const int rem = U - R * ch.P1;
+    const int want = (rem + R * tail_chunks - 1) / (R * tail_chunks);
+    ch.P2 = want > kMinTailChunk ? want : kMinTailChunk;
+    ch.C = R + (rem + ch.P2 - 1) / ch.P2;
+    return ch;
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <class KV, class QT, int D, int BS, int G, int HG, bool PFX = false>
@@ -369,7 +407,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
     uint64_t* empty = full + S;
     int* skip = reinterpret_cast<int*>(empty + S);
     volatile int* abort_flag = skip + S;
-    int* prefix = const_cast<int*>(abort_flag + 1);                           // [num_seqs + 1]
+    int* chunk_ring = const_cast<int*>(abort_flag + 1);                       // [kChunkRing] chunk ids
+    int* prefix = chunk_ring + kChunkRing;                                     // [num_seqs + 1]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -400,10 +439,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 
     const int total = prefix[p.num_seqs];
     const int nruns = gridDim.x;
-    const int per_run = (total + nruns - 1) / nruns;
-    const int run_begin = min(total, (int)blockIdx.x * per_run);
-    const int run_end = min(total, run_begin + per_run);
-    const int nunits = run_end - run_begin;
+    const Chunks ch = make_chunks(total, nruns, p.tail_chunks);
 
     // zero rows of empty sequences (one run per sequence); a prefix pass writes no rows, and a
     // suffix pass leaves the rows of sequences with shared blocks to the merge
@@ -428,87 +464,120 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 
     // =========================== producer warp ===============================
     if (warp == W) {
-        if (nunits <= 0)
-            return;
         if (lane == 0) {
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
         }
-        // lane l resolves unit (batch + l): pool row of its head group, or -1 for a bad block id;
-        // `app` is the stream (sequence * NHG + head group) whose new token lands in this unit
-        // (its last block) when the launch also appends, else -1
-        auto locate = [&](int k, int& app) -> int {
-            app = -1;
-            if (k >= nunits)
-                return -1;
-            const int x = run_begin + k;
-            const int s = find_seq(prefix, p.num_seqs, x);
-            const int nb = (prefix[s + 1] - prefix[s]) / NHG;
-            const int r = x - prefix[s];
-            const int hg = r / nb, j = r - hg * nb;
-            if (p.new_k != nullptr && j == nb - 1)
-                app = s * NHG + hg;
-            int skipb = 0;
-            if (p.skip_blocks != nullptr) {   // a suffix pass starts past the shared blocks
-                int e = 0;
-                (void)stream_tokens(p, s, BS, capacity, skipb, e);
-            }
-            const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + skipb + j);
-            if (phys < 0 || phys >= p.num_blocks) {
-                atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
-                return -1;
-            }
-            return (phys * Hkv + hg * HG) * BS;
-        };
-        int cur_app, ahead_app;
-        int cur = locate(lane, cur_app), ahead = locate(32 + lane, ahead_app);
+        // chunks: this CTA's own, then tail chunks claimed one ahead (the claim's round trip
+        // overlaps the current chunk's copies)
+        int cur = blockIdx.x;
+        int nxt = ch.C;
+        if (lane == 0 && ch.C > ch.R)
+            nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
         bool aborted = false;
         int issued = 0;
-        for (int k0 = 0; k0 < nunits; k0 += 32) {
-            if (k0 > 0) {
-                cur = ahead;
-                cur_app = ahead_app;
-                ahead = locate(k0 + 32 + lane, ahead_app);
+        int k = 0;                 // stages issued so far (ring position)
+        int published = 0;         // chunks announced to the consumers
+        while (cur < ch.C && !aborted) {
+            const int cb = ch.begin(cur);
+            const int nunits = ch.end(cur) - cb;
+            if (nunits > 0) {
+                if (lane == 0)
+                    chunk_ring[published % kChunkRing] = cur;   // read after this chunk's first stage fills
+                ++published;
             }
-            const int cnt = min(32, nunits - k0);
-            for (int i = 0; i < cnt; ++i) {
-                const int row = __shfl_sync(kFullMask, cur, i);
-                const int app = __shfl_sync(kFullMask, cur_app, i);
-                if (app >= 0)   // the decode-step append of this stream, before its last block is read
-                    append_new_token_impl<KV>(p, app / NHG, (app % NHG) * HG, HG, D, BS, lane,
-                                                      row < 0 ? -1 : row / (Hkv * BS));
-                if (lane == 0 && !aborted) {
-                    const int k = k0 + i;
-                    const int st = k % S;
-                    if (*abort_flag) {
-                        aborted = true;
-                    } else if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
-                        aborted = true;
-                        *abort_flag = 1;
-                        atomicOr(p.err, PKV_DEVERR_TIMEOUT);
-                    } else if (p.withheld_unit != 0 && run_begin + k == p.withheld_unit - 1) {
-                        aborted = true;   // test hook: this stage never fills; issue nothing more
-                    } else if (row < 0) {
-                        skip[st] = 1;
-                        mbar_arrive(&full[st]);
-                        issued = k + 1;
-                    } else {
-                        skip[st] = 0;
-                        uint8_t* dst = stages + (size_t)st * C::kStage;
-                        mbar_arrive_expect_tx(&full[st], C::kStage);
-#pragma unroll
-                        for (int bx = 0; bx < C::kBoxes; ++bx) {
-                            tma_load_2d(dst + bx * C::kBoxBytes, &kmap, bx * C::kBoxCols, row, &full[st]);
-                            tma_load_2d(dst + C::kHalf + bx * C::kBoxBytes, &vmap, bx * C::kBoxCols, row, &full[st]);
-                        }
-                        issued = k + 1;
-                    }
+            // lane l resolves unit (batch + l): pool row of its head group, or -1 for a bad block
+            // id; `app` is the stream (sequence * NHG + head group) whose new token lands in this
+            // unit (its last block) when the launch also appends, else -1
+            auto locate = [&](int kk, int& app) -> int {
+                app = -1;
+                if (kk >= nunits)
+                    return -1;
+                const int x = cb + kk;
+                const int s = find_seq(prefix, p.num_seqs, x);
+                const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+                const int r = x - prefix[s];
+                const int hg = r / nb, j = r - hg * nb;
+                if (p.new_k != nullptr && j == nb - 1)
+                    app = s * NHG + hg;
+                int skipb = 0;
+                if (p.skip_blocks != nullptr) {   // a suffix pass starts past the shared blocks
+                    int e = 0;
+                    (void)stream_tokens(p, s, BS, capacity, skipb, e);
                 }
+                const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + skipb + j);
+                if (phys < 0 || phys >= p.num_blocks) {
+                    atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
+                    return -1;
+                }
+                return (phys * Hkv + hg * HG) * BS;
+            };
+            int cur_app, ahead_app;
+            int cur_row = locate(lane, cur_app), ahead = locate(32 + lane, ahead_app);
+            for (int k0 = 0; k0 < nunits && !aborted; k0 += 32) {
+                if (k0 > 0) {
+                    cur_row = ahead;
+                    cur_app = ahead_app;
+                    ahead = locate(k0 + 32 + lane, ahead_app);
+                }
+                const int cnt = min(32, nunits - k0);
+                for (int i = 0; i < cnt; ++i) {
+                    const int row = __shfl_sync(kFullMask, cur_row, i);
+                    const int app = __shfl_sync(kFullMask, cur_app, i);
+                    if (app >= 0)   // the decode-step append of this stream, before its last block is read
+                        append_new_token_impl<KV>(p, app / NHG, (app % NHG) * HG, HG, D, BS, lane,
+                                                  row < 0 ? -1 : row / (Hkv * BS));
+                    if (lane == 0 && !aborted) {
+                        const int st = k % S;
+                        if (*abort_flag) {
+                            aborted = true;
+                        } else if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
+                            aborted = true;
+                            *abort_flag = 1;
+                            atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                        } else if (p.withheld_unit != 0 && cb + k0 + i == p.withheld_unit - 1) {
+                            aborted = true;   // test hook: this stage never fills; issue nothing more
+                        } else if (row < 0) {
+                            skip[st] = 1;
+                            mbar_arrive(&full[st]);
+                            issued = k + 1;
+                        } else {
+                            skip[st] = 0;
+                            uint8_t* dst = stages + (size_t)st * C::kStage;
+                            mbar_arrive_expect_tx(&full[st], C::kStage);
+#pragma unroll
+                            for (int bx = 0; bx < C::kBoxes; ++bx) {
+                                tma_load_2d(dst + bx * C::kBoxBytes, &kmap, bx * C::kBoxCols, row, &full[st]);
+                                tma_load_2d(dst + C::kHalf + bx * C::kBoxBytes, &vmap, bx * C::kBoxCols, row,
+                                            &full[st]);
+                            }
+                            issued = k + 1;
+                        }
+                    }
+                    ++k;
+                }
+                aborted = __shfl_sync(kFullMask, aborted ? 1 : 0, 0) != 0;
+            }
+            cur = __shfl_sync(kFullMask, nxt, 0);
+            if (lane == 0 && cur < ch.C)
+                nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
+        }
+        // end of the work: a stage without bytes whose chunk id is -1 tells the consumers
+        if (lane == 0 && !aborted) {
+            const int st = k % S;
+            if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
+                aborted = true;
+                *abort_flag = 1;
+                atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+            } else {
+                chunk_ring[published % kChunkRing] = -1;
+                skip[st] = 1;
+                mbar_arrive(&full[st]);
             }
         }
         if (lane == 0 && aborted) {
-            for (int k = max(0, issued - S); k < issued; ++k)
-                (void)mbar_wait_bounded(&full[k % S], (k / S) & 1);
+            for (int kk = max(0, issued - S); kk < issued; ++kk)
+                (void)mbar_wait_bounded(&full[kk % S], (kk / S) & 1);
         }
         return;
     }
@@ -518,411 +587,429 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
     const int t = lane & 3;    // MMA column pair
 
 
-    int x = run_begin;
-    int k = 0;                 // unit index within the run
-    while (x < run_end) {
-        const int s = find_seq(prefix, p.num_seqs, x);
-        const int nb = (prefix[s + 1] - prefix[s]) / NHG;
-        const int hg = (x - prefix[s]) / nb;
-        const int stream_begin = prefix[s] + hg * nb;
-        const int stream_end = stream_begin + nb;
-        const int seg_end = min(run_end, stream_end);
-        const int head = hg * HG + warp / C::kNT;   // this warp's KV head
-        const int tile = warp % C::kNT;             // prefix pass: this warp's 8 of the 32 columns
-        int skipb = 0, lerr = 0;
-        const int L = stream_tokens(p, s, BS, capacity, skipb, lerr);
-        const int QL = p.q_len > 1 ? p.q_len : 1;
-        const int Gq = p.num_heads / p.num_kv_heads;
-        // FP8 per-head scales (when given): this head's into the score and output factors
-        const float qk_scale = p.k_head_scales ? p.q_scale * __ldg(p.k_head_scales + head) : p.q_scale;
-        const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
-        // Query column c (0..7) of this warp: its row of q / out, and how many of the stream's
-        // tokens it sees. Decode: column c is new token c / Gq of q_len and sees the tokens before
-        // position L - q_len + 1 + c / Gq (all L when q_len = 1); columns >= G are padding.
-        // Prefix pass: column tile * 8 + c is query head (.. % Gq) of member (.. / Gq) of group s,
-        // which sees its own shared blocks of the group's row; columns past the members: padding.
-        auto column = [&](int c, size_t& row) -> int {
-            row = 0;
-            if constexpr (PFX) {
-                const int cg = tile * 8 + c, mem = cg / Gq;
-                const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
-                if (mem >= cnt || mem >= p.pfx_max_group)
-                    return 0;
-                const int seq = p.pfx_members[off + mem];
-                if (seq < 0 || seq >= p.pfx_num_seqs)
-                    return 0;
-                row = (size_t)seq * p.num_heads + (size_t)head * Gq + (cg - mem * Gq);
-                const int lim = p.pfx_shared[seq] * BS;
-                return lim < 0 ? 0 : (lim < L ? lim : L);
-            } else {
-                if (c >= G)
-                    return 0;
-                row = query_row(p, s, head, c);
-                return L - QL + 1 + c / Gq;
-            }
-        };
-        size_t row_g, row0, row1;
-        const int lim_g = column(g, row_g);
-        const int lim0 = column(2 * t, row0);
-        const int lim1 = column(2 * t + 1, row1);
-        const bool qcol = PFX ? lim_g > 0 : g < G;   // this lane holds a real column g of Q^T
-        if constexpr (PFX) {
-            if (tile == 0 && lane == 0) {
-                const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
-                bool bad = cnt > p.pfx_max_group;
-                for (int i = 0; i < cnt && i < p.pfx_max_group; ++i) {
-                    const int seq = p.pfx_members[off + i];
-                    bad |= seq < 0 || seq >= p.pfx_num_seqs || p.pfx_shared[seq] * BS > L;
-                }
-                if (bad)
-                    atomicOr(p.err, PKV_DEVERR_PLAN);
-            }
-        }
-
-        // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
-        uint32_t qb[C::kKS][2];
-        float qk0 = qk_scale, qk1 = qk_scale;   // score factors of this lane's columns 2t, 2t+1
-        if constexpr (F8) {
-            // FP8 products: column g of Q^T times a power of two sigma_g (max |q| * sigma_g < 256),
-            // as E4M3 hi + lo codes (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3,
-            // b1 = d 32kk + 16 + 4t .. +3. 1 / sigma goes into the column's score factor.
-            constexpr int K8 = D / 32;
-            const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
-            float f[K8][2][4];
-            float mx = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < K8; ++kk)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    if (qcol)
-                        load_q<4>(qp + kk * 32 + hh * 16 + 4 * t, f[kk][hh]);
-                    else
-                        f[kk][hh][0] = f[kk][hh][1] = f[kk][hh][2] = f[kk][hh][3] = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        mx = fmaxf(mx, fabsf(f[kk][hh][i]));
-                }
-            mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
-            // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
-            int se = 127;
-            if (mx > 0.f) {
-                se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
-                se = se < 2 ? 2 : (se > 252 ? 252 : se);
-            }
-            const float sig = __uint_as_float((uint32_t)se << 23);
-            const float inv_sig = __uint_as_float((uint32_t)(254 - se) << 23);
-#pragma unroll
-            for (int kk = 0; kk < K8; ++kk)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t h01, l01, h23, l23;
-                    split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
-                    split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
-                    qb[kk][hh] = h01 | (h23 << 16);
-                    qb[K8 + kk][hh] = l01 | (l23 << 16);
-                }
-            qk0 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t) * 4);
-            qk1 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t + 1) * 4);
-        } else {
-            const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
-#pragma unroll
-            for (int ks = 0; ks < C::kKS; ++ks) {
-                if (qcol) {
-                    if constexpr (F16) {
-                        // k order permuted to match the widened INT8 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
-                        float f[4];
-                        load_q<4>(qp + ks * 16 + 4 * t, f);
-                        qb[ks][0] = pack2<true>(f[0], f[1]);
-                        qb[ks][1] = pack2<true>(f[2], f[3]);
-                    } else {
-                        qb[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t));
-                        qb[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t + 8));
-                    }
-                } else {
-                    qb[ks][0] = qb[ks][1] = 0u;
-                }
-            }
-        }
-        float o[C::kDT][4];
-#pragma unroll
-        for (int dt = 0; dt < C::kDT; ++dt)
-            o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-        float m[2] = {-INFINITY, -INFINITY};   // running reference for heads 2t, 2t+1
-        float l[2] = {0.f, 0.f};
-
-        for (; x < seg_end; ++x, ++k) {
+    int k = 0;                 // stages consumed so far (ring position)
+    for (int ordinal = 0;; ++ordinal) {
+        // the first stage of the CTA's next chunk carries the chunk's id (-1: no more work)
+        {
             const int st = k % S;
-            bool ok = !*abort_flag && mbar_wait_bounded(&full[st], (k / S) & 1);
-            if (__any_sync(kFullMask, !ok)) {
+            const bool ok = !*abort_flag && mbar_wait_bounded(&full[st], (k / S) & 1);
+            if (!__all_sync(kFullMask, ok)) {
                 if (lane == 0 && !*abort_flag) {
                     *abort_flag = 1;
                     atomicOr(p.err, PKV_DEVERR_TIMEOUT);
                 }
-                ok = false;
-            }
-            const int jb = x - stream_begin;         // logical block
-            const int valid = min(BS, L - jb * BS);
-            bool released = false;
-            if (ok && skip[st] == 0 && valid > 0) {
-                const uint32_t kbase = smem_addr(stages + (size_t)st * C::kStage);
-                const uint32_t vbase = kbase + C::kHalf;
-                const int r0 = warp * BS;            // this head's first box row
-#pragma unroll
-                for (int tt = 0; tt < C::kTT; ++tt) {
-                    // ---- S^T = K Q^T : 16 tokens x 8 heads
-                    float sc[4] = {0.f, 0.f, 0.f, 0.f};
-                    float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
-                    const int mi = lane >> 3, rr = lane & 7;
-                    if constexpr (F8) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 32; ++kk) {
-                            // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment
-                            // of 16 tokens x d 32kk .. 32kk+31 as it lies in the stage, no conversion
-                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                            uint32_t a[4];
-                            ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
-                            mma_16832_f8<KV::kFmt>(sc, a, qb[kk][0], qb[kk][1]);                 // q hi
-                            mma_16832_f8<KV::kFmt>(sd, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);   // q lo
-                        }
-                    } else if constexpr (F16) {
-#pragma unroll
-                        for (int ks = 0; ks < C::kKS; ks += 2) {
-                            // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each
-                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                            uint32_t r[4];
-                            ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
-#pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
-                                const uint32_t a[4] = {fp8x2_to_f16x2<KV>(lo), fp8x2_to_f16x2<KV>(hi),
-                                                       fp8x2_to_f16x2<KV>(lo >> 16), fp8x2_to_f16x2<KV>(hi >> 16)};
-                                mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int ks = 0; ks < C::kKS; ++ks) {
-                            // matrices: (tok 0-7, d 0-7), (tok 8-15, d 0-7), (tok 0-7, d 8-15), (tok 8-15, d 8-15)
-                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                            const int box = ks / 4, chunk = (ks % 4) * 2 + (mi >> 1);
-                            uint32_t a[4];
-                            ldsm_x4(kbase + box * C::kBoxBytes + swz(row, chunk), a);
-                            mma_16816<false>((ks & 1) ? sd : sc, a, qb[ks][0], qb[ks][1]);
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        sc[i] += sd[i];
-                    // V fragments of this tile into registers; after the block's last tile the
-                    // stage goes back to the producer before the softmax and p.V arithmetic
-                    uint32_t vf[C::kDT * 4 / ((F16 || F8) ? 2 : 1)];
-                    if constexpr (F16 || F8) {
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; dt += 2) {
-                            // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
-                            const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                            uint32_t r[4];
-                            ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                vf[2 * dt + i] = r[i];
-                        }
-                    } else {
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; ++dt) {
-                            // matrices: (d 0-7, tok 0-7), (d 8-15, tok 0-7), (d 0-7, tok 8-15), (d 8-15, tok 8-15)
-                            const int row = r0 + tt * 16 + (mi >> 1) * 8 + rr;
-                            const int box = dt / 4, chunk = (dt % 4) * 2 + (mi & 1);
-                            uint32_t r[4];
-                            ldsm_x4_t(vbase + box * C::kBoxBytes + swz(row, chunk), r);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                vf[4 * dt + i] = r[i];
-                        }
-                    }
-                    if (tt == C::kTT - 1) {
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&empty[st]);
-                        released = true;
-                    }
-                    // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
-                    const int tok0 = jb * BS + tt * 16 + g;   // position in the sequence
-                    sc[0] = (tok0 < lim0) ? sc[0] * qk0 : -INFINITY;
-                    sc[1] = (tok0 < lim1) ? sc[1] * qk1 : -INFINITY;
-                    sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk0 : -INFINITY;
-                    sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk1 : -INFINITY;
-                    // The reference moves only when some score passes it by the slack; each lane
-                    // tests its own scores first, so the butterfly max runs only when one does
-                    // (same result as reducing first: the tile max passes iff some lane's does).
-                    float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
-                    if (__any_sync(kFullMask, bm0 > m[0] + kSlack || bm1 > m[1] + kSlack)) {
-#pragma unroll
-                        for (int off = 4; off < 32; off <<= 1) {
-                            bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
-                            bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
-                        }
-                        const bool up0 = bm0 > m[0] + kSlack, up1 = bm1 > m[1] + kSlack;
-                        const float n0 = up0 ? bm0 : m[0], n1 = up1 ? bm1 : m[1];
-                        const float a0 = up0 ? fast_exp2(m[0] - n0) : 1.f, a1 = up1 ? fast_exp2(m[1] - n1) : 1.f;
-                        m[0] = n0;
-                        m[1] = n1;
-                        l[0] *= a0;
-                        l[1] *= a1;
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; ++dt) {
-                            o[dt][0] *= a0;
-                            o[dt][1] *= a1;
-                            o[dt][2] *= a0;
-                            o[dt][3] *= a1;
-                        }
-                    }
-                    float pr[4];
-                    const float mo0 = m[0] - kPOff, mo1 = m[1] - kPOff;
-                    pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - mo0);
-                    pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - mo1);
-                    pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - mo0);
-                    pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - mo1);
-                    l[0] += pr[0] + pr[2];
-                    l[1] += pr[1] + pr[3];
-                    const int srcA = (2 * t) * 4 + (g >> 1), srcB = (2 * t + 1) * 4 + (g >> 1);
-                    uint32_t pb0, pb1;
-                    if constexpr (F8) {
-                        // ---- P^T as E4M3 hi (b0) and lo (b1) codes, k = tokens 2t, 2t+1, 2t+8, 2t+9 of column g
-                        uint32_t h0, l0, h1, l1;
-                        split_e4m3x2(pack2<true>(pr[0], pr[2]), h0, l0);   // column 2t:   tokens g, g+8
-                        split_e4m3x2(pack2<true>(pr[1], pr[3]), h1, l1);   // column 2t+1: tokens g, g+8
-                        const uint32_t wh = h0 | (h1 << 16), wl = l0 | (l1 << 16);
-                        const uint32_t ah = __shfl_sync(kFullMask, wh, srcA), bh = __shfl_sync(kFullMask, wh, srcB);
-                        const uint32_t al = __shfl_sync(kFullMask, wl, srcA), bl = __shfl_sync(kFullMask, wl, srcB);
-                        const uint32_t sel = (g & 1) ? 0x7362u : 0x5140u;
-                        pb0 = qcol ? __byte_perm(ah, bh, sel) : 0u;
-                        pb1 = qcol ? __byte_perm(al, bl, sel) : 0u;
-                    } else {
-                        // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
-                        const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
-                        const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
-                        const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
-                        const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
-                        const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
-                        pb0 = qcol ? __byte_perm(va, vb, 0x5410) : 0u;
-                        pb1 = qcol ? __byte_perm(va, vb, 0x7632) : 0u;
-                    }
-                    // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
-                    const bool partial = valid < tt * 16 + 16;
-                    if constexpr (F8) {
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; dt += 2) {
-#pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
-                                if (partial) {
-                                    const int tk = tt * 16 + 2 * t;
-                                    lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
-                                    hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
-                                }
-                                // rows g / g+8 of the m-tile = d 2g / 2g+1 of chunk dt + h2; k = tokens
-                                // 2t, 2t+1, 2t+8, 2t+9 against P hi, then the same tokens against P lo
-                                const uint32_t a0 = __byte_perm(lo, hi, 0x6420), a1 = __byte_perm(lo, hi, 0x7531);
-                                const uint32_t a[4] = {a0, a1, a0, a1};
-                                mma_16832_f8<KV::kFmt>(o[dt + h2], a, pb0, pb1);
-                            }
-                        }
-                    } else if constexpr (F16) {
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; dt += 2) {
-#pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
-                                if (partial) {
-                                    const int tk = tt * 16 + 2 * t;
-                                    lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
-                                    hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
-                                }
-                                // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1)
-                                const uint32_t a[4] = {fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0020)),
-                                                       fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0031)),
-                                                       fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0020)),
-                                                       fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0031))};
-                                mma_16816<true>(o[dt + h2], a, pb0, pb1);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int dt = 0; dt < C::kDT; ++dt) {
-                            uint32_t a[4] = {vf[4 * dt], vf[4 * dt + 1], vf[4 * dt + 2], vf[4 * dt + 3]};
-                            if (partial) {
-                                const int tk = tt * 16 + 2 * t;
-                                const uint32_t m01 = (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
-                                const uint32_t m89 = (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
-                                a[0] &= m01;
-                                a[1] &= m01;
-                                a[2] &= m89;
-                                a[3] &= m89;
-                            }
-                            mma_16816<false>(o[dt], a, pb0, pb1);
-                        }
-                    }
-                }
-            }
-            if (!released) {
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&empty[st]);
+                break;
             }
         }
+        const int cur = chunk_ring[ordinal % kChunkRing];
+        if (cur < 0 || cur >= ch.C)
+            break;
+        const int run_end = ch.end(cur);
+        int x = ch.begin(cur);
+        while (x < run_end) {
+            const int s = find_seq(prefix, p.num_seqs, x);
+            const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+            const int hg = (x - prefix[s]) / nb;
+            const int stream_begin = prefix[s] + hg * nb;
+            const int stream_end = stream_begin + nb;
+            const int seg_end = min(run_end, stream_end);
+            const int head = hg * HG + warp / C::kNT;   // this warp's KV head
+            const int tile = warp % C::kNT;             // prefix pass: this warp's 8 of the 32 columns
+            int skipb = 0, lerr = 0;
+            const int L = stream_tokens(p, s, BS, capacity, skipb, lerr);
+            const int QL = p.q_len > 1 ? p.q_len : 1;
+            const int Gq = p.num_heads / p.num_kv_heads;
+            // FP8 per-head scales (when given): this head's into the score and output factors
+            const float qk_scale = p.k_head_scales ? p.q_scale * __ldg(p.k_head_scales + head) : p.q_scale;
+            const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
+            // Query column c (0..7) of this warp: its row of q / out, and how many of the stream's
+            // tokens it sees. Decode: column c is new token c / Gq of q_len and sees the tokens before
+            // position L - q_len + 1 + c / Gq (all L when q_len = 1); columns >= G are padding.
+            // Prefix pass: column tile * 8 + c is query head (.. % Gq) of member (.. / Gq) of group s,
+            // which sees its own shared blocks of the group's row; columns past the members: padding.
+            auto column = [&](int c, size_t& row) -> int {
+                row = 0;
+                if constexpr (PFX) {
+                    const int cg = tile * 8 + c, mem = cg / Gq;
+                    const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
+                    if (mem >= cnt || mem >= p.pfx_max_group)
+                        return 0;
+                    const int seq = p.pfx_members[off + mem];
+                    if (seq < 0 || seq >= p.pfx_num_seqs)
+                        return 0;
+                    row = (size_t)seq * p.num_heads + (size_t)head * Gq + (cg - mem * Gq);
+                    const int lim = p.pfx_shared[seq] * BS;
+                    return lim < 0 ? 0 : (lim < L ? lim : L);
+                } else {
+                    if (c >= G)
+                        return 0;
+                    row = query_row(p, s, head, c);
+                    return L - QL + 1 + c / Gq;
+                }
+            };
+            size_t row_g, row0, row1;
+            const int lim_g = column(g, row_g);
+            const int lim0 = column(2 * t, row0);
+            const int lim1 = column(2 * t + 1, row1);
+            const bool qcol = PFX ? lim_g > 0 : g < G;   // this lane holds a real column g of Q^T
+            if constexpr (PFX) {
+                if (tile == 0 && lane == 0) {
+                    const int off = p.pfx_offsets[s], cnt = p.pfx_offsets[s + 1] - off;
+                    bool bad = cnt > p.pfx_max_group;
+                    for (int i = 0; i < cnt && i < p.pfx_max_group; ++i) {
+                        const int seq = p.pfx_members[off + i];
+                        bad |= seq < 0 || seq >= p.pfx_num_seqs || p.pfx_shared[seq] * BS > L;
+                    }
+                    if (bad)
+                        atomicOr(p.err, PKV_DEVERR_PLAN);
+                }
+            }
 
-        // ---- end of this warp's segment: l over the 8 row groups, then write or merge
+            // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
+            uint32_t qb[C::kKS][2];
+            float qk0 = qk_scale, qk1 = qk_scale;   // score factors of this lane's columns 2t, 2t+1
+            if constexpr (F8) {
+                // FP8 products: column g of Q^T times a power of two sigma_g (max |q| * sigma_g < 256),
+                // as E4M3 hi + lo codes (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3,
+                // b1 = d 32kk + 16 + 4t .. +3. 1 / sigma goes into the column's score factor.
+                constexpr int K8 = D / 32;
+                const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
+                float f[K8][2][4];
+                float mx = 0.f;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l[0] += __shfl_xor_sync(kFullMask, l[0], off);
-            l[1] += __shfl_xor_sync(kFullMask, l[1], off);
-        }
-        const int first_run = stream_begin / per_run;
-        const int last_run = (stream_end - 1) / per_run;
-        const int stream = s * NHG + hg;
-        // element (head column c, row d) of this lane's accumulators
-        auto d_of = [&](int dt, int half) -> int {
-            return (F16 || F8) ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
-        };
-        // a whole stream writes `out`; pieces of split streams, every stream of a prefix pass and
-        // the suffix of a sequence with shared blocks leave (o, m, l) for the merge
-        if (first_run == last_run && !PFX && skipb == 0) {
-            QT* out0 = reinterpret_cast<QT*>(p.out) + row0 * D;
-            QT* out1 = reinterpret_cast<QT*>(p.out) + row1 * D;
-            const float inv0 = l[0] > 0.f ? out_scale / l[0] : 0.f;
-            const float inv1 = l[1] > 0.f ? out_scale / l[1] : 0.f;
+                for (int kk = 0; kk < K8; ++kk)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (qcol)
+                            load_q<4>(qp + kk * 32 + hh * 16 + 4 * t, f[kk][hh]);
+                        else
+                            f[kk][hh][0] = f[kk][hh][1] = f[kk][hh][2] = f[kk][hh][3] = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            mx = fmaxf(mx, fabsf(f[kk][hh][i]));
+                    }
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
+                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
+                int se = 127;
+                if (mx > 0.f) {
+                    se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
+                    se = se < 2 ? 2 : (se > 252 ? 252 : se);
+                }
+                const float sig = __uint_as_float((uint32_t)se << 23);
+                const float inv_sig = __uint_as_float((uint32_t)(254 - se) << 23);
+#pragma unroll
+                for (int kk = 0; kk < K8; ++kk)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t h01, l01, h23, l23;
+                        split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
+                        split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
+                        qb[kk][hh] = h01 | (h23 << 16);
+                        qb[K8 + kk][hh] = l01 | (l23 << 16);
+                    }
+                qk0 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t) * 4);
+                qk1 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t + 1) * 4);
+            } else {
+                const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
+#pragma unroll
+                for (int ks = 0; ks < C::kKS; ++ks) {
+                    if (qcol) {
+                        if constexpr (F16) {
+                            // k order permuted to match the widened INT8 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
+                            float f[4];
+                            load_q<4>(qp + ks * 16 + 4 * t, f);
+                            qb[ks][0] = pack2<true>(f[0], f[1]);
+                            qb[ks][1] = pack2<true>(f[2], f[3]);
+                        } else {
+                            qb[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t));
+                            qb[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t + 8));
+                        }
+                    } else {
+                        qb[ks][0] = qb[ks][1] = 0u;
+                    }
+                }
+            }
+            float o[C::kDT][4];
 #pragma unroll
             for (int dt = 0; dt < C::kDT; ++dt)
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int d = d_of(dt, half);
-                    if (2 * t < G)
-                        from_float(o[dt][2 * half] * inv0, out0 + d);
-                    if (2 * t + 1 < G)
-                        from_float(o[dt][2 * half + 1] * inv1, out1 + d);
+                o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+            float m[2] = {-INFINITY, -INFINITY};   // running reference for heads 2t, 2t+1
+            float l[2] = {0.f, 0.f};
+
+            for (; x < seg_end; ++x, ++k) {
+                const int st = k % S;
+                bool ok = !*abort_flag && mbar_wait_bounded(&full[st], (k / S) & 1);
+                if (__any_sync(kFullMask, !ok)) {
+                    if (lane == 0 && !*abort_flag) {
+                        *abort_flag = 1;
+                        atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                    }
+                    ok = false;
                 }
-        } else {
-            float* part = p.partials + ((size_t)(blockIdx.x + stream) * W + warp) * p.slot_floats;
+                const int jb = x - stream_begin;         // logical block
+                const int valid = min(BS, L - jb * BS);
+                bool released = false;
+                if (ok && skip[st] == 0 && valid > 0) {
+                    const uint32_t kbase = smem_addr(stages + (size_t)st * C::kStage);
+                    const uint32_t vbase = kbase + C::kHalf;
+                    const int r0 = warp * BS;            // this head's first box row
 #pragma unroll
-            for (int dt = 0; dt < C::kDT; ++dt)
+                    for (int tt = 0; tt < C::kTT; ++tt) {
+                        // ---- S^T = K Q^T : 16 tokens x 8 heads
+                        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                        float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
+                        const int mi = lane >> 3, rr = lane & 7;
+                        if constexpr (F8) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int d = d_of(dt, half);
-                    if (2 * t < G)
-                        part[(2 * t) * D + d] = o[dt][2 * half];
-                    if (2 * t + 1 < G)
-                        part[(2 * t + 1) * D + d] = o[dt][2 * half + 1];
+                            for (int kk = 0; kk < D / 32; ++kk) {
+                                // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment
+                                // of 16 tokens x d 32kk .. 32kk+31 as it lies in the stage, no conversion
+                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                uint32_t a[4];
+                                ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
+                                mma_16832_f8<KV::kFmt>(sc, a, qb[kk][0], qb[kk][1]);                 // q hi
+                                mma_16832_f8<KV::kFmt>(sd, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);   // q lo
+                            }
+                        } else if constexpr (F16) {
+#pragma unroll
+                            for (int ks = 0; ks < C::kKS; ks += 2) {
+                                // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each
+                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                uint32_t r[4];
+                                ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2) {
+                                    const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
+                                    const uint32_t a[4] = {fp8x2_to_f16x2<KV>(lo), fp8x2_to_f16x2<KV>(hi),
+                                                           fp8x2_to_f16x2<KV>(lo >> 16), fp8x2_to_f16x2<KV>(hi >> 16)};
+                                    mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int ks = 0; ks < C::kKS; ++ks) {
+                                // matrices: (tok 0-7, d 0-7), (tok 8-15, d 0-7), (tok 0-7, d 8-15), (tok 8-15, d 8-15)
+                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                const int box = ks / 4, chunk = (ks % 4) * 2 + (mi >> 1);
+                                uint32_t a[4];
+                                ldsm_x4(kbase + box * C::kBoxBytes + swz(row, chunk), a);
+                                mma_16816<false>((ks & 1) ? sd : sc, a, qb[ks][0], qb[ks][1]);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            sc[i] += sd[i];
+                        // V fragments of this tile into registers; after the block's last tile the
+                        // stage goes back to the producer before the softmax and p.V arithmetic
+                        uint32_t vf[C::kDT * 4 / ((F16 || F8) ? 2 : 1)];
+                        if constexpr (F16 || F8) {
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; dt += 2) {
+                                // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
+                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                uint32_t r[4];
+                                ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    vf[2 * dt + i] = r[i];
+                            }
+                        } else {
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; ++dt) {
+                                // matrices: (d 0-7, tok 0-7), (d 8-15, tok 0-7), (d 0-7, tok 8-15), (d 8-15, tok 8-15)
+                                const int row = r0 + tt * 16 + (mi >> 1) * 8 + rr;
+                                const int box = dt / 4, chunk = (dt % 4) * 2 + (mi & 1);
+                                uint32_t r[4];
+                                ldsm_x4_t(vbase + box * C::kBoxBytes + swz(row, chunk), r);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    vf[4 * dt + i] = r[i];
+                            }
+                        }
+                        if (tt == C::kTT - 1) {
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(&empty[st]);
+                            released = true;
+                        }
+                        // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
+                        const int tok0 = jb * BS + tt * 16 + g;   // position in the sequence
+                        sc[0] = (tok0 < lim0) ? sc[0] * qk0 : -INFINITY;
+                        sc[1] = (tok0 < lim1) ? sc[1] * qk1 : -INFINITY;
+                        sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk0 : -INFINITY;
+                        sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk1 : -INFINITY;
+                        // The reference moves only when some score passes it by the slack; each lane
+                        // tests its own scores first, so the butterfly max runs only when one does
+                        // (same result as reducing first: the tile max passes iff some lane's does).
+                        float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
+                        if (__any_sync(kFullMask, bm0 > m[0] + kSlack || bm1 > m[1] + kSlack)) {
+#pragma unroll
+                            for (int off = 4; off < 32; off <<= 1) {
+                                bm0 = fmaxf(bm0, __shfl_xor_sync(kFullMask, bm0, off));
+                                bm1 = fmaxf(bm1, __shfl_xor_sync(kFullMask, bm1, off));
+                            }
+                            const bool up0 = bm0 > m[0] + kSlack, up1 = bm1 > m[1] + kSlack;
+                            const float n0 = up0 ? bm0 : m[0], n1 = up1 ? bm1 : m[1];
+                            const float a0 = up0 ? fast_exp2(m[0] - n0) : 1.f, a1 = up1 ? fast_exp2(m[1] - n1) : 1.f;
+                            m[0] = n0;
+                            m[1] = n1;
+                            l[0] *= a0;
+                            l[1] *= a1;
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; ++dt) {
+                                o[dt][0] *= a0;
+                                o[dt][1] *= a1;
+                                o[dt][2] *= a0;
+                                o[dt][3] *= a1;
+                            }
+                        }
+                        float pr[4];
+                        const float mo0 = m[0] - kPOff, mo1 = m[1] - kPOff;
+                        pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - mo0);
+                        pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - mo1);
+                        pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - mo0);
+                        pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - mo1);
+                        l[0] += pr[0] + pr[2];
+                        l[1] += pr[1] + pr[3];
+                        const int srcA = (2 * t) * 4 + (g >> 1), srcB = (2 * t + 1) * 4 + (g >> 1);
+                        uint32_t pb0, pb1;
+                        if constexpr (F8) {
+                            // ---- P^T as E4M3 hi (b0) and lo (b1) codes, k = tokens 2t, 2t+1, 2t+8, 2t+9 of column g
+                            uint32_t h0, l0, h1, l1;
+                            split_e4m3x2(pack2<true>(pr[0], pr[2]), h0, l0);   // column 2t:   tokens g, g+8
+                            split_e4m3x2(pack2<true>(pr[1], pr[3]), h1, l1);   // column 2t+1: tokens g, g+8
+                            const uint32_t wh = h0 | (h1 << 16), wl = l0 | (l1 << 16);
+                            const uint32_t ah = __shfl_sync(kFullMask, wh, srcA), bh = __shfl_sync(kFullMask, wh, srcB);
+                            const uint32_t al = __shfl_sync(kFullMask, wl, srcA), bl = __shfl_sync(kFullMask, wl, srcB);
+                            const uint32_t sel = (g & 1) ? 0x7362u : 0x5140u;
+                            pb0 = qcol ? __byte_perm(ah, bh, sel) : 0u;
+                            pb1 = qcol ? __byte_perm(al, bl, sel) : 0u;
+                        } else {
+                            // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
+                            const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
+                            const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
+                            const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
+                            const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
+                            const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
+                            pb0 = qcol ? __byte_perm(va, vb, 0x5410) : 0u;
+                            pb1 = qcol ? __byte_perm(va, vb, 0x7632) : 0u;
+                        }
+                        // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
+                        const bool partial = valid < tt * 16 + 16;
+                        if constexpr (F8) {
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; dt += 2) {
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2) {
+                                    uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
+                                    if (partial) {
+                                        const int tk = tt * 16 + 2 * t;
+                                        lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                        hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                    }
+                                    // rows g / g+8 of the m-tile = d 2g / 2g+1 of chunk dt + h2; k = tokens
+                                    // 2t, 2t+1, 2t+8, 2t+9 against P hi, then the same tokens against P lo
+                                    const uint32_t a0 = __byte_perm(lo, hi, 0x6420), a1 = __byte_perm(lo, hi, 0x7531);
+                                    const uint32_t a[4] = {a0, a1, a0, a1};
+                                    mma_16832_f8<KV::kFmt>(o[dt + h2], a, pb0, pb1);
+                                }
+                            }
+                        } else if constexpr (F16) {
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; dt += 2) {
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2) {
+                                    uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
+                                    if (partial) {
+                                        const int tk = tt * 16 + 2 * t;
+                                        lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                        hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                    }
+                                    // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1)
+                                    const uint32_t a[4] = {fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0020)),
+                                                           fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0031)),
+                                                           fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0020)),
+                                                           fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0031))};
+                                    mma_16816<true>(o[dt + h2], a, pb0, pb1);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int dt = 0; dt < C::kDT; ++dt) {
+                                uint32_t a[4] = {vf[4 * dt], vf[4 * dt + 1], vf[4 * dt + 2], vf[4 * dt + 3]};
+                                if (partial) {
+                                    const int tk = tt * 16 + 2 * t;
+                                    const uint32_t m01 = (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
+                                    const uint32_t m89 = (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                    a[0] &= m01;
+                                    a[1] &= m01;
+                                    a[2] &= m89;
+                                    a[3] &= m89;
+                                }
+                                mma_16816<false>(o[dt], a, pb0, pb1);
+                            }
+                        }
+                    }
                 }
-            if (g == 0) {
-                if (2 * t < G) {
-                    part[G * D + 2 * t] = m[0];
-                    part[G * D + G + 2 * t] = l[0];
+                if (!released) {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&empty[st]);
                 }
-                if (2 * t + 1 < G) {
-                    part[G * D + 2 * t + 1] = m[1];
-                    part[G * D + G + 2 * t + 1] = l[1];
+            }
+
+            // ---- end of this warp's segment: l over the 8 row groups, then write or merge
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                l[0] += __shfl_xor_sync(kFullMask, l[0], off);
+                l[1] += __shfl_xor_sync(kFullMask, l[1], off);
+            }
+            const int first_run = ch.of(stream_begin);   // chunks holding pieces of this stream
+            const int last_run = ch.of(stream_end - 1);
+            const int stream = s * NHG + hg;
+            // element (head column c, row d) of this lane's accumulators
+            auto d_of = [&](int dt, int half) -> int {
+                return (F16 || F8) ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
+            };
+            // a whole stream writes `out`; pieces of split streams, every stream of a prefix pass and
+            // the suffix of a sequence with shared blocks leave (o, m, l) for the merge
+            if (first_run == last_run && !PFX && skipb == 0) {
+                QT* out0 = reinterpret_cast<QT*>(p.out) + row0 * D;
+                QT* out1 = reinterpret_cast<QT*>(p.out) + row1 * D;
+                const float inv0 = l[0] > 0.f ? out_scale / l[0] : 0.f;
+                const float inv1 = l[1] > 0.f ? out_scale / l[1] : 0.f;
+#pragma unroll
+                for (int dt = 0; dt < C::kDT; ++dt)
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int d = d_of(dt, half);
+                        if (2 * t < G)
+                            from_float(o[dt][2 * half] * inv0, out0 + d);
+                        if (2 * t + 1 < G)
+                            from_float(o[dt][2 * half + 1] * inv1, out1 + d);
+                    }
+            } else {
+                float* part = p.partials + ((size_t)(cur + stream) * W + warp) * p.slot_floats;
+#pragma unroll
+                for (int dt = 0; dt < C::kDT; ++dt)
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int d = d_of(dt, half);
+                        if (2 * t < G)
+                            part[(2 * t) * D + d] = o[dt][2 * half];
+                        if (2 * t + 1 < G)
+                            part[(2 * t + 1) * D + d] = o[dt][2 * half + 1];
+                    }
+                if (g == 0) {
+                    if (2 * t < G) {
+                        part[G * D + 2 * t] = m[0];
+                        part[G * D + G + 2 * t] = l[0];
+                    }
+                    if (2 * t + 1 < G) {
+                        part[G * D + 2 * t + 1] = m[1];
+                        part[G * D + G + 2 * t + 1] = l[1];
+                    }
                 }
             }
         }
@@ -1071,10 +1158,12 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     const int NHG = p.num_kv_heads / HG;
     (void)build_unit_prefix(p, prefix, BS, NHG, p.max_blocks_per_seq * BS);
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x == 0)   // the decode grid is done claiming: ready for the next call
+        *p.chunk_ctr = 0;
     const int total = prefix[p.num_seqs];
     if (total == 0)
         return;
-    const int per_run = (total + decode_runs - 1) / decode_runs;
+    const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kMergeThreads / 32);
     const int items = p.num_seqs * NHG * HG;
@@ -1085,7 +1174,7 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
         if (nb == 0)
             continue;
         const int sb = prefix[s] + hg * nb;
-        const int first_run = sb / per_run, last_run = (sb + nb - 1) / per_run;
+        const int first_run = ch.of(sb), last_run = ch.of(sb + nb - 1);
         if (first_run != last_run)
             merge_split<QT, D, G, HG>(p, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
     }
@@ -1113,8 +1202,12 @@ __global__ void __launch_bounds__(kMergeThreads)
     (void)build_unit_prefix(pp, prefix_p, BS, Hkv, capacity);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int total_s = prefix_s[ps.num_seqs], total_p = prefix_p[pp.num_seqs];
-    const int per_run_s = total_s > 0 ? (total_s + runs_s - 1) / runs_s : 1;
-    const int per_run_p = total_p > 0 ? (total_p + runs_p - 1) / runs_p : 1;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {   // both passes are done claiming
+        *ps.chunk_ctr = 0;
+        *pp.chunk_ctr = 0;
+    }
+    const Chunks ch_s = make_chunks(total_s, runs_s, ps.tail_chunks);
+    const Chunks ch_p = make_chunks(total_p, runs_p, pp.tail_chunks);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kMergeThreads / 32);
     const int wid = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
@@ -1164,7 +1257,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         if (nb_p > 0) {
             const int pstream = gi * Hkv + h, sb = prefix_p[gi] + h * nb_p;
             const int cg = mi * Gq + gq, tile = cg >> 3, c = cg & 7;
-            for (int r = sb / per_run_p; r <= (sb + nb_p - 1) / per_run_p; ++r) {
+            for (int r = ch_p.of(sb); r <= ch_p.of(sb + nb_p - 1); ++r) {
                 const float* base = pp.partials + ((size_t)(r + pstream) * 4 + tile) * pp.slot_floats;
                 add(base + c * D, __ldcg(base + 8 * D + c), __ldcg(base + 8 * D + 8 + c));
             }
@@ -1173,7 +1266,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         const int nb_s = (prefix_s[seq + 1] - prefix_s[seq]) / NHG;
         if (nb_s > 0) {
             const int hg = h / HG, w = h - hg * HG, stream = seq * NHG + hg, sb = prefix_s[seq] + hg * nb_s;
-            for (int r = sb / per_run_s; r <= (sb + nb_s - 1) / per_run_s; ++r) {
+            for (int r = ch_s.of(sb); r <= ch_s.of(sb + nb_s - 1); ++r) {
                 const float* base = ps.partials + ((size_t)(r + stream) * HG + w) * ps.slot_floats;
                 add(base + gq * D, __ldcg(base + G * D + gq), __ldcg(base + G * D + G + gq));
             }
@@ -1202,7 +1295,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         if (skipb > 0)
             continue;
         const int sb = prefix_s[s] + hg * nb;
-        const int first_run = sb / per_run_s, last_run = (sb + nb - 1) / per_run_s;
+        const int first_run = ch_s.of(sb), last_run = ch_s.of(sb + nb - 1);
         if (first_run != last_run)
             merge_split<QT, D, G, HG>(ps, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
     }
@@ -1221,19 +1314,20 @@ struct MmaLauncher {
 
     static size_t smem_bytes(int num_seqs, int S)
     {
-        return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + (size_t)(num_seqs + 1) * 4 + 64;
+        return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + kChunkRing * 4 + (size_t)(num_seqs + 1) * 4 + 64;
     }
 
     // Ring depth: the SM's shared memory split between kCtasPerSM CTAs (~96 KB or ~64 KB of stages).
     static int stages(int num_seqs)
     {
         const long long budget = kMaxSmemPerBlock / C::kCtasPerSM - 1024;
-        const long long room = budget - 16 - (long long)(num_seqs + 1) * 4 - 64;
+        const long long room = budget - 16 - kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64;
         long long S = room / (C::kStage + 20);
         if (S > 8)
             S = 8;
         if (S < 2) {   // many sequences: fall back to one CTA per SM
-            S = ((long long)kMaxSmemPerBlock - 1024 - 16 - (long long)(num_seqs + 1) * 4 - 64) / (C::kStage + 20);
+            S = ((long long)kMaxSmemPerBlock - 1024 - 16 - kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64) /
+                (C::kStage + 20);
             if (S > 8)
                 S = 8;
         }

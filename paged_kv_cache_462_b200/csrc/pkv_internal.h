@@ -15,6 +15,11 @@ constexpr int kMaxSeqs = 16384;         // per call: the per-sequence tile prefi
 constexpr int kMaxRunsPerSM = 3;        // automatic partition count is at most 3 runs per SM
 constexpr size_t kWorkspaceHeader = 256;
 constexpr int kMaxHeadGroup = 4;        // KV heads per MMA work unit (partial slots reserved per run)
+// Tensor-core kernels: a CTA's first chunk is its share of three quarters of the work; the last
+// quarter is cut into up to kTailChunksPerRun chunks per CTA, claimed as CTAs run dry. The
+// workspace keeps partial slots for (1 + kTailChunksPerRun) chunks per run.
+constexpr int kTailChunksPerRun = 4;
+constexpr int kMinTailChunk = 8;        // units
 constexpr float kLog2e = 1.4426950408889634074f;
 
 struct DecodeParams {
@@ -73,6 +78,10 @@ struct DecodeParams {
     // 1: execute griddepcontrol.wait before the grid exits (a suffix pass launched behind the
     // prefix pass, so that the merge's wait covers both)
     int wait_prior_at_exit;
+    // Tensor-core kernels: tail chunks per run (0: one static run per CTA) and the workspace
+    // counter they are claimed from (zero before the launch; the merge kernel clears it after)
+    int tail_chunks;
+    int32_t* chunk_ctr;
 };
 
 // One request to the warp-MMA kernels of a shape (decode_mma_dispatch.cuh).
