@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--prefix-sharing", choices=["auto", "on", "off"], default="auto",
                     help="shared-prefix decode (blocks a plan shares read once per group): auto = on for "
                          "workloads whose sequences share prefix blocks (config 3)")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="cut the workload down to its first N sequences' draw (same distributions; for profiling "
+                         "captures that must stay small)")
     ap.add_argument("--no-targets", action="store_true",
                     help="skip the extra target points (long-context and mixed batch, bf16 and E4M3 caches)")
     return ap.parse_args()
@@ -77,6 +80,9 @@ def workload_spec(args) -> W.Spec:
     """The config's workload, with the cache dtype replaced when --kv-dtype asks for it (q and the
     appended rows stay bf16; an E4M3 cache gets per-tensor absmax/448 scales)."""
     spec = W.config_spec(args.config)
+    if args.num_seqs is not None:
+        spec.num_seqs = args.num_seqs
+        spec.name = f"{spec.name}_{args.num_seqs}seqs"
     if args.kv_dtype is not None:
         if spec.q_dtype != "bf16":
             raise SystemExit("--kv-dtype applies to the bf16-query workloads (configs 1-4)")
@@ -573,7 +579,8 @@ def ours_arm(args):
 
     # the other points of the throughput target, timed the same way (same K and W), one at a time
     targets = []
-    if not args.no_targets and args.q_len == 1 and args.kv_dtype is None and args.partitions == 0:
+    if (not args.no_targets and args.q_len == 1 and args.kv_dtype is None and args.partitions == 0
+            and args.num_seqs is None):
         main_kv = spec.kv_dtype
         del state
         torch.cuda.empty_cache()

@@ -753,7 +753,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                 if (ok && skip[st] == 0 && valid > 0) {
                     const uint32_t kbase = smem_addr(stages + (size_t)st * C::kStage);
                     const uint32_t vbase = kbase + C::kHalf;
-                    const int r0 = warp * BS;            // this head's first box row
+                    const int r0 = (warp / C::kNT) * BS;   // this warp's KV head's first box row
 #pragma unroll
                     for (int tt = 0; tt < C::kTT; ++tt) {
                         // ---- S^T = K Q^T : 16 tokens x 8 heads
