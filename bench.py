@@ -122,22 +122,26 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_traffic(config: int):
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches this kernel build."""
+def kernel_traffic(config: int, kv: str, prefix: bool):
+    """DRAM bytes (read + written) per step of the decode kernels, from the committed ncu summary
+    of this workload, if it was captured on this kernel build (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)
+            recs = json.load(f)["records"]
     except Exception:
         return None
-    if rec.get("kernel_sha") != kernel_sha() or int(rec.get("config", -1)) != config:
-        return None
-    return rec.get("dram_bytes_per_launch")
+    for rec in recs:
+        if (rec.get("kernel_sha") == kernel_sha() and int(rec.get("config", -1)) == config
+                and rec.get("kv") == kv and bool(rec.get("prefix_sharing")) == prefix
+                and rec.get("num_seqs") is None):
+            return rec.get("dram_bytes_per_step")
+    return None
 
 
 def kernel_sha() -> str:
     h = hashlib.sha256()
-    for name in ("decode_mma.cuh", "decode_kernel.cuh", "device.cuh"):
+    for name in ("decode_mma.cuh", "decode_kernel.cuh", "device.cuh", "decode_mma_dispatch.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_462_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -608,6 +612,7 @@ def ours_arm(args):
                             "kv_logical_gbs": tdec["kv_logical"] / (sum(tms) / K * 1e-3) / 1e9,
                             "seq_steps_per_s": world * tb.spec.num_seqs / (agg_t["ms"] * 1e-3),
                             "device_errors": int(agg_t["errors"]),
+                            "traffic": kernel_traffic(cfg, kv, tplan is not None),
                             "clocks": clocks.summary(t0, t1) if clocks else None})
             del ts
             torch.cuda.empty_cache()
@@ -672,7 +677,7 @@ def ours_arm(args):
                 "peak_kind": peak_kind,
                 "unit": "GB/s",
                 "frac": kern_gbs / peak,
-                "traffic": kernel_traffic(args.config),
+                "traffic": kernel_traffic(args.config, spec.kv_dtype, plan is not None) if args.q_len == 1 else None,
                 "algorithmic_bytes": kern_bytes,
             },
             # fused: the decode kernel (append inside) + the merge kernel; else append + decode

@@ -106,6 +106,30 @@ __device__ __forceinline__ void mma_16832_f8(float (&c)[4], const uint32_t (&a)[
     }
 }
 
+// D += A B with A 16x32 and B 32x8 of signed 8-bit integers, exact int32 sums
+__device__ __forceinline__ void mma_16832_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four values as signed 8-bit hi and lo codes of x = rint(v): hi = floor((x + 64) / 128), lo = x - 128 hi
+// (hi + lo / 128 = x / 128 exactly; |x| < 8192 keeps hi in [-64, 64], lo in [-64, 63]). Byte i = value i.
+__device__ __forceinline__ void split_s8x4(const float (&v)[4], uint32_t& hi, uint32_t& lo)
+{
+    hi = lo = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int x = __float2int_rn(v[i]);
+        const int h = (x + 64) >> 7;
+        hi |= (uint32_t)(h & 0xff) << (8 * i);
+        lo |= (uint32_t)((x - (h << 7)) & 0xff) << (8 * i);
+    }
+}
+
 // Two values (f16x2, low half first) as E4M3 hi and lo codes with hi + lo ~ x: hi = E4M3(x) and
 // lo = E4M3(x - hi), the difference exact in f16 (hi is x rounded to 4 significant bits). Each
 // result holds its two codes in bits 0-15, low half's code first. |x| must stay below 448.
@@ -256,8 +280,10 @@ __device__ __forceinline__ size_t query_row(const DecodeParams& p, int s, int he
 template <class KV, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaCfg {
     // products: bf16 caches in bf16 MMA; E4M3 / E5M2 codes straight into FP8 MMA (q and p as E4M3
-    // hi + lo pairs); INT8 codes widened exactly to f16 for f16 MMA
+    // hi + lo pairs); INT8: q.K on integer MMA (K codes as they are, q as s8 hi + lo), V codes
+    // widened exactly to f16 for f16 MMA
     static constexpr bool kF8 = KV::kBytes == 1 && !KV::kInt8;
+    static constexpr bool kI8 = KV::kInt8;
     static constexpr bool kF16 = KV::kInt8;
     static constexpr int kRowBytes = D * KV::kBytes;          // one token row of one head
     static constexpr int kBoxCols = 128 / KV::kBytes;         // elements per 128-byte box row
@@ -278,7 +304,7 @@ struct MmaCfg {
     static_assert(kRowBytes % 128 == 0, "rows are whole 128-byte swizzle spans");
     static_assert(BS % 16 == 0 && G <= 8 && HG <= 8, "tile shape");
     static_assert(kRows <= 256, "TMA box height");
-    static_assert(!kF8 || D == 128, "FP8 MMA tiles: one 128-byte box across head_dim");
+    static_assert(KV::kBytes == 2 || D == 128, "8-bit MMA tiles: one 128-byte box across head_dim");
     static_assert(!PFX || (HG == 1 && G == 8), "prefix pass: one KV head per unit, 8 columns per warp");
 };
 
@@ -391,6 +417,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
     constexpr int W = C::W;
     constexpr bool F16 = C::kF16;
     constexpr bool F8 = C::kF8;
+    constexpr bool I8 = C::kI8;
     // lazy running max: moved when a tile max passes it by kSlack (log2 units). FP8 products take
     // p * 2^kPOff <= 2^(kSlack + kPOff) = 256 (E4M3 holds up to 448), which keeps small weights in
     // E4M3's normal range; the factor cancels between o and l.
@@ -668,10 +695,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
             // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
             uint32_t qb[C::kKS][2];
             float qk0 = qk_scale, qk1 = qk_scale;   // score factors of this lane's columns 2t, 2t+1
-            if constexpr (F8) {
-                // FP8 products: column g of Q^T times a power of two sigma_g (max |q| * sigma_g < 256),
-                // as E4M3 hi + lo codes (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3,
-                // b1 = d 32kk + 16 + 4t .. +3. 1 / sigma goes into the column's score factor.
+            if constexpr (F8 || I8) {
+                // 8-bit products: column g of Q^T times a power of two sigma_g, as hi + lo codes
+                // (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3, b1 = d 32kk + 16 + 4t .. +3.
+                // FP8: max |q| * sigma_g < 256, E4M3 hi and lo; INT8: max |q| * sigma_g < 2^13,
+                // rounded to an integer x = 128 hi + lo. 1 / sigma goes into the column's score factor.
                 constexpr int K8 = D / 32;
                 const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
                 float f[K8][2][4];
@@ -690,10 +718,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                     }
                 mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
-                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
+                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E) (FP8) or
+                // 2^(139 - E) (INT8), kept normal both ways
                 int se = 127;
                 if (mx > 0.f) {
-                    se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
+                    se = 127 + (I8 ? 139 : 134) - (int)((__float_as_uint(mx) >> 23) & 0xffu);
                     se = se < 2 ? 2 : (se > 252 ? 252 : se);
                 }
                 const float sig = __uint_as_float((uint32_t)se << 23);
@@ -702,11 +731,17 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                 for (int kk = 0; kk < K8; ++kk)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t h01, l01, h23, l23;
-                        split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
-                        split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
-                        qb[kk][hh] = h01 | (h23 << 16);
-                        qb[K8 + kk][hh] = l01 | (l23 << 16);
+                        if constexpr (I8) {
+                            const float v[4] = {f[kk][hh][0] * sig, f[kk][hh][1] * sig, f[kk][hh][2] * sig,
+                                                f[kk][hh][3] * sig};
+                            split_s8x4(v, qb[kk][hh], qb[K8 + kk][hh]);
+                        } else {
+                            uint32_t h01, l01, h23, l23;
+                            split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
+                            split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
+                            qb[kk][hh] = h01 | (h23 << 16);
+                            qb[K8 + kk][hh] = l01 | (l23 << 16);
+                        }
                     }
                 qk0 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t) * 4);
                 qk1 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t + 1) * 4);
@@ -715,16 +750,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 #pragma unroll
                 for (int ks = 0; ks < C::kKS; ++ks) {
                     if (qcol) {
-                        if constexpr (F16) {
-                            // k order permuted to match the widened INT8 A fragments: (4t, 4t+1 | 4t+2, 4t+3)
-                            float f[4];
-                            load_q<4>(qp + ks * 16 + 4 * t, f);
-                            qb[ks][0] = pack2<true>(f[0], f[1]);
-                            qb[ks][1] = pack2<true>(f[2], f[3]);
-                        } else {
-                            qb[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t));
-                            qb[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t + 8));
-                        }
+                        qb[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t));
+                        qb[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t + 8));
                     } else {
                         qb[ks][0] = qb[ks][1] = 0u;
                     }
@@ -771,21 +798,21 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                                 mma_16832_f8<KV::kFmt>(sc, a, qb[kk][0], qb[kk][1]);                 // q hi
                                 mma_16832_f8<KV::kFmt>(sd, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);   // q lo
                             }
-                        } else if constexpr (F16) {
+                        } else if constexpr (I8) {
+                            // the same A fragments of INT8 codes against q's s8 hi and lo: exact
+                            // int32 sums, combined as 128 hi + lo
+                            int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
 #pragma unroll
-                            for (int ks = 0; ks < C::kKS; ks += 2) {
-                                // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each
+                            for (int kk = 0; kk < D / 32; ++kk) {
                                 const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                                uint32_t r[4];
-                                ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
-#pragma unroll
-                                for (int h2 = 0; h2 < 2; ++h2) {
-                                    const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
-                                    const uint32_t a[4] = {fp8x2_to_f16x2<KV>(lo), fp8x2_to_f16x2<KV>(hi),
-                                                           fp8x2_to_f16x2<KV>(lo >> 16), fp8x2_to_f16x2<KV>(hi >> 16)};
-                                    mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
-                                }
+                                uint32_t a[4];
+                                ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
+                                mma_16832_s8(ih, a, qb[kk][0], qb[kk][1]);
+                                mma_16832_s8(il, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);
                             }
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                sc[i] = (float)(ih[i] * 128 + il[i]);
                         } else {
 #pragma unroll
                             for (int ks = 0; ks < C::kKS; ++ks) {
