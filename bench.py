@@ -476,6 +476,25 @@ def reference_arm(args):
     return 0
 
 
+def pack_step_inputs(torch, tensors: dict, dev):
+    """One device buffer and one pinned host buffer holding copies of `tensors` at the same
+    256-byte-aligned offsets: ({name: device view, "_buffer": device buffer}, {..host..})."""
+    offs, total = {}, 0
+    for n, t in tensors.items():
+        offs[n] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+    hbuf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    dv, hv = {"_buffer": dbuf}, {"_buffer": hbuf}
+    for n, t in tensors.items():
+        nb = t.numel() * t.element_size()
+        dv[n] = dbuf[offs[n]:offs[n] + nb].view(t.dtype).view(t.shape)
+        hv[n] = hbuf[offs[n]:offs[n] + nb].view(t.dtype).view(t.shape)
+        dv[n].copy_(t)
+        hv[n].copy_(t.cpu())
+    return dv, hv
+
+
 def use_prefix_plan(args, spec) -> bool:
     """The shared-prefix decode for workloads whose sequences share prefix blocks (or when asked)."""
     if args.q_len != 1 or args.prefix_sharing == "off" or spec.kv_dtype == "f32":
@@ -529,6 +548,7 @@ def ours_arm(args):
     state = DeviceState(torch, pkv, b, dev, args.partitions)
     state.set_q_len(args.q_len)
     plan = state.use_prefix_plan(spec.share_group) if use_prefix_plan(args, spec) else None
+    plan_host_ms = state.plan_host_ms if plan is not None else None
     dec, app = step_bytes(b, args.q_len, plan)
     bytes_step = dec["total"] + app
     # a read (not a write) of a buffer twice the size of L2: the L2 ends up holding clean lines of
@@ -555,14 +575,18 @@ def ours_arm(args):
     e2e = None
     if not args.no_e2e:
         names = ("q_mq", "sl", "bt") if args.q_len > 1 else ("q", "new_k", "new_v", "new_slots", "sl", "bt")
-        dev_in = {n: getattr(state, n) for n in names}
+        owners = {n: state for n in names}
         if state.plan is not None:   # the plan's arrays travel with the tables they come from
-            dev_in.update({f"plan_{n}": getattr(state.plan, n) for n in ("members", "offsets", "tables", "lens",
-                                                                          "shared")})
-        host = {n: t.detach().cpu().pin_memory() for n, t in dev_in.items()}
+            owners.update({n: state.plan for n in ("members", "offsets", "tables", "lens", "shared")})
+        # the step's inputs live in one device buffer with a pinned host mirror of the same layout,
+        # so each step's upload is a single copy
+        dev_in, host_in = pack_step_inputs(torch, {n: getattr(o, n) for n, o in owners.items()}, dev)
+        for n, o in owners.items():
+            setattr(o, n, dev_in[n])
+        dev_buf, host_buf = dev_in["_buffer"], host_in["_buffer"]
         dev_out = state.out_mq if args.q_len > 1 else state.out
         out_h = torch.empty(dev_out.shape, dtype=dev_out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        h2d = host_buf.numel()
         d2h = out_h.numel() * out_h.element_size()
         Ke = K
         ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
@@ -571,8 +595,7 @@ def ours_arm(args):
             rec = i >= args.warmup
             if rec:
                 ee[i - args.warmup][0].record(stream)
-            for n, t in host.items():
-                dev_in[n].copy_(t, non_blocking=True)
+            dev_buf.copy_(host_buf, non_blocking=True)
             state.step()
             out_h.copy_(dev_out, non_blocking=True)
             if rec:
@@ -653,7 +676,7 @@ def ours_arm(args):
                 "step": (f"paged_attention_decode_mq: the last {args.q_len} tokens of every sequence as queries, "
                          "causal within the chunk (their K/V already cached)" if args.q_len > 1 else
                          f"paged_decode_step_shared_prefix: prefix pass over the {plan.num_groups} groups' shared "
-                         f"blocks (plan made once on the host in {state.plan_host_ms:.2f} ms, outside the timed "
+                         f"blocks (plan made once on the host in {plan_host_ms:.2f} ms, outside the timed "
                          "region), suffix pass with the append fused, merge" if plan is not None else
                          "paged_decode_step: append of one new token per sequence fused into the paged "
                          "decode launch" if fused else
