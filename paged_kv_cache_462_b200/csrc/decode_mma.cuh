@@ -51,6 +51,8 @@
 namespace pkv {
 
 constexpr float kMmaRescaleSlack = 8.0f;  // log2 units
+// INT8 caches: q.K on the integer tensor cores (true) or on f16 after widening the K codes (false)
+constexpr bool kInt8Imma = true;
 constexpr int kChunkRing = 16;             // chunk ids in flight between producer and consumers (> stages)
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -87,25 +89,6 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
     }
 }
 
-// D += A B with A 16x32 and B 32x8 of 8-bit floats (A: the cache's format, B: E4M3), fp32 sums
-template <__nv_fp8_interpretation_t AFMT>
-__device__ __forceinline__ void mma_16832_f8(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    if constexpr (AFMT == __NV_E5M2) {
-        asm volatile(
-            "mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-            "{%0, %1, %2, %3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    } else {
-        asm volatile(
-            "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-            "{%0, %1, %2, %3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-    }
-}
-
 // D += A B with A 16x32 and B 32x8 of signed 8-bit integers, exact int32 sums
 __device__ __forceinline__ void mma_16832_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
@@ -130,39 +113,37 @@ __device__ __forceinline__ void split_s8x4(const float (&v)[4], uint32_t& hi, ui
     }
 }
 
-// Two values (f16x2, low half first) as E4M3 hi and lo codes with hi + lo ~ x: hi = E4M3(x) and
-// lo = E4M3(x - hi), the difference exact in f16 (hi is x rounded to 4 significant bits). Each
-// result holds its two codes in bits 0-15, low half's code first. |x| must stay below 448.
-__device__ __forceinline__ void split_e4m3x2(uint32_t x, uint32_t& hi, uint32_t& lo)
+// Bytes B0 and B1 of r (two 8-bit codes) as an f16x2 (byte B0 in the low half), exact:
+//  * E5M2 codes are the high bytes of the f16 of the same value: one byte permute.
+//  * E4M3 s.eeee.mmm placed as f16 bits s.0eeee.mmm0000000 is the code's value times 2^-8, normal
+//    and subnormal alike (the f16 exponent bias is 8 more than E4M3's, and E4M3's subnormal step
+//    2^-9 lands on f16's subnormal step 2^-24 shifted by 7): a permute, a shift and two logic
+//    operations; the launcher puts the 2^8 back into the score and output factors.
+//  * INT8: the offset byte x + 128 as the mantissa of 1024.0 gives the f16 1152 + x; less 1152.
+template <class KV, int B0, int B1>
+__device__ __forceinline__ uint32_t widen2(uint32_t r)
 {
-    uint16_t h, l;
-    uint32_t hv;
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h) : "r"(x));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hv) : "h"(h));
-    const __half2 d = __hsub2(*reinterpret_cast<const __half2*>(&x), *reinterpret_cast<const __half2*>(&hv));
-    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l) : "r"(*reinterpret_cast<const uint32_t*>(&d)));
-    hi = h;
-    lo = l;
-}
-
-// two 8-bit codes (low byte first) -> f16x2, exact for E4M3, E5M2 and INT8
-template <class KV>
-__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t two_codes)
-{
-    uint32_t r;
     if constexpr (KV::kInt8) {
-        // the offset byte x + 128 as the mantissa of 1024.0: f16 value 1152 + x, less 1152 (exact)
-        r = __byte_perm(two_codes ^ 0x8080u, 0x64646464u, 0x4140);
-        const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&r), __halves2half2(__ushort_as_half(0x6480),
+        const uint32_t x = __byte_perm(r ^ 0x80808080u, 0x64646464u, B0 | (4 << 4) | (B1 << 8) | (4 << 12));
+        const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&x), __halves2half2(__ushort_as_half(0x6480),
                                                                                       __ushort_as_half(0x6480)));
         return *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+        const uint32_t x = __byte_perm(r, 0u, 4 | (B0 << 4) | (4 << 8) | (B1 << 12));   // [0, c0, 0, c1]
+        if constexpr (KV::kFmt == __NV_E5M2)
+            return x;
+        else
+            return ((x >> 1) & 0x3F803F80u) | (x & 0x80008000u);
     }
-    const uint16_t v = static_cast<uint16_t>(two_codes);
-    if constexpr (KV::kFmt == __NV_E5M2)
-        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(r) : "h"(v));
-    else
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-    return r;
+}
+
+// factor between an 8-bit code's widened f16 and its format value (see widen2)
+template <class KV>
+constexpr float widen_factor()
+{
+    if constexpr (KV::kBytes == 1 && !KV::kInt8)
+        return KV::kFmt == __NV_E4M3 ? 256.0f : 1.0f;
+    return 1.0f;
 }
 
 template <bool F16>
@@ -279,12 +260,11 @@ __device__ __forceinline__ size_t query_row(const DecodeParams& p, int s, int he
 // their query heads), 8 each, against the same staged K/V tile.
 template <class KV, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaCfg {
-    // products: bf16 caches in bf16 MMA; E4M3 / E5M2 codes straight into FP8 MMA (q and p as E4M3
-    // hi + lo pairs); INT8: q.K on integer MMA (K codes as they are, q as s8 hi + lo), V codes
-    // widened exactly to f16 for f16 MMA
-    static constexpr bool kF8 = KV::kBytes == 1 && !KV::kInt8;
-    static constexpr bool kI8 = KV::kInt8;
-    static constexpr bool kF16 = KV::kInt8;
+    // products: bf16 caches in bf16 MMA; 8-bit codes widened exactly to f16 (widen2) for f16 MMA,
+    // q scaled per column by a power of two into f16's range; INT8 q.K on integer MMA (K codes as
+    // they are, q as s8 hi + lo) when kInt8Imma
+    static constexpr bool kF16 = KV::kBytes == 1;
+    static constexpr bool kI8 = KV::kInt8 && kInt8Imma;
     static constexpr int kRowBytes = D * KV::kBytes;          // one token row of one head
     static constexpr int kBoxCols = 128 / KV::kBytes;         // elements per 128-byte box row
     static constexpr int kBoxes = kRowBytes / 128;            // boxes across head_dim
@@ -416,13 +396,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
     using C = MmaCfg<KV, D, BS, G, HG, PFX>;
     constexpr int W = C::W;
     constexpr bool F16 = C::kF16;
-    constexpr bool F8 = C::kF8;
     constexpr bool I8 = C::kI8;
-    // lazy running max: moved when a tile max passes it by kSlack (log2 units). FP8 products take
-    // p * 2^kPOff <= 2^(kSlack + kPOff) = 256 (E4M3 holds up to 448), which keeps small weights in
-    // E4M3's normal range; the factor cancels between o and l.
-    constexpr float kSlack = F8 ? 2.0f : kMmaRescaleSlack;
-    constexpr float kPOff = F8 ? 6.0f : 0.0f;
+    // lazy running max: moved only when a tile max passes it by kSlack (log2 units), so p <= 2^8
+    constexpr float kSlack = kMmaRescaleSlack;
     const int S = p.stages_per_warp;   // ring depth (stages of the CTA)
     const int Hkv = p.num_kv_heads;
     const int NHG = Hkv / HG;          // head groups per sequence
@@ -695,11 +671,13 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
             // Q^T as the B operand: b0 = (k: d pair, n: query column g); columns g >= G are zero.
             uint32_t qb[C::kKS][2];
             float qk0 = qk_scale, qk1 = qk_scale;   // score factors of this lane's columns 2t, 2t+1
-            if constexpr (F8 || I8) {
-                // 8-bit products: column g of Q^T times a power of two sigma_g, as hi + lo codes
-                // (qb[kk] hi, qb[D/32 + kk] lo); b0 = d 32kk + 4t .. +3, b1 = d 32kk + 16 + 4t .. +3.
-                // FP8: max |q| * sigma_g < 256, E4M3 hi and lo; INT8: max |q| * sigma_g < 2^13,
-                // rounded to an integer x = 128 hi + lo. 1 / sigma goes into the column's score factor.
+            if constexpr (F16) {
+                // 8-bit caches: column g of Q^T times a power of two sigma_g, 1 / sigma_g going into
+                // the column's score factor. f16 MMA: max |q| * sigma_g < 2^14 (exact for a bf16 q at
+                // any magnitude), k order permuted to match the widened A fragments:
+                // qb[ks] = (d 16ks + 4t, +1 | +2, +3). Integer MMA (INT8): max |q| * sigma_g < 2^13,
+                // rounded to x = 128 hi + lo, qb[kk] hi and qb[D/32 + kk] lo as s8, b0 = d 32kk + 4t
+                // .. +3, b1 = d 32kk + 16 + 4t .. +3.
                 constexpr int K8 = D / 32;
                 const QT* qp = reinterpret_cast<const QT*>(p.q) + row_g * D;
                 float f[K8][2][4];
@@ -718,11 +696,11 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                     }
                 mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, 2));
-                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E) (FP8) or
-                // 2^(139 - E) (INT8), kept normal both ways
+                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(140 - E) (f16) or
+                // 2^(139 - E) (s8), kept normal both ways
                 int se = 127;
                 if (mx > 0.f) {
-                    se = 127 + (I8 ? 139 : 134) - (int)((__float_as_uint(mx) >> 23) & 0xffu);
+                    se = 127 + (I8 ? 139 : 140) - (int)((__float_as_uint(mx) >> 23) & 0xffu);
                     se = se < 2 ? 2 : (se > 252 ? 252 : se);
                 }
                 const float sig = __uint_as_float((uint32_t)se << 23);
@@ -736,11 +714,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                                                 f[kk][hh][3] * sig};
                             split_s8x4(v, qb[kk][hh], qb[K8 + kk][hh]);
                         } else {
-                            uint32_t h01, l01, h23, l23;
-                            split_e4m3x2(pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig), h01, l01);
-                            split_e4m3x2(pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig), h23, l23);
-                            qb[kk][hh] = h01 | (h23 << 16);
-                            qb[K8 + kk][hh] = l01 | (l23 << 16);
+                            qb[2 * kk + hh][0] = pack2<true>(f[kk][hh][0] * sig, f[kk][hh][1] * sig);
+                            qb[2 * kk + hh][1] = pack2<true>(f[kk][hh][2] * sig, f[kk][hh][3] * sig);
                         }
                     }
                 qk0 = qk_scale * __shfl_sync(kFullMask, inv_sig, (2 * t) * 4);
@@ -787,20 +762,10 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         float sc[4] = {0.f, 0.f, 0.f, 0.f};
                         float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
                         const int mi = lane >> 3, rr = lane & 7;
-                        if constexpr (F8) {
-#pragma unroll
-                            for (int kk = 0; kk < D / 32; ++kk) {
-                                // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment
-                                // of 16 tokens x d 32kk .. 32kk+31 as it lies in the stage, no conversion
-                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
-                                uint32_t a[4];
-                                ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
-                                mma_16832_f8<KV::kFmt>(sc, a, qb[kk][0], qb[kk][1]);                 // q hi
-                                mma_16832_f8<KV::kFmt>(sd, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);   // q lo
-                            }
-                        } else if constexpr (I8) {
-                            // the same A fragments of INT8 codes against q's s8 hi and lo: exact
-                            // int32 sums, combined as 128 hi + lo
+                        if constexpr (I8) {
+                            // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment of
+                            // 16 tokens x d 32kk .. 32kk+31 of INT8 codes as it lies in the stage, against
+                            // q's s8 hi and lo: exact int32 sums, combined as 128 hi + lo
                             int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
 #pragma unroll
                             for (int kk = 0; kk < D / 32; ++kk) {
@@ -813,6 +778,22 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 #pragma unroll
                             for (int i = 0; i < 4; ++i)
                                 sc[i] = (float)(ih[i] * 128 + il[i]);
+                        } else if constexpr (F16) {
+#pragma unroll
+                            for (int ks = 0; ks < C::kKS; ks += 2) {
+                                // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each;
+                                // each lane's 4 codes of a row widen to the A pairs (d 4t, 4t+1 | 4t+2, 4t+3)
+                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                uint32_t r[4];
+                                ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2) {
+                                    const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
+                                    const uint32_t a[4] = {widen2<KV, 0, 1>(lo), widen2<KV, 0, 1>(hi),
+                                                           widen2<KV, 2, 3>(lo), widen2<KV, 2, 3>(hi)};
+                                    mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
+                                }
+                            }
                         } else {
 #pragma unroll
                             for (int ks = 0; ks < C::kKS; ++ks) {
@@ -829,8 +810,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             sc[i] += sd[i];
                         // V fragments of this tile into registers; after the block's last tile the
                         // stage goes back to the producer before the softmax and p.V arithmetic
-                        uint32_t vf[C::kDT * 4 / ((F16 || F8) ? 2 : 1)];
-                        if constexpr (F16 || F8) {
+                        uint32_t vf[C::kDT * 4 / (F16 ? 2 : 1)];
+                        if constexpr (F16) {
 #pragma unroll
                             for (int dt = 0; dt < C::kDT; dt += 2) {
                                 // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
@@ -892,27 +873,15 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             }
                         }
                         float pr[4];
-                        const float mo0 = m[0] - kPOff, mo1 = m[1] - kPOff;
-                        pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - mo0);
-                        pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - mo1);
-                        pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - mo0);
-                        pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - mo1);
+                        pr[0] = (sc[0] == -INFINITY) ? 0.f : fast_exp2(sc[0] - m[0]);
+                        pr[1] = (sc[1] == -INFINITY) ? 0.f : fast_exp2(sc[1] - m[1]);
+                        pr[2] = (sc[2] == -INFINITY) ? 0.f : fast_exp2(sc[2] - m[0]);
+                        pr[3] = (sc[3] == -INFINITY) ? 0.f : fast_exp2(sc[3] - m[1]);
                         l[0] += pr[0] + pr[2];
                         l[1] += pr[1] + pr[3];
                         const int srcA = (2 * t) * 4 + (g >> 1), srcB = (2 * t + 1) * 4 + (g >> 1);
                         uint32_t pb0, pb1;
-                        if constexpr (F8) {
-                            // ---- P^T as E4M3 hi (b0) and lo (b1) codes, k = tokens 2t, 2t+1, 2t+8, 2t+9 of column g
-                            uint32_t h0, l0, h1, l1;
-                            split_e4m3x2(pack2<true>(pr[0], pr[2]), h0, l0);   // column 2t:   tokens g, g+8
-                            split_e4m3x2(pack2<true>(pr[1], pr[3]), h1, l1);   // column 2t+1: tokens g, g+8
-                            const uint32_t wh = h0 | (h1 << 16), wl = l0 | (l1 << 16);
-                            const uint32_t ah = __shfl_sync(kFullMask, wh, srcA), bh = __shfl_sync(kFullMask, wh, srcB);
-                            const uint32_t al = __shfl_sync(kFullMask, wl, srcA), bl = __shfl_sync(kFullMask, wl, srcB);
-                            const uint32_t sel = (g & 1) ? 0x7362u : 0x5140u;
-                            pb0 = qcol ? __byte_perm(ah, bh, sel) : 0u;
-                            pb1 = qcol ? __byte_perm(al, bl, sel) : 0u;
-                        } else {
+                        {
                             // ---- P^T as the B operand: b0 = (tokens 2t, 2t+1; head g), b1 = (tokens 2t+8, 2t+9; head g)
                             const uint32_t X = pack2<F16>(pr[0], pr[2]);   // head 2t:   tokens g, g+8
                             const uint32_t Y = pack2<F16>(pr[1], pr[3]);   // head 2t+1: tokens g, g+8
@@ -924,7 +893,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         }
                         // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
                         const bool partial = valid < tt * 16 + 16;
-                        if constexpr (F8) {
+                        if constexpr (F16) {
 #pragma unroll
                             for (int dt = 0; dt < C::kDT; dt += 2) {
 #pragma unroll
@@ -935,29 +904,10 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                                         lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
                                         hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
                                     }
-                                    // rows g / g+8 of the m-tile = d 2g / 2g+1 of chunk dt + h2; k = tokens
-                                    // 2t, 2t+1, 2t+8, 2t+9 against P hi, then the same tokens against P lo
-                                    const uint32_t a0 = __byte_perm(lo, hi, 0x6420), a1 = __byte_perm(lo, hi, 0x7531);
-                                    const uint32_t a[4] = {a0, a1, a0, a1};
-                                    mma_16832_f8<KV::kFmt>(o[dt + h2], a, pb0, pb1);
-                                }
-                            }
-                        } else if constexpr (F16) {
-#pragma unroll
-                            for (int dt = 0; dt < C::kDT; dt += 2) {
-#pragma unroll
-                                for (int h2 = 0; h2 < 2; ++h2) {
-                                    uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
-                                    if (partial) {
-                                        const int tk = tt * 16 + 2 * t;
-                                        lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
-                                        hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
-                                    }
-                                    // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1)
-                                    const uint32_t a[4] = {fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0020)),
-                                                           fp8x2_to_f16x2<KV>(__byte_perm(lo, 0u, 0x0031)),
-                                                           fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0020)),
-                                                           fp8x2_to_f16x2<KV>(__byte_perm(hi, 0u, 0x0031))};
+                                    // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1):
+                                    // A pairs (tok a, a+1) of d 2g from bytes 0, 2 and of d 2g+1 from 1, 3
+                                    const uint32_t a[4] = {widen2<KV, 0, 2>(lo), widen2<KV, 1, 3>(lo),
+                                                           widen2<KV, 0, 2>(hi), widen2<KV, 1, 3>(hi)};
                                     mma_16816<true>(o[dt + h2], a, pb0, pb1);
                                 }
                             }
@@ -997,7 +947,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
             const int stream = s * NHG + hg;
             // element (head column c, row d) of this lane's accumulators
             auto d_of = [&](int dt, int half) -> int {
-                return (F16 || F8) ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
+                return F16 ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
             };
             // a whole stream writes `out`; pieces of split streams, every stream of a prefix pass and
             // the suffix of a sequence with shared blocks leave (o, m, l) for the merge
@@ -1046,136 +996,99 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
         asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Log-sum-exp merge of the nseg partials of KV head (stream's head group) * HG + warp of sequence
-// s, written by runs first_run .. first_run + nseg - 1, into out. One warp.
-template <class QT, int D, int G, int HG>
-__device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int stream, int first_run, int nseg, int NHG,
-                                           int warp, int lane)
+// One piece of a query column: its o (D floats), m and l.
+struct PieceRef {
+    const float* o;
+    const float* m;
+    const float* l;
+};
+
+// Log-sum-exp combination of the n pieces of one query column into dst (one warp; lane i owns
+// floats 4i .. 4i + 3 of the D): out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, times
+// out_scale. Every lane loads one piece's (m, l), then the o slices stream in eight pieces at a
+// time, so a column split into many pieces costs a few round trips, not one per piece.
+template <class QT, int D, class Piece>
+__device__ __forceinline__ void merge_column(int n, Piece piece, float out_scale, QT* dst, int lane)
 {
-    const int head = (stream - s * NHG) * HG + warp;
-    const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
-    QT* out = reinterpret_cast<QT*>(p.out);
-    auto slot = [&](int c) -> const float* {
-        return p.partials + ((size_t)(first_run + c + stream) * HG + warp) * p.slot_floats;
-    };
-    constexpr int NV = (G * D + 127) / 128;    // float4 groups per lane
-    float4 acc[NV];
-#pragma unroll
-    for (int v = 0; v < NV; ++v)
-        acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Lsum[G];
-    float Mcur[G];                             // running reference over the 32-segment chunks
-#pragma unroll
-    for (int gq = 0; gq < G; ++gq) {
-        Lsum[gq] = 0.f;
-        Mcur[gq] = -INFINITY;
-    }
-    for (int c0 = 0; c0 < nseg; c0 += 32) {
-        const int cnt = min(32, nseg - c0);
-        const bool mine = lane < cnt;
-        // one round trip: lane c's segment (m, l), and every lane's slice of the first four segments' o
-        float mc[G], lc[G];
-#pragma unroll
-        for (int gq = 0; gq < G; ++gq) {
-            mc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + gq) : -INFINITY;
-            lc[gq] = mine ? __ldcg(slot(c0 + lane) + G * D + G + gq) : 0.f;
+    const bool mine = 4 * lane < D;
+    float M = -INFINITY, Lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < n; c0 += 32) {
+        const int cnt = min(32, n - c0);
+        float mi = -INFINITY, li = 0.f;
+        if (lane < cnt) {
+            const PieceRef r = piece(c0 + lane);
+            mi = __ldcg(r.m);
+            li = __ldcg(r.l);
         }
-        float4 ov[4][NV];
+        float mx = mi;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int off = 16; off >= 1; off >>= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+        const float Mn = fmaxf(M, mx);
+        if (Mn == -INFINITY)
+            continue;                                   // no token in any of these pieces (warp-uniform)
+        const float rescale = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+        Lsum *= rescale;
+        acc.x *= rescale;
+        acc.y *= rescale;
+        acc.z *= rescale;
+        acc.w *= rescale;
+        M = Mn;
+        const float w = mi == -INFINITY ? 0.f : fast_exp2(mi - M);
+        float lw = w * li;
 #pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                const int idx = 4 * lane + 128 * v;
-                ov[u][v] = (u < cnt && idx < G * D) ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + u) + idx))
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        // chunk reference max, rescale what earlier chunks accumulated
-        float w[G];
+        for (int off = 16; off >= 1; off >>= 1)
+            lw += __shfl_xor_sync(kFullMask, lw, off);
+        Lsum += lw;
+        for (int j = 0; j < cnt; j += 8) {
+            float4 v[8];
+            float wu[8];
 #pragma unroll
-        for (int gq = 0; gq < G; ++gq) {
-            float mx = mc[gq];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
-            const float Mn = fmaxf(Mcur[gq], mx);
-            const float rescale = (Mcur[gq] == -INFINITY) ? 0.f : fast_exp2(Mcur[gq] - Mn);
-            Lsum[gq] *= rescale;
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                if ((4 * lane + 128 * v) / D == gq) {
-                    acc[v].x *= rescale;
-                    acc[v].y *= rescale;
-                    acc[v].z *= rescale;
-                    acc[v].w *= rescale;
-                }
-            }
-            Mcur[gq] = Mn;
-            w[gq] = (mc[gq] == -INFINITY || Mn == -INFINITY) ? 0.f : fast_exp2(mc[gq] - Mn);
-            float lw = w[gq] * lc[gq];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                lw += __shfl_xor_sync(kFullMask, lw, off);
-            Lsum[gq] += lw;
-        }
-        for (int j = 0; j < cnt; j += 4) {
-            if (j > 0) {                         // later groups of four segments
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                    for (int v = 0; v < NV; ++v) {
-                        const int idx = 4 * lane + 128 * v;
-                        ov[u][v] = (j + u < cnt && idx < G * D)
-                                       ? __ldcg(reinterpret_cast<const float4*>(slot(c0 + j + u) + idx))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
+            for (int u = 0; u < 8; ++u) {
+                wu[u] = __shfl_sync(kFullMask, w, (j + u) & 31);
+                v[u] = (j + u < cnt && mine) ? __ldcg(reinterpret_cast<const float4*>(piece(c0 + j + u).o) + lane)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float wu[G];
-#pragma unroll
-                for (int gq = 0; gq < G; ++gq)
-                    wu[gq] = __shfl_sync(kFullMask, w[gq], (j + u) & 31);
-                if (j + u < cnt) {
-#pragma unroll
-                    for (int v = 0; v < NV; ++v) {
-                        const int gv = (4 * lane + 128 * v) / D;
-                        float a = 0.f;
-#pragma unroll
-                        for (int gq = 0; gq < G; ++gq)
-                            a = (gq == gv) ? wu[gq] : a;
-                        acc[v].x = fmaf(a, ov[u][v].x, acc[v].x);
-                        acc[v].y = fmaf(a, ov[u][v].y, acc[v].y);
-                        acc[v].z = fmaf(a, ov[u][v].z, acc[v].z);
-                        acc[v].w = fmaf(a, ov[u][v].w, acc[v].w);
-                    }
-                }
+            for (int u = 0; u < 8; ++u) {
+                acc.x = fmaf(wu[u], v[u].x, acc.x);
+                acc.y = fmaf(wu[u], v[u].y, acc.y);
+                acc.z = fmaf(wu[u], v[u].z, acc.z);
+                acc.w = fmaf(wu[u], v[u].w, acc.w);
             }
         }
     }
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-        const int idx = 4 * lane + 128 * v;
-        if (idx < G * D) {
-            const int gv = idx / D;
-            float L = 0.f;
-#pragma unroll
-            for (int gq = 0; gq < G; ++gq)
-                L = (gq == gv) ? Lsum[gq] : L;
-            const float inv = L > 0.f ? out_scale / L : 0.f;
-            QT* dst = out + query_row(p, s, head, gv) * D + (idx - gv * D);
-            from_float(acc[v].x * inv, dst);
-            from_float(acc[v].y * inv, dst + 1);
-            from_float(acc[v].z * inv, dst + 2);
-            from_float(acc[v].w * inv, dst + 3);
-        }
+    if (mine) {
+        const float inv = Lsum > 0.f ? out_scale / Lsum : 0.f;
+        QT* o = dst + 4 * lane;
+        from_float(acc.x * inv, o);
+        from_float(acc.y * inv, o + 1);
+        from_float(acc.z * inv, o + 2);
+        from_float(acc.w * inv, o + 3);
     }
 }
 
+// Merge of query column gq of KV head (stream's head group) * HG + w of sequence s, whose stream
+// left pieces in chunks first_chunk .. first_chunk + n - 1 (slot (chunk + stream) * HG + w).
+template <class QT, int D, int G, int HG>
+__device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int stream, int first_chunk, int n, int NHG,
+                                           int w, int gq, int lane)
+{
+    const int head = (stream - s * NHG) * HG + w;
+    const float out_scale = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
+    auto piece = [&](int i) -> PieceRef {
+        const float* b = p.partials + ((size_t)(first_chunk + i + stream) * HG + w) * p.slot_floats;
+        return PieceRef{b + gq * D, b + G * D + gq, b + G * D + G + gq};
+    };
+    merge_column<QT, D>(n, piece, out_scale, reinterpret_cast<QT*>(p.out) + query_row(p, s, head, gq) * D, lane);
+}
 
-// Merge of the streams the decode kernel split across runs: one warp per (stream, KV head of its
-// group), launched behind the decode kernel as a programmatic dependent launch. The prefix is
-// built while the decode kernel still runs (it reads only seq_lens); griddepcontrol.wait then
-// holds until the decode grid has finished and its partials are visible.
+
+// Merge of the streams the decode kernel split across chunks: one warp per (stream, KV head of
+// its group, query column), launched behind the decode kernel as a programmatic dependent launch.
+// The prefix is built while the decode kernel still runs (it reads only seq_lens);
+// griddepcontrol.wait then holds until the decode grid has finished and its partials are visible.
 constexpr int kMergeThreads = 128;
 
 template <class QT, int D, int BS, int G, int HG>
@@ -1193,9 +1106,10 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kMergeThreads / 32);
-    const int items = p.num_seqs * NHG * HG;
+    const int items = p.num_seqs * NHG * HG * G;
     for (int it = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5); it < items; it += warps) {
-        const int stream = it / HG, w = it - stream * HG;
+        const int gq = it % G, sw = it / G;
+        const int stream = sw / HG, w = sw - stream * HG;
         const int s = stream / NHG, hg = stream - s * NHG;
         const int nb = (prefix[s + 1] - prefix[s]) / NHG;
         if (nb == 0)
@@ -1203,7 +1117,7 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
         const int sb = prefix[s] + hg * nb;
         const int first_run = ch.of(sb), last_run = ch.of(sb + nb - 1);
         if (first_run != last_run)
-            merge_split<QT, D, G, HG>(p, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
+            merge_split<QT, D, G, HG>(p, s, stream, first_run, last_run - first_run + 1, NHG, w, gq, lane);
     }
 }
 
@@ -1228,11 +1142,11 @@ __global__ void __launch_bounds__(kMergeThreads)
     (void)build_unit_prefix(ps, prefix_s, BS, NHG, capacity);
     (void)build_unit_prefix(pp, prefix_p, BS, Hkv, capacity);
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int total_s = prefix_s[ps.num_seqs], total_p = prefix_p[pp.num_seqs];
     if (blockIdx.x == 0 && threadIdx.x == 0) {   // both passes are done claiming
         *ps.chunk_ctr = 0;
         *pp.chunk_ctr = 0;
     }
+    const int total_s = prefix_s[ps.num_seqs], total_p = prefix_p[pp.num_seqs];
     const Chunks ch_s = make_chunks(total_s, runs_s, ps.tail_chunks);
     const Chunks ch_p = make_chunks(total_p, runs_p, pp.tail_chunks);
     const int lane = threadIdx.x & 31;
@@ -1261,58 +1175,34 @@ __global__ void __launch_bounds__(kMergeThreads)
         (void)stream_tokens(ps, seq, BS, capacity, skipb, e);
         if (skipb == 0)
             continue;                                 // nothing shared: the suffix pass wrote it whole
-        float M = -INFINITY, Lsum = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const bool mine = 4 * lane < D;
-        auto add = [&](const float* o, float m, float l) {
-            if (m == -INFINITY)
-                return;
-            const float Mn = fmaxf(M, m);
-            const float a = M == -INFINITY ? 0.f : fast_exp2(M - Mn), b = fast_exp2(m - Mn);
-            Lsum = Lsum * a + l * b;
-            if (mine) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(o + 4 * lane));
-                acc.x = acc.x * a + b * v.x;
-                acc.y = acc.y * a + b * v.y;
-                acc.z = acc.z * a + b * v.z;
-                acc.w = acc.w * a + b * v.w;
-            }
-            M = Mn;
-        };
         // prefix pieces: stream (gi, h) of the prefix pass, column mi * Gq + gq (tile cg / 8)
         const int nb_p = (prefix_p[gi + 1] - prefix_p[gi]) / Hkv;
-        if (nb_p > 0) {
-            const int pstream = gi * Hkv + h, sb = prefix_p[gi] + h * nb_p;
-            const int cg = mi * Gq + gq, tile = cg >> 3, c = cg & 7;
-            for (int r = ch_p.of(sb); r <= ch_p.of(sb + nb_p - 1); ++r) {
-                const float* base = pp.partials + ((size_t)(r + pstream) * 4 + tile) * pp.slot_floats;
-                add(base + c * D, __ldcg(base + 8 * D + c), __ldcg(base + 8 * D + 8 + c));
-            }
-        }
+        const int pstream = gi * Hkv + h, sbp = prefix_p[gi] + h * nb_p;
+        const int cg = mi * Gq + gq, tile = cg >> 3, c = cg & 7;
+        const int fp = nb_p > 0 ? ch_p.of(sbp) : 0, np = nb_p > 0 ? ch_p.of(sbp + nb_p - 1) - fp + 1 : 0;
         // suffix pieces: stream (seq, h / HG) of the suffix pass, warp h % HG, column gq
         const int nb_s = (prefix_s[seq + 1] - prefix_s[seq]) / NHG;
-        if (nb_s > 0) {
-            const int hg = h / HG, w = h - hg * HG, stream = seq * NHG + hg, sb = prefix_s[seq] + hg * nb_s;
-            for (int r = ch_s.of(sb); r <= ch_s.of(sb + nb_s - 1); ++r) {
-                const float* base = ps.partials + ((size_t)(r + stream) * HG + w) * ps.slot_floats;
-                add(base + gq * D, __ldcg(base + G * D + gq), __ldcg(base + G * D + G + gq));
+        const int hg = h / HG, w = h - hg * HG, stream = seq * NHG + hg, sbs = prefix_s[seq] + hg * nb_s;
+        const int fs = nb_s > 0 ? ch_s.of(sbs) : 0, ns = nb_s > 0 ? ch_s.of(sbs + nb_s - 1) - fs + 1 : 0;
+        auto piece = [&](int i) -> PieceRef {
+            if (i < np) {
+                const float* b = pp.partials + ((size_t)(fp + i + pstream) * 4 + tile) * pp.slot_floats;
+                return PieceRef{b + c * D, b + 8 * D + c, b + 8 * D + 8 + c};
             }
-        }
+            const float* b = ps.partials + ((size_t)(fs + (i - np) + stream) * HG + w) * ps.slot_floats;
+            return PieceRef{b + gq * D, b + G * D + gq, b + G * D + G + gq};
+        };
         const float out_scale = ps.v_head_scales ? ps.v_scale * __ldg(ps.v_head_scales + h) : ps.v_scale;
-        const float inv = Lsum > 0.f ? out_scale / Lsum : 0.f;
-        if (mine) {
-            QT* dst = reinterpret_cast<QT*>(ps.out) + ((size_t)seq * ps.num_heads + (size_t)h * Gq + gq) * D + 4 * lane;
-            from_float(acc.x * inv, dst);
-            from_float(acc.y * inv, dst + 1);
-            from_float(acc.z * inv, dst + 2);
-            from_float(acc.w * inv, dst + 3);
-        }
+        merge_column<QT, D>(np + ns, piece, out_scale,
+                            reinterpret_cast<QT*>(ps.out) + ((size_t)seq * ps.num_heads + (size_t)h * Gq + gq) * D,
+                            lane);
     }
 
     // (b) split streams of sequences without shared blocks
-    const int items_b = ps.num_seqs * NHG * HG;
+    const int items_b = ps.num_seqs * NHG * HG * G;
     for (int it = wid; it < items_b; it += warps) {
-        const int stream = it / HG, w = it - stream * HG;
+        const int gq = it % G, sw = it / G;
+        const int stream = sw / HG, w = sw - stream * HG;
         const int s = stream / NHG, hg = stream - s * NHG;
         const int nb = (prefix_s[s + 1] - prefix_s[s]) / NHG;
         if (nb == 0)
@@ -1324,7 +1214,7 @@ __global__ void __launch_bounds__(kMergeThreads)
         const int sb = prefix_s[s] + hg * nb;
         const int first_run = ch_s.of(sb), last_run = ch_s.of(sb + nb - 1);
         if (first_run != last_run)
-            merge_split<QT, D, G, HG>(ps, s, stream, first_run, last_run - first_run + 1, NHG, w, lane);
+            merge_split<QT, D, G, HG>(ps, s, stream, first_run, last_run - first_run + 1, NHG, w, gq, lane);
     }
 }
 
@@ -1396,9 +1286,10 @@ struct MmaLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
-        // 8-bit codes enter the products as their format's values: only the per-tensor scales remain
-        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
-        p.v_scale = KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f;
+        // 8-bit codes enter the products widened (E4M3 as its value times 2^-8): the per-tensor scales
+        // and the widening factor remain
+        p.q_scale = p.scale * kLog2e * widen_factor<KV>() * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
+        p.v_scale = widen_factor<KV>() * (KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(nruns);
         cfg.blockDim = dim3(C::kThreads);
@@ -1435,11 +1326,11 @@ struct MmaLauncher {
         if (st != PKV_OK)
             return st;
         // the merge of split streams, allowed to start while the decode grid drains
-        const int items = p.num_seqs * p.num_kv_heads;
+        const int items = p.num_seqs * p.num_kv_heads * G;
         const int per_cta = kMergeThreads / 32;
         int mgrid = (items + per_cta - 1) / per_cta;
-        if (mgrid > nruns)
-            mgrid = nruns;
+        if (mgrid > 2 * nruns)
+            mgrid = 2 * nruns;
         void* args[] = {&p, &nruns};
         return launch_merge_pdl((const void*)paged_decode_merge_kernel<QT, D, BS, G, HG>, args, mgrid,
                                 (size_t)(p.num_seqs + 1) * 4, stream);
@@ -1461,13 +1352,11 @@ struct MmaLauncher {
         const int st = launch_decode(ps, runs_s, stream, any_groups);
         if (st != PKV_OK)
             return st;
-        const long long members_items = any_groups ? 1ll * ps.num_seqs * ps.num_heads : 0;
-        const long long items = members_items > 1ll * ps.num_seqs * ps.num_kv_heads
-                                    ? members_items : 1ll * ps.num_seqs * ps.num_kv_heads;
+        const long long items = 1ll * ps.num_seqs * ps.num_kv_heads * G;   // >= members x query heads
         const int per_cta = kMergeThreads / 32;
         long long mgrid = (items + per_cta - 1) / per_cta;
-        if (mgrid > runs_s)
-            mgrid = runs_s;
+        if (mgrid > 2ll * runs_s)
+            mgrid = 2ll * runs_s;
         if (mgrid < 1)
             mgrid = 1;
         void* args[] = {&ps, &pp, &runs_s, &runs_p};

@@ -19,7 +19,7 @@ constexpr int kMaxHeadGroup = 4;        // KV heads per MMA work unit (partial s
 // quarter is cut into up to kTailChunksPerRun chunks per CTA, claimed as CTAs run dry. The
 // workspace keeps partial slots for (1 + kTailChunksPerRun) chunks per run.
 constexpr int kTailChunksPerRun = 4;
-constexpr int kMinTailChunk = 8;        // units
+constexpr int kMinTailChunk = 16;       // units
 constexpr float kLog2e = 1.4426950408889634074f;
 
 struct DecodeParams {
