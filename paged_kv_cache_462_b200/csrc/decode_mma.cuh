@@ -115,10 +115,9 @@ __device__ __forceinline__ void split_s8x4(const float (&v)[4], uint32_t& hi, ui
 
 // Bytes B0 and B1 of r (two 8-bit codes) as an f16x2 (byte B0 in the low half), exact:
 //  * E5M2 codes are the high bytes of the f16 of the same value: one byte permute.
-//  * E4M3 s.eeee.mmm placed as f16 bits s.0eeee.mmm0000000 is the code's value times 2^-8, normal
-//    and subnormal alike (the f16 exponent bias is 8 more than E4M3's, and E4M3's subnormal step
-//    2^-9 lands on f16's subnormal step 2^-24 shifted by 7): a permute, a shift and two logic
-//    operations; the launcher puts the 2^8 back into the score and output factors.
+//  * E4M3: the hardware conversion of the code pair. (Placing s.eeee.mmm as the f16 bits
+//    s.0eeee.mmm0000000, the value times 2^-8 for normal and subnormal codes alike, takes a
+//    permute, a shift and two logic operations instead and measured slower.)
 //  * INT8: the offset byte x + 128 as the mantissa of 1024.0 gives the f16 1152 + x; less 1152.
 template <class KV, int B0, int B1>
 __device__ __forceinline__ uint32_t widen2(uint32_t r)
@@ -129,21 +128,15 @@ __device__ __forceinline__ uint32_t widen2(uint32_t r)
                                                                                       __ushort_as_half(0x6480)));
         return *reinterpret_cast<const uint32_t*>(&h);
     } else {
-        const uint32_t x = __byte_perm(r, 0u, 4 | (B0 << 4) | (4 << 8) | (B1 << 12));   // [0, c0, 0, c1]
-        if constexpr (KV::kFmt == __NV_E5M2)
-            return x;
-        else
-            return ((x >> 1) & 0x3F803F80u) | (x & 0x80008000u);
+        if constexpr (KV::kFmt == __NV_E5M2) {
+            return __byte_perm(r, 0u, 4 | (B0 << 4) | (4 << 8) | (B1 << 12));   // [0, c0, 0, c1]
+        } else {
+            uint32_t o;
+            const uint16_t v = static_cast<uint16_t>(__byte_perm(r, 0u, B0 | (B1 << 4)));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(o) : "h"(v));
+            return o;
+        }
     }
-}
-
-// factor between an 8-bit code's widened f16 and its format value (see widen2)
-template <class KV>
-constexpr float widen_factor()
-{
-    if constexpr (KV::kBytes == 1 && !KV::kInt8)
-        return KV::kFmt == __NV_E4M3 ? 256.0f : 1.0f;
-    return 1.0f;
 }
 
 template <bool F16>
@@ -372,7 +365,7 @@ __device__ __forceinline__ Chunks make_chunks(int U, int R, int tail_chunks)
     ch.R = R;
     ch.U = U;
     const int per = (U + R - 1) / R;
-    if (tail_chunks <= 0 || U < 2 * R * kMinTailChunk) {   // static: one run per CTA
+    if (tail_chunks <= 0 || U < kMinUnitsForTail * R) {   // static: one run per CTA
         ch.P1 = per > 0 ? per : 1;
         ch.P2 = 1;
         ch.C = R;
@@ -1286,10 +1279,9 @@ struct MmaLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
-        // 8-bit codes enter the products widened (E4M3 as its value times 2^-8): the per-tensor scales
-        // and the widening factor remain
-        p.q_scale = p.scale * kLog2e * widen_factor<KV>() * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
-        p.v_scale = widen_factor<KV>() * (KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f);
+        // 8-bit codes enter the products widened exactly: only the per-tensor scales remain
+        p.q_scale = p.scale * kLog2e * (KV::kBytes == 1 && !p.k_head_scales ? p.k_scale : 1.0f);
+        p.v_scale = KV::kBytes == 1 && !p.v_head_scales ? p.v_scale_in : 1.0f;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(nruns);
         cfg.blockDim = dim3(C::kThreads);

@@ -20,6 +20,10 @@ constexpr int kMaxHeadGroup = 4;        // KV heads per MMA work unit (partial s
 // workspace keeps partial slots for (1 + kTailChunksPerRun) chunks per run.
 constexpr int kTailChunksPerRun = 4;
 constexpr int kMinTailChunk = 16;       // units
+// below this many units per CTA the split stays static: there a CTA's whole run lasts only some
+// tens of microseconds, and tail chunks (and the merging of the extra pieces they cut) cost more
+// than the imbalance they remove (measured on the long-context and Llama-3-8B-layer workloads)
+constexpr int kMinUnitsForTail = 256;
 constexpr float kLog2e = 1.4426950408889634074f;
 
 struct DecodeParams {

@@ -602,3 +602,29 @@ def test_int8_workloads_fused_step(cfg, over):
     assert g.device_errors() == 0
     assert np.array_equal(cache_bytes(g.kc), okc) and np.array_equal(cache_bytes(g.vc), ovc)
     assert max_err(out, ref) <= TOL["int8"]
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
+def test_every_8bit_code_reads_back_exactly(kv):
+    """One cached token (softmax weight exactly 1) whose V rows hold every finite code of the
+    format across two KV heads: with a unit scale the output row is each code's value, bit for
+    bit in bf16 (all of them are bf16 values): the kernel's widening of each code is exact."""
+    D, BS = 128, 16
+    codes = np.arange(256, dtype=np.uint8)
+    if kv == "e4m3":
+        vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    elif kv == "e5m2":
+        vals = torch.from_numpy(codes).view(torch.float8_e5m2).float().numpy()
+    else:
+        vals = codes.view(np.int8).astype(np.float32)
+    bad = ~np.isfinite(vals)
+    codes[bad], vals[bad] = 0, 0.0                          # NaN / infinite codes are not values
+    kc = torch.zeros((4, 2, BS, D), dtype=TORCH_DT[kv], device="cuda")
+    vc = torch.zeros_like(kc)
+    vc.view(torch.uint8)[0, :, 0, :] = torch.from_numpy(codes.reshape(2, D)).cuda()
+    q = torch.ones((1, 2, D), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q)
+    pkv.paged_attention_decode(out, q, kc, vc, torch.zeros((1, 1), dtype=torch.int32, device="cuda"),
+                               torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, 1.0, 1.0)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.float().cpu().numpy().reshape(-1), vals)
