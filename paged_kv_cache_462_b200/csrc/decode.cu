@@ -1,7 +1,8 @@
-// Dispatch of paged_attention_decode: the warp-MMA kernel (decode_mma.cuh) for
-// bf16 / E4M3 / E5M2 caches of the shapes it covers, the CUDA-core kernel
-// (decode_kernel.cuh) for fp32 caches and the other bf16 / E4M3 shapes (E5M2
-// has no CUDA-core form).
+// Dispatch of paged_attention_decode: the tcgen05 kernel (decode_tc05.cuh) for E4M3 / E5M2
+// caches with head_dim 128 and block size 16 or 32, the warp-MMA kernel (decode_mma.cuh) for
+// bf16 and INT8 caches of the shapes it covers (and the shared-prefix passes of every 8-bit and
+// bf16 cache), the CUDA-core kernel (decode_kernel.cuh) for fp32 caches and the other bf16 /
+// E4M3 shapes (E5M2 has no CUDA-core form).
 #include "decode_kernel.cuh"
 
 namespace pkv {
@@ -71,9 +72,22 @@ int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads)
     return 0;
 }
 
+int decode_tc05_dispatch(int kv_dtype, int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st,
+                         int* occ);
+
+bool tc05_supported(int q_dtype, int kv_dtype, int head_dim, int block_size, int group)
+{
+    return q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2) && head_dim == 128 &&
+           (block_size == 16 || block_size == 32) && (group == 1 || group == 2 || group == 4 || group == 5 ||
+                                                        group == 8);
+}
+
 int decode_dispatch(int q_dtype, int kv_dtype, int D, int BS, int G, const DecodeParams& p, int nruns,
                     cudaStream_t st, int* occupancy_out)
 {
+    // FP8 caches: the tcgen05 kernel (8-bit products on the fifth-generation tensor cores)
+    if (tc05_supported(q_dtype, kv_dtype, D, BS, G))
+        return decode_tc05_dispatch(kv_dtype, D, BS, G, p, nruns, st, occupancy_out);
     if (q_dtype == PKV_BF16 && mma_supported(kv_dtype, D, BS, G, p.num_kv_heads))
         return decode_mma_dispatch(kv_dtype, D, BS, G, mma_head_group(kv_dtype, D, BS, p.num_kv_heads), p, nruns,
                                    st, occupancy_out);

@@ -305,17 +305,19 @@ __device__ __forceinline__ int stream_tokens(const DecodeParams& p, int s, int B
     return L - skip * BS;
 }
 
-// prefix[s] = units (head group x logical block) of sequences before s, units of a sequence =
-// ceil(L / block_size) * groups with L the tokens the pass streams (stream_tokens). All threads
-// of the CTA; ends with a barrier. Returns the PKV_DEVERR_* bits of clamped lengths or skips.
-__device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity)
+// prefix[s] = units (head group x UT tokens) of sequences before s, units of a sequence =
+// ceil(L / UT) * groups with L the tokens the pass streams (stream_tokens, blocks of BS tokens;
+// UT = BS for the warp-MMA kernel, whose unit is one block). All threads of the CTA; ends with a
+// barrier. Returns the PKV_DEVERR_* bits of clamped lengths or skips.
+__device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity,
+                                                 int UT)
 {
     const int tid = threadIdx.x, lane = tid & 31;
     int bad = 0;
     for (int s = tid; s < p.num_seqs; s += blockDim.x) {
         int skip;
         const int L = stream_tokens(p, s, BS, capacity, skip, bad);
-        prefix[s + 1] = ((L + BS - 1) / BS) * NHG;
+        prefix[s + 1] = ((L + UT - 1) / UT) * NHG;
     }
     if (tid == 0)
         prefix[0] = 0;
@@ -428,7 +430,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
         fence_mbar_init();
     }
     {
-        const int bad = build_unit_prefix(p, prefix, BS, NHG, capacity);
+        const int bad = build_unit_prefix(p, prefix, BS, NHG, capacity, BS);
         if (bad && blockIdx.x == 0 && tid == 0)
             atomicOr(p.err, bad);
     }
@@ -1084,12 +1086,14 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
 // griddepcontrol.wait then holds until the decode grid has finished and its partials are visible.
 constexpr int kMergeThreads = 128;
 
-template <class QT, int D, int BS, int G, int HG>
+// UT: tokens per unit of the decode kernel (the block size for the warp-MMA kernel, 128 for the
+// tcgen05 kernel).
+template <class QT, int D, int BS, int G, int HG, int UT = BS>
 __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const DecodeParams p, int decode_runs)
 {
     extern __shared__ int prefix[];   // [num_seqs + 1]
     const int NHG = p.num_kv_heads / HG;
-    (void)build_unit_prefix(p, prefix, BS, NHG, p.max_blocks_per_seq * BS);
+    (void)build_unit_prefix(p, prefix, BS, NHG, p.max_blocks_per_seq * BS, UT);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (blockIdx.x == 0 && threadIdx.x == 0)   // the decode grid is done claiming: ready for the next call
         *p.chunk_ctr = 0;
@@ -1132,8 +1136,8 @@ __global__ void __launch_bounds__(kMergeThreads)
     int* prefix_p = smem_prefix + ps.num_seqs + 1;   // [num_groups + 1]
     const int Hkv = ps.num_kv_heads, NHG = Hkv / HG, Gq = ps.num_heads / Hkv;
     const int capacity = ps.max_blocks_per_seq * BS;
-    (void)build_unit_prefix(ps, prefix_s, BS, NHG, capacity);
-    (void)build_unit_prefix(pp, prefix_p, BS, Hkv, capacity);
+    (void)build_unit_prefix(ps, prefix_s, BS, NHG, capacity, BS);
+    (void)build_unit_prefix(pp, prefix_p, BS, Hkv, capacity, BS);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (blockIdx.x == 0 && threadIdx.x == 0) {   // both passes are done claiming
         *ps.chunk_ctr = 0;
