@@ -385,6 +385,23 @@ PKV_API int pkv_validate_tables(const int32_t* block_tables, const int32_t* seq_
 /* Number of partitions num_partitions = 0 resolves to for this configuration on the current device. */
 PKV_API int pkv_default_partitions(int head_dim, int block_size, int num_heads, int num_kv_heads, int kv_dtype);
 
+/*
+ * Kernel for decodes of FP8 (E4M3 / E5M2) caches, process-wide:
+ *   PKV_FP8_KERNEL_MMA (0, the default): warp-level tensor-core products on codes widened
+ *     exactly to f16 (every FP8 shape the library covers);
+ *   PKV_FP8_KERNEL_TCGEN05 (1): fifth-generation tensor cores (tcgen05.mma, accumulators in
+ *     tensor memory) reading the 8-bit K and V tiles as they lie, for head_dim 128, block size 16
+ *     or 32 and a multiple of 128 / block_size KV heads; other FP8 shapes keep the default
+ *     kernel. Same results within the FP8 tolerance; on the measured workloads it is slower
+ *     than the default.
+ * Applies to calls queued after it (plain and fused decode steps, several new tokens per
+ * sequence, per-head scales and the no-allocation entry point; the shared-prefix passes always
+ * use the default). Returns the previous choice, or -PKV_ERR_SHAPE for an unknown value.
+ */
+#define PKV_FP8_KERNEL_MMA 0
+#define PKV_FP8_KERNEL_TCGEN05 1
+PKV_API int pkv_set_fp8_kernel(int which);
+
 /* Static description of a status code. */
 PKV_API const char* pkv_status_string(int status);
 

@@ -76,6 +76,8 @@ def load_library():
     lib.pkv_read_device_error.restype = i32
     lib.pkv_default_partitions.argtypes = [i32, i32, i32, i32, i32]
     lib.pkv_default_partitions.restype = i32
+    lib.pkv_set_fp8_kernel.argtypes = [i32]
+    lib.pkv_set_fp8_kernel.restype = i32
     lib.paged_attention_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.paged_attention_shared_prefix_workspace_size.restype = sz
     lib.paged_attention_decode_shared_prefix.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32,
@@ -152,6 +154,18 @@ def new_workspace(num_seqs, num_heads, num_kv_heads, head_dim, num_partitions=0,
 def workspace_init(workspace: torch.Tensor, stream=None) -> None:
     _check("pkv_workspace_init",
            load_library().pkv_workspace_init(_cuda("workspace", workspace), workspace.numel(), _stream_handle(stream)))
+
+
+FP8_KERNEL_MMA = 0        # warp-level tensor cores on codes widened to f16 (the default)
+FP8_KERNEL_TCGEN05 = 1    # fifth-generation tensor cores reading the 8-bit tiles (tcgen05.mma)
+
+
+def set_fp8_kernel(which: int) -> int:
+    """Process-wide kernel for FP8-cache decodes (pkv_set_fp8_kernel); returns the previous choice."""
+    prev = load_library().pkv_set_fp8_kernel(int(which))
+    if prev < 0:
+        raise PkvError("pkv_set_fp8_kernel", -prev)
+    return prev
 
 
 def default_partitions(head_dim, block_size, num_heads, num_kv_heads, kv_dtype) -> int:

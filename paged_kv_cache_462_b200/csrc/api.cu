@@ -224,6 +224,8 @@ int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_
     p.k_head_scales = k_head_scales;
     p.v_head_scales = v_head_scales;
     p.tail_chunks = kTailChunksPerRun;
+    p.tail_min_units = kMinUnitsForTail;
+    p.tail_min_chunk = kMinTailChunk;
     p.chunk_ctr = reinterpret_cast<int32_t*>(ws) + 1;   // header word 1
     if (withheld_unit >= 0) {
         if (!(q_dtype == PKV_BF16 && mma_supported(kv_dtype, head_dim, block_size, group, num_kv_heads)))

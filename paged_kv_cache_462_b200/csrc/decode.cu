@@ -1,8 +1,11 @@
 // Dispatch of paged_attention_decode: the tcgen05 kernel (decode_tc05.cuh) for E4M3 / E5M2
-// caches with head_dim 128 and block size 16 or 32, the warp-MMA kernel (decode_mma.cuh) for
-// bf16 and INT8 caches of the shapes it covers (and the shared-prefix passes of every 8-bit and
-// bf16 cache), the CUDA-core kernel (decode_kernel.cuh) for fp32 caches and the other bf16 /
-// E4M3 shapes (E5M2 has no CUDA-core form).
+// caches with head_dim 128, block size 16 or 32 and a multiple of 128 / block size KV heads; the
+// warp-MMA kernel (decode_mma.cuh) for bf16 and INT8 caches and the other E4M3 / E5M2 shapes it
+// covers (and the shared-prefix passes of every 8-bit and bf16 cache); the CUDA-core kernel
+// (decode_kernel.cuh) for fp32 caches and the other bf16 / E4M3 shapes (E5M2 has no CUDA-core
+// form).
+#include <atomic>
+
 #include "decode_kernel.cuh"
 
 namespace pkv {
@@ -75,18 +78,23 @@ int mma_head_group(int kv_dtype, int head_dim, int block_size, int num_kv_heads)
 int decode_tc05_dispatch(int kv_dtype, int D, int BS, int G, const DecodeParams& p, int nruns, cudaStream_t st,
                          int* occ);
 
-bool tc05_supported(int q_dtype, int kv_dtype, int head_dim, int block_size, int group)
+// the tcgen05 kernel's unit is one block of 128 / block_size KV heads
+bool tc05_supported(int q_dtype, int kv_dtype, int head_dim, int block_size, int group, int num_kv_heads)
 {
     return q_dtype == PKV_BF16 && (kv_dtype == PKV_FP8_E4M3 || kv_dtype == PKV_FP8_E5M2) && head_dim == 128 &&
-           (block_size == 16 || block_size == 32) && (group == 1 || group == 2 || group == 4 || group == 5 ||
-                                                        group == 8);
+           (block_size == 16 || block_size == 32) && num_kv_heads % (128 / block_size) == 0 &&
+           (group == 1 || group == 2 || group == 4 || group == 5 || group == 8);
 }
+
+std::atomic<int> g_fp8_kernel{PKV_FP8_KERNEL_MMA};
 
 int decode_dispatch(int q_dtype, int kv_dtype, int D, int BS, int G, const DecodeParams& p, int nruns,
                     cudaStream_t st, int* occupancy_out)
 {
-    // FP8 caches: the tcgen05 kernel (8-bit products on the fifth-generation tensor cores)
-    if (tc05_supported(q_dtype, kv_dtype, D, BS, G))
+    // FP8 caches on the tcgen05 kernel (8-bit products on the fifth-generation tensor cores)
+    // when it is chosen and covers the shape
+    if (g_fp8_kernel.load(std::memory_order_relaxed) == PKV_FP8_KERNEL_TCGEN05 &&
+        tc05_supported(q_dtype, kv_dtype, D, BS, G, p.num_kv_heads))
         return decode_tc05_dispatch(kv_dtype, D, BS, G, p, nruns, st, occupancy_out);
     if (q_dtype == PKV_BF16 && mma_supported(kv_dtype, D, BS, G, p.num_kv_heads))
         return decode_mma_dispatch(kv_dtype, D, BS, G, mma_head_group(kv_dtype, D, BS, p.num_kv_heads), p, nruns,
@@ -101,3 +109,10 @@ int decode_dispatch(int q_dtype, int kv_dtype, int D, int BS, int G, const Decod
 }
 
 }  // namespace pkv
+
+extern "C" PKV_API int pkv_set_fp8_kernel(int which)
+{
+    if (which != PKV_FP8_KERNEL_MMA && which != PKV_FP8_KERNEL_TCGEN05)
+        return -PKV_ERR_SHAPE;
+    return pkv::g_fp8_kernel.exchange(which);
+}

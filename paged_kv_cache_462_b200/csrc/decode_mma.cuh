@@ -308,9 +308,10 @@ __device__ __forceinline__ int stream_tokens(const DecodeParams& p, int s, int B
 // prefix[s] = units (head group x UT tokens) of sequences before s, units of a sequence =
 // ceil(L / UT) * groups with L the tokens the pass streams (stream_tokens, blocks of BS tokens;
 // UT = BS for the warp-MMA kernel, whose unit is one block). All threads of the CTA; ends with a
-// barrier. Returns the PKV_DEVERR_* bits of clamped lengths or skips.
+// barrier. Returns the PKV_DEVERR_* bits of clamped lengths or skips. With `info`, also
+// info[s] = (streamed tokens, skipped blocks) of every sequence.
 __device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* prefix, int BS, int NHG, int capacity,
-                                                 int UT)
+                                                 int UT, int2* info = nullptr)
 {
     const int tid = threadIdx.x, lane = tid & 31;
     int bad = 0;
@@ -318,6 +319,8 @@ __device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* pre
         int skip;
         const int L = stream_tokens(p, s, BS, capacity, skip, bad);
         prefix[s + 1] = ((L + UT - 1) / UT) * NHG;
+        if (info != nullptr)
+            info[s] = make_int2(L, skip);
     }
     if (tid == 0)
         prefix[0] = 0;
@@ -346,10 +349,10 @@ __device__ __forceinline__ int build_unit_prefix(const DecodeParams& p, int* pre
 
 // The units of a launch, in (sequence, head group, block) order, cut into chunks. Chunk c < R (R =
 // the grid's CTAs) is CTA c's own: [c * P1, (c + 1) * P1), three quarters of the work shared out
-// evenly. The last quarter is cut into chunks of P2 >= kMinTailChunk units, about
-// tail_chunks per CTA, which CTAs claim from a counter as they finish: SMs that stream slower
-// take fewer of them, so the grid ends together. With tail_chunks = 0 (or too little work) the
-// R own chunks cover everything. Chunks are contiguous and in order: the pieces of a stream are
+// evenly. The last quarter is cut into chunks of P2 >= min_chunk units, about tail_chunks per
+// CTA, which CTAs claim from a counter as they finish: SMs that stream slower take fewer of
+// them, so the grid ends together. With tail_chunks = 0 (or fewer than min_units units per CTA)
+// the R own chunks cover everything. Chunks are contiguous and in order: the pieces of a stream are
 // chunks of(begin) .. of(end - 1), the same for every schedule.
 struct Chunks {
     int R, P1, P2, C, U;
@@ -361,13 +364,13 @@ struct Chunks {
     __device__ __forceinline__ int of(int x) const { return x < R * P1 ? x / P1 : R + (x - R * P1) / P2; }
 };
 
-__device__ __forceinline__ Chunks make_chunks(int U, int R, int tail_chunks)
+__device__ __forceinline__ Chunks make_chunks(int U, int R, int tail_chunks, int min_units, int min_chunk)
 {
     Chunks ch;
     ch.R = R;
     ch.U = U;
     const int per = (U + R - 1) / R;
-    if (tail_chunks <= 0 || U < kMinUnitsForTail * R) {   // static: one run per CTA
+    if (tail_chunks <= 0 || U < min_units * R) {   // static: one run per CTA
         ch.P1 = per > 0 ? per : 1;
         ch.P2 = 1;
         ch.C = R;
@@ -376,7 +379,7 @@ __device__ __forceinline__ Chunks make_chunks(int U, int R, int tail_chunks)
     ch.P1 = (int)(3ll * U / (4ll * R));
     const int rem = U - R * ch.P1;
     const int want = (rem + R * tail_chunks - 1) / (R * tail_chunks);
-    ch.P2 = want > kMinTailChunk ? want : kMinTailChunk;
+    ch.P2 = want > min_chunk ? want : min_chunk;
     ch.C = R + (rem + ch.P2 - 1) / ch.P2;
     return ch;
 }
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 
     const int total = prefix[p.num_seqs];
     const int nruns = gridDim.x;
-    const Chunks ch = make_chunks(total, nruns, p.tail_chunks);
+    const Chunks ch = make_chunks(total, nruns, p.tail_chunks, p.tail_min_units, p.tail_min_chunk);
 
     // zero rows of empty sequences (one run per sequence); a prefix pass writes no rows, and a
     // suffix pass leaves the rows of sequences with shared blocks to the merge
@@ -1100,7 +1103,7 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     const int total = prefix[p.num_seqs];
     if (total == 0)
         return;
-    const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks);
+    const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks, p.tail_min_units, p.tail_min_chunk);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kMergeThreads / 32);
     const int items = p.num_seqs * NHG * HG * G;
@@ -1144,8 +1147,8 @@ __global__ void __launch_bounds__(kMergeThreads)
         *pp.chunk_ctr = 0;
     }
     const int total_s = prefix_s[ps.num_seqs], total_p = prefix_p[pp.num_seqs];
-    const Chunks ch_s = make_chunks(total_s, runs_s, ps.tail_chunks);
-    const Chunks ch_p = make_chunks(total_p, runs_p, pp.tail_chunks);
+    const Chunks ch_s = make_chunks(total_s, runs_s, ps.tail_chunks, ps.tail_min_units, ps.tail_min_chunk);
+    const Chunks ch_p = make_chunks(total_p, runs_p, pp.tail_chunks, pp.tail_min_units, pp.tail_min_chunk);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kMergeThreads / 32);
     const int wid = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
@@ -1222,6 +1225,24 @@ __global__ void __launch_bounds__(kMergeThreads)
 bool make_cache_tensormap(CUtensorMap* map, const void* base, int kv_dtype, int head_dim, long long rows,
                           int box_rows);
 
+// A merge kernel as a programmatic dependent launch behind the decode grid on `stream`.
+inline int launch_merge_pdl(const void* kern, void** args, int grid, size_t smem, cudaStream_t stream)
+{
+    if (!ensure_smem_attribute(kern, smem))
+        return PKV_ERR_LAUNCH;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, kern, args) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
+}
+
 template <class KV, class QT, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaLauncher {
     using C = MmaCfg<KV, D, BS, G, HG, PFX>;
@@ -1297,23 +1318,6 @@ struct MmaLauncher {
         cfg.attrs = attr;
         cfg.numAttrs = pdl ? 1 : 0;
         return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, p) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
-    }
-
-    static int launch_merge_pdl(const void* kern, void** args, int grid, size_t smem, cudaStream_t stream)
-    {
-        if (!ensure_smem_attribute(kern, smem))
-            return PKV_ERR_LAUNCH;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(kMergeThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelExC(&cfg, kern, args) == cudaSuccess ? PKV_OK : PKV_ERR_LAUNCH;
     }
 
     static int launch(DecodeParams p, int nruns, cudaStream_t stream)

@@ -5,44 +5,52 @@
 // Same result as the other decode kernels: for every sequence s and query head g,
 // out[s][g] = softmax_t(scale * q . K_t) V_t over the seq_lens[s] cached tokens, K_t / V_t read
 // through the block table ("vLLM inference cost optimisation", developer.aliyun.com, sections 2
-// and 4; wzjinhao.cn vLLM write-up, section 2.1), GQA head g -> KV head g / G.
+// and 4; wzjinhao.cn vLLM write-up, section 2.1), GQA head g -> KV head g / Gq.
 //
 // Layout of the work:
-//  * Unit = 128 consecutive tokens (128 / block_size logical blocks) of one (sequence, KV head)
-//    stream; units in (sequence, KV head, position) order are shared out in chunks exactly as in
-//    the warp-MMA kernel (Chunks), and streams cut by a chunk boundary leave pieces for the merge.
-//  * Warp 4 (producer): per unit, one 2-D TMA copy per block for K and one for V, each a box of
-//    block_size rows x 128 bytes with 128-byte swizzle, landing at row (block index in the unit)
-//    * block_size of the stage's 128-row K (V) tile, so a stage holds the unit as two
-//    128 x 128-byte tiles in the layout the tensor cores read (K-major for K, MN-major for V).
-//  * Warp 5 (MMA issuer, lane 0): S^T = K Q^T as four tcgen05.mma kind::f8f6f4 (M = 128 tokens,
-//    N = 16: the 8 query columns as E4M3 hi codes, then the same 8 as lo codes, K = 32 bytes of d
-//    each) into a TMEM S tile; when the softmax warps have written P, O^T += V^T P^T as eight
-//    (M = 128 d, N = 8 columns, K = 32 tokens, P hi then P lo) into the stream's TMEM O tile.
-//    Unit k+1's scores are issued before unit k's p.V, so the tensor cores work while the
-//    softmax of unit k runs.
-//  * Warps 0-3 (softmax, 128 threads): thread i is TMEM lane i, i.e. token i of the unit for S and
-//    row d = i of O. It loads its token's 16 S values, forms the 8 columns' scaled scores, keeps
-//    the online softmax (a lazy running max common to the 128 threads, partial sums per thread),
-//    writes its token's weights as E4M3 hi and lo bytes into the P^T tile, and at the end of a
-//    stream reads its row of O and writes the output row (or a partial piece).
+//  * Unit = one cache block of a (sequence, head group) stream: the block's rows of HPU = 128 /
+//    block_size consecutive KV heads, 128 rows of 128 bytes that lie contiguously in the cache
+//    ([block][KV head][token][d]). One 2-D TMA box (128 rows, 128-byte swizzle) brings its K tile
+//    and one its V tile: big copies, few of them (the TMA unit's cost is per copy). Units in
+//    (sequence, head group, block) order are shared out in chunks as in the warp-MMA kernel
+//    (Chunks); streams cut by a chunk boundary leave pieces for the merge.
+//  * Tile row r = (head hl = r / block_size, token t = r % block_size). The scores are one
+//    tcgen05.mma product S = K Q^T over all rows and all HPU heads' query columns (kind::f8f6f4,
+//    M = 128 rows, N = the HPU heads x (E4M3 hi codes, lo codes) x G columns, padded so that each
+//    softmax warp's heads start a 16-column group; four K = 32-byte steps of d); row r keeps only
+//    its own head's columns. The weights go into P^T, where row
+//    (head hl, column c) is non-zero only in the bytes of head hl's tokens, so O^T += V^T P^T
+//    (M = 128 d, N = (head, column) pairs, K = 32 rows per step, P hi then P lo) sums each head's
+//    own tokens only: the block-diagonal structure is exact, the extra tensor-core work is free.
+//  * Warp 4 (producer): per unit, a table lookup (32 units resolved at once, one per lane, the
+//    next 32 loaded while these are issued), the decode-step append of a stream's last block,
+//    the unit's descriptor (sequence, head group, block, segment flags) and the two copies.
+//  * Warp 5 issues the scores of every unit in order (once its tiles have landed and the S tile
+//    has been read), warp 6 its p.V product (once the weights are in): a tcgen05.mma holds its
+//    issuing thread for the tensor pipe's whole time (about 50 cycles for these shapes), so the
+//    issuers are threads of their own, off the softmax warps' path.
+//  * Warps 0-3 (softmax, 128 threads): thread i is TMEM lane i: tile row i for S (token t of head
+//    hl), row d = i of O.
+//  * One CTA per SM (the driver grants no more to a kernel that allocates tensor memory): the
+//    SM's shared memory goes to a deep stage ring; the last quarter of the work is cut into small
+//    chunks that CTAs claim as they run dry, so that slower SMs take fewer.
 //  * q and p enter the 8-bit products as E4M3 hi + lo pairs: q scaled per column by a power of two
 //    sigma (max |q| sigma < 256; a bf16 q is then held exactly down to 2^-2 of sigma's unit), p
 //    times 2^6 under a lazy-max slack of 2 (so p 2^6 <= 256 and weights down to 2^-12 of the
 //    running max stay E4M3-normal; the factor cancels between O and l).
-//  * S and P tiles are double-buffered by unit parity, Q and O tiles by stream (segment) parity.
+//  * P tiles are double-buffered by unit parity; one S tile, one O tile (hi and lo parts) and one
+//    Q tile, written at a segment's start (every score of the previous segment is done by then).
 //  * Every wait is bounded; a wait that runs out sets PKV_DEVERR_TIMEOUT, every role leaves its
-//    loop, the MMA issuer drains its MMAs, and TMEM is released before the CTA exits.
+//    loop, thread 0 waits for the MMAs it issued, and TMEM is released before the CTA exits.
 #pragma once
 
 #include "decode_mma.cuh"
 
 namespace pkv {
 
-constexpr int kTcUnit = 128;          // tokens per unit
+constexpr int kTcRows = 128;          // cache rows per unit (HPU heads x block_size tokens)
 constexpr int kTcStage = 32768;       // K tile + V tile, 128 rows x 128 bytes each
-constexpr int kTcTmemCols = 64;       // S0 [0,16) S1 [16,32) O0 [32,40) O1 [40,48)
-constexpr int kTcThreads = 192;       // warps 0-3 softmax, 4 producer, 5 MMA issuer
+constexpr int kTcThreads = 224;       // warps 0-3 softmax, 4 producer, 5 scores issuer, 6 p.V issuer
 
 // ------------------------------------------------------------------ tcgen05 wrappers
 
@@ -86,7 +94,8 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16])
+// TMEM loads / stores of this warp's 32 lanes, n consecutive 32-bit columns from `taddr`.
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r)
 {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -96,7 +105,7 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "memory");
 }
 
-__device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t (&r)[8])
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t* r)
 {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
@@ -104,11 +113,57 @@ __device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t (&r)[8])
                  : "memory");
 }
 
-__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&r)[8])
+__device__ __forceinline__ void tc_ld4(uint32_t taddr, uint32_t* r)
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
                  : "memory");
+}
+
+__device__ __forceinline__ void tc_ld2(uint32_t taddr, uint32_t* r)
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr) : "memory");
+}
+
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// n columns (a multiple of 2) in pieces of 16, 8, 4 and 2
+template <int N>
+__device__ __forceinline__ void tc_ld_cols(uint32_t taddr, uint32_t* r)
+{
+    static_assert(N % 2 == 0, "even column count");
+    if constexpr (N >= 16) {
+        tc_ld16(taddr, r);
+        tc_ld_cols<N - 16>(taddr + 16, r + 16);
+    } else if constexpr (N >= 8) {
+        tc_ld8(taddr, r);
+        tc_ld_cols<N - 8>(taddr + 8, r + 8);
+    } else if constexpr (N >= 4) {
+        tc_ld4(taddr, r);
+        tc_ld_cols<N - 4>(taddr + 4, r + 4);
+    } else if constexpr (N >= 2) {
+        tc_ld2(taddr, r);
+    }
+}
+
+// n columns, a multiple of 16
+template <int N>
+__device__ __forceinline__ void tc_st_cols(uint32_t taddr, const uint32_t* r)
+{
+    static_assert(N % 16 == 0, "multiple of 16 columns");
+    if constexpr (N >= 16) {
+        tc_st16(taddr, r);
+        tc_st_cols<N - 16>(taddr + 16, r + 16);
+    }
 }
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -135,90 +190,122 @@ __device__ __forceinline__ uint32_t swz_byte(int r, int b)
     return (uint32_t)(r * 128 + ((((b >> 4) ^ (r & 7)) << 4) | (b & 15)));
 }
 
-// ------------------------------------------------------------------ unit walk
 
-// The CTA's units in order: chunk after chunk (ids from the producer's ring, read once the
-// chunk's first stage has filled), units of a chunk in order, a segment = the units of one
-// stream inside one chunk. Every role walks the same sequence.
-struct TcUnit {
-    int k;            // unit ordinal in the CTA (stage k % S, S/P buffer k & 1)
-    int seg;          // segment ordinal in the CTA (Q/O buffer seg & 1)
-    int chunk;        // chunk id
-    int x;            // unit index
-    int s, h;         // sequence, KV head
-    int u;            // unit within the stream (tokens 128 u ..)
-    int stream_begin, stream_end;
-    bool first, last; // first / last unit of its segment
-};
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t* r)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
 
-struct TcWalk {
-    int ordinal;      // chunks consumed
-    int chunk, x, end;
-    int k, seg;
-    bool done;
+// TMEM loads / stores of n columns (a multiple of 8) in pieces of 8, from an 8-aligned column
+template <int N>
+__device__ __forceinline__ void tc_ld_cols8(uint32_t taddr, uint32_t* r)
+{
+    static_assert(N % 8 == 0, "multiple of 8 columns");
+    if constexpr (N >= 8) {
+        tc_ld8(taddr, r);
+        tc_ld_cols8<N - 8>(taddr + 8, r + 8);
+    }
+}
 
-    __device__ __forceinline__ void init()
+template <int N>
+__device__ __forceinline__ void tc_st_cols8(uint32_t taddr, const uint32_t* r)
+{
+    static_assert(N % 8 == 0, "multiple of 8 columns");
+    if constexpr (N >= 8) {
+        tc_st8(taddr, r);
+        tc_st_cols8<N - 8>(taddr + 8, r + 8);
+    }
+}
+
+// ------------------------------------------------------------------ configuration
+
+template <class KV, class QT, int BS, int G>
+struct TcCfg {
+    static constexpr int HPU = kTcRows / BS;                  // KV heads per unit
+    static constexpr int WH = 32 / BS;                        // heads per softmax warp
+    static constexpr int NO = HPU * G;                        // (head, column) pairs of a unit
+    static constexpr int NOp = (NO + 7) / 8 * 8;              // P^T rows per part = O columns per part
+    static constexpr int kLdS = WH * 2 * G;                   // S columns of one softmax warp's heads
+    static constexpr int kLdSp = (kLdS + 7) / 8 * 8;          // ... padded: each warp's columns start 8-aligned
+    static constexpr int NQ = 4 * kLdSp;                      // Q^T rows = S columns per tile
+    static constexpr int kTmemUsed = 2 * NQ + 2 * NOp;        // S0, S1, O (hi part, lo part)
+    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                                          : kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kQBytes = (NQ * 128 + 1023) / 1024 * 1024;
+    static constexpr int kPBytes = 2 * NOp * 128;             // one buffer: hi rows, then lo rows
+    // one CTA per SM (the occupancy the driver grants a kernel that allocates tensor memory)
+    static constexpr int kCtasPerSm = 1;
+    static constexpr uint32_t kFmt = KV::kFmt == __NV_E5M2 ? 1u : 0u;
+    static_assert(KV::kBytes == 1 && !KV::kInt8, "FP8 caches");
+    static_assert(BS == 16 || BS == 32, "block size");
+    static_assert(G >= 1 && G <= 8, "query columns per KV head");
+    static_assert(kTmemUsed <= 512 && NQ <= 256 && NQ % 16 == 0 && 2 * NOp <= 256, "tensor memory, MMA N");
+    // Q^T row (= S column) of head hl of the unit, part 0 (hi codes) or 1 (lo codes), column c
+    __device__ __forceinline__ static constexpr int qrow(int hl, int part, int c)
     {
-        ordinal = 0;
-        chunk = -1;
-        x = end = 0;
-        k = -1;
-        seg = -1;
-        done = false;
+        return (hl / WH) * kLdSp + (hl % WH) * 2 * G + part * G + c;
     }
 };
+
+// What the producer tells the softmax warps about the unit in a stage (written before the stage's
+// full barrier is signalled).
+struct TcDesc {
+    int s, hg, j, flags;   // sequence, head group, block of the stream, kTc* flags
+    int chunk, L, skip, pad;
+};
+constexpr int kTcFirst = 1;    // first unit of a segment (the units of one stream inside one chunk)
+constexpr int kTcLast = 2;     // last unit of a segment
+constexpr int kTcEnd = 4;      // no unit: the CTA's work is done
+constexpr int kTcBad = 8;      // the block id was out of range: nothing was copied
+constexpr int kTcDirect = 16;  // the stream lies in one chunk: output written directly
 
 // ------------------------------------------------------------------ kernel
 
 template <class KV, class QT, int BS, int G>
-struct TcCfg {
-    static constexpr int kBPU = kTcUnit / BS;       // blocks per unit
-    static constexpr uint32_t kFmt = KV::kFmt == __NV_E5M2 ? 1u : 0u;
-    static_assert(KV::kBytes == 1 && !KV::kInt8, "FP8 caches");
-    static_assert(BS == 16 || BS == 32, "block size");
-    static_assert(G <= 8, "query columns per KV head");
-};
-
-template <class KV, class QT, int BS, int G>
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kTcThreads, (TcCfg<KV, QT, BS, G>::kCtasPerSm))
     paged_decode_tc05_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                              const DecodeParams p)
 {
     using C = TcCfg<KV, QT, BS, G>;
     constexpr int D = 128;
+    constexpr int HPU = C::HPU, NO = C::NO, NOp = C::NOp, NQ = C::NQ;
     constexpr float kSlack = 2.0f;     // log2 units
     constexpr float kPOff = 6.0f;      // p * 2^6 enters the products
     const int S = p.stages_per_warp;
     const int Hkv = p.num_kv_heads;
+    const int NHG = Hkv / HPU;
     const int capacity = p.max_blocks_per_seq * BS;
     const int QL = p.q_len > 1 ? p.q_len : 1;
     const int Gq = p.num_heads / p.num_kv_heads;
 
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* stages = smem;                                        // [S][32 KB]
-    uint8_t* qtile = stages + (size_t)S * kTcStage;                // [2][2 KB]
-    uint8_t* ptile = qtile + 2 * 2048;                             // [2][2 KB]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(ptile + 2 * 2048);
-    uint64_t* full = bars;                    // [S]
-    uint64_t* empty = full + S;               // [S]
-    uint64_t* s_full = empty + S;             // [2]
-    uint64_t* s_empty = s_full + 2;           // [2]
-    uint64_t* p_full = s_empty + 2;           // [2]
-    uint64_t* p_empty = p_full + 2;           // [2]
-    uint64_t* o_full = p_empty + 2;           // [2]
-    uint64_t* o_empty = o_full + 2;           // [2]
-    uint64_t* q_full = o_empty + 2;           // [2]
-    uint64_t* q_empty = q_full + 2;           // [2]
-    uint64_t* drain = q_empty + 2;            // [1]
-    uint64_t* gbar = drain + 1;               // [1] the four softmax warps' group barrier
-    int* stage_bad = reinterpret_cast<int*>(gbar + 1);             // [S] bad-block bit masks
-    int* chunk_ring = stage_bad + S;                               // [kChunkRing]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(chunk_ring + kChunkRing);
+    uint8_t* qtile = stages + (size_t)S * kTcStage;                // Q^T: NQ rows of 128 bytes
+    uint8_t* ptile = qtile + C::kQBytes;                           // [2] P^T: NOp hi rows, NOp lo rows
+    TcDesc* desc = reinterpret_cast<TcDesc*>(ptile + 2 * C::kPBytes);   // [S]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(desc + S);
+    uint64_t* full = bars;                    // [S] the stage's copies have landed
+    uint64_t* empty = full + S;               // [S] the stage's products are done
+    uint64_t* s_full = empty + S;             // [2] the scores are in S tile b
+    uint64_t* s_empty = s_full + 2;           // [2] every softmax warp has read S tile b
+    uint64_t* p_full = s_empty + 2;           // [2] every softmax warp has written P
+    uint64_t* p_empty = p_full + 2;           // [2] the p.V product reading P is done
+    uint64_t* o_full = p_empty + 2;           // [1] the segment's last p.V is done
+    uint64_t* o_empty = o_full + 1;           // [1] every softmax warp has read O
+    uint64_t* q_full = o_empty + 1;           // [1] the segment's Q tile is written
+    uint64_t* drain = q_full + 1;             // [2] each issuer's MMAs are done
+    uint64_t* gbar = drain + 2;               // [1] the four softmax warps' group barrier
+    int2* info = reinterpret_cast<int2*>(gbar + 1);                // [num_seqs] (tokens, skipped blocks)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(info + p.num_seqs);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* red = reinterpret_cast<float*>(tmem_slot + 2);          // [4][8] cross-warp reductions
-    float* colq = red + 32;                                        // [2][8] per-column score factors
-    int* votes = reinterpret_cast<int*>(colq + 16);                // [2][4] lazy-max votes per warp
-    int* prefix = votes + 8;                                       // [num_seqs + 1]
+    int* votes = reinterpret_cast<int*>(tmem_slot + 2);            // [2][4] lazy-max votes per warp
+    float* colq = reinterpret_cast<float*>(votes + 8);             // [NO] score factor per (head, column)
+    float* ash = colq + NO;                                        // [NO] rescale factors
+    float* msh = ash + NO;                                         // [NO] running max at a segment's end
+    float* lsh = msh + NO;                                         // [NO] weight sums at a segment's end
+    int* prefix = reinterpret_cast<int*>(lsh + NO);                // [num_seqs + 1]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -233,28 +320,27 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             mbar_init(&s_empty[i], 4);
             mbar_init(&p_full[i], 4);
             mbar_init(&p_empty[i], 1);
-            mbar_init(&o_full[i], 1);
-            mbar_init(&o_empty[i], 4);
-            mbar_init(&q_full[i], 4);
-            mbar_init(&q_empty[i], 1);
+            mbar_init(&drain[i], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, 4);
+        mbar_init(q_full, 1);
         mbar_init(gbar, 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
-                     "r"(kTcTmemCols)
+                     "r"(C::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // tiles read by the tensor cores start as zeros (rows no copy fills must not hold NaN codes)
-    for (int i = tid; i < (S * kTcStage + 4 * 2048) / 16; i += kTcThreads)
-        reinterpret_cast<uint4*>(stages)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // Q^T padding rows and the off-diagonal bytes of P^T are read by the tensor cores as zeros
+    for (int i = tid; i < (C::kQBytes + 2 * C::kPBytes) / 16; i += kTcThreads)
+        reinterpret_cast<uint4*>(qtile)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
     {
-        const int bad = build_unit_prefix(p, prefix, BS, Hkv, capacity, kTcUnit);   // ends with __syncthreads
+        const int bad = build_unit_prefix(p, prefix, BS, NHG, capacity, BS, info);   // ends with __syncthreads
         if (bad && blockIdx.x == 0 && tid == 0)
             atomicOr(p.err, bad);
     }
@@ -264,19 +350,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const int total = prefix[p.num_seqs];
     const int nruns = gridDim.x;
-    const Chunks ch = make_chunks(total, nruns, p.tail_chunks);
+    const Chunks ch = make_chunks(total, nruns, p.tail_chunks, p.tail_min_units, p.tail_min_chunk);
 
     // zero rows of empty sequences (one run per sequence)
     for (int s = blockIdx.x; s < p.num_seqs; s += nruns) {
         if (prefix[s + 1] == prefix[s]) {
             if (tid == 0 && p.new_k != nullptr && __ldg(p.new_slots + s) >= 0)
                 atomicOr(p.err, PKV_DEVERR_SLOT);
-            if (p.skip_blocks != nullptr) {
-                int skipb, e = 0;
-                (void)stream_tokens(p, s, BS, capacity, skipb, e);
-                if (skipb > 0)
-                    continue;
-            }
+            if (info[s].y > 0)
+                continue;
             const int rows = p.num_heads * QL;
             QT* o = reinterpret_cast<QT*>(p.out) + (size_t)s * rows * D;
             for (int i = tid; i < rows * D; i += kTcThreads)
@@ -290,142 +372,104 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             atomicOr(p.err, PKV_DEVERR_TIMEOUT);
         }
     };
-    // next unit of the walk (false at the end of the CTA's work or on a failed wait); a chunk's
-    // id is read once the chunk's first stage has filled
-    auto next_unit = [&](TcWalk& w, TcUnit& u) -> bool {
-        if (w.done)
-            return false;
-        if (w.x >= w.end) {
-            const int kk = w.k + 1;
-            if (*abort_flag || !mbar_wait_bounded(&full[kk % S], (kk / S) & 1)) {
-                fail();
-                w.done = true;
-                return false;
-            }
-            const int c = chunk_ring[w.ordinal % kChunkRing];
-            ++w.ordinal;
-            if (c < 0 || c >= ch.C) {
-                w.done = true;
-                return false;
-            }
-            w.chunk = c;
-            w.x = ch.begin(c);
-            w.end = ch.end(c);
-        }
-        u.k = ++w.k;
-        u.chunk = w.chunk;
-        u.x = w.x;
-        u.s = find_seq(prefix, p.num_seqs, w.x);
-        const int nu = (prefix[u.s + 1] - prefix[u.s]) / Hkv;
-        const int r = w.x - prefix[u.s];
-        u.h = r / nu;
-        u.u = r - u.h * nu;
-        u.stream_begin = prefix[u.s] + u.h * nu;
-        u.stream_end = u.stream_begin + nu;
-        u.first = w.x == ch.begin(w.chunk) || w.x == u.stream_begin;
-        u.last = w.x + 1 == w.end || w.x + 1 == u.stream_end;
-        if (u.first)
-            ++w.seg;
-        u.seg = w.seg;
-        ++w.x;
-        return true;
-    };
 
     if (warp == 4) {
         // =========================== producer ===============================
+        // Units are resolved 32 at a time, one per lane; the next 32 table entries are loaded
+        // while these units' copies are issued. Each stage gets the unit's descriptor.
         if (lane == 0) {
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
         }
+        struct Look {
+            int s, hg, j, nbl, phys, flags;
+            bool has;
+        };
+        // unit x0 + lane of chunk [cb, ce): sequence, head group, block of the stream, blocks of the
+        // stream, the raw table entry and the segment flags
+        auto look = [&](int x0, int cb, int ce) -> Look {
+            Look r{0, 0, 0, 0, 0, 0, false};
+            const int x = x0 + lane;
+            if (x < ce) {
+                r.s = find_seq(prefix, p.num_seqs, x);
+                const int nu = (prefix[r.s + 1] - prefix[r.s]) / NHG;
+                const int rr = x - prefix[r.s];
+                r.hg = rr / nu;
+                r.j = rr - r.hg * nu;
+                r.nbl = nu;
+                r.has = true;
+                const int skip = info[r.s].y;
+                r.phys = __ldg(p.block_tables + (long long)r.s * p.max_blocks_per_seq + skip + r.j);
+                const int sb = x - r.j;   // the stream's first unit
+                r.flags = (x == cb || r.j == 0 ? kTcFirst : 0) | (x + 1 == ce || r.j == nu - 1 ? kTcLast : 0) |
+                          (ch.of(sb) == ch.of(sb + nu - 1) && skip == 0 ? kTcDirect : 0);
+            }
+            return r;
+        };
         int cur = blockIdx.x;
         int nxt = ch.C;
         if (lane == 0 && ch.C > ch.R)
             nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
         bool aborted = false;
-        int k = 0, issued = 0, published = 0;
+        int k = 0, issued = 0;
         while (cur < ch.C && !aborted) {
             const int cb = ch.begin(cur), ce = ch.end(cur);
-            if (ce > cb) {
-                if (lane == 0)
-                    chunk_ring[published % kChunkRing] = cur;
-                ++published;
-            }
-            for (int x = cb; x < ce && !aborted; ++x, ++k) {
-                const int s = find_seq(prefix, p.num_seqs, x);
-                const int nu = (prefix[s + 1] - prefix[s]) / Hkv;
-                const int r = x - prefix[s];
-                const int h = r / nu, uu = r - h * nu;
-                int skipb = 0, L = 0;
-                {
-                    int e = 0;
-                    L = stream_tokens(p, s, BS, capacity, skipb, e);
-                }
-                const int nbl = (L + BS - 1) / BS;               // blocks of the stream
-                const int j0 = uu * C::kBPU;
-                // lane b < kBPU: block j0 + b of the stream -> pool row, -1 when past the stream or bad
-                int row = -1, bad = 0;
-                if (lane < C::kBPU && j0 + lane < nbl) {
-                    const int phys = __ldg(p.block_tables + (long long)s * p.max_blocks_per_seq + skipb + j0 + lane);
-                    if (phys < 0 || phys >= p.num_blocks) {
-                        atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
-                        bad = 1;
-                    } else {
-                        row = (phys * Hkv + h) * BS;
+            Look lk = look(cb, cb, ce);
+            for (int x0 = cb; x0 < ce && !aborted; x0 += 32) {
+                const Look nx = look(x0 + 32, cb, ce);   // loads in flight while this batch is issued
+                const bool bad = lk.has && (lk.phys < 0 || lk.phys >= p.num_blocks);
+                if (bad)
+                    atomicOr(p.err, PKV_DEVERR_BLOCK_ID);
+                // first cache row of the unit: block phys, KV head hg * HPU, token 0
+                const int row = lk.has && !bad ? (lk.phys * Hkv + lk.hg * HPU) * BS : -1;
+                const int nb = ce - x0 < 32 ? ce - x0 : 32;
+                for (int q = 0; q < nb && !aborted; ++q, ++k) {
+                    const int sq = __shfl_sync(kFullMask, lk.s, q), hgq = __shfl_sync(kFullMask, lk.hg, q);
+                    const int jq = __shfl_sync(kFullMask, lk.j, q), nblq = __shfl_sync(kFullMask, lk.nbl, q);
+                    const int rowq = __shfl_sync(kFullMask, row, q), fq = __shfl_sync(kFullMask, lk.flags, q);
+                    // the decode-step append of this stream's heads, before its last block is read
+                    if (p.new_k != nullptr && jq == nblq - 1)
+                        append_new_token_impl<KV>(p, sq, hgq * HPU, HPU, D, BS, lane, rowq < 0 ? -1 : rowq / (Hkv * BS));
+                    if (lane == 0) {
+                        const int st = k % S;
+                        if (*abort_flag) {
+                            aborted = true;
+                        } else if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
+                            aborted = true;
+                            fail();
+                        } else if (p.withheld_unit != 0 && x0 + q == p.withheld_unit - 1) {
+                            aborted = true;   // test hook: this stage never fills; issue nothing more
+                        } else {
+                            const int2 inf = info[sq];
+                            reinterpret_cast<int4*>(desc + st)[0] = make_int4(sq, hgq, jq, fq | (rowq < 0 ? kTcBad : 0));
+                            reinterpret_cast<int4*>(desc + st)[1] = make_int4(cur, inf.x, inf.y, 0);
+                            if (rowq < 0) {
+                                mbar_arrive(&full[st]);
+                            } else {
+                                mbar_arrive_expect_tx(&full[st], (uint32_t)kTcStage);
+                                uint8_t* dst = stages + (size_t)st * kTcStage;
+                                tma_load_2d(dst, &kmap, 0, rowq, &full[st]);
+                                tma_load_2d(dst + kTcStage / 2, &vmap, 0, rowq, &full[st]);
+                            }
+                            issued = k + 1;
+                        }
                     }
+                    aborted = __shfl_sync(kFullMask, aborted ? 1 : 0, 0) != 0;
                 }
-                const unsigned badmask = __ballot_sync(kFullMask, bad != 0);
-                const unsigned loadmask = __ballot_sync(kFullMask, row >= 0);
-                // the decode-step append of this stream, before its last block is read
-                if (p.new_k != nullptr && j0 + C::kBPU >= nbl && nbl > 0) {
-                    const int lastrow = __shfl_sync(kFullMask, row, (nbl - 1 - j0) & 31);
-                    append_new_token_impl<KV>(p, s, h, 1, D, BS, lane, lastrow < 0 ? -1 : lastrow / (Hkv * BS));
-                }
-                if (lane == 0) {
-                    const int st = k % S;
-                    if (*abort_flag) {
-                        aborted = true;
-                    } else if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
-                        aborted = true;
-                        fail();
-                    } else if (p.withheld_unit != 0 && x == p.withheld_unit - 1) {
-                        aborted = true;   // test hook: this stage never fills; issue nothing more
-                    } else {
-                        stage_bad[st] = (int)badmask;
-                        const int n = __popc(loadmask);
-                        if (n == 0)
-                            mbar_arrive(&full[st]);
-                        else
-                            mbar_arrive_expect_tx(&full[st], (uint32_t)n * BS * 128 * 2);
-                        issued = k + 1;
-                    }
-                }
-                // the copies (lane 0 issues; rows broadcast from the lanes that resolved them)
-                const int st = k % S;
-                const bool go = __shfl_sync(kFullMask, (int)(!aborted && issued == k + 1), 0) != 0;
-                aborted = __shfl_sync(kFullMask, aborted ? 1 : 0, 0) != 0;
-#pragma unroll
-                for (int b = 0; b < C::kBPU; ++b) {
-                    const int rb = __shfl_sync(kFullMask, row, b);
-                    if (go && lane == 0 && rb >= 0) {
-                        uint8_t* dst = stages + (size_t)st * kTcStage + b * BS * 128;
-                        tma_load_2d(dst, &kmap, 0, rb, &full[st]);
-                        tma_load_2d(dst + kTcStage / 2, &vmap, 0, rb, &full[st]);
-                    }
-                }
+                lk = nx;
             }
             cur = __shfl_sync(kFullMask, nxt, 0);
             if (lane == 0 && cur < ch.C)
                 nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
         }
-        // end of the work: a stage without bytes whose chunk id is -1 tells the other roles
+        // end of the work: a stage without bytes whose descriptor says so
         if (lane == 0 && !aborted) {
             const int st = k % S;
             if (k >= S && !mbar_wait_bounded(&empty[st], ((k / S) - 1) & 1)) {
                 aborted = true;
                 fail();
             } else {
-                chunk_ring[published % kChunkRing] = -1;
-                stage_bad[st] = 0;
+                reinterpret_cast<int4*>(desc + st)[0] = make_int4(0, 0, 0, kTcEnd);
                 mbar_arrive(&full[st]);
             }
         }
@@ -434,91 +478,109 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 (void)mbar_wait_bounded(&full[kk % S], (kk / S) & 1);
         }
     } else if (warp == 5) {
-        // =========================== MMA issuer ==============================
+        // =========================== scores issuer ===========================
+        // S = K Q^T of every unit in order into S tile k & 1: once its tiles have landed, the
+        // softmax warps have read that tile (unit k - 2) and (a segment's first unit) the
+        // segment's Q tile is written.
         if (lane == 0) {
-            const uint32_t id_qk = tc_idesc(C::kFmt, 0u, 0u, 16, 128);
-            const uint32_t id_pv = tc_idesc(C::kFmt, 0u, 1u, 8, 128);
-            TcWalk wq, wp;
-            wq.init();
-            wp.init();
-            TcUnit uq, up;
-            auto issue_qk = [&](const TcUnit& u) -> bool {
-                const int st = u.k % S, b = u.k & 1, n = u.k >> 1, j = u.seg & 1;
-                // next_unit already waited for the first stage of a chunk; wait for this one
-                if (!mbar_wait_bounded(&full[st], (u.k / S) & 1))
-                    return false;
-                if (n >= 1 && !mbar_wait_bounded(&s_empty[b], (n - 1) & 1))
-                    return false;
-                if (u.first && !mbar_wait_bounded(&q_full[j], (u.seg >> 1) & 1))
-                    return false;
-                tc_fence_after();
-                const uint32_t kbase = smem_addr(stages + (size_t)st * kTcStage);
-                const uint32_t qbase = smem_addr(qtile + j * 2048);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc_mma(tmem + 16u * b, tc_sdesc(kbase + ks * 32, 1024), tc_sdesc(qbase + ks * 32, 1024), id_qk,
-                           ks > 0 ? 1u : 0u);
-                tc_commit(&s_full[b]);
-                if (u.last)
-                    tc_commit(&q_empty[j]);
-                return true;
-            };
+            const uint32_t id_qk = tc_idesc(C::kFmt, 0u, 0u, NQ, 128);   // M 128 rows, N (head, hi/lo, column)
+            const uint64_t q_desc = tc_sdesc(smem_addr(qtile), 1024);
+            int seg = 0;
             bool ok = true;
-            bool have_q = next_unit(wq, uq);
-            if (have_q)
-                ok = issue_qk(uq);
-            while (ok && next_unit(wp, up)) {
-                if (next_unit(wq, uq))
-                    ok = issue_qk(uq);
-                if (!ok)
-                    break;
-                const int st = up.k % S, b = up.k & 1, n = up.k >> 1, j = up.seg & 1;
-                if (!mbar_wait_bounded(&p_full[b], n & 1)) {
+            for (int k = 0; ok; ++k) {
+                const int st = k % S;
+                if (!mbar_wait_bounded(&full[st], (k / S) & 1)) {
                     ok = false;
                     break;
                 }
-                if (up.first && up.seg >= 2 && !mbar_wait_bounded(&o_empty[j], ((up.seg >> 1) - 1) & 1)) {
+                const int flags = reinterpret_cast<const int4*>(desc + st)[0].w;
+                if (flags & kTcEnd)
+                    break;
+                if ((k >= 2 && !mbar_wait_bounded(&s_empty[k & 1], ((k >> 1) - 1) & 1)) ||
+                    ((flags & kTcFirst) && !mbar_wait_bounded(q_full, seg & 1))) {
                     ok = false;
                     break;
                 }
+                if (flags & kTcFirst)
+                    ++seg;
                 tc_fence_after();
-                const uint32_t vbase = smem_addr(stages + (size_t)st * kTcStage + kTcStage / 2);
-                const uint32_t pbase = smem_addr(ptile + b * 2048);
-                const uint32_t od = tmem + 32u + 8u * j;
+                const uint64_t k_desc = tc_sdesc(smem_addr(stages + (size_t)st * kTcStage), 1024);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t a = tc_sdesc(vbase + ks * 4096, 1024);
-                    tc_mma(od, a, tc_sdesc(pbase + ks * 32, 1024), id_pv, (up.first && ks == 0) ? 0u : 1u);
-                    tc_mma(od, a, tc_sdesc(pbase + 1024 + ks * 32, 1024), id_pv, 1u);
-                }
-                tc_commit(&empty[st]);
-                tc_commit(&p_empty[b]);
-                if (up.last)
-                    tc_commit(&o_full[j]);
+                for (int ks = 0; ks < 4; ++ks)   // K steps of 32 bytes of d: start address + 32 bytes
+                    tc_mma(tmem + (uint32_t)((k & 1) * NQ), k_desc + 2 * ks, q_desc + 2 * ks, id_qk, ks > 0 ? 1u : 0u);
+                tc_commit(&s_full[k & 1]);
             }
             if (!ok)
                 fail();
-            // every MMA issued has completed before TMEM is released
-            tc_commit(drain);
-            (void)mbar_wait_bounded(drain, 0);
+            tc_commit(&drain[0]);   // every MMA issued has completed before TMEM is released
+            (void)mbar_wait_bounded(&drain[0], 0);
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // =========================== p.V issuer ==============================
+        // O^T += V^T [P_hi^T | P_lo^T] of every unit in order, once the softmax warps have written
+        // its weights (a segment's first unit: once they have read the previous segment's O); its
+        // completion frees the stage and the P buffer.
+        if (lane == 0) {
+            const uint32_t id_pv = tc_idesc(C::kFmt, 0u, 1u, 2 * NOp, 128);   // M 128 d (V^T MN-major)
+            const uint32_t od = tmem + (uint32_t)(2 * NQ);
+            int seg = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int st = k % S, b = k & 1;
+                if (!mbar_wait_bounded(&full[st], (k / S) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int flags = reinterpret_cast<const int4*>(desc + st)[0].w;
+                if (flags & kTcEnd)
+                    break;
+                const bool first = (flags & kTcFirst) != 0;
+                if (!mbar_wait_bounded(&p_full[b], (k >> 1) & 1) ||
+                    (first && seg >= 1 && !mbar_wait_bounded(o_empty, (seg - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                if (first)
+                    ++seg;
+                tc_fence_after();
+                const uint64_t v_desc = tc_sdesc(smem_addr(stages + (size_t)st * kTcStage + kTcStage / 2), 1024);
+                const uint64_t p_desc = tc_sdesc(smem_addr(ptile + b * C::kPBytes), 1024);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // 32 tile rows per step: V + 4096 bytes, P + 32 bytes
+                    tc_mma(od, v_desc + 256 * ks, p_desc + 2 * ks, id_pv, (first && ks == 0) ? 0u : 1u);
+                tc_commit(&empty[st]);
+                tc_commit(&p_empty[b]);
+                if (flags & kTcLast)
+                    tc_commit(o_full);
+            }
+            if (!ok)
+                fail();
+            tc_commit(&drain[1]);
+            (void)mbar_wait_bounded(&drain[1], 0);
         }
         __syncwarp();
     } else {
         // =========================== softmax warps ===========================
-        const float qk_head_scale = p.q_scale;   // per-tensor factor (head scales applied per stream)
-        TcWalk w;
-        w.init();
-        TcUnit u;
-        float m[8], lp[8], qk[8];
-        int lim[8];
+        const int hl = tid / BS, t = tid - (tid / BS) * BS;            // this thread's tile row
+        // this row's bytes of P^T (rows (hl, c), hi then lo; the byte is the tile row)
+        uint32_t poh[G], pol[G];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < G; ++c) {
+            poh[c] = swz_byte(hl * G + c, tid);
+            pol[c] = swz_byte(NOp + hl * G + c, tid);
+        }
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t o_hi = tmem + (uint32_t)(2 * NQ) + lane_base, o_lo = o_hi + (uint32_t)NOp;   // row d = tid of O
+        float m[G], lp[G], qk[G];
+        int lim[G];
+#pragma unroll
+        for (int c = 0; c < G; ++c) {
             m[c] = -INFINITY;
             lp[c] = 0.f;
             qk[c] = 0.f;
             lim[c] = 0;
         }
-        int q_written = -1;   // last segment whose Q tile is written
         // Barrier of the four softmax warps with a bounded wait (an mbarrier, one arrival per warp;
         // a warp is never more than one phase ahead). No wait here can block for good: a warp
         // whose wait runs out leaves, and the others' waits run out in turn.
@@ -533,104 +595,135 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 fail();
             return __all_sync(kFullMask, okg);
         };
-        // Q tile of segment u.seg: thread i -> column i >> 4, d (i & 15) * 8 .. + 7
-        auto write_q = [&](const TcUnit& uu) -> bool {
-            const int j = uu.seg & 1;
-            if (uu.seg >= 2 && !mbar_wait_bounded(&q_empty[j], ((uu.seg >> 1) - 1) & 1))
-                return false;
-            const int c = tid >> 4, d0 = (tid & 15) * 8;
-            float f[8];
-            if (c < G) {
-                const QT* qp = reinterpret_cast<const QT*>(p.q) + query_row(p, uu.s, uu.h, c) * D + d0;
-                load_q<8>(qp, f);
-            } else {
+        // Q^T of stream (s, hg): rows (head h2, hi / lo part, column c) at C::qrow, 16 threads per
+        // (head, column) pair, 8 d each; colq = the pair's score factor (scale, log2 e, K scale,
+        // 1 / sigma)
+        auto write_q = [&](int s, int hg) {
+            for (int task = tid; task < NO * 16; task += 128) {
+                const int nn = task >> 4, d0 = (task & 15) * 8;
+                const int h2 = nn / G, c = nn - (nn / G) * G;
+                const int head = hg * HPU + h2;
+                float f[8];
+                load_q<8>(reinterpret_cast<const QT*>(p.q) + query_row(p, s, head, c) * D + d0, f);
+                float mx = 0.f;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    f[i] = 0.f;
-            }
-            float mx = 0.f;
+                    mx = fmaxf(mx, fabsf(f[i]));
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                mx = fmaxf(mx, fabsf(f[i]));
+                for (int off = 1; off < 16; off <<= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
+                // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
+                int se = 127;
+                if (mx > 0.f) {
+                    se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
+                    se = se < 2 ? 2 : (se > 252 ? 252 : se);
+                }
+                const float sig = __uint_as_float((uint32_t)se << 23);
+                const float inv_sig = __uint_as_float((uint32_t)(254 - se) << 23);
+                uint32_t hw[2], lw[2];
 #pragma unroll
-            for (int off = 1; off < 16; off <<= 1)
-                mx = fmaxf(mx, __shfl_xor_sync(kFullMask, mx, off));
-            // mx < 2^(E - 126) with E its biased exponent; sigma = 2^(134 - E), kept normal both ways
-            int se = 127;
-            if (mx > 0.f) {
-                se = 127 + 134 - (int)((__float_as_uint(mx) >> 23) & 0xffu);
-                se = se < 2 ? 2 : (se > 252 ? 252 : se);
+                for (int i = 0; i < 2; ++i) {
+                    uint32_t h01, l01, h23, l23;
+                    split_e4m3x2(pack2<true>(f[4 * i] * sig, f[4 * i + 1] * sig), h01, l01);
+                    split_e4m3x2(pack2<true>(f[4 * i + 2] * sig, f[4 * i + 3] * sig), h23, l23);
+                    hw[i] = h01 | (h23 << 16);
+                    lw[i] = l01 | (l23 << 16);
+                }
+                *reinterpret_cast<uint2*>(qtile + swz_byte(C::qrow(h2, 0, c), d0)) = make_uint2(hw[0], hw[1]);
+                *reinterpret_cast<uint2*>(qtile + swz_byte(C::qrow(h2, 1, c), d0)) = make_uint2(lw[0], lw[1]);
+                if ((task & 15) == 0) {
+                    const float hs = p.k_head_scales ? __ldg(p.k_head_scales + head) : 1.0f;
+                    colq[nn] = p.q_scale * hs * inv_sig;
+                }
             }
-            const float sig = __uint_as_float((uint32_t)se << 23);
-            const float inv_sig = __uint_as_float((uint32_t)(254 - se) << 23);
-            uint32_t hw[2], lw[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                uint32_t h01, l01, h23, l23;
-                split_e4m3x2(pack2<true>(f[4 * i] * sig, f[4 * i + 1] * sig), h01, l01);
-                split_e4m3x2(pack2<true>(f[4 * i + 2] * sig, f[4 * i + 3] * sig), h23, l23);
-                hw[i] = h01 | (h23 << 16);
-                lw[i] = l01 | (l23 << 16);
-            }
-            uint8_t* qt = qtile + j * 2048;
-            *reinterpret_cast<uint2*>(qt + swz_byte(c, d0)) = make_uint2(hw[0], hw[1]);
-            *reinterpret_cast<uint2*>(qt + swz_byte(8 + c, d0)) = make_uint2(lw[0], lw[1]);
-            const float hs = p.k_head_scales ? __ldg(p.k_head_scales + uu.h) : 1.0f;
-            if ((tid & 15) == 0)
-                colq[j * 8 + c] = qk_head_scale * hs * inv_sig;
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&q_full[j]);
-            return true;
+            fence_proxy_async_smem();   // read by the tensor cores once q_full is signalled
         };
-        bool ok = next_unit(w, u);
-        if (ok)
-            ok = write_q(u);
-        if (ok)
-            q_written = u.seg;
-        while (ok) {
-            const int st = u.k % S, b = u.k & 1, n = u.k >> 1, j = u.seg & 1;
-            int skipb = 0, L = 0;
-            {
-                int e = 0;
-                L = stream_tokens(p, u.s, BS, capacity, skipb, e);
+        int nseg = 0;      // segments finished (O tile phases)
+        // Two units per iteration (unit k and, when k is not the last of its segment, unit k + 1 of
+        // the same stream): the syncs, fences and waits of an iteration are paid once for both.
+        for (int k = 0;;) {
+            const int st0 = k % S;
+            if (!mbar_wait_bounded(&full[st0], (k / S) & 1)) {
+                fail();
+                break;
             }
-            if (u.first) {
-                // the segment's column factors and limits (column c: new token c / Gq of q_len)
-                if (!group_sync())   // colq of this segment written by write_q
+            // the units (their stages' copies are done: the V rows below are read and written after them)
+            const int4 da = reinterpret_cast<const int4*>(desc + st0)[0];
+            const int4 db = reinterpret_cast<const int4*>(desc + st0)[1];
+            const int flags = da.w;
+            if (flags & kTcEnd)
+                break;
+            const int s = da.x, hg = da.y, chunk = db.x, L = db.y;
+            const bool first = (flags & kTcFirst) != 0;
+            const int nu = (flags & kTcLast) ? 1 : 2;   // units this iteration
+            const int st1 = (k + 1) % S;
+            int flags1 = kTcLast, j1 = 0;
+            if (nu == 2) {
+                if (!mbar_wait_bounded(&full[st1], ((k + 1) / S) & 1)) {
+                    fail();
                     break;
+                }
+                const int4 d1 = reinterpret_cast<const int4*>(desc + st1)[0];
+                flags1 = d1.w;
+                j1 = d1.z;
+            }
+            const bool last = (flags1 & kTcLast) != 0;
+            if (first) {
+                // a new stream: its Q tile (the previous segment's scores are all done: their S tiles
+                // were read) and the column factors and limits (column c: new token c / Gq of q_len)
+                write_q(s, hg);
+                if (!group_sync())
+                    break;
+                if (tid == 0)
+                    mbar_arrive(q_full);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    qk[c] = colq[j * 8 + c];
-                    lim[c] = c < G ? L - QL + 1 + c / Gq : 0;
+                for (int c = 0; c < G; ++c) {
+                    qk[c] = colq[hl * G + c];
+                    lim[c] = L - QL + 1 + c / Gq;
                     m[c] = -INFINITY;
                     lp[c] = 0.f;
                 }
             }
-            // ---- scores of token tid of this unit (the stage's copies are done: stage_bad and the V
-            // rows below are read and written after them)
-            if (!mbar_wait_bounded(&full[st], (u.k / S) & 1) || !mbar_wait_bounded(&s_full[b], n & 1)) {
+            // ---- this row's scores in both units: the warp's heads' columns, then this head's hi and lo
+            const int b0 = k & 1, b1 = (k + 1) & 1;
+            if (!mbar_wait_bounded(&s_full[b0], (k >> 1) & 1) ||
+                (nu == 2 && !mbar_wait_bounded(&s_full[b1], ((k + 1) >> 1) & 1))) {
                 fail();
                 break;
             }
             tc_fence_after();
-            uint32_t r[16];
-            tc_ld16(tmem + 16u * b + ((uint32_t)(warp * 32) << 16), r);
+            uint32_t r0[C::kLdSp], r1[C::kLdSp];
+            tc_ld_cols8<C::kLdSp>(tmem + (uint32_t)(b0 * NQ + warp * C::kLdSp) + lane_base, r0);
+            if (nu == 2)
+                tc_ld_cols8<C::kLdSp>(tmem + (uint32_t)(b1 * NQ + warp * C::kLdSp) + lane_base, r1);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&s_empty[b]);
-            const int pos = u.u * kTcUnit + tid;
-            const bool valid = pos < L && !((stage_bad[st] >> (tid / BS)) & 1);
-            float sc[8];
+            if (lane == 0) {
+                mbar_arrive(&s_empty[b0]);
+                if (nu == 2)
+                    mbar_arrive(&s_empty[b1]);
+            }
+            const bool valid0 = da.z * BS + t < L && (flags & kTcBad) == 0;
+            const bool valid1 = nu == 2 && j1 * BS + t < L && (flags1 & kTcBad) == 0;
+            float sc0[G], sc1[G];
             bool exceed = false;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float raw = __uint_as_float(r[c]) + __uint_as_float(r[8 + c]);
-                sc[c] = (valid && pos < lim[c]) ? raw * qk[c] : -INFINITY;
-                exceed |= sc[c] > m[c] + kSlack;
+            for (int c = 0; c < G; ++c) {
+                uint32_t h0 = r0[c], l0 = r0[G + c], h1 = r1[c], l1 = r1[G + c];
+                if constexpr (C::WH == 2) {
+                    if (lane >= 16) {
+                        h0 = r0[2 * G + c];
+                        l0 = r0[3 * G + c];
+                        h1 = r1[2 * G + c];
+                        l1 = r1[3 * G + c];
+                    }
+                }
+                sc0[c] = (valid0 && da.z * BS + t < lim[c]) ? (__uint_as_float(h0) + __uint_as_float(l0)) * qk[c]
+                                                            : -INFINITY;
+                sc1[c] = (valid1 && j1 * BS + t < lim[c]) ? (__uint_as_float(h1) + __uint_as_float(l1)) * qk[c]
+                                                          : -INFINITY;
+                exceed |= fmaxf(sc0[c], sc1[c]) > m[c] + kSlack;
             }
             {
                 const int vote = __any_sync(kFullMask, exceed);
@@ -642,75 +735,96 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 break;
             const int any = votes[vb] | votes[vb + 1] | votes[vb + 2] | votes[vb + 3];
             if (any) {
-                // new reference: the 128 tokens' max per column where it passes the old one by the slack
+                // new reference per (head, column): the blocks' max where it passes the old one by
+                // the slack (a head's tokens are lanes of one warp)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float v = sc[c];
+                for (int c = 0; c < G; ++c) {
+                    float v = fmaxf(sc0[c], sc1[c]);
 #pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1)
+                    for (int off = BS / 2; off >= 1; off >>= 1)
                         v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
-                    if (lane == 0)
-                        red[warp * 8 + c] = v;
+                    float a = 1.f;
+                    if (v > m[c] + kSlack) {
+                        a = m[c] == -INFINITY ? 1.f : fast_exp2(m[c] - v);
+                        m[c] = v;
+                    }
+                    lp[c] *= a;
+                    if (t == 0)
+                        ash[hl * G + c] = a;
                 }
                 if (!group_sync())
                     break;
-                float a[8];
-                bool rescale = false;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float M = fmaxf(fmaxf(red[c], red[8 + c]), fmaxf(red[16 + c], red[24 + c]));
-                    a[c] = 1.f;
-                    if (M > m[c] + kSlack) {
-                        a[c] = m[c] == -INFINITY ? 1.f : fast_exp2(m[c] - M);
-                        rescale |= m[c] != -INFINITY;
-                        m[c] = M;
-                    }
-                    lp[c] *= a[c];
-                }
-                if (!group_sync())   // red reused later
-                    break;
-                if (rescale && !u.first) {
-                    // O holds the segment's earlier units: scale it once their p.V products are done
-                    const int kp = u.k - 1;
+                if (!first) {
+                    // O holds the segment's earlier blocks: scale row d's columns once their p.V is done
+                    const int kp = k - 1;
                     if (!mbar_wait_bounded(&p_empty[kp & 1], (kp >> 1) & 1)) {
                         fail();
                         break;
                     }
                     tc_fence_after();
-                    uint32_t o[8];
-                    const uint32_t ot = tmem + 32u + 8u * j + ((uint32_t)(warp * 32) << 16);
-                    tc_ld8(ot, o);
-                    tc_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        o[c] = __float_as_uint(__uint_as_float(o[c]) * a[c]);
-                    tc_st8(ot, o);
+                    for (int c0 = 0; c0 < NOp; c0 += 8) {   // 8 columns of both parts at a time
+                        uint32_t oh[8], ol[8];
+                        tc_ld8(o_hi + c0, oh);
+                        tc_ld8(o_lo + c0, ol);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float a = c0 + i < NO ? ash[c0 + i] : 1.f;
+                            oh[i] = __float_as_uint(__uint_as_float(oh[i]) * a);
+                            ol[i] = __float_as_uint(__uint_as_float(ol[i]) * a);
+                        }
+                        tc_st8(o_hi + c0, oh);
+                        tc_st8(o_lo + c0, ol);
+                    }
                     tc_wait_st();
                 }
             }
-            // ---- weights, their hi / lo codes into P^T (row c hi, row 8 + c lo; byte = token)
-            float pr[8];
+            // ---- weights, their hi / lo codes into P^T of each unit: row (head hl, column c),
+            // byte = tile row; P buffer b was last read by the p.V of unit k - 2 (k - 1 for b1)
+            float pr0[G], pr1[G];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                pr[c] = sc[c] == -INFINITY ? 0.f : fast_exp2(sc[c] - m[c] + kPOff);
-                lp[c] += pr[c];
+            for (int c = 0; c < G; ++c) {
+                pr0[c] = sc0[c] == -INFINITY ? 0.f : fast_exp2(sc0[c] - m[c] + kPOff);
+                pr1[c] = sc1[c] == -INFINITY ? 0.f : fast_exp2(sc1[c] - m[c] + kPOff);
+                lp[c] += pr0[c] + pr1[c];
             }
-            if (n >= 1 && !mbar_wait_bounded(&p_empty[b], (n - 1) & 1)) {
+            if ((k >= 2 && !mbar_wait_bounded(&p_empty[b0], ((k >> 1) - 1) & 1)) ||
+                (nu == 2 && k >= 1 && !mbar_wait_bounded(&p_empty[b1], (((k + 1) >> 1) - 1) & 1))) {
                 fail();
                 break;
             }
-            uint8_t* pt = ptile + b * 2048;
+            uint8_t* pt0 = ptile + b0 * C::kPBytes;
+            uint8_t* pt1 = ptile + b1 * C::kPBytes;
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) {
+            for (int c = 0; c < G; c += 2) {
                 uint32_t hi, lo;
-                split_e4m3x2(pack2<true>(pr[c], pr[c + 1]), hi, lo);
-                pt[swz_byte(c, tid)] = (uint8_t)(hi & 0xff);
-                pt[swz_byte(c + 1, tid)] = (uint8_t)(hi >> 8);
-                pt[swz_byte(8 + c, tid)] = (uint8_t)(lo & 0xff);
-                pt[swz_byte(9 + c, tid)] = (uint8_t)(lo >> 8);
+                split_e4m3x2(pack2<true>(pr0[c], c + 1 < G ? pr0[c + 1] : 0.f), hi, lo);
+                pt0[poh[c]] = (uint8_t)(hi & 0xff);
+                pt0[pol[c]] = (uint8_t)(lo & 0xff);
+                if (c + 1 < G) {
+                    pt0[poh[c + 1]] = (uint8_t)(hi >> 8);
+                    pt0[pol[c + 1]] = (uint8_t)(lo >> 8);
+                }
+                if (nu == 2) {
+                    split_e4m3x2(pack2<true>(pr1[c], c + 1 < G ? pr1[c + 1] : 0.f), hi, lo);
+                    pt1[poh[c]] = (uint8_t)(hi & 0xff);
+                    pt1[pol[c]] = (uint8_t)(lo & 0xff);
+                    if (c + 1 < G) {
+                        pt1[poh[c + 1]] = (uint8_t)(hi >> 8);
+                        pt1[pol[c + 1]] = (uint8_t)(lo >> 8);
+                    }
+                }
             }
-            if (!valid) {   // weight 0 against V codes that may be NaN: zero this token's V row
-                uint4* vr = reinterpret_cast<uint4*>(stages + (size_t)st * kTcStage + kTcStage / 2 + tid * 128);
+            // weight 0 against V codes that may be NaN: zero this row of an invalid token's V tile
+            if (!valid0) {
+                uint4* vr = reinterpret_cast<uint4*>(stages + (size_t)st0 * kTcStage + kTcStage / 2 + tid * 128);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    vr[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (nu == 2 && !valid1) {
+                uint4* vr = reinterpret_cast<uint4*>(stages + (size_t)st1 * kTcStage + kTcStage / 2 + tid * 128);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     vr[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -718,82 +832,71 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&p_full[b]);
-
-            if (!u.last) {
-                ok = next_unit(w, u);
+            if (lane == 0) {
+                mbar_arrive(&p_full[b0]);
+                if (nu == 2)
+                    mbar_arrive(&p_full[b1]);
+            }
+            k += nu;
+            if (!last)
                 continue;
-            }
-            // ---- end of the segment: next segment's Q first (the tensor cores can start on it),
-            // then this segment's output
-            const TcUnit cur = u;
-            const int curL = L;
-            bool more = next_unit(w, u);
-            if (more) {
-                if (!write_q(u)) {
-                    fail();
-                    more = false;
-                } else {
-                    q_written = u.seg;
-                }
-            }
-            if (!mbar_wait_bounded(&o_full[j], (cur.seg >> 1) & 1)) {
+
+            // ---- end of the segment: its output
+            if (!mbar_wait_bounded(o_full, nseg & 1)) {
                 fail();
                 break;
             }
+            ++nseg;
             tc_fence_after();
-            uint32_t o[8];
-            tc_ld8(tmem + 32u + 8u * j + ((uint32_t)(warp * 32) << 16), o);
-            tc_wait_ld();
+            // l and the reference per (head, column) over the head's tokens
+#pragma unroll
+            for (int c = 0; c < G; ++c) {
+                float v = lp[c];
+#pragma unroll
+                for (int off = BS / 2; off >= 1; off >>= 1)
+                    v += __shfl_xor_sync(kFullMask, v, off);
+                if (t == 0) {
+                    lsh[hl * G + c] = v;
+                    msh[hl * G + c] = m[c];
+                }
+            }
+            if (!group_sync())
+                break;
+            const int stream = s * NHG + hg;
+            const bool direct = (flags & kTcDirect) != 0;
+#pragma unroll
+            for (int c0 = 0; c0 < NOp; c0 += 8) {   // row d = tid of O, 8 columns of both parts at a time
+                uint32_t oh[8], ol[8];
+                tc_ld8(o_hi + c0, oh);
+                tc_ld8(o_lo + c0, ol);
+                tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int nn = c0 + i;
+                    if (nn >= NO)
+                        continue;
+                    const int h2 = nn / G, c2 = nn - (nn / G) * G, head = hg * HPU + h2;
+                    const float o = __uint_as_float(oh[i]) + __uint_as_float(ol[i]);
+                    if (direct) {   // thread tid writes element d = tid of every row
+                        const float vs = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + head) : p.v_scale;
+                        const float l = lsh[nn];
+                        from_float(o * (l > 0.f ? vs / l : 0.f),
+                                   reinterpret_cast<QT*>(p.out) + query_row(p, s, head, c2) * D + tid);
+                    } else {        // a piece per (chunk, stream, head): o, then m, then l
+                        float* part = p.partials + ((size_t)(chunk + stream) * HPU + h2) * p.slot_floats;
+                        part[c2 * D + tid] = o;
+                        if (tid == nn) {
+                            part[G * D + c2] = msh[nn] - kPOff;   // the reference the weights were taken against
+                            part[G * D + G + c2] = lsh[nn];
+                        }
+                    }
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&o_empty[j]);
-            // l per column over the 128 tokens
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float v = lp[c];
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1)
-                    v += __shfl_xor_sync(kFullMask, v, off);
-                if (lane == 0)
-                    red[warp * 8 + c] = v;
-            }
-            if (!group_sync())
-                break;
-            float lsum[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                lsum[c] = red[c] + red[8 + c] + red[16 + c] + red[24 + c];
-            if (!group_sync())
-                break;
-            const float vs = p.v_head_scales ? p.v_scale * __ldg(p.v_head_scales + cur.h) : p.v_scale;
-            const int stream = cur.s * Hkv + cur.h;
-            const int first_chunk = ch.of(cur.stream_begin), last_chunk = ch.of(cur.stream_end - 1);
-            if (first_chunk == last_chunk && skipb == 0) {
-#pragma unroll
-                for (int c = 0; c < G; ++c) {
-                    const float inv = lsum[c] > 0.f ? vs / lsum[c] : 0.f;
-                    QT* dst = reinterpret_cast<QT*>(p.out) + query_row(p, cur.s, cur.h, c) * D + tid;
-                    from_float(__uint_as_float(o[c]) * inv, dst);
-                }
-            } else {
-                float* part = p.partials + (size_t)(cur.chunk + stream) * p.slot_floats;
-#pragma unroll
-                for (int c = 0; c < G; ++c)
-                    part[c * D + tid] = __uint_as_float(o[c]);
-#pragma unroll
-                for (int c = 0; c < G; ++c)
-                    if (tid == c) {
-                        part[G * D + c] = m[c] - kPOff;   // the reference the weights were taken against
-                        part[G * D + G + c] = lsum[c];
-                    }
-            }
-            (void)curL;
-            ok = more;
+                mbar_arrive(o_empty);   // O has been read: the next segment's p.V may overwrite it
         }
-        (void)q_written;
     }
 
     // a suffix pass launched behind a prefix pass completes only after it
@@ -802,36 +905,46 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols)
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
                      : "memory");
 }
 
 // ------------------------------------------------------------------ host side
 
+constexpr int kTcMaxStages = 8;
+constexpr int kTcTailChunksPerRun = 0;
+constexpr int kTcMinUnitsForTail = 32;
+constexpr int kTcMinTailChunk = 8;
+static_assert((1 + kTcTailChunksPerRun) * (kTcRows / 16) <= (1 + kTailChunksPerRun) * kMaxHeadGroup,
+              "piece slots of the workspace");
+
 template <class KV, class QT, int BS, int G>
 struct TcLauncher {
+    using C = TcCfg<KV, QT, BS, G>;
+
     static size_t smem_bytes(int num_seqs, int S)
     {
-        return (size_t)S * kTcStage + 4 * 2048 + (size_t)(2 * S + 18) * 8 + (size_t)S * 4 + kChunkRing * 4 + 8 +
-               (32 + 16 + 8) * 4 + (size_t)(num_seqs + 1) * 4 + 64;
+        return (size_t)S * (kTcStage + sizeof(TcDesc) + 2 * 8) + C::kQBytes + 2 * C::kPBytes + 14 * 8 +
+               (size_t)num_seqs * 8 + 8 + 8 * 4 + 4 * C::NO * 4 + (size_t)(num_seqs + 1) * 4 + 64;
     }
 
-    // Ring depth: two CTAs per SM, the rest of the SM's shared memory in stages
-    static int stages(int num_seqs)
+    // Ring depth: one CTA per SM, the SM's shared memory in stages
+    static int stages(int num_seqs, int* ctas)
     {
-        for (int S = 3; S >= 2; --S)
-            if (smem_bytes(num_seqs, S) + 1024 <= (size_t)kMaxSmemPerBlock / 2)
+        for (int S = kTcMaxStages; S >= 2; --S)
+            if (smem_bytes(num_seqs, S) <= (size_t)kMaxSmemPerBlock - 1024) {
+                *ctas = C::kCtasPerSm;
                 return S;
-        for (int S = 4; S >= 2; --S)   // many sequences: one CTA per SM
-            if (smem_bytes(num_seqs, S) + 1024 <= (size_t)kMaxSmemPerBlock)
-                return S;
+            }
+        *ctas = 0;
         return 0;
     }
 
     static int occupancy(int num_seqs)
     {
-        const int S = stages(num_seqs);
+        int cps = 0;
+        const int S = stages(num_seqs, &cps);
         if (S < 2)
             return 0;
         auto kern = paged_decode_tc05_kernel<KV, QT, BS, G>;
@@ -841,40 +954,48 @@ struct TcLauncher {
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kTcThreads, smem) != cudaSuccess)
             return 0;
-        return n < 2 ? n : 2;   // 2 x 64 TMEM columns per SM at most is what the kernel plans for
+        return n < cps ? n : cps;
     }
 
     static int launch(DecodeParams p, int nruns, cudaStream_t stream)
     {
-        const int S = stages(p.num_seqs);
-        if (S < 2)
+        int cps = 0;
+        const int S = stages(p.num_seqs, &cps);
+        if (S < 2 || p.num_kv_heads % C::HPU != 0)
             return PKV_ERR_SHAPE;
         const long long rows = (long long)p.num_blocks * p.num_kv_heads * BS;
         const int kvdt = KV::kFmt == __NV_E5M2 ? PKV_FP8_E5M2 : PKV_FP8_E4M3;
         CUtensorMap kmap, vmap;
-        if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, 128, rows, BS) ||
-            !make_cache_tensormap(&vmap, p.v_cache, kvdt, 128, rows, BS))
+        if (!make_cache_tensormap(&kmap, p.k_cache, kvdt, 128, rows, kTcRows) ||
+            !make_cache_tensormap(&vmap, p.v_cache, kvdt, 128, rows, kTcRows))
             return PKV_ERR_LAUNCH;
         auto kern = paged_decode_tc05_kernel<KV, QT, BS, G>;
         const size_t smem = smem_bytes(p.num_seqs, S);
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
+        // Units of 32 KB: a static split (tail chunks, of any size measured, cost more in extra
+        // segments and merges than the imbalance they remove). At most one tail chunk per run
+        // would keep the pieces within the workspace: a chunk leaves pieces of HPU (8) heads at
+        // slots (chunk + stream) * HPU + head, and 2 R chunks x 8 fit the R x 5 chunks x 4 heads
+        // the workspace reserves.
+        p.tail_chunks = kTcTailChunksPerRun;
+        p.tail_min_units = kTcMinUnitsForTail;
+        p.tail_min_chunk = kTcMinTailChunk;
         p.q_scale = p.scale * kLog2e * (!p.k_head_scales ? p.k_scale : 1.0f);
         p.v_scale = !p.v_head_scales ? p.v_scale_in : 1.0f;
         kern<<<nruns, kTcThreads, smem, stream>>>(kmap, vmap, p);
         if (cudaGetLastError() != cudaSuccess)
             return PKV_ERR_LAUNCH;
-        // the merge of split streams (one KV head per stream, 128-token units)
+        // the merge of split streams (head groups of HPU KV heads, one block per unit)
         const int items = p.num_seqs * p.num_kv_heads * G;
         const int per_cta = kMergeThreads / 32;
         int mgrid = (items + per_cta - 1) / per_cta;
         if (mgrid > 2 * nruns)
             mgrid = 2 * nruns;
         void* args[] = {&p, &nruns};
-        return MmaLauncher<KV, QT, 128, BS, G, 1>::launch_merge_pdl(
-            (const void*)paged_decode_merge_kernel<QT, 128, BS, G, 1, kTcUnit>, args, mgrid,
-            (size_t)(p.num_seqs + 1) * 4, stream);
+        return launch_merge_pdl((const void*)paged_decode_merge_kernel<QT, 128, BS, G, C::HPU, BS>, args, mgrid,
+                                (size_t)(p.num_seqs + 1) * 4, stream);
     }
 };
 

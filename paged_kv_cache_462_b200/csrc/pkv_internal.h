@@ -86,6 +86,10 @@ struct DecodeParams {
     // counter they are claimed from (zero before the launch; the merge kernel clears it after)
     int tail_chunks;
     int32_t* chunk_ctr;
+    // the chunk schedule's thresholds: units per CTA below which the split stays static, and the
+    // smallest tail chunk (kMinUnitsForTail / kMinTailChunk unless a kernel's units are larger)
+    int tail_min_units;
+    int tail_min_chunk;
 };
 
 // One request to the warp-MMA kernels of a shape (decode_mma_dispatch.cuh).

@@ -36,6 +36,18 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
+def test_fp8_kernel_choice(lib):
+    """The process-wide FP8 kernel choice: unknown values rejected, the previous value returned."""
+    assert lib.pkv_set_fp8_kernel(7) == -2
+    assert lib.pkv_set_fp8_kernel(-1) == -2
+    prev = lib.pkv_set_fp8_kernel(pkv.FP8_KERNEL_TCGEN05)
+    assert prev == pkv.FP8_KERNEL_MMA                      # the default
+    assert lib.pkv_set_fp8_kernel(pkv.FP8_KERNEL_MMA) == pkv.FP8_KERNEL_TCGEN05
+    assert pkv.set_fp8_kernel(pkv.FP8_KERNEL_MMA) == pkv.FP8_KERNEL_MMA
+    with pytest.raises(pkv.PkvError):
+        pkv.set_fp8_kernel(3)
+
+
 def test_status_strings(lib):
     for code in range(7):
         assert pkv.status_string(code)

@@ -134,10 +134,12 @@ def test_split_invariance_sweep():
     assert g.device_errors() == 0
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
-def test_full_size_sampled(cfg):
+@pytest.mark.parametrize("cfg,kv", [(1, None), (2, None), (3, None), (4, None), (2, "e4m3"), (3, "e4m3")])
+def test_full_size_sampled(cfg, kv, fp8_kernel):
     """Full workload in the benchmark's launch configuration; sampled sequences checked one by one."""
-    b = W.config_batch(cfg)
+    if fp8_kernel == "tcgen05" and (kv or W.config_spec(cfg).kv_dtype) not in ("e4m3", "e5m2"):
+        pytest.skip("the FP8 kernel choice only concerns FP8 caches")
+    b = W.config_batch(cfg) if kv is None else W.with_cache_dtype(W.config_batch(cfg), kv)
     g = GpuStep(b)
     out = g.step(0)
     torch.cuda.synchronize()
@@ -400,9 +402,41 @@ def test_e5m2_shapes(BS, G):
     assert np.all(g.out.float().cpu().numpy()[0] == 0)
 
 
+@pytest.fixture
+def tcgen05():
+    """FP8-cache decodes on the tcgen05 kernel for the test, the default kernel after it."""
+    prev = pkv.set_fp8_kernel(pkv.FP8_KERNEL_TCGEN05)
+    yield
+    pkv.set_fp8_kernel(prev)
+
+
+@pytest.fixture(params=["mma", "tcgen05"])
+def fp8_kernel(request):
+    """Both FP8-cache kernels in turn."""
+    prev = pkv.set_fp8_kernel(pkv.FP8_KERNEL_TCGEN05 if request.param == "tcgen05" else pkv.FP8_KERNEL_MMA)
+    yield request.param
+    pkv.set_fp8_kernel(prev)
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("BS", [16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 5, 8])
+def test_fp8_tensor_core_shapes(kv, BS, G, fp8_kernel):
+    """FP8 caches whose KV heads fill whole 128-row tiles (128 / block_size heads of a block per
+    unit, one and two head groups): ragged lengths, one and several partitions (streams split
+    across CTAs and merged), every output element against the oracle."""
+    hpu = 128 // BS
+    for Hkv in (hpu, 2 * hpu):
+        lengths = [0, 1, BS, BS + 1, 3 * BS - 1, 97, 200, 700]
+        b = W.build_batch(_spec(f"tc_{kv}_{BS}_{G}_{Hkv}", len(lengths), G * Hkv, Hkv, 128, BS, kv, lengths,
+                                seed=7000 + BS * 10 + G + Hkv))
+        g, _ = _check_step(b, partitions=(0, 5, 40))
+        assert np.all(g.out.float().cpu().numpy()[0] == 0)
+
+
 @pytest.mark.parametrize("cfg,over", [(1, dict(num_seqs=6)), (4, dict(num_seqs=5)), (3, dict(num_seqs=16)),
                                       (2, dict(num_seqs=2, lengths=("fixed", 2000)))])
-def test_e5m2_workloads_fused_step(cfg, over):
+def test_e5m2_workloads_fused_step(cfg, over, fp8_kernel):
     b = W.config_batch(cfg, kv_dtype="e5m2", **over)
     ref, okc, ovc = oracle.run_step(b)
     g = GpuStep(b)
@@ -439,6 +473,34 @@ def test_multi_query_causal(kv, BS, q_len, Hq, Hkv):
     g = GpuStep(b)
     g.append()
     rng = np.random.default_rng(q_len * 100 + Hq)
+    qm = W.f32_to_bf16_bits(rng.standard_normal((b.num_seqs, q_len, Hq, 128)).astype(np.float32))
+    ref = oracle.paged_decode(qm, "bf16", okc, ovc, kv, b.block_tables, b.seq_lens, Hq, Hkv, 128, BS, b.num_blocks,
+                              b.scale, b.k_scale, b.v_scale, q_len=q_len)
+    q = to_dev(qm, "bf16")
+    for parts in (0, 3):
+        out = torch.full_like(q, float("nan"))
+        ws = pkv.new_workspace(b.num_seqs, Hq * q_len, Hkv, 128, parts)
+        pkv.paged_attention_decode_mq(out, q, g.kc, g.vc, g.bt, g.sl, float(b.scale), float(b.k_scale),
+                                      float(b.v_scale), parts, ws)
+        torch.cuda.synchronize()
+        assert pkv.read_device_error(ws) == 0
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert np.max(np.abs(got - ref)) <= TOL[kv], parts
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("BS,q_len,Hq,Hkv", [(16, 2, 16, 8), (16, 4, 16, 8), (16, 5, 8, 8), (32, 2, 8, 4)])
+def test_multi_query_causal_fp8_tensor_core(kv, BS, q_len, Hq, Hkv, fp8_kernel):
+    """Several new tokens per sequence on FP8 caches whose heads fill whole 128-row tiles (the
+    columns of a KV head are its query heads x new tokens), against the oracle's causal definition."""
+    lengths = [1, q_len - 1, q_len, BS + 3, 3 * BS - 1, 97, 300]
+    b = W.build_batch(_spec(f"mqtc_{kv}_{BS}_{q_len}_{Hq}", len(lengths), Hq, Hkv, 128, BS, kv, lengths,
+                            seed=1900 + BS + q_len * 10 + Hq))
+    _, okc, ovc = oracle.run_step(b)
+    g = GpuStep(b)
+    g.append()
+    rng = np.random.default_rng(q_len * 100 + Hq + 7)
     qm = W.f32_to_bf16_bits(rng.standard_normal((b.num_seqs, q_len, Hq, 128)).astype(np.float32))
     ref = oracle.paged_decode(qm, "bf16", okc, ovc, kv, b.block_tables, b.seq_lens, Hq, Hkv, 128, BS, b.num_blocks,
                               b.scale, b.k_scale, b.v_scale, q_len=q_len)
@@ -520,7 +582,7 @@ def _head_scale_case(kv, parts, gain_k, gain_v):
 
 @pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
 @pytest.mark.parametrize("parts", [0, 5])
-def test_head_scales_append_and_decode(kv, parts):
+def test_head_scales_append_and_decode(kv, parts, fp8_kernel):
     """FP8 caches with one scale per KV head (heads of very different ranges): appends bit-exact
     and outputs within tolerance of the oracle using the same head scales, relative to each
     head's V range (outputs scale with it)."""
@@ -532,7 +594,7 @@ def test_head_scales_append_and_decode(kv, parts):
 
 @pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
 @pytest.mark.parametrize("parts", [0, 5])
-def test_head_scales_unit_range_values_absolute_tolerance(kv, parts):
+def test_head_scales_unit_range_values_absolute_tolerance(kv, parts, fp8_kernel):
     """Per-head scales that differ widely for K (ranges 0.05x .. 40x) and moderately for V
     (0.5x .. 2x, values of order one): every output within the plain absolute tolerance."""
     gain_k = np.geomspace(0.05, 40.0, 8).astype(np.float32)
@@ -543,7 +605,7 @@ def test_head_scales_unit_range_values_absolute_tolerance(kv, parts):
 
 @pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
 @pytest.mark.parametrize("qgain", [2.0 ** 8, 2.0 ** -16])
-def test_8bit_cache_query_magnitudes(kv, qgain):
+def test_8bit_cache_query_magnitudes(kv, qgain, fp8_kernel):
     """Queries far from unit size with 8-bit caches (q times 2^8: sharply peaked softmax; q times
     2^-16: nearly uniform): the fused step against the oracle on the same bf16 q."""
     b = W.config_batch(1, num_seqs=6, kv_dtype=kv)
@@ -605,10 +667,11 @@ def test_int8_workloads_fused_step(cfg, over):
 
 
 @pytest.mark.parametrize("kv", ["e4m3", "e5m2", "int8"])
-def test_every_8bit_code_reads_back_exactly(kv):
+@pytest.mark.parametrize("Hkv", [2, 8])
+def test_every_8bit_code_reads_back_exactly(kv, Hkv, fp8_kernel):
     """One cached token (softmax weight exactly 1) whose V rows hold every finite code of the
     format across two KV heads: with a unit scale the output row is each code's value, bit for
-    bit in bf16 (all of them are bf16 values): the kernel's widening of each code is exact."""
+    bit in bf16 (all of them are bf16 values): the kernel's use of each code is exact."""
     D, BS = 128, 16
     codes = np.arange(256, dtype=np.uint8)
     if kv == "e4m3":
@@ -619,12 +682,14 @@ def test_every_8bit_code_reads_back_exactly(kv):
         vals = codes.view(np.int8).astype(np.float32)
     bad = ~np.isfinite(vals)
     codes[bad], vals[bad] = 0, 0.0                          # NaN / infinite codes are not values
-    kc = torch.zeros((4, 2, BS, D), dtype=TORCH_DT[kv], device="cuda")
+    kc = torch.zeros((4, Hkv, BS, D), dtype=TORCH_DT[kv], device="cuda")
     vc = torch.zeros_like(kc)
-    vc.view(torch.uint8)[0, :, 0, :] = torch.from_numpy(codes.reshape(2, D)).cuda()
-    q = torch.ones((1, 2, D), dtype=torch.bfloat16, device="cuda")
+    vc.view(torch.uint8)[0, :2, 0, :] = torch.from_numpy(codes.reshape(2, D)).cuda()
+    q = torch.ones((1, Hkv, D), dtype=torch.bfloat16, device="cuda")
     out = torch.empty_like(q)
     pkv.paged_attention_decode(out, q, kc, vc, torch.zeros((1, 1), dtype=torch.int32, device="cuda"),
                                torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, 1.0, 1.0)
     torch.cuda.synchronize()
-    assert np.array_equal(out.float().cpu().numpy().reshape(-1), vals)
+    got = out.float().cpu().numpy()
+    assert np.array_equal(got[0, :2].reshape(-1), vals)
+    assert np.all(got[0, 2:] == 0)
