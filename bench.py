@@ -65,6 +65,9 @@ def parse_args():
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="cut the workload down to its first N sequences' draw (same distributions; for profiling "
                          "captures that must stay small)")
+    ap.add_argument("--fp8-kernel", choices=["mma", "tcgen05"], default="mma",
+                    help="kernel for E4M3 / E5M2 caches (pkv_set_fp8_kernel): warp-level MMA on widened codes "
+                         "(default) or tcgen05 on the 8-bit tiles")
     ap.add_argument("--no-targets", action="store_true",
                     help="skip the extra target points (long-context and mixed batch, bf16 and E4M3 caches)")
     return ap.parse_args()
@@ -542,8 +545,10 @@ def ours_arm(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pkv.load_library()
+    pkv.set_fp8_kernel(pkv.FP8_KERNEL_TCGEN05 if args.fp8_kernel == "tcgen05" else pkv.FP8_KERNEL_MMA)
 
     spec = workload_spec(args)
+    tc05 = args.fp8_kernel == "tcgen05" and spec.kv_dtype in ("e4m3", "e5m2")
     b = W.build_batch(spec, seed=spec.seed + 1000 * rank)
     state = DeviceState(torch, pkv, b, dev, args.partitions)
     state.set_q_len(args.q_len)
@@ -683,6 +688,7 @@ def ours_arm(args):
                          "paged_decode_step: reshape_and_cache then paged_attention_decode (two launches)"),
                 "l2": "cold: a 256 MiB read before every step, outside the step's CUDA events",
                 "replicas": world,
+                **({"fp8_kernel": args.fp8_kernel} if spec.kv_dtype in ("e4m3", "e5m2") else {}),
             },
             "seq_steps_per_s": world * spec.num_seqs / (ms_max * 1e-3),
             "step_us": dec_max * 1e3,
@@ -693,14 +699,16 @@ def ours_arm(args):
                 # events bracket the whole step: the decode kernel (append fused) and its merge kernel
                 "kernel": ("paged_decode_mma_kernel prefix pass + suffix pass (append fused) + "
                            "paged_decode_prefix_merge_kernel" if plan is not None and plan.num_groups > 0 else
-                           "paged_decode_mma_kernel (append fused) + paged_decode_merge_kernel" if fused
+                           "paged_decode_tc05_kernel (append fused) + paged_decode_merge_kernel" if fused and tc05
+                           else "paged_decode_mma_kernel (append fused) + paged_decode_merge_kernel" if fused
                            else "reshape_and_cache_kernel + paged_decode_kernel"),
                 "achieved": kern_gbs,
                 "peak": peak,
                 "peak_kind": peak_kind,
                 "unit": "GB/s",
                 "frac": kern_gbs / peak,
-                "traffic": kernel_traffic(args.config, spec.kv_dtype, plan is not None) if args.q_len == 1 else None,
+                "traffic": (kernel_traffic(args.config, spec.kv_dtype, plan is not None)
+                            if args.q_len == 1 and not tc05 else None),
                 "algorithmic_bytes": kern_bytes,
             },
             # fused: the decode kernel (append inside) + the merge kernel; else append + decode
