@@ -220,6 +220,7 @@ int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_
     p.counters = reinterpret_cast<int32_t*>(ws + lay.counters_off);
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
+    p.partial_slots = (long long)((workspace_bytes - lay.partials_off) / ((size_t)p.slot_floats * 4));
     p.q_len = q_len;
     p.k_head_scales = k_head_scales;
     p.v_head_scales = v_head_scales;

@@ -407,13 +407,26 @@ __global__ void __launch_bounds__(kTcThreads, (TcCfg<KV, QT, BS, G>::kCtasPerSm)
             return r;
         };
         int cur = blockIdx.x;
-        int nxt = ch.C;
-        if (lane == 0 && ch.C > ch.R)
-            nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
         bool aborted = false;
         int k = 0, issued = 0;
         while (cur < ch.C && !aborted) {
             const int cb = ch.begin(cur), ce = ch.end(cur);
+            // The next chunk is claimed as this one's last unit is issued: the claim's round trip
+            // overlaps the units still in the stages, and a CTA claims only once it is that far,
+            // so the CTAs of slower SMs take fewer tail chunks.
+            int nxt = ch.C;
+            bool claimed = false;
+            auto claim = [&]() {
+                if (claimed)
+                    return;
+                claimed = true;
+                if (ch.C > ch.R) {
+                    int v = 0;
+                    if (lane == 0)
+                        v = ch.R + atomicAdd(p.chunk_ctr, 1);
+                    nxt = __shfl_sync(kFullMask, v, 0);
+                }
+            };
             Look lk = look(cb, cb, ce);
             for (int x0 = cb; x0 < ce && !aborted; x0 += 32) {
                 const Look nx = look(x0 + 32, cb, ce);   // loads in flight while this batch is issued
@@ -424,6 +437,8 @@ __global__ void __launch_bounds__(kTcThreads, (TcCfg<KV, QT, BS, G>::kCtasPerSm)
                 const int row = lk.has && !bad ? (lk.phys * Hkv + lk.hg * HPU) * BS : -1;
                 const int nb = ce - x0 < 32 ? ce - x0 : 32;
                 for (int q = 0; q < nb && !aborted; ++q, ++k) {
+                    if (x0 + q == ce - 1)
+                        claim();
                     const int sq = __shfl_sync(kFullMask, lk.s, q), hgq = __shfl_sync(kFullMask, lk.hg, q);
                     const int jq = __shfl_sync(kFullMask, lk.j, q), nblq = __shfl_sync(kFullMask, lk.nbl, q);
                     const int rowq = __shfl_sync(kFullMask, row, q), fq = __shfl_sync(kFullMask, lk.flags, q);
@@ -458,9 +473,9 @@ __global__ void __launch_bounds__(kTcThreads, (TcCfg<KV, QT, BS, G>::kCtasPerSm)
                 }
                 lk = nx;
             }
-            cur = __shfl_sync(kFullMask, nxt, 0);
-            if (lane == 0 && cur < ch.C)
-                nxt = ch.R + atomicAdd(p.chunk_ctr, 1);
+            if (!aborted)
+                claim();   // an empty chunk
+            cur = nxt;
         }
         // end of the work: a stage without bytes whose descriptor says so
         if (lane == 0 && !aborted) {
@@ -913,11 +928,13 @@ __global__ void __launch_bounds__(kTcThreads, (TcCfg<KV, QT, BS, G>::kCtasPerSm)
 // ------------------------------------------------------------------ host side
 
 constexpr int kTcMaxStages = 8;
+// Static split by default: tail chunks, claimed late (as a CTA issues its chunk's last unit),
+// were measured at 8 to 16 units: each chunk is a new segment, and a segment boundary serialises
+// this kernel's pipeline (the output, then the next Q tile, then the first scores), so the extra
+// boundaries cost more than the per-SM imbalance they remove.
 constexpr int kTcTailChunksPerRun = 0;
 constexpr int kTcMinUnitsForTail = 32;
-constexpr int kTcMinTailChunk = 8;
-static_assert((1 + kTcTailChunksPerRun) * (kTcRows / 16) <= (1 + kTailChunksPerRun) * kMaxHeadGroup,
-              "piece slots of the workspace");
+constexpr int kTcMinTailChunk = 16;
 
 template <class KV, class QT, int BS, int G>
 struct TcLauncher {
@@ -974,12 +991,15 @@ struct TcLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
-        // Units of 32 KB: a static split (tail chunks, of any size measured, cost more in extra
-        // segments and merges than the imbalance they remove). At most one tail chunk per run
-        // would keep the pieces within the workspace: a chunk leaves pieces of HPU (8) heads at
-        // slots (chunk + stream) * HPU + head, and 2 R chunks x 8 fit the R x 5 chunks x 4 heads
-        // the workspace reserves.
-        p.tail_chunks = kTcTailChunksPerRun;
+        // Units of 32 KB: up to kTcTailChunksPerRun tail chunks per CTA, from kTcMinUnitsForTail
+        // units per CTA on, of kTcMinTailChunk units at least, claimed as CTAs run dry. A chunk
+        // leaves pieces of HPU heads at slots (chunk + stream) * HPU + head: as many tail chunks
+        // as the workspace's partial slots hold.
+        const long long pairs = (long long)p.num_seqs * p.num_kv_heads;
+        int tail = kTcTailChunksPerRun;
+        while (tail > 0 && (long long)nruns * (1 + tail) * C::HPU + pairs > p.partial_slots)
+            --tail;
+        p.tail_chunks = tail;
         p.tail_min_units = kTcMinUnitsForTail;
         p.tail_min_chunk = kTcMinTailChunk;
         p.q_scale = p.scale * kLog2e * (!p.k_head_scales ? p.k_scale : 1.0f);

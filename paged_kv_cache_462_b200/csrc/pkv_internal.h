@@ -90,6 +90,8 @@ struct DecodeParams {
     // smallest tail chunk (kMinUnitsForTail / kMinTailChunk unless a kernel's units are larger)
     int tail_min_units;
     int tail_min_chunk;
+    // partial slots the workspace holds (pieces of split streams, slot_floats floats each)
+    long long partial_slots;
 };
 
 // One request to the warp-MMA kernels of a shape (decode_mma_dispatch.cuh).
