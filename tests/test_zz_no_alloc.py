@@ -51,6 +51,25 @@ def test_static_matches_workspace_entry_point_twice(cfg):
         assert err <= TOL[b.spec.kv_dtype], err
 
 
+@pytest.mark.parametrize("cfg", [1, 4])
+def test_static_call_leaves_device_memory_unchanged(cfg):
+    """After two warm-up calls (the first resolves the array's address), further calls change
+    neither the device's free memory nor torch's allocation count: nothing is allocated."""
+    b = W.config_batch(cfg, num_seqs=24)
+    g = GpuStep(b)
+    g.append()
+    out = torch.empty_like(g.q)
+    for _ in range(2):
+        assert _call_static(g, out) == 0
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for _ in range(3):
+        assert _call_static(g, out) == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+
+
 def test_static_rejects_oversized_batch():
     # 16384 sequences x 8 KV heads need far more than the 32 MiB array: refused before any launch
     assert _fn()(None, None, None, None, None, None, 16384, 32, 8, 128, 16, 0.1, 64, 1024, 1, 1, 1.0, 1.0, 0,
