@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(Cfg<KV, QT, D, BS, G>::kThreads, 1) paged_deco
             bool ok = true;
             if (!aborted)
                 ok = !*abort_flag && mbar_wait_bounded(&full[st], parity);
-            if (__any_sync(kFullMask, !ok)) {   // one verdict for the whole warp
+            if (__any_sync(kFullMask, !ok)) {   // one decision for the whole warp
                 if (!aborted && lane == 0 && !*abort_flag) {
                     *abort_flag = 1;
                     atomicOr(p.err, PKV_DEVERR_TIMEOUT);
