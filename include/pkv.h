@@ -100,7 +100,8 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2, PKV_FP8_E5M2 = 3, PK
 /*
  * Bytes of device workspace paged_attention_decode needs: a 256-byte header
  * (error word, work-claim counters), one arrival counter per (sequence, kv
- * head) and fp32 split-KV partials (o[G][head_dim], m[G], l[G]) for up to
+ * head), one 8-byte completion stamp per work chunk (5 * num_partitions) and
+ * fp32 split-KV partials (o[G][head_dim], m[G], l[G]) for up to
  * 4 * (5 * num_partitions) + num_seqs * num_kv_heads segments (a partition's
  * share of the work is cut into at most 5 chunks). num_partitions = 0 sizes it
  * for the automatic partition count on the current device. Returns 0 for

@@ -2,6 +2,7 @@
 // Every entry point validates what the host can see and returns a pkv_status
 // before launching anything; nothing here allocates, frees or synchronises
 // (pkv_read_device_error excepted, which synchronises by design).
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <map>
@@ -53,7 +54,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int slot_floats_for(int group, int head_dim) { return (int)round_up((size_t)group * (head_dim + 2), 4); }
 
 struct WorkspaceLayout {
-    size_t counters_off, partials_off, bytes;
+    size_t counters_off, done_off, partials_off, bytes;
 };
 
 WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_dim, long long runs)
@@ -61,7 +62,9 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
     WorkspaceLayout w;
     const long long pairs = (long long)num_seqs * num_kv_heads;
     w.counters_off = kWorkspaceHeader;
-    w.partials_off = w.counters_off + round_up((size_t)pairs * 4, 256);
+    w.done_off = w.counters_off + round_up((size_t)pairs * 4, 256);
+    // one completion stamp (8 bytes) per chunk
+    w.partials_off = w.done_off + round_up((size_t)(runs * (1 + kTailChunksPerRun)) * 8, 256);
     // a chunk (a run's own or a tail chunk, 1 + kTailChunksPerRun per run at most) writes at most
     // one partial per (stream it touches, head of the stream's group)
     w.bytes = w.partials_off +
@@ -70,6 +73,16 @@ WorkspaceLayout layout_for(int num_seqs, int num_kv_heads, int group, int head_d
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A new value for every call (never 0, whose stamp a fresh zeroed workspace cannot hold anyway).
+uint32_t next_epoch()
+{
+    static std::atomic<uint32_t> g_epoch{0};
+    uint32_t e = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    if (e == 0)
+        e = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    return e;
+}
 
 // 8-bit caches quantised with scales (FP8 formats and INT8)
 bool is_fp8(int dtype) { return dtype == PKV_FP8_E4M3 || dtype == PKV_FP8_E5M2 || dtype == PKV_INT8; }
@@ -221,6 +234,8 @@ int decode_prepare(void* out, const void* q, const void* k_cache, const void* v_
     p.partials = reinterpret_cast<float*>(ws + lay.partials_off);
     p.slot_floats = slot_floats_for(group, head_dim);
     p.partial_slots = (long long)((workspace_bytes - lay.partials_off) / ((size_t)p.slot_floats * 4));
+    p.chunk_done = reinterpret_cast<unsigned long long*>(ws + lay.done_off);
+    p.epoch = next_epoch();
     p.q_len = q_len;
     p.k_head_scales = k_head_scales;
     p.v_head_scales = v_head_scales;
@@ -544,6 +559,7 @@ int shared_prefix_impl(void* out, const void* q, const void* k_cache, const void
     if (workspace_bytes < prefix_off + prefix_partials_bytes(num_groups, num_kv_heads, head_dim, runs_p))
         return PKV_ERR_WORKSPACE;
 
+    ps.chunk_done = nullptr;   // the shared-prefix merge waits for both passes' grids instead
     DecodeParams pp = ps;
     pp.num_seqs = num_groups;
     pp.seq_lens = group_lens;

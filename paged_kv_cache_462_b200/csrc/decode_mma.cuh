@@ -409,7 +409,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
     int* skip = reinterpret_cast<int*>(empty + S);
     volatile int* abort_flag = skip + S;
     int* chunk_ring = const_cast<int*>(abort_flag + 1);                       // [kChunkRing] chunk ids
-    int* prefix = chunk_ring + kChunkRing;                                     // [num_seqs + 1]
+    int* chunk_cnt = chunk_ring + kChunkRing;                                  // [kChunkRing] warps done
+    int* prefix = chunk_cnt + kChunkRing;                                      // [num_seqs + 1]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -430,6 +431,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
             mbar_init(&empty[i], W);
         }
         *abort_flag = 0;
+        for (int i = 0; i < kChunkRing; ++i)
+            chunk_cnt[i] = 0;
         fence_mbar_init();
     }
     {
@@ -988,6 +991,23 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                 }
             }
         }
+        // The chunk is done for this warp. The last of the W consumer warps to get here stamps it:
+        // every lane's writes are made visible device-wide first, so a merge that sees the stamp
+        // sees the pieces.
+        if (p.chunk_done != nullptr) {
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                int* cnt = &chunk_cnt[ordinal % kChunkRing];
+                if (atomicAdd(cnt, 1) == W - 1) {
+                    *cnt = 0;
+                    __threadfence();
+                    const unsigned long long v = chunk_stamp(p.epoch);
+                    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p.chunk_done + cur), "l"(v) : "memory");
+                }
+            }
+            __syncwarp();
+        }
     }
     // a suffix pass launched behind a prefix pass completes only after it (see the launcher)
     if (p.wait_prior_at_exit && tid == 0)
@@ -1085,8 +1105,10 @@ __device__ __forceinline__ void merge_split(const DecodeParams& p, int s, int st
 
 // Merge of the streams the decode kernel split across chunks: one warp per (stream, KV head of
 // its group, query column), launched behind the decode kernel as a programmatic dependent launch.
-// The prefix is built while the decode kernel still runs (it reads only seq_lens);
-// griddepcontrol.wait then holds until the decode grid has finished and its partials are visible.
+// The prefix is built while the decode kernel still runs (it reads only seq_lens). With chunk
+// completion stamps (DecodeParams::chunk_done) each split stream is merged once its chunks are
+// stamped, overlapping the decode grid's tail; otherwise griddepcontrol.wait holds until the
+// decode grid has finished and its partials are visible.
 constexpr int kMergeThreads = 128;
 
 // UT: tokens per unit of the decode kernel (the block size for the warp-MMA kernel, 128 for the
@@ -1097,27 +1119,64 @@ __global__ void __launch_bounds__(kMergeThreads) paged_decode_merge_kernel(const
     extern __shared__ int prefix[];   // [num_seqs + 1]
     const int NHG = p.num_kv_heads / HG;
     (void)build_unit_prefix(p, prefix, BS, NHG, p.max_blocks_per_seq * BS, UT);
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (blockIdx.x == 0 && threadIdx.x == 0)   // the decode grid is done claiming: ready for the next call
-        *p.chunk_ctr = 0;
+    // With completion stamps, a split stream is merged as soon as the chunks holding its pieces
+    // carry this call's stamp, while the decode grid still runs; without, after the whole grid.
+    const bool stamped = p.chunk_done != nullptr;
+    if (!stamped)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
     const int total = prefix[p.num_seqs];
-    if (total == 0)
-        return;
-    const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks, p.tail_min_units, p.tail_min_chunk);
     const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (kMergeThreads / 32);
-    const int items = p.num_seqs * NHG * HG * G;
-    for (int it = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5); it < items; it += warps) {
-        const int gq = it % G, sw = it / G;
-        const int stream = sw / HG, w = sw - stream * HG;
-        const int s = stream / NHG, hg = stream - s * NHG;
-        const int nb = (prefix[s + 1] - prefix[s]) / NHG;
-        if (nb == 0)
-            continue;
-        const int sb = prefix[s] + hg * nb;
-        const int first_run = ch.of(sb), last_run = ch.of(sb + nb - 1);
-        if (first_run != last_run)
+    if (total > 0) {
+        const Chunks ch = make_chunks(total, decode_runs, p.tail_chunks, p.tail_min_units, p.tail_min_chunk);
+        const unsigned long long want = chunk_stamp(p.epoch);
+        const int warps = gridDim.x * (kMergeThreads / 32);
+        const int items = p.num_seqs * NHG * HG * G;
+        for (int it = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5); it < items; it += warps) {
+            const int gq = it % G, sw = it / G;
+            const int stream = sw / HG, w = sw - stream * HG;
+            const int s = stream / NHG, hg = stream - s * NHG;
+            const int nb = (prefix[s + 1] - prefix[s]) / NHG;
+            if (nb == 0)
+                continue;
+            const int sb = prefix[s] + hg * nb;
+            const int first_run = ch.of(sb), last_run = ch.of(sb + nb - 1);
+            if (first_run == last_run)
+                continue;
+            if (stamped) {
+                // every chunk of the stream stamped (a bounded wait; a chunk whose CTA gave up is
+                // never stamped, and the call has flagged that already)
+                bool ok = true;
+                for (int c = first_run + lane; c <= last_run; c += 32) {
+                    const uint64_t t0 = global_ns();
+                    for (uint32_t polls = 0;; ++polls) {
+                        unsigned long long v;
+                        asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p.chunk_done + c) : "memory");
+                        if (v == want)
+                            break;
+                        if (polls >= kWaitLimitPolls || ((polls & 15u) == 15u && global_ns() - t0 > kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(200);
+                    }
+                    if (!ok)
+                        break;
+                }
+                __threadfence();
+                if (!__all_sync(kFullMask, ok)) {
+                    if (lane == 0)
+                        atomicOr(p.err, PKV_DEVERR_TIMEOUT);
+                    continue;
+                }
+            }
             merge_split<QT, D, G, HG>(p, s, stream, first_run, last_run - first_run + 1, NHG, w, gq, lane);
+        }
+    }
+    // the decode grid is done claiming: the counter is ready for the next call
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (stamped)
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+        *p.chunk_ctr = 0;
     }
 }
 
@@ -1249,19 +1308,19 @@ struct MmaLauncher {
 
     static size_t smem_bytes(int num_seqs, int S)
     {
-        return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + kChunkRing * 4 + (size_t)(num_seqs + 1) * 4 + 64;
+        return (size_t)S * C::kStage + (size_t)S * (8 + 8 + 4) + 16 + 2 * kChunkRing * 4 + (size_t)(num_seqs + 1) * 4 + 64;
     }
 
     // Ring depth: the SM's shared memory split between kCtasPerSM CTAs (~96 KB or ~64 KB of stages).
     static int stages(int num_seqs)
     {
         const long long budget = kMaxSmemPerBlock / C::kCtasPerSM - 1024;
-        const long long room = budget - 16 - kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64;
+        const long long room = budget - 16 - 2 * kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64;
         long long S = room / (C::kStage + 20);
         if (S > 8)
             S = 8;
         if (S < 2) {   // many sequences: fall back to one CTA per SM
-            S = ((long long)kMaxSmemPerBlock - 1024 - 16 - kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64) /
+            S = ((long long)kMaxSmemPerBlock - 1024 - 16 - 2 * kChunkRing * 4 - (long long)(num_seqs + 1) * 4 - 64) /
                 (C::kStage + 20);
             if (S > 8)
                 S = 8;

@@ -991,6 +991,7 @@ struct TcLauncher {
         if (!ensure_smem_attribute((const void*)kern, smem))
             return PKV_ERR_LAUNCH;
         p.stages_per_warp = S;
+        p.chunk_done = nullptr;   // this kernel does not stamp chunks: its merge waits for the grid
         // Units of 32 KB: up to kTcTailChunksPerRun tail chunks per CTA, from kTcMinUnitsForTail
         // units per CTA on, of kTcMinTailChunk units at least, claimed as CTAs run dry. A chunk
         // leaves pieces of HPU heads at slots (chunk + stream) * HPU + head: as many tail chunks

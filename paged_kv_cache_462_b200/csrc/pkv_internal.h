@@ -92,7 +92,19 @@ struct DecodeParams {
     int tail_min_chunk;
     // partial slots the workspace holds (pieces of split streams, slot_floats floats each)
     long long partial_slots;
+    // Per-chunk completion stamps (null: none): a CTA stores chunk_stamp(epoch) at
+    // chunk_done[chunk] once the chunk's pieces are written, and the merge starts on a split stream
+    // as soon as its chunks carry this call's stamp. epoch differs from call to call.
+    unsigned long long* chunk_done;
+    uint32_t epoch;
 };
+
+// The completion stamp of a chunk in the call with this epoch: the epoch and its complement, a
+// pattern that no value the workspace held before (partials, stamps of other calls) can match.
+__host__ __device__ __forceinline__ unsigned long long chunk_stamp(uint32_t epoch)
+{
+    return ((unsigned long long)epoch << 32) | (unsigned long long)(~epoch);
+}
 
 // One request to the warp-MMA kernels of a shape (decode_mma_dispatch.cuh).
 struct MmaOp {

@@ -55,11 +55,11 @@ def test_status_strings(lib):
 
 
 def test_workspace_size_with_explicit_partitions(lib):
-    # 64 seqs, 32/8 heads, d=128, 296 runs of up to 5 chunks: header + counters + (296 * 5 * 4 + 512) slots
-    # of 4*(128+2) floats
+    # 64 seqs, 32/8 heads, d=128, 296 runs of up to 5 chunks: header + counters + a completion stamp per
+    # chunk (296 * 5 * 8 bytes, rounded to 256) + (296 * 5 * 4 + 512) slots of 4*(128+2) floats
     n = lib.paged_attention_workspace_size(64, 32, 8, 128, 296)
     slot = 4 * (128 + 2)
-    assert n == 256 + 2048 + (296 * 5 * 4 + 512) * slot * 4
+    assert n == 256 + 2048 + (296 * 5 * 8 + 255) // 256 * 256 + (296 * 5 * 4 + 512) * slot * 4
     assert lib.paged_attention_workspace_size(64, 30, 8, 128, 296) == 0     # 30 % 8 != 0
     assert lib.paged_attention_workspace_size(64, 24, 8, 128, 296) == 0     # group 3 unsupported
     assert lib.paged_attention_workspace_size(64, 32, 8, 96, 296) == 0      # head_dim 96 unsupported
