@@ -35,13 +35,16 @@
 //  * Split streams (a stream cut by a run boundary): each run's warp stores its
 //    piece's fp32 partial (o, m, l) and moves on. A second, small kernel
 //    launched as a programmatic dependent launch merges them (log-sum-exp, a
-//    warp per stream and KV head) once the decode grid has finished: no fence,
-//    atomic or merge ever sits in the streaming kernel, whose memory system is
-//    saturated (a global round trip there costs microseconds), and the result
-//    does not depend on timing.
+//    warp per stream and KV head). The streaming kernel only stamps each chunk
+//    once its warps have written the chunk's pieces (a fence and one release
+//    store per chunk), and a merge warp starts on a stream when the stream's
+//    chunks carry this call's stamp: no atomic or merge sits in the streaming
+//    kernel, whose memory system is saturated (a global round trip there costs
+//    microseconds), and the result does not depend on timing.
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include <cuda.h>
 
@@ -67,6 +70,16 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
 {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// Two 16x16 byte matrices, transposed (sm_100a): lane i gives the address of row i & 15 of matrix
+// i >> 4 (16 bytes); lane (g = lane >> 2, t = lane & 3) receives in r[2j] byte g and in r[2j + 1]
+// byte g + 8 of rows 4t .. 4t + 3 of matrix j (row 4t + e in byte e).
+__device__ __forceinline__ void ldsm_b8_x2_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
@@ -136,6 +149,26 @@ __device__ __forceinline__ uint32_t widen2(uint32_t r)
             asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(o) : "h"(v));
             return o;
         }
+    }
+}
+
+// The code pairs (bytes 0, 1) and (bytes 2, 3) of r widened exactly to f16x2 (the lower byte in
+// the low half). E4M3 and E5M2: the hardware conversion of each 16-bit half of r, which takes no
+// permute (every E5M2 value is an f16 value too); INT8 as widen2 does.
+template <class KV>
+__device__ __forceinline__ void widen_halves(uint32_t r, uint32_t& w01, uint32_t& w23)
+{
+    if constexpr (!KV::kInt8 && KV::kFmt == __NV_E4M3) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+            : "=r"(w01), "=r"(w23) : "r"(r));
+    } else if constexpr (!KV::kInt8) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "cvt.rn.f16x2.e5m2x2 %0, lo;\n\tcvt.rn.f16x2.e5m2x2 %1, hi;\n\t}"
+            : "=r"(w01), "=r"(w23) : "r"(r));
+    } else {
+        w01 = widen2<KV, 0, 1>(r);
+        w23 = widen2<KV, 2, 3>(r);
     }
 }
 
@@ -283,6 +316,18 @@ struct MmaCfg {
 
 // Byte offset of the 16-byte chunk `c` (0..7) of box row `r` in a 128B-swizzled box.
 __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// 8-bit caches: the token (0-15 within a 16-token tile) that row r of the q.K MMA holds. Rows
+// 0-3, 4-7, 8-11, 12-15 hold tokens 0-3, 12-15, 4-7, 8-11: each 8-row half reads 8 distinct swizzle
+// positions, and so do the halves of the p.V loads (v_tok).
+__device__ __forceinline__ constexpr int tok_of_row(int r) { return r < 4 ? r : (r < 8 ? r + 8 : r - 4); }
+// The token at row i of the transposed p.V byte loads: lane (g, t) then holds tokens v_tok(4t),
+// v_tok(4t + 1) of the q.K row 2t (scores of rows 2t and 2t + 8) and v_tok(4t + 2), v_tok(4t + 3) of
+// row 2t + 1, so the softmax weights reach the p.V operand as packed pairs.
+__device__ __forceinline__ constexpr int v_tok(int i)
+{
+    return tok_of_row(2 * (i >> 2) + ((i >> 1) & 1) + 8 * (i & 1));
+}
 
 // Tokens of sequence s this pass streams: seq_lens[s] clamped to [0, capacity], less the
 // skip_blocks[s] leading blocks of a shared-prefix suffix pass (at most the full blocks). `err`
@@ -763,6 +808,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         float sc[4] = {0.f, 0.f, 0.f, 0.f};
                         float sd[4] = {0.f, 0.f, 0.f, 0.f};   // second accumulator: halves the MMA dependency chain
                         const int mi = lane >> 3, rr = lane & 7;
+                        // 8-bit caches: MMA row r of the tile holds token tok_of_row(r), so that this
+                        // lane's scores (rows g, g + 8) are the token pair its P^T value carries
+                        const int krow = r0 + tt * 16 + (F16 ? tok_of_row((mi & 1) * 8 + rr) : (mi & 1) * 8 + rr);
                         if constexpr (I8) {
                             // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment of
                             // 16 tokens x d 32kk .. 32kk+31 of INT8 codes as it lies in the stage, against
@@ -770,9 +818,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
 #pragma unroll
                             for (int kk = 0; kk < D / 32; ++kk) {
-                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
                                 uint32_t a[4];
-                                ldsm_x4(kbase + swz(row, 2 * kk + (mi >> 1)), a);
+                                ldsm_x4(kbase + swz(krow, 2 * kk + (mi >> 1)), a);
                                 mma_16832_s8(ih, a, qb[kk][0], qb[kk][1]);
                                 mma_16832_s8(il, a, qb[D / 32 + kk][0], qb[D / 32 + kk][1]);
                             }
@@ -784,14 +831,13 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             for (int ks = 0; ks < C::kKS; ks += 2) {
                                 // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each;
                                 // each lane's 4 codes of a row widen to the A pairs (d 4t, 4t+1 | 4t+2, 4t+3)
-                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
                                 uint32_t r[4];
-                                ldsm_x4(kbase + swz(row, ks + (mi >> 1)), r);
+                                ldsm_x4(kbase + swz(krow, ks + (mi >> 1)), r);
 #pragma unroll
                                 for (int h2 = 0; h2 < 2; ++h2) {
-                                    const uint32_t lo = r[2 * h2], hi = r[2 * h2 + 1];
-                                    const uint32_t a[4] = {widen2<KV, 0, 1>(lo), widen2<KV, 0, 1>(hi),
-                                                           widen2<KV, 2, 3>(lo), widen2<KV, 2, 3>(hi)};
+                                    uint32_t a[4];
+                                    widen_halves<KV>(r[2 * h2], a[0], a[2]);
+                                    widen_halves<KV>(r[2 * h2 + 1], a[1], a[3]);
                                     mma_16816<true>(h2 ? sd : sc, a, qb[ks + h2][0], qb[ks + h2][1]);
                                 }
                             }
@@ -799,10 +845,9 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
 #pragma unroll
                             for (int ks = 0; ks < C::kKS; ++ks) {
                                 // matrices: (tok 0-7, d 0-7), (tok 8-15, d 0-7), (tok 0-7, d 8-15), (tok 8-15, d 8-15)
-                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
                                 const int box = ks / 4, chunk = (ks % 4) * 2 + (mi >> 1);
                                 uint32_t a[4];
-                                ldsm_x4(kbase + box * C::kBoxBytes + swz(row, chunk), a);
+                                ldsm_x4(kbase + box * C::kBoxBytes + swz(krow, chunk), a);
                                 mma_16816<false>((ks & 1) ? sd : sc, a, qb[ks][0], qb[ks][1]);
                             }
                         }
@@ -815,10 +860,12 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         if constexpr (F16) {
 #pragma unroll
                             for (int dt = 0; dt < C::kDT; dt += 2) {
-                                // matrices: (tok 0-7 | 8-15) x (chunk dt | dt+1), transposed: pairs of tokens per code pair
-                                const int row = r0 + tt * 16 + (mi & 1) * 8 + rr;
+                                // matrices: the tile's 16 tokens x chunk dt | dt + 1 (d 16dt .. 16dt + 31),
+                                // transposed: r[0] = d 16dt + g of tokens v_tok(4t .. 4t + 3), r[1] = d +8,
+                                // r[2], r[3] the same for chunk dt + 1
+                                const int row = r0 + tt * 16 + v_tok(lane & 15);
                                 uint32_t r[4];
-                                ldsm_x4_t(vbase + swz(row, dt + (mi >> 1)), r);
+                                ldsm_b8_x2_t(vbase + swz(row, dt + (lane >> 4)), r);
 #pragma unroll
                                 for (int i = 0; i < 4; ++i)
                                     vf[2 * dt + i] = r[i];
@@ -843,11 +890,13 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             released = true;
                         }
                         // sc: (token g | g+8) x (heads 2t, 2t+1), in log2 units after the scale
-                        const int tok0 = jb * BS + tt * 16 + g;   // position in the sequence
+                        // positions in the sequence of rows g and g + 8
+                        const int tok0 = jb * BS + tt * 16 + (F16 ? tok_of_row(g) : g);
+                        const int tok8 = jb * BS + tt * 16 + (F16 ? tok_of_row(g + 8) : g + 8);
                         sc[0] = (tok0 < lim0) ? sc[0] * qk0 : -INFINITY;
                         sc[1] = (tok0 < lim1) ? sc[1] * qk1 : -INFINITY;
-                        sc[2] = (tok0 + 8 < lim0) ? sc[2] * qk0 : -INFINITY;
-                        sc[3] = (tok0 + 8 < lim1) ? sc[3] * qk1 : -INFINITY;
+                        sc[2] = (tok8 < lim0) ? sc[2] * qk0 : -INFINITY;
+                        sc[3] = (tok8 < lim1) ? sc[3] * qk1 : -INFINITY;
                         // The reference moves only when some score passes it by the slack; each lane
                         // tests its own scores first, so the butterfly max runs only when one does
                         // (same result as reducing first: the tile max passes iff some lane's does).
@@ -889,28 +938,49 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                             const uint32_t xa = __shfl_sync(kFullMask, X, srcA), ya = __shfl_sync(kFullMask, Y, srcA);
                             const uint32_t xb = __shfl_sync(kFullMask, X, srcB), yb = __shfl_sync(kFullMask, Y, srcB);
                             const uint32_t va = (g & 1) ? ya : xa, vb = (g & 1) ? yb : xb;
-                            pb0 = qcol ? __byte_perm(va, vb, 0x5410) : 0u;
-                            pb1 = qcol ? __byte_perm(va, vb, 0x7632) : 0u;
+                            if constexpr (F16) {
+                                // 8-bit caches: lane 4(2t) + g/2 holds tokens v_tok(4t), v_tok(4t + 1) of
+                                // head g, lane 4(2t + 1) + g/2 tokens v_tok(4t + 2), v_tok(4t + 3)
+                                pb0 = qcol ? va : 0u;
+                                pb1 = qcol ? vb : 0u;
+                            } else {
+                                pb0 = qcol ? __byte_perm(va, vb, 0x5410) : 0u;
+                                pb1 = qcol ? __byte_perm(va, vb, 0x7632) : 0u;
+                            }
                         }
                         // ---- O^T += V^T P^T : head_dim x 8 heads, k = the tile's 16 tokens
                         const bool partial = valid < tt * 16 + 16;
                         if constexpr (F16) {
+                            // byte e of a V register is token v_tok(4t + e): in a partial tile the codes
+                            // past the sequence's end are cleared (stale codes may be NaN); full tiles
+                            // run a copy of the loop without the masks
+                            auto pv = [&](auto masked, uint32_t keep) {
 #pragma unroll
-                            for (int dt = 0; dt < C::kDT; dt += 2) {
+                                for (int dt = 0; dt < C::kDT; dt += 2) {
 #pragma unroll
-                                for (int h2 = 0; h2 < 2; ++h2) {
-                                    uint32_t lo = vf[2 * dt + 2 * h2], hi = vf[2 * dt + 2 * h2 + 1];   // tokens 2t,2t+1 | 2t+8,2t+9
-                                    if (partial) {
-                                        const int tk = tt * 16 + 2 * t;
-                                        lo &= (tk < valid ? 0x0000ffffu : 0u) | (tk + 1 < valid ? 0xffff0000u : 0u);
-                                        hi &= (tk + 8 < valid ? 0x0000ffffu : 0u) | (tk + 9 < valid ? 0xffff0000u : 0u);
+                                    for (int h2 = 0; h2 < 2; ++h2) {
+                                        // d 16(dt + h2) + g (row g) and + 8 (row g + 8); k 2t, 2t+1 are tokens
+                                        // v_tok(4t), v_tok(4t + 1) (bytes 0, 1), k 2t+8, 2t+9 bytes 2, 3
+                                        uint32_t rg = vf[2 * dt + 2 * h2], rg8 = vf[2 * dt + 2 * h2 + 1];
+                                        if constexpr (decltype(masked)::value) {
+                                            rg &= keep;
+                                            rg8 &= keep;
+                                        }
+                                        uint32_t a[4];
+                                        widen_halves<KV>(rg, a[0], a[2]);
+                                        widen_halves<KV>(rg8, a[1], a[3]);
+                                        mma_16816<true>(o[dt + h2], a, pb0, pb1);
                                     }
-                                    // bytes (d 2g, tok a), (d 2g+1, tok a), (d 2g, tok a+1), (d 2g+1, tok a+1):
-                                    // A pairs (tok a, a+1) of d 2g from bytes 0, 2 and of d 2g+1 from 1, 3
-                                    const uint32_t a[4] = {widen2<KV, 0, 2>(lo), widen2<KV, 1, 3>(lo),
-                                                           widen2<KV, 0, 2>(hi), widen2<KV, 1, 3>(hi)};
-                                    mma_16816<true>(o[dt + h2], a, pb0, pb1);
                                 }
+                            };
+                            if (partial) {
+                                uint32_t keep = 0u;
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    keep |= (tt * 16 + v_tok(4 * t + e) < valid) ? 0xffu << (8 * e) : 0u;
+                                pv(std::true_type{}, keep);
+                            } else {
+                                pv(std::false_type{}, 0u);
                             }
                         } else {
 #pragma unroll
@@ -948,7 +1018,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
             const int stream = s * NHG + hg;
             // element (head column c, row d) of this lane's accumulators
             auto d_of = [&](int dt, int half) -> int {
-                return F16 ? dt * 16 + 2 * g + half : dt * 16 + g + 8 * half;
+                return dt * 16 + g + 8 * half;
             };
             // a whole stream writes `out`; pieces of split streams, every stream of a prefix pass and
             // the suffix of a sequence with shared blocks leave (o, m, l) for the merge
