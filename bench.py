@@ -61,7 +61,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--prefix-sharing", choices=["auto", "on", "off"], default="auto",
                     help="shared-prefix decode (blocks a plan shares read once per group): auto = on for "
-                         "workloads whose sequences share prefix blocks (config 3)")
+                         "workloads whose sequences share prefix blocks (config 3) with a bf16 cache, off with "
+                         "an 8-bit cache (there the plain step measured faster)")
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="cut the workload down to its first N sequences' draw (same distributions; for profiling "
                          "captures that must stay small)")
@@ -499,10 +500,17 @@ def pack_step_inputs(torch, tensors: dict, dev):
 
 
 def use_prefix_plan(args, spec) -> bool:
-    """The shared-prefix decode for workloads whose sequences share prefix blocks (or when asked)."""
+    """The shared-prefix decode for workloads whose sequences share prefix blocks (or when asked).
+
+    By default only with a bf16 cache: there the step is HBM-bound and reading each shared block
+    once per group saves its bytes (config 3: 398 against 418 us per step). With an 8-bit cache
+    the decode is bound by its consumer warps, not HBM, so the bytes saved buy nothing while the
+    prefix pass and its merge add work (config 3 with an E4M3 cache: 261 against 245 us)."""
     if args.q_len != 1 or args.prefix_sharing == "off" or spec.kv_dtype == "f32":
         return False
-    return args.prefix_sharing == "on" or spec.share_group > 1
+    if args.prefix_sharing == "on":
+        return True
+    return spec.share_group > 1 and spec.kv_dtype == "bf16"
 
 
 def time_steps(torch, state, K: int, warmup: int, flush_l2, stream, dev):
