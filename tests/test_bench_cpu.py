@@ -58,3 +58,32 @@ def test_oracle_timing_on_all_cores():
     one = bench.time_oracle_threads(items, 0.3, 1)
     many = bench.time_oracle_threads(items, 0.3, 4)
     assert one[0] > 0 and one[1] > 0 and many[1] >= 4
+
+
+def test_prefix_sharing_choice():
+    """`--prefix-sharing auto` takes the shared-prefix step for bf16 caches of workloads that share
+    prefix blocks and the plain step for 8-bit caches; `on` / `off` override it, and multi-query
+    decode and f32 caches never take it."""
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    import workloads as W
+    spec = W.config_spec(3)
+    assert spec.share_group > 1 and spec.kv_dtype == "bf16"
+
+    def args(mode="auto", q_len=1):
+        return argparse.Namespace(prefix_sharing=mode, q_len=q_len)
+
+    def typed(kv):
+        s = W.config_spec(3)
+        s.kv_dtype = kv
+        return s
+
+    assert bench.use_prefix_plan(args(), spec)
+    for kv in ("e4m3", "e5m2", "int8"):
+        assert not bench.use_prefix_plan(args(), typed(kv))
+        assert bench.use_prefix_plan(args("on"), typed(kv))
+    assert not bench.use_prefix_plan(args("off"), spec)
+    assert not bench.use_prefix_plan(args(q_len=2), spec)
+    assert not bench.use_prefix_plan(args("on"), typed("f32"))
+    assert not bench.use_prefix_plan(args(), W.config_spec(2))   # no shared prefixes
