@@ -29,9 +29,13 @@
 //    running max (moved only when a tile max passes it by 8, in log2 units),
 //    P^T re-laid out with 4 shuffles into the B operand of O^T += V^T P^T
 //    (head_dim x 8 heads, k = 16 tokens). bf16 caches use bf16 MMA; 8-bit codes
-//    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2 / .e5m2x2; for INT8 a byte
-//    permute and one f16 subtraction) and use f16 MMA, the per-tensor or
-//    per-head scales applied to the fp32 scores and outputs.
+//    are widened exactly to f16 (cvt.rn.f16x2.e4m3x2 / .e5m2x2 on a 16-bit half
+//    of the loaded register; for INT8 a byte permute and one f16 subtraction)
+//    and use f16 MMA, the per-tensor or per-head scales applied to the fp32
+//    scores and outputs. For 8-bit caches the V codes come through the
+//    transposed byte ldmatrix (four consecutive tokens of one d per lane) and
+//    the tile's tokens take a fixed order (tok_of_row, v_tok) so that each
+//    shuffled P^T word holds the two tokens of its MMA k pair.
 //  * Split streams (a stream cut by a run boundary): each run's warp stores its
 //    piece's fp32 partial (o, m, l) and moves on. A second, small kernel
 //    launched as a programmatic dependent launch merges them (log-sum-exp, a
@@ -126,35 +130,21 @@ __device__ __forceinline__ void split_s8x4(const float (&v)[4], uint32_t& hi, ui
     }
 }
 
-// Bytes B0 and B1 of r (two 8-bit codes) as an f16x2 (byte B0 in the low half), exact:
-//  * E5M2 codes are the high bytes of the f16 of the same value: one byte permute.
-//  * E4M3: the hardware conversion of the code pair. (Placing s.eeee.mmm as the f16 bits
-//    s.0eeee.mmm0000000, the value times 2^-8 for normal and subnormal codes alike, takes a
-//    permute, a shift and two logic operations instead and measured slower.)
-//  * INT8: the offset byte x + 128 as the mantissa of 1024.0 gives the f16 1152 + x; less 1152.
-template <class KV, int B0, int B1>
-__device__ __forceinline__ uint32_t widen2(uint32_t r)
+// INT8 codes in bytes B0 and B1 of r as an exact f16x2 (byte B0 in the low half): the offset
+// byte x + 128 as the mantissa of 1024.0 gives the f16 1152 + x; less 1152.
+template <int B0, int B1>
+__device__ __forceinline__ uint32_t widen2_i8(uint32_t r)
 {
-    if constexpr (KV::kInt8) {
-        const uint32_t x = __byte_perm(r ^ 0x80808080u, 0x64646464u, B0 | (4 << 4) | (B1 << 8) | (4 << 12));
-        const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&x), __halves2half2(__ushort_as_half(0x6480),
-                                                                                      __ushort_as_half(0x6480)));
-        return *reinterpret_cast<const uint32_t*>(&h);
-    } else {
-        if constexpr (KV::kFmt == __NV_E5M2) {
-            return __byte_perm(r, 0u, 4 | (B0 << 4) | (4 << 8) | (B1 << 12));   // [0, c0, 0, c1]
-        } else {
-            uint32_t o;
-            const uint16_t v = static_cast<uint16_t>(__byte_perm(r, 0u, B0 | (B1 << 4)));
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(o) : "h"(v));
-            return o;
-        }
-    }
+    const uint32_t x = __byte_perm(r ^ 0x80808080u, 0x64646464u, B0 | (4 << 4) | (B1 << 8) | (4 << 12));
+    const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&x), __halves2half2(__ushort_as_half(0x6480),
+                                                                                  __ushort_as_half(0x6480)));
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // The code pairs (bytes 0, 1) and (bytes 2, 3) of r widened exactly to f16x2 (the lower byte in
 // the low half). E4M3 and E5M2: the hardware conversion of each 16-bit half of r, which takes no
-// permute (every E5M2 value is an f16 value too); INT8 as widen2 does.
+// permute (every E5M2 value is an f16 value too; placing E4M3 bits in an f16 instead, the value
+// times 2^-8, took more instructions and measured slower); INT8: widen2_i8.
 template <class KV>
 __device__ __forceinline__ void widen_halves(uint32_t r, uint32_t& w01, uint32_t& w23)
 {
@@ -167,8 +157,8 @@ __device__ __forceinline__ void widen_halves(uint32_t r, uint32_t& w01, uint32_t
             "cvt.rn.f16x2.e5m2x2 %0, lo;\n\tcvt.rn.f16x2.e5m2x2 %1, hi;\n\t}"
             : "=r"(w01), "=r"(w23) : "r"(r));
     } else {
-        w01 = widen2<KV, 0, 1>(r);
-        w23 = widen2<KV, 2, 3>(r);
+        w01 = widen2_i8<0, 1>(r);
+        w23 = widen2_i8<2, 3>(r);
     }
 }
 
@@ -286,7 +276,7 @@ __device__ __forceinline__ size_t query_row(const DecodeParams& p, int s, int he
 // their query heads), 8 each, against the same staged K/V tile.
 template <class KV, int D, int BS, int G, int HG, bool PFX = false>
 struct MmaCfg {
-    // products: bf16 caches in bf16 MMA; 8-bit codes widened exactly to f16 (widen2) for f16 MMA,
+    // products: bf16 caches in bf16 MMA; 8-bit codes widened exactly to f16 (widen_halves) for f16 MMA,
     // q scaled per column by a power of two into f16's range; INT8 q.K on integer MMA (K codes as
     // they are, q as s8 hi + lo) when kInt8Imma
     static constexpr bool kF16 = KV::kBytes == 1;
@@ -812,8 +802,8 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         // lane's scores (rows g, g + 8) are the token pair its P^T value carries
                         const int krow = r0 + tt * 16 + (F16 ? tok_of_row((mi & 1) * 8 + rr) : (mi & 1) * 8 + rr);
                         if constexpr (I8) {
-                            // matrices (tok 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment of
-                            // 16 tokens x d 32kk .. 32kk+31 of INT8 codes as it lies in the stage, against
+                            // matrices (MMA rows 0-7 | 8-15) x (chunk 2kk | 2kk+1): the m16n8k32 A fragment
+                            // of 16 tokens x d 32kk .. 32kk+31 of INT8 codes as it lies in the stage, against
                             // q's s8 hi and lo: exact int32 sums, combined as 128 hi + lo
                             int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -829,7 +819,7 @@ __global__ void __launch_bounds__(MmaCfg<KV, D, BS, G, HG, PFX>::kThreads, MmaCf
                         } else if constexpr (F16) {
 #pragma unroll
                             for (int ks = 0; ks < C::kKS; ks += 2) {
-                                // matrices: (tok 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each;
+                                // matrices: (MMA rows 0-7 | 8-15) x (chunk ks | ks+1), 8 tokens x 16 codes each;
                                 // each lane's 4 codes of a row widen to the A pairs (d 4t, 4t+1 | 4t+2, 4t+3)
                                 uint32_t r[4];
                                 ldsm_x4(kbase + swz(krow, ks + (mi >> 1)), r);
